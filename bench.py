@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Benchmark of the gated delta-rule chunk forward+backward on B200.
+
+One step = one pass of the whole path on one batch of synthetic input:
+sf_segment_run over the sequence split into N segments (forward over the
+segments with the state handed on, then backward in reverse with the state
+gradient handed back), i.e. UT transform, chunk scan, output, recompute,
+reverse state-gradient scan and the parallel gradient kernel for every segment.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--segments N] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `value` is Mtokens/s of forward+backward over
+all ranks (each rank runs its own independent batch: weak scaling, no
+collective on the data path).  `--impl reference` times the fp64 CPU oracle on
+a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "gated-delta chunk fwd+bwd Mtokens/s at H=16,d=128; % of bf16 roofline"
+UNIT = "Mtokens/s"
+DEFAULT_WORKLOAD = "headline_h16_t64k"
+DEFAULT_SEGMENTS = 16
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ------------------------------------------------------------ work model ----
+# Algorithmic work of the method (its GEMMs, no recompute; bytes across the
+# boundary with bf16 I/O and fp32 g/beta), per token per head.
+
+def algo_flops_per_token_head(C, dk, dv, use_beta=True):
+    if use_beta:
+        fwd = 2 * C * (3 * dk + 2 * dv) + 6 * dk * dv
+        bwd = 2 * C * (5 * dk + 4 * dv) + 12 * dk * dv
+    else:
+        fwd = 2 * C * (dk + dv) + 4 * dk * dv
+        bwd = 2 * C * (2 * dk + 2 * dv) + 8 * dk * dv
+    return fwd, bwd
+
+
+def algo_bytes_per_token_head(dk, dv, esize=2, use_beta=True):
+    gb = 8 if use_beta else 4
+    fwd = esize * (2 * dk + dv) + gb + esize * dv
+    bwd = esize * (2 * dk + dv) + gb + esize * dv + esize * (2 * dk + dv) + gb
+    return fwd, bwd
+
+
+def kernel_work(name, w, T_seg):
+    """(bound, algorithmic flops, algorithmic bytes) of ONE launch of `name`
+    on a segment of T_seg tokens (all B*H heads)."""
+    C, dk, dv = w.C, w.dk, w.dv
+    es = 2 if w.io == "bf16" else 4
+    n = w.B * w.H * T_seg                      # token-heads in the launch
+    nch = w.B * w.H * ((T_seg + C - 1) // C)   # chunk-heads in the launch
+    wu = 4 if name.startswith("simt") else 2   # W/U/V_new storage bytes per element
+    if name.endswith("prep"):
+        flops = nch * (2 * C * C * dk + 2 * C * C * dk + 2 * C * C * dv)
+        byts = n * (es * (dk + dv) + 8 + wu * (dk + dv))
+        return "hbm", flops, byts
+    if name.endswith("scan_fwd"):
+        flops = nch * 2 * (2 * C * dk * dv)
+        byts = n * (wu * (dk + dv) + es * dk + wu * dv)
+        return "tensor", flops, byts
+    if name.endswith("scan_bwd"):
+        flops = nch * 2 * (2 * C * dk * dv) + nch * 2 * C * dk * dv
+        byts = n * (es * (2 * dk + dv) + wu * dv * 2)
+        return "tensor", flops, byts
+    if name.endswith("out"):
+        flops = nch * (2 * C * dk * dv + 2 * C * C * dk + 2 * C * C * dv)
+        byts = n * (es * (2 * dk + dv)) + nch * dk * dv * 4
+        return "hbm", flops, byts
+    if name.endswith("bwd_intra"):
+        flops = nch * (2 * C * C * dk + 2 * C * C * dv)
+        byts = n * (es * (2 * dk + dv) + wu * dv)
+        return "hbm", flops, byts
+    # parallel gradient kernel: dP K, dP^T Q, dW (gamma K)^T, T^T dW, dA K (C^2 dk each),
+    # dO V_new^T, dU V^T, T^T dU (C^2 dv each), dO S0^T, V_new dS^T, dV_new S0^T (C dk dv each)
+    flops = nch * (2 * C * C * 5 * dk + 2 * C * C * 3 * dv + 3 * 2 * C * dk * dv)
+    byts = (n * (es * (2 * dk + 2 * dv) + 8 + 2 * wu * dv + es * (2 * dk + dv) + 8)
+            + nch * 2 * dk * dv * 4)
+    return "hbm", flops, byts
+
+
+# ---------------------------------------------------------------- helpers ---
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.idx = device_index
+        self.out = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.idx)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------- reference arm ---
+
+def run_reference(args):
+    """Time the fp64 CPU oracle (as it stands) on a bounded sample of the workload."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import numpy as np  # noqa: F401
+    import oracle
+    from chunked_gated_delta_13_b200.inputs import CONFIGS, as_f64, make_inputs
+
+    w = CONFIGS[args.workload]
+    seg = args.segments if args.segments else w.N
+    budget_s = float(os.environ.get("SF_REF_STEP_SECONDS", "1.5"))
+
+    def sample_inputs(T):
+        f = as_f64(make_inputs(w.with_(T=T)))
+        return f
+
+    def one_step(f, T):
+        N = max(1, min(seg, T // w.C)) if T >= w.C else 1
+        oracle.segment_run(f["q"], f["k"], f["v"], f["g"], f["beta"], f["S_in"], f["dO"],
+                           f["dS_out"], N=N)
+
+    # calibrate the T-prefix so that one step takes about `budget_s`
+    T_cal = min(w.T, 256)
+    f = sample_inputs(T_cal)
+    t = time.perf_counter()
+    one_step(f, T_cal)
+    dt = time.perf_counter() - t
+    T_s = int(max(w.C, min(w.T, T_cal * budget_s / max(dt, 1e-6))) // w.C * w.C)
+    f = sample_inputs(T_s)
+    for _ in range(args.warmup):
+        one_step(f, T_s)
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        one_step(f, T_s)
+        times.append(time.perf_counter() - t)
+    per = sum(times) / len(times)
+    value = w.B * T_s / per / 1e6
+    sample = (f"{w.B}x{w.H} heads x first {T_s} of {w.T} tokens (fp64, fwd+bwd, "
+              f"{min(seg, max(1, T_s // w.C))} segments); cost is linear in tokens")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": T_s, "T_full": w.T, "dk": w.dk,
+                   "dv": w.dv, "C": w.C, "segments": seg},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline(w, seg, seconds=15.0):
+    """The oracle on a bounded T-prefix of the workload, all heads (rank 0, N=1)."""
+    import oracle
+    from chunked_gated_delta_13_b200.inputs import as_f64, make_inputs
+    T_cal = min(w.T, 256)
+    f = as_f64(make_inputs(w.with_(T=T_cal)))
+    t = time.perf_counter()
+    oracle.segment_run(f["q"], f["k"], f["v"], f["g"], f["beta"], f["S_in"], f["dO"], f["dS_out"],
+                       N=1)
+    dt = time.perf_counter() - t
+    T_s = int(max(w.C, min(w.T, T_cal * seconds / max(dt, 1e-6))) // w.C * w.C)
+    f = as_f64(make_inputs(w.with_(T=T_s)))
+    N = max(1, min(seg, T_s // w.C))
+    t = time.perf_counter()
+    oracle.segment_run(f["q"], f["k"], f["v"], f["g"], f["beta"], f["S_in"], f["dO"], f["dS_out"],
+                       N=N)
+    dt = time.perf_counter() - t
+    return {"value": w.B * T_s / dt / 1e6, "unit": UNIT, "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": f"{w.B}x{w.H} heads x first {T_s} of {w.T} tokens, fp64 fwd+bwd, "
+                      f"{N} segments, {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------- our arm ---
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import chunked_gated_delta_13_b200 as sf
+    from chunked_gated_delta_13_b200.inputs import CONFIGS, make_inputs
+
+    ws, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", rank=rank, world_size=ws,
+                                timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = CONFIGS[args.workload].with_(seed=CONFIGS[args.workload].seed + rank)
+    seg = args.segments if args.segments else w.N
+    inp_cpu = make_inputs(w)
+    d = {k: None if v is None else v.to(dev).contiguous() for k, v in inp_cpu.items()}
+    shape = sf.make_shape(w.B, w.H, w.T, w.dk, w.dv, w.C, w.io, w.use_beta, w.scale)
+    stream = torch.cuda.current_stream(dev)
+    nbytes = sf.segment_workspace_bytes(shape, seg)
+    wsbuf = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    out = {"o": torch.empty_like(d["v"]),
+           "S_out": torch.empty(w.B, w.H, w.dk, w.dv, dtype=torch.float32, device=dev),
+           "dq": torch.empty_like(d["q"]), "dk": torch.empty_like(d["k"]),
+           "dv": torch.empty_like(d["v"]),
+           "dg": torch.empty(w.B, w.H, w.T, dtype=torch.float32, device=dev),
+           "dbeta": None if d["beta"] is None else torch.empty_like(d["beta"]),
+           "dS_in": torch.empty(w.B, w.H, w.dk, w.dv, dtype=torch.float32, device=dev)}
+
+    def step(src=d):
+        sf.segment_run(src["q"], src["k"], src["v"], src["g"], src["beta"], src["S_in"], src["dO"],
+                       src["dS_out"], N=seg, C=w.C, scale=w.scale, out=out, workspace=wsbuf,
+                       stream=stream)
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if ws == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else local)
+    clocks.start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    # kernel launch observer: CUDA events around every kernel on its stream
+    rec = []
+
+    def hook(name, after, stream_handle):
+        # every launch of this step goes to `stream` (the handle passed to the library)
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(stream)
+        rec.append((name, after, ev))
+
+    sf.set_launch_hook(hook)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    sf.set_launch_hook(None)
+    ms = t0.elapsed_time(t1) / args.steps
+    ms = max_over_ranks(ms)
+    clk = clocks.stop()
+
+    # per-kernel durations inside the timed region
+    per = {}
+    open_ev = {}
+    for name, after, ev in rec:
+        if not after:
+            open_ev[name] = ev
+        else:
+            per.setdefault(name, []).append(open_ev.pop(name).elapsed_time(ev))
+    launches = sum(len(v) for v in per.values()) // args.steps
+
+    # end-to-end: pinned host inputs -> device -> step -> results back to host
+    pin = {k: None if v is None else v.pin_memory() for k, v in inp_cpu.items()}
+    host_out = {k: None if v is None else torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+                for k, v in out.items()}
+    h2d = sum(v.numel() * v.element_size() for v in pin.values() if v is not None)
+    d2h = sum(v.numel() * v.element_size() for v in host_out.values() if v is not None)
+    dst = {k: None if v is None else torch.empty_like(v) for k, v in d.items()}
+
+    def e2e_step():
+        for k, v in pin.items():
+            if v is not None:
+                dst[k].copy_(v, non_blocking=True)
+        step(dst)
+        for k, v in out.items():
+            if v is not None:
+                host_out[k].copy_(v, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n_e2e = max(1, min(args.steps, 5))
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e)
+
+    tokens = w.B * w.T * ws
+    value = tokens / (ms * 1e-3) / 1e6
+    pk = peaks()
+
+    # roofline of the dominant kernel
+    tot = {k: sum(v) for k, v in per.items()}
+    dom = max(tot, key=tot.get) if tot else None
+    roof = None
+    if dom:
+        T_seg = -(-w.T // seg)
+        bound, flops, byts = kernel_work(dom, w, T_seg)
+        avg_ms = tot[dom] / len(per[dom])
+        if bound == "hbm":
+            ach = byts / (avg_ms * 1e-3) / 1e9
+            peak = pk["hbm_gbs"]
+            unit = "GB/s"
+        else:
+            ach = flops / (avg_ms * 1e-3) / 1e12
+            peak = pk["bf16_tflops_sustained"]
+            unit = "TFLOP/s"
+        roof = {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+                "traffic": None, "kernel": dom, "avg_launch_ms": avg_ms,
+                "share": tot[dom] / sum(tot.values()), "peak_source": pk["source"]}
+
+    # whole-step roofline (the metric's "% of bf16 roofline")
+    ff, fb = algo_flops_per_token_head(w.C, w.dk, w.dv, w.use_beta)
+    bf_, bb = algo_bytes_per_token_head(w.dk, w.dv, 2 if w.io == "bf16" else 4, w.use_beta)
+    th = w.B * w.H * w.T
+    t_flop = th * (ff + fb) / (pk["bf16_tflops"] * 1e12)
+    t_hbm = th * (bf_ + bb) / (pk["hbm_gbs"] * 1e9)
+    t_roof = max(t_flop, t_hbm)
+    step_roof = {"bound": "hbm" if t_hbm >= t_flop else "tensor", "t_roof_ms": t_roof * 1e3,
+                 "frac": t_roof / (ms * 1e-3), "algo_tflops": th * (ff + fb) / (ms * 1e-3) / 1e12,
+                 "algo_gbs": th * (bf_ + bb) / (ms * 1e-3) / 1e9}
+
+    if rank == 0:
+        cpu = None
+        if ws == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(CONFIGS[args.workload], seg)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.io, "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
+                       "C": w.C, "segments": seg, "path": sf.path(shape),
+                       "parallelism": f"replicas x{ws} (independent batches)",
+                       "l2": (f"inputs {sum(v.numel() * v.element_size() for v in d.values() if v is not None) / 2**20:.0f} MiB"
+                              f" > L2 {L2_BYTES / 2**20:.0f} MiB, no flush")},
+            "roofline": roof, "roofline_step": step_roof,
+            "kernels_ms": {k: {"launches": len(v), "total_ms": sum(v), "share": sum(v) / sum(tot.values())}
+                           for k, v in per.items()},
+            "cpu_baseline": cpu,
+            "e2e": {"value": tokens / (e2e_ms * 1e-3) / 1e6, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--segments", type=int, default=DEFAULT_SEGMENTS)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

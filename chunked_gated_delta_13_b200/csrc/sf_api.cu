@@ -1,0 +1,357 @@
+// C ABI of libsf_gdn: argument checks, workspace sizing, dispatch to a kernel
+// family, and the segment chain (StateFlow, arXiv 2608.06838, section 3.1:
+// the sequence split X = C_0 || ... || C_{N-1}, Fwd/Bwd per segment, the state
+// handed forward and the state gradient handed backward).
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "../../include/sf_gdn.h"
+#include "sf_common.cuh"
+#include "tc_kernels.cuh"
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+sf_launch_hook g_hook = nullptr;
+void* g_hook_user = nullptr;
+
+sf_status cuda_fail(cudaError_t e) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+                  cudaGetErrorString(e));
+    return SF_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool head_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool chunk_ok(int C) { return C == 16 || C == 32 || C == 64 || C == 128; }
+
+sf_status check_shape(const sf_gdn_shape* s) {
+    if (!s) return SF_ERR_INVALID_ARG;
+    if (s->B < 0 || s->H < 0 || s->T < 0) return SF_ERR_INVALID_ARG;
+    if (s->io != SF_F32 && s->io != SF_BF16) return SF_ERR_INVALID_ARG;
+    if (s->use_beta != 0 && s->use_beta != 1) return SF_ERR_INVALID_ARG;
+    if (!(s->scale == s->scale) || s->scale > 3.0e38f || s->scale < -3.0e38f) return SF_ERR_INVALID_ARG;
+    if (!head_ok(s->dk) || !head_ok(s->dv) || !chunk_ok(s->C)) return SF_ERR_UNSUPPORTED;
+    if ((long long)s->B * s->H > 65535) return SF_ERR_UNSUPPORTED;
+    return SF_OK;
+}
+
+enum class Path { Simt, Tc };
+
+Path pick_path(const sf_gdn_shape& s) {
+    return sf::tc_supports(s.io == SF_BF16, s.dk, s.dv, s.C, s.use_beta != 0) ? Path::Tc : Path::Simt;
+}
+
+// View of a segment [t0, t0+T) of a sequence of T_full tokens.
+sf::SeqView make_view(const sf_gdn_shape& s, int T, long long T_full) {
+    sf::SeqView v{};
+    v.BH = s.B * s.H;
+    v.T = T;
+    v.dk = s.dk;
+    v.dv = s.dv;
+    v.C = s.C;
+    v.NC = (T + s.C - 1) / s.C;
+    v.use_beta = s.use_beta;
+    v.scale = s.scale;
+    v.hs_k = T_full * s.dk;
+    v.hs_v = T_full * s.dv;
+    v.hs_g = T_full;
+    return v;
+}
+
+size_t call_ws(const sf_gdn_shape& s, int T, bool backward) {
+    if (T == 0 || s.B * s.H == 0) return 0;
+    const sf::SeqView v = make_view(s, T, T);
+    return pick_path(s) == Path::Tc ? sf::tc_workspace_bytes(v, backward)
+                                    : sf::simt_workspace_bytes(v, backward);
+}
+
+size_t elem_size(const sf_gdn_shape& s) { return s.io == SF_BF16 ? 2 : 4; }
+
+// Offset a [B,H,T,d] pointer to token t0.
+template <typename T>
+T* at_token(T* p, long long t0, int d, size_t esize) {
+    return p ? reinterpret_cast<T*>(reinterpret_cast<char*>(p) + (size_t)t0 * d * esize) : p;
+}
+template <typename T>
+const T* at_token(const T* p, long long t0, int d, size_t esize) {
+    return p ? reinterpret_cast<const T*>(reinterpret_cast<const char*>(p) + (size_t)t0 * d * esize) : p;
+}
+
+// State copy helper: dst = src (or zeros when src is NULL).
+cudaError_t copy_state(float* dst, const float* src, size_t n, cudaStream_t st) {
+    if (!dst) return cudaSuccess;
+    if (src) return cudaMemcpyAsync(dst, src, n * sizeof(float), cudaMemcpyDeviceToDevice, st);
+    return cudaMemsetAsync(dst, 0, n * sizeof(float), st);
+}
+
+// Forward of the segment [t0, t0+T) of a T_full-token sequence.
+sf_status fwd_segment(const sf_gdn_shape& s, int T, long long t0, long long T_full,
+                      const sf::FwdArgs& full, void* ws, cudaStream_t st) {
+    const size_t es = elem_size(s);
+    const size_t nstate = (size_t)s.B * s.H * s.dk * s.dv;
+    if (s.B * s.H == 0) return SF_OK;
+    if (T == 0) {
+        cudaError_t e = copy_state(full.S_out, full.S_in, nstate, st);
+        return e == cudaSuccess ? SF_OK : cuda_fail(e);
+    }
+    sf::FwdArgs a = full;
+    a.q = at_token(full.q, t0, s.dk, es);
+    a.k = at_token(full.k, t0, s.dk, es);
+    a.v = at_token(full.v, t0, s.dv, es);
+    a.o = at_token(full.o, t0, s.dv, es);
+    a.g = at_token(full.g, t0, 1, 4);
+    a.beta = at_token(full.beta, t0, 1, 4);
+    const sf::SeqView v = make_view(s, T, T_full);
+    const bool bf16 = s.io == SF_BF16;
+    cudaError_t e = pick_path(s) == Path::Tc ? sf::tc_fwd(v, a, ws, st) : sf::simt_fwd(v, bf16, a, ws, st);
+    return e == cudaSuccess ? SF_OK : cuda_fail(e);
+}
+
+sf_status bwd_segment(const sf_gdn_shape& s, int T, long long t0, long long T_full,
+                      const sf::BwdArgs& full, void* ws, cudaStream_t st) {
+    const size_t es = elem_size(s);
+    const size_t nstate = (size_t)s.B * s.H * s.dk * s.dv;
+    if (s.B * s.H == 0) return SF_OK;
+    if (T == 0) {
+        cudaError_t e = copy_state(full.dS_in, full.dS_out, nstate, st);
+        return e == cudaSuccess ? SF_OK : cuda_fail(e);
+    }
+    sf::BwdArgs a = full;
+    a.q = at_token(full.q, t0, s.dk, es);
+    a.k = at_token(full.k, t0, s.dk, es);
+    a.v = at_token(full.v, t0, s.dv, es);
+    a.dO = at_token(full.dO, t0, s.dv, es);
+    a.dq = at_token(full.dq, t0, s.dk, es);
+    a.dk = at_token(full.dk, t0, s.dk, es);
+    a.dv = at_token(full.dv, t0, s.dv, es);
+    a.g = at_token(full.g, t0, 1, 4);
+    a.beta = at_token(full.beta, t0, 1, 4);
+    a.dg = at_token(full.dg, t0, 1, 4);
+    a.dbeta = at_token(full.dbeta, t0, 1, 4);
+    const sf::SeqView v = make_view(s, T, T_full);
+    const bool bf16 = s.io == SF_BF16;
+    cudaError_t e = pick_path(s) == Path::Tc ? sf::tc_bwd(v, a, ws, st) : sf::simt_bwd(v, bf16, a, ws, st);
+    return e == cudaSuccess ? SF_OK : cuda_fail(e);
+}
+
+bool all_aligned(std::initializer_list<const void*> ps) {
+    for (const void* p : ps)
+        if (p && !aligned16(p)) return false;
+    return true;
+}
+
+sf_status check_fwd_ptrs(const sf_gdn_shape& s, const void* q, const void* k, const void* v,
+                         const float* g, const float* beta, const float* S_in, const void* o,
+                         const float* S_out) {
+    const bool empty = (long long)s.B * s.H * s.T == 0;
+    if (!empty && (!q || !k || !v || !g || !o)) return SF_ERR_INVALID_ARG;
+    if (!empty && s.use_beta && !beta) return SF_ERR_INVALID_ARG;
+    if (!s.use_beta && beta) return SF_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, g, beta, S_in, o, S_out})) return SF_ERR_ALIGNMENT;
+    return SF_OK;
+}
+
+sf_status check_bwd_ptrs(const sf_gdn_shape& s, const void* q, const void* k, const void* v,
+                         const float* g, const float* beta, const float* S_in, const void* dO,
+                         const float* dS_out, const void* dq, const void* dk, const void* dv,
+                         const float* dg, const float* dbeta, const float* dS_in) {
+    sf_status st = check_fwd_ptrs(s, q, k, v, g, beta, S_in, dO, nullptr);
+    if (st != SF_OK) return st;
+    const bool empty = (long long)s.B * s.H * s.T == 0;
+    if (!empty && (!dq || !dk || !dv || !dg)) return SF_ERR_INVALID_ARG;
+    if (!empty && s.use_beta && !dbeta) return SF_ERR_INVALID_ARG;
+    if (!s.use_beta && dbeta) return SF_ERR_INVALID_ARG;
+    if (!all_aligned({dO, dS_out, dq, dk, dv, dg, dbeta, dS_in})) return SF_ERR_ALIGNMENT;
+    return SF_OK;
+}
+
+sf_status check_ws(size_t need, const void* ws, size_t ws_bytes) {
+    if (need == 0) return SF_OK;
+    if (!ws || ws_bytes < need) return SF_ERR_WORKSPACE;
+    if (!aligned16(ws)) return SF_ERR_ALIGNMENT;
+    return SF_OK;
+}
+
+bool segment_lengths(const sf_gdn_shape& s, int N, const int* seg_len, std::vector<int>& out) {
+    if (N <= 0) return false;
+    out.assign(N, 0);
+    if (seg_len) {
+        long long sum = 0;
+        for (int i = 0; i < N; ++i) {
+            if (seg_len[i] < 0) return false;
+            out[i] = seg_len[i];
+            sum += seg_len[i];
+        }
+        return sum == s.T;
+    }
+    const int base = s.T / N, rem = s.T % N;
+    for (int i = 0; i < N; ++i) out[i] = base + (i < rem ? 1 : 0);
+    return true;
+}
+
+}  // namespace
+
+namespace sf {
+void launch_hook(const char* kernel, int after, cudaStream_t st) {
+    sf_launch_hook h = g_hook;
+    if (h) h(kernel, after, static_cast<void*>(st), g_hook_user);
+}
+}  // namespace sf
+
+extern "C" {
+
+void sf_set_launch_hook(sf_launch_hook hook, void* user) {
+    g_hook_user = user;
+    g_hook = hook;
+}
+
+const char* sf_status_str(sf_status s) {
+    switch (s) {
+        case SF_OK: return "SF_OK";
+        case SF_ERR_INVALID_ARG: return "SF_ERR_INVALID_ARG";
+        case SF_ERR_UNSUPPORTED: return "SF_ERR_UNSUPPORTED";
+        case SF_ERR_ALIGNMENT: return "SF_ERR_ALIGNMENT";
+        case SF_ERR_WORKSPACE: return "SF_ERR_WORKSPACE";
+        case SF_ERR_CUDA: return "SF_ERR_CUDA";
+        case SF_ERR_TIMEOUT: return "SF_ERR_TIMEOUT";
+    }
+    return "SF_ERR_UNKNOWN";
+}
+
+const char* sf_last_cuda_error(void) { return g_last_cuda_error; }
+
+size_t sf_gdn_fwd_workspace_bytes(const sf_gdn_shape* s) {
+    if (check_shape(s) != SF_OK) return 0;
+    return call_ws(*s, s->T, false);
+}
+
+size_t sf_gdn_bwd_workspace_bytes(const sf_gdn_shape* s) {
+    if (check_shape(s) != SF_OK) return 0;
+    return call_ws(*s, s->T, true);
+}
+
+sf_status sf_gdn_fwd(const sf_gdn_shape* s, const void* q, const void* k, const void* v,
+                     const float* g, const float* beta, const float* S_in, void* o, float* S_out,
+                     void* ws, size_t ws_bytes, void* stream) {
+    sf_status st = check_shape(s);
+    if (st != SF_OK) return st;
+    st = check_fwd_ptrs(*s, q, k, v, g, beta, S_in, o, S_out);
+    if (st != SF_OK) return st;
+    st = check_ws(call_ws(*s, s->T, false), ws, ws_bytes);
+    if (st != SF_OK) return st;
+    sf::FwdArgs a{q, k, v, g, beta, S_in, o, S_out};
+    return fwd_segment(*s, s->T, 0, s->T, a, ws, static_cast<cudaStream_t>(stream));
+}
+
+sf_status sf_gdn_bwd(const sf_gdn_shape* s, const void* q, const void* k, const void* v,
+                     const float* g, const float* beta, const float* S_in, const void* dO,
+                     const float* dS_out, void* dq, void* dk, void* dv, float* dg, float* dbeta,
+                     float* dS_in, void* ws, size_t ws_bytes, void* stream) {
+    sf_status st = check_shape(s);
+    if (st != SF_OK) return st;
+    st = check_bwd_ptrs(*s, q, k, v, g, beta, S_in, dO, dS_out, dq, dk, dv, dg, dbeta, dS_in);
+    if (st != SF_OK) return st;
+    st = check_ws(call_ws(*s, s->T, true), ws, ws_bytes);
+    if (st != SF_OK) return st;
+    sf::BwdArgs a{q, k, v, g, beta, S_in, dO, dS_out, dq, dk, dv, dg, dbeta, dS_in};
+    return bwd_segment(*s, s->T, 0, s->T, a, ws, static_cast<cudaStream_t>(stream));
+}
+
+size_t sf_segment_workspace_bytes(const sf_gdn_shape* s, int N, const int* seg_len) {
+    if (check_shape(s) != SF_OK) return 0;
+    std::vector<int> lens;
+    if (!segment_lengths(*s, N, seg_len, lens)) return 0;
+    size_t per = 0;
+    for (int L : lens) {
+        const size_t f = call_ws(*s, L, false), b = call_ws(*s, L, true);
+        per = per > f ? per : f;
+        per = per > b ? per : b;
+    }
+    const size_t nstate = (size_t)s->B * s->H * s->dk * s->dv;
+    // N+1 boundary states, two boundary state gradients (ping-pong), then the
+    // per-segment workspace; every piece 256-byte aligned.
+    return sf::align_up(nstate * sizeof(float), 256) * (size_t)(N + 3) + per + 256;
+}
+
+sf_status sf_segment_run(const sf_gdn_shape* s, int N, const int* seg_len, const void* q,
+                         const void* k, const void* v, const float* g, const float* beta,
+                         const float* S_in, const void* dO, const float* dS_out, void* o,
+                         float* S_out, void* dq, void* dk, void* dv, float* dg, float* dbeta,
+                         float* dS_in, void* ws, size_t ws_bytes, void* stream) {
+    sf_status st = check_shape(s);
+    if (st != SF_OK) return st;
+    std::vector<int> lens;
+    if (!segment_lengths(*s, N, seg_len, lens)) return SF_ERR_INVALID_ARG;
+    st = check_fwd_ptrs(*s, q, k, v, g, beta, S_in, o, S_out);
+    if (st != SF_OK) return st;
+    if (dO) {
+        st = check_bwd_ptrs(*s, q, k, v, g, beta, S_in, dO, dS_out, dq, dk, dv, dg, dbeta, dS_in);
+        if (st != SF_OK) return st;
+    }
+    const size_t need = sf_segment_workspace_bytes(s, N, seg_len);
+    st = check_ws(need, ws, ws_bytes);
+    if (st != SF_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (s->B * s->H == 0) return SF_OK;
+
+    const size_t nstate = (size_t)s->B * s->H * s->dk * s->dv;
+    const size_t sstride = sf::align_up(nstate * sizeof(float), 256);
+    char* base = reinterpret_cast<char*>(sf::align_up(reinterpret_cast<uintptr_t>(ws), 256));
+    auto state = [&](int i) { return reinterpret_cast<float*>(base + sstride * (size_t)i); };
+    float* dS_a = state(N + 1);
+    float* dS_b = state(N + 2);
+    void* seg_ws = base + sstride * (size_t)(N + 3);
+
+    cudaError_t e = copy_state(state(0), S_in, nstate, cs);
+    if (e != cudaSuccess) return cuda_fail(e);
+    std::vector<long long> t0(N);
+    long long t = 0;
+    for (int i = 0; i < N; ++i) {
+        t0[i] = t;
+        t += lens[i];
+    }
+    for (int i = 0; i < N; ++i) {
+        sf::FwdArgs a{q, k, v, g, beta, state(i), o, state(i + 1)};
+        st = fwd_segment(*s, lens[i], t0[i], s->T, a, seg_ws, cs);
+        if (st != SF_OK) return st;
+    }
+    if (S_out) {
+        e = copy_state(S_out, state(N), nstate, cs);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    if (!dO) return SF_OK;
+    e = copy_state(dS_a, dS_out, nstate, cs);
+    if (e != cudaSuccess) return cuda_fail(e);
+    float* cur = dS_a;
+    float* nxt = dS_b;
+    for (int i = N - 1; i >= 0; --i) {
+        sf::BwdArgs a{q, k, v, g, beta, state(i), dO, cur, dq, dk, dv, dg, dbeta, nxt};
+        st = bwd_segment(*s, lens[i], t0[i], s->T, a, seg_ws, cs);
+        if (st != SF_OK) return st;
+        float* tmp = cur;
+        cur = nxt;
+        nxt = tmp;
+    }
+    if (dS_in) {
+        e = copy_state(dS_in, cur, nstate, cs);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return SF_OK;
+}
+
+const char* sf_gdn_path(const sf_gdn_shape* s) {
+    if (check_shape(s) != SF_OK) return nullptr;
+    return pick_path(*s) == Path::Tc ? "tc" : "simt";
+}
+
+int sf_gdn_launches(const sf_gdn_shape* s, int backward) {
+    if (check_shape(s) != SF_OK) return -1;
+    return pick_path(*s) == Path::Tc ? sf::tc_launches(backward != 0) : sf::simt_launches(backward != 0);
+}
+
+}  // extern "C"

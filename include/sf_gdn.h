@@ -1,0 +1,151 @@
+/*
+ * sf_gdn.h — C ABI of libsf_gdn.so: forward and backward of one sequence
+ * segment of a Gated DeltaNet (gated delta-rule) linear-recurrence layer with
+ * an explicit boundary state, and the segment chain that runs a long sequence
+ * as N segments on one GPU.
+ *
+ * The operations (StateFlow: Sequence Pipeline Parallelism for Long-Context
+ * Modeling with Linear Recurrence, arXiv 2608.06838):
+ *   - section 2.1 (the generic linear recurrence, with the Gated DeltaNet
+ *     "scalar-plus-low-rank" transition), written with the state S in
+ *     R^{dk x dv} per (batch, head):
+ *         alpha_t = exp(g_t)
+ *         S_t     = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+ *         o_t     = scale * S_t^T q_t
+ *     and with the beta path off (the scalar-identity transition of Mamba-2):
+ *         S_t     = alpha_t S_{t-1} + k_t v_t^T
+ *   - section 3.1, the chunk forward  Fwd(C_in, S_in) -> (C_out, S_out)
+ *     and backward Bwd(C_in, S_in, dC_out, dS_out) -> (dC_in, dS_in):
+ *     sf_gdn_fwd / sf_gdn_bwd.  The backward gives the gradients of
+ *         L = sum_t <o_t, dO_t> + <S_out, dS_out>
+ *     with respect to q, k, v, g, beta and S_in.  It recomputes everything it
+ *     needs from its inputs and S_in; nothing is saved between the calls.
+ *   - section 3.1, the sequence split X = C_0 || ... || C_{N-1} with the state
+ *     handed forward (S_{i+1}^in = S_i^out) and the state gradient handed
+ *     backward (dS_i^out = dS_{i+1}^in): sf_segment_run.
+ *
+ * Layouts (row-major, contiguous unless stated):
+ *   q, k, dq, dk          [B, H, T, dk]   in the I/O dtype
+ *   v, o, dO, dv          [B, H, T, dv]   in the I/O dtype
+ *   g, beta, dg, dbeta    [B, H, T]       fp32   (g is the log-decay, <= 0 in practice)
+ *   S_in, S_out, dS_out, dS_in  [B, H, dk, dv]  fp32
+ * All device pointers must be 16-byte aligned.
+ *
+ * Ownership: the caller owns every buffer, including the workspace; the library
+ * allocates no device or host memory and keeps no state between calls, so calls
+ * on different streams with different workspaces may run concurrently.  All
+ * work is enqueued on `stream` (a cudaStream_t, NULL = the legacy default
+ * stream); the calls return as soon as the work is enqueued.
+ *
+ * Errors: arguments are checked before anything is enqueued; a failed check
+ * returns its status and leaves every output untouched.  A launch failure
+ * returns SF_ERR_CUDA (the CUDA error string is kept per thread, see
+ * sf_last_cuda_error).  No exception crosses the ABI.
+ */
+#ifndef SF_GDN_H_
+#define SF_GDN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SF_OK = 0,
+    SF_ERR_INVALID_ARG = 1,   /* null pointer where one is required, negative size, bad flag */
+    SF_ERR_UNSUPPORTED = 2,   /* head size, chunk size or dtype this build does not implement */
+    SF_ERR_ALIGNMENT = 3,     /* a device pointer is not 16-byte aligned */
+    SF_ERR_WORKSPACE = 4,     /* workspace missing or smaller than the *_workspace_bytes query */
+    SF_ERR_CUDA = 5,          /* a CUDA launch or copy failed */
+    SF_ERR_TIMEOUT = 6        /* reserved: no kernel of this build waits on another */
+} sf_status;
+
+typedef enum { SF_F32 = 0, SF_BF16 = 1 } sf_dtype;
+
+/* Shape of one call.  B, H >= 0 and T >= 0 (T need not be a multiple of C:
+ * the last chunk is ragged and is handled exactly).  dk, dv in {16, 32, 64, 128}.
+ * C (the kernel chunk length) in {16, 32, 64, 128}.  io = dtype of q, k, v, o,
+ * dO, dq, dk, dv.  use_beta = 0 selects the recurrence without the delta term
+ * (beta must then be NULL).  scale multiplies q (1.0 = none). */
+typedef struct {
+    int B, H, T;
+    int dk, dv;
+    int C;
+    sf_dtype io;
+    int use_beta;
+    float scale;
+} sf_gdn_shape;
+
+/* Human-readable name of a status. */
+const char* sf_status_str(sf_status s);
+
+/* Text of the last CUDA error seen by a call on this thread ("" if none). */
+const char* sf_last_cuda_error(void);
+
+/* Bytes of device workspace the call needs for this shape (0 when the shape
+ * is invalid).  The workspace must be 16-byte aligned; its contents on entry
+ * do not matter and are clobbered. */
+size_t sf_gdn_fwd_workspace_bytes(const sf_gdn_shape* shape);
+size_t sf_gdn_bwd_workspace_bytes(const sf_gdn_shape* shape);
+
+/* Forward of one segment (StateFlow section 3.1, Fwd).
+ *   q, k, v, g           inputs (device); beta: device [B,H,T] fp32 iff use_beta, else NULL
+ *   S_in                 device state entering the segment, NULL = zeros
+ *   o                    device output [B,H,T,dv] (io dtype)
+ *   S_out                device state leaving the segment, NULL = not written
+ *   ws, ws_bytes         device workspace of at least sf_gdn_fwd_workspace_bytes(shape)
+ *   stream               cudaStream_t */
+sf_status sf_gdn_fwd(const sf_gdn_shape* shape, const void* q, const void* k, const void* v,
+                     const float* g, const float* beta, const float* S_in, void* o,
+                     float* S_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Backward of one segment (StateFlow section 3.1, Bwd).  Inputs as for
+ * sf_gdn_fwd plus dO [B,H,T,dv] (io dtype) and dS_out (NULL = zeros).
+ * Outputs dq, dk, dv (io dtype), dg (fp32), dbeta (fp32; NULL iff !use_beta)
+ * and dS_in (fp32; NULL = not written).  All outputs are overwritten. */
+sf_status sf_gdn_bwd(const sf_gdn_shape* shape, const void* q, const void* k, const void* v,
+                     const float* g, const float* beta, const float* S_in, const void* dO,
+                     const float* dS_out, void* dq, void* dk, void* dv, float* dg,
+                     float* dbeta, float* dS_in, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace for sf_segment_run: the per-segment workspace of the longest
+ * segment plus N+1 fp32 boundary states and N+1 boundary state gradients.
+ * seg_len: host array of N lengths summing to shape->T, or NULL for the equal
+ * split (the first T % N segments one token longer). */
+size_t sf_segment_workspace_bytes(const sf_gdn_shape* full, int N, const int* seg_len);
+
+/* The segment chain on one GPU (StateFlow section 3.1): split the sequence of
+ * `full` into N segments, run sf_gdn_fwd on segments 0..N-1 with each S_out
+ * handed on as the next S_in, then (when dO != NULL) sf_gdn_bwd on segments
+ * N-1..0 with each dS_in handed back as the previous dS_out.  Arguments are the
+ * full-sequence tensors of sf_gdn_fwd and sf_gdn_bwd; with dO == NULL the
+ * backward is skipped and dq, dk, dv, dg, dbeta, dS_in are ignored.  The
+ * boundary states stay fp32 on the device, so when every segment length is a
+ * multiple of C the results are bit-identical to N = 1. */
+sf_status sf_segment_run(const sf_gdn_shape* full, int N, const int* seg_len, const void* q,
+                         const void* k, const void* v, const float* g, const float* beta,
+                         const float* S_in, const void* dO, const float* dS_out, void* o,
+                         float* S_out, void* dq, void* dk, void* dv, float* dg, float* dbeta,
+                         float* dS_in, void* ws, size_t ws_bytes, void* stream);
+
+/* Optional launch observer, for profiling.  When set, every kernel this
+ * library launches is bracketed by hook(name, 0, stream, user) just before the
+ * launch and hook(name, 1, stream, user) just after it, on the calling thread,
+ * so the caller can record CUDA events on `stream` around each kernel.  NULL
+ * removes the observer.  The setting is process-wide; set it while no other
+ * thread is inside the library. */
+typedef void (*sf_launch_hook)(const char* kernel, int after, void* stream, void* user);
+void sf_set_launch_hook(sf_launch_hook hook, void* user);
+
+/* Introspection for tests and benchmarks: the kernel family a shape runs on
+ * ("tc" = tensor-core kernels, "simt" = fp32 CUDA-core kernels; NULL if the
+ * shape is unsupported) and how many kernels one call launches. */
+const char* sf_gdn_path(const sf_gdn_shape* shape);
+int sf_gdn_launches(const sf_gdn_shape* shape, int backward);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SF_GDN_H_ */

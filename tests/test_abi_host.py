@@ -1,0 +1,145 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds and loads,
+it exports every function the header declares, and argument checks return
+their status before anything is enqueued (so fake device addresses are fine)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import chunked_gated_delta_13_b200 as sf
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sf_gdn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sf_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = sf.lib()
+    names = declared_functions()
+    assert names, "no declarations parsed"
+    assert sorted(names) == sorted(sf.EXPORTED_SYMBOLS)
+    for name in names:
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    L = sf.lib()
+    for code, name in enumerate(sf.STATUS_NAMES):
+        assert L.sf_status_str(code).decode() == name
+
+
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced: the checks return first
+
+
+def fake(off=0):
+    return ctypes.c_void_p(FAKE + off)
+
+
+def call_fwd(shape, q=fake(), k=fake(), v=fake(), g=fake(), beta=fake(), S_in=None, o=fake(),
+             S_out=None, ws=fake(), nbytes=1 << 40):
+    return sf.lib().sf_gdn_fwd(ctypes.byref(shape), q, k, v, g, beta, S_in, o, S_out, ws, nbytes,
+                               None)
+
+
+def call_bwd(shape, **kw):
+    args = dict(q=fake(), k=fake(), v=fake(), g=fake(), beta=fake(), S_in=None, dO=fake(),
+                dS_out=None, dq=fake(), dk=fake(), dv=fake(), dg=fake(), dbeta=fake(),
+                dS_in=None, ws=fake(), nbytes=1 << 40)
+    args.update(kw)
+    a = args
+    return sf.lib().sf_gdn_bwd(ctypes.byref(shape), a["q"], a["k"], a["v"], a["g"], a["beta"],
+                               a["S_in"], a["dO"], a["dS_out"], a["dq"], a["dk"], a["dv"], a["dg"],
+                               a["dbeta"], a["dS_in"], a["ws"], a["nbytes"], None)
+
+
+def test_invalid_shapes():
+    bad = [sf.make_shape(-1, 1, 64, 64, 64), sf.make_shape(1, 1, -5, 64, 64)]
+    for s in bad:
+        assert call_fwd(s) == 1
+    s = sf.make_shape(1, 1, 64, 64, 64)
+    s.io = 7
+    assert call_fwd(s) == 1
+    s = sf.make_shape(1, 1, 64, 64, 64)
+    s.use_beta = 3
+    assert call_fwd(s) == 1
+    s = sf.make_shape(1, 1, 64, 64, 64, scale=float("nan"))
+    assert call_fwd(s) == 1
+    assert sf.lib().sf_gdn_fwd(None, fake(), fake(), fake(), fake(), fake(), None, fake(), None,
+                               fake(), 1, None) == 1
+
+
+def test_unsupported_sizes():
+    assert call_fwd(sf.make_shape(1, 1, 64, 96, 64)) == 2
+    assert call_fwd(sf.make_shape(1, 1, 64, 64, 256)) == 2
+    assert call_fwd(sf.make_shape(1, 1, 64, 64, 64, C=48)) == 2
+    assert call_fwd(sf.make_shape(300, 300, 64, 64, 64)) == 2
+
+
+def test_null_pointers_and_beta_flag():
+    s = sf.make_shape(1, 2, 64, 64, 64)
+    assert call_fwd(s, q=None) == 1
+    assert call_fwd(s, o=None) == 1
+    assert call_fwd(s, beta=None) == 1            # use_beta=1 needs beta
+    s_off = sf.make_shape(1, 2, 64, 64, 64, use_beta=False)
+    assert call_fwd(s_off) == 1                    # beta given although the beta path is off
+    assert call_bwd(s, dq=None) == 1
+    assert call_bwd(s, dbeta=None) == 1
+    assert call_bwd(s_off, beta=None) == 1        # dbeta given without beta
+
+
+def test_alignment():
+    s = sf.make_shape(1, 2, 64, 64, 64)
+    assert call_fwd(s, k=fake(8)) == 3
+    assert call_fwd(s, S_in=fake(4)) == 3
+    assert call_bwd(s, dg=fake(2)) == 3
+
+
+def test_workspace_checks():
+    s = sf.make_shape(1, 2, 200, 64, 64, C=64)
+    need = sf.fwd_workspace_bytes(s)
+    assert need > 0
+    assert call_fwd(s, ws=None, nbytes=0) == 4
+    assert call_fwd(s, nbytes=need - 1) == 4
+    assert sf.bwd_workspace_bytes(s) >= need
+    assert call_bwd(s, nbytes=sf.bwd_workspace_bytes(s) - 1) == 4
+    assert sf.fwd_workspace_bytes(sf.make_shape(1, 2, 0, 64, 64)) == 0
+    assert sf.fwd_workspace_bytes(sf.make_shape(1, 1, 64, 100, 64)) == 0
+
+
+def test_segment_run_checks():
+    s = sf.make_shape(1, 2, 256, 64, 64)
+    L = sf.lib()
+    nb = sf.segment_workspace_bytes(s, 4)
+    assert nb > 0
+    assert sf.segment_workspace_bytes(s, 0) == 0
+    assert sf.segment_workspace_bytes(s, 2, [100, 100]) == 0      # lengths must sum to T
+    assert sf.segment_workspace_bytes(s, 2, [0, 256]) > 0
+
+    def run(N, seg, nbytes):
+        arr = None if seg is None else (ctypes.c_int * N)(*seg)
+        return L.sf_segment_run(ctypes.byref(s), N, arr, fake(), fake(), fake(), fake(), fake(),
+                                None, None, None, fake(), None, None, None, None, None, None, None,
+                                fake(), nbytes, None)
+    assert run(0, None, nb) == 1
+    assert run(2, [100, 100], nb) == 1
+    assert run(4, None, nb - 1) == 4
+
+
+def test_path_and_launch_counts():
+    s = sf.make_shape(1, 2, 256, 64, 64, io="f32")
+    assert sf.path(s) == "simt"
+    assert sf.launches(s, False) >= 1 and sf.launches(s, True) >= 1
+    assert sf.path(sf.make_shape(1, 1, 64, 100, 64)) is None
+
+
+def test_cpu_tensors_rejected():
+    torch = pytest.importorskip("torch")
+    q = torch.zeros(1, 1, 8, 16)
+    with pytest.raises(RuntimeError):
+        sf.fwd(q, q, q, torch.zeros(1, 1, 8), torch.zeros(1, 1, 8))
