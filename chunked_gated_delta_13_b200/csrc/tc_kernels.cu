@@ -1,12 +1,1399 @@
-// Tensor-core kernel family of libsf_gdn (bf16 I/O, fp32 state).
+// Tensor-core kernel family of libsf_gdn: bf16 I/O, fp32 state and
+// accumulation, key head size 128, value head size 64 or 128, chunk length 64.
+//
+// Decomposition (StateFlow, arXiv 2608.06838, section 2.2: Pre / ST / Out per
+// chunk; section 3.4.2: the backward stages SR, OG, STB, PG):
+//   forward  : prep (Pre: UT/WY transform)  -> scan (ST, sequential over chunks)
+//              -> out (Out)
+//   backward : prep (Pre again, plus the intra-chunk output gradient OG)
+//              -> one launch running the forward state recompute (SR) and the
+//                 reverse state-gradient scan (STB) side by side: the two
+//                 chains do not depend on each other
+//              -> grad (PG: every input gradient of every chunk)
+// With G_i = sum_{s<=i} g_s inside a chunk, gamma_i = exp(G_i),
+// Gamma_ij = exp(G_i - G_j) (j <= i), Khat = K * exp(G_C - G):
+//   A = strictly-lower(diag(beta)(K K^T * Gamma)), L = (I + A)^{-1}, T = L diag(beta)
+//   W = T (gamma * K), U = T V;  V_new = U - W S0;  S_C = gamma_C S0 + Khat^T V_new
+//   O = scale (gamma * Q) S0 + scale ((Q K^T) * Gamma) V_new
+// The state chains keep S (or dS) in fp32 registers as the accumulator of
+// warp-level m16n8k16 products: each warp owns 16 state columns, so the
+// recurrence never leaves the register file; only the operands W, Khat, U
+// stream in through double-buffered asynchronous copies.
 #include "tc_kernels.cuh"
+#include "tc_mma.cuh"
 
 namespace sf {
+namespace {
 
-bool tc_supports(bool, int, int, int, bool) { return false; }
-size_t tc_workspace_bytes(const SeqView&, bool) { return 0; }
-cudaError_t tc_fwd(const SeqView&, const FwdArgs&, void*, cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t tc_bwd(const SeqView&, const BwdArgs&, void*, cudaStream_t) { return cudaErrorNotSupported; }
-int tc_launches(bool) { return 0; }
+using bf16 = __nv_bfloat16;
+using namespace tc;
+
+constexpr int C = 64;        // chunk length
+constexpr int DK = 128;      // key head size
+constexpr int LDK = DK + 8;  // shared row stride of [*][DK] tiles
+constexpr int LDC = C + 8;   // shared row stride of [*][C] tiles
+constexpr int LDF = 72;      // shared row stride of fp32 [C][C] tiles
+
+struct TcWs {
+    float* Gc;   // [BH][Tp]           chunk-local cumulative log-decay
+    bf16* W;     // [BH][Tp][DK]
+    bf16* Kh;    // [BH][Tp][DK]       K * exp(G_C - G)
+    bf16* Ut;    // [BH][NC][DV][C]    U transposed per chunk (V^T without the beta path)
+    bf16* Vnt;   // [BH][NC][DV][C]    V_new transposed per chunk
+    bf16* S0t;   // [BH][NC][DV][DK]   state entering each chunk, transposed
+    bf16* dVit;  // [BH][NC][DV][C]    intra-chunk part of dV_new, transposed
+    bf16* dVnt;  // [BH][NC][DV][C]    dV_new transposed
+    bf16* dSCt;  // [BH][NC][DV][DK]   gradient of the state leaving each chunk, transposed
+    size_t total;
+};
+
+TcWs tc_layout(const SeqView& s, bool backward, char* base) {
+    TcWs w{};
+    const size_t BH = s.BH, NC = s.NC, Tp = NC * C, DV = s.dv;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char* p = base ? base + off : nullptr;
+        off = align_up(off + bytes, 256);
+        return p;
+    };
+    w.Gc = reinterpret_cast<float*>(take(BH * Tp * 4));
+    w.W = reinterpret_cast<bf16*>(take(s.use_beta ? BH * Tp * DK * 2 : 0));
+    w.Kh = reinterpret_cast<bf16*>(take(BH * Tp * DK * 2));
+    w.Ut = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
+    w.Vnt = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
+    w.S0t = reinterpret_cast<bf16*>(take(BH * NC * DV * DK * 2));
+    if (backward) {
+        w.dVit = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
+        w.dVnt = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
+        w.dSCt = reinterpret_cast<bf16*>(take(BH * NC * DV * DK * 2));
+    }
+    w.total = off + 256;
+    return w;
+}
+
+// Inclusive cumulative sum of the 64 log-decays of a chunk by warp 0 (fixed
+// shuffle order, so every launch adds in the same order).  Tokens past the end
+// contribute g = 0.
+__device__ __forceinline__ void chunk_cumsum(const float* g, int nval, float* Gs, int lane) {
+    const float x0 = (2 * lane < nval) ? g[2 * lane] : 0.f;
+    const float x1 = (2 * lane + 1 < nval) ? g[2 * lane + 1] : 0.f;
+    float inc = x0 + x1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    float exc = __shfl_up_sync(0xffffffffu, inc, 1);
+    if (lane == 0) exc = 0.f;
+    const float a = exc + x0;
+    Gs[2 * lane] = a;
+    Gs[2 * lane + 1] = a + x1;
+}
+
+// (I + A)^{-1} of a strictly lower-triangular 64x64 fp32 matrix A (row stride
+// la) into L (row stride ll; its strictly upper part must be zero on entry).
+// Forward substitution inside the four 16x16 diagonal blocks (warps 0-3, one
+// column per lane), then the off-diagonal blocks one block row at a time:
+// L_IJ = -L_II * sum_{m=J}^{I-1} A_Im L_mJ.  Y: 768 floats of scratch.
+__device__ void block_inverse(const float* A, int la, float* L, int ll, float* Y, int tid, int nthr) {
+    const int lane = tid & 31, w = tid >> 5;
+    if (w < 4 && lane < 16) {
+        const int o = 16 * w, cc = lane;
+        for (int r = cc; r < 16; ++r) {
+            float x = (r == cc) ? 1.f : 0.f;
+            for (int j = cc; j < r; ++j) x -= A[(o + r) * la + o + j] * L[(o + j) * ll + o + cc];
+            L[(o + r) * ll + o + cc] = x;
+        }
+    }
+    __syncthreads();
+    for (int I = 1; I < 4; ++I) {
+        for (int e = tid; e < I * 256; e += nthr) {
+            const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+            float y = 0.f;
+            for (int m = J; m < I; ++m)
+                for (int p = 0; p < 16; ++p)
+                    y += A[(16 * I + r) * la + 16 * m + p] * L[(16 * m + p) * ll + 16 * J + cc];
+            Y[e] = y;
+        }
+        __syncthreads();
+        for (int e = tid; e < I * 256; e += nthr) {
+            const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+            float x = 0.f;
+            for (int p = 0; p <= r; ++p) x += L[(16 * I + r) * ll + 16 * I + p] * Y[(J << 8) + p * 16 + cc];
+            L[(16 * I + r) * ll + 16 * J + cc] = -x;
+        }
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------------ prep ---
+template <int DV, bool BWD>
+constexpr size_t prep_smem() {
+    return (size_t)C * LDK * 2 + (size_t)C * (DV + 8) * 2 + (BWD ? (size_t)C * LDK * 2 + (size_t)C * (DV + 8) * 2 : 0) +
+           (size_t)C * LDF * 4 * 2 + (size_t)C * LDC * 2 * 2 + 768 * 4 + 2 * C * 4;
+}
+
+// One CTA (4 warps) per (chunk, head).  Writes G, Khat, W, U^T; in backward
+// mode also dVi^T = (P^T dO)^T with P = scale (Q K^T) * Gamma.
+template <int DV, bool BETA, bool BWD>
+__global__ void __launch_bounds__(128)
+tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
+               const bf16* __restrict__ v, const float* __restrict__ g,
+               const float* __restrict__ beta, const bf16* __restrict__ dO, float* __restrict__ Gc,
+               bf16* __restrict__ Wo, bf16* __restrict__ Kho, bf16* __restrict__ Uto,
+               bf16* __restrict__ dVito) {
+    constexpr int LDV = DV + 8;
+    extern __shared__ __align__(16) unsigned char smem[];
+    bf16* Ks = reinterpret_cast<bf16*>(smem);
+    bf16* Vs = Ks + C * LDK;
+    bf16* Qs = Vs + C * LDV;
+    bf16* dOs = Qs + (BWD ? C * LDK : 0);
+    float* Af = reinterpret_cast<float*>(dOs + (BWD ? C * LDV : 0));  // later: W staging
+    float* Lf = Af + C * LDF;                                          // later: U^T staging
+    bf16* Tw = reinterpret_cast<bf16*>(Lf + C * LDF);                  // later: P
+    bf16* Tu = Tw + C * LDC;
+    float* Yb = reinterpret_cast<float*>(Tu + C * LDC);
+    float* Gs = Yb + 768;
+    float* Bs = Gs + C;
+
+    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int gq = lane >> 2, tq = lane & 3;
+    const int t0 = c * C;
+    const int nval = min(C, s.T - t0);
+    const size_t Tp = (size_t)s.NC * C;
+    load_tile<C, DK, 128>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+    load_tile<C, DV, 128>(Vs, LDV, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+    if (BWD) {
+        load_tile<C, DK, 128>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+        load_tile<C, DV, 128>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+    }
+    cp_async_commit();
+    if (w == 0) chunk_cumsum(g + bh * s.hs_g + t0, nval, Gs, lane);
+    for (int i = tid; i < C; i += 128) Bs[i] = (BETA && i < nval) ? beta[bh * s.hs_g + t0 + i] : 0.f;
+    if (BETA)
+        for (int e = tid; e < C * LDF; e += 128) Lf[e] = 0.f;
+    cp_async_wait<0>();
+    __syncthreads();
+
+    for (int i = tid; i < C; i += 128) Gc[bh * Tp + t0 + i] = Gs[i];
+    const float gC = Gs[C - 1];
+    for (int e = tid; e < C * (DK / 8); e += 128) {
+        const int r = e >> 4, cc = (e & 15) * 8;
+        const float d = expf(gC - Gs[r]);
+        uint4 x = *reinterpret_cast<const uint4*>(Ks + r * LDK + cc);
+        x.x = scale2(x.x, d, d);
+        x.y = scale2(x.y, d, d);
+        x.z = scale2(x.z, d, d);
+        x.w = scale2(x.w, d, d);
+        *reinterpret_cast<uint4*>(Kho + (bh * Tp + t0 + r) * DK + cc) = x;
+    }
+
+    bf16* Ust = reinterpret_cast<bf16*>(Lf);  // [DV][LDC]
+    if (BETA) {
+        {  // A = strictly-lower(diag(beta) (K K^T * Gamma))
+            float acc[8][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                uint32_t a[4];
+                ldA(a, Ks, LDK, 16 * w, 16 * kk, lane);
+#pragma unroll
+                for (int nn = 0; nn < 8; nn += 2) {
+                    uint32_t b[4];
+                    ldBnk(b, Ks, LDK, 8 * nn, 16 * kk, lane);
+                    mma(acc[nn], a, b[0], b[1]);
+                    mma(acc[nn + 1], a, b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int nn = 0; nn < 8; ++nn)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 16 * w + gq + 8 * (e >> 1), j = 8 * nn + 2 * tq + (e & 1);
+                    Af[i * LDF + j] = (j < i) ? Bs[i] * expf(Gs[i] - Gs[j]) * acc[nn][e] : 0.f;
+                }
+        }
+        __syncthreads();
+        block_inverse(Af, LDF, Lf, LDF, Yb, tid, 128);
+        for (int e = tid; e < C * C; e += 128) {
+            const int i = e >> 6, j = e & 63;
+            const float l = Lf[i * LDF + j];
+            Tw[i * LDC + j] = __float2bfloat16_rn(l * Bs[j] * expf(Gs[j]));
+            Tu[i * LDC + j] = __float2bfloat16_rn(l * Bs[j]);
+        }
+        __syncthreads();
+        bf16* Wst = reinterpret_cast<bf16*>(Af);  // [C][LDK]
+        {  // W = T (gamma * K)
+            float acc[16][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                uint32_t a[4];
+                ldA(a, Tw, LDC, 16 * w, 16 * kk, lane);
+#pragma unroll
+                for (int nn = 0; nn < 16; nn += 2) {
+                    uint32_t b[4];
+                    ldBkn(b, Ks, LDK, 8 * nn, 16 * kk, lane);
+                    mma(acc[nn], a, b[0], b[1]);
+                    mma(acc[nn + 1], a, b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int nn = 0; nn < 16; ++nn) {
+                const int i = 16 * w + gq, col = 8 * nn + 2 * tq;
+                *reinterpret_cast<uint32_t*>(Wst + i * LDK + col) = pack(acc[nn][0], acc[nn][1]);
+                *reinterpret_cast<uint32_t*>(Wst + (i + 8) * LDK + col) = pack(acc[nn][2], acc[nn][3]);
+            }
+        }
+        {  // U = T V, staged transposed
+            float acc[DV / 8][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                uint32_t a[4];
+                ldA(a, Tu, LDC, 16 * w, 16 * kk, lane);
+#pragma unroll
+                for (int nn = 0; nn < DV / 8; nn += 2) {
+                    uint32_t b[4];
+                    ldBkn(b, Vs, LDV, 8 * nn, 16 * kk, lane);
+                    mma(acc[nn], a, b[0], b[1]);
+                    mma(acc[nn + 1], a, b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int nn = 0; nn < DV / 8; ++nn)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 16 * w + gq + 8 * (e >> 1), col = 8 * nn + 2 * tq + (e & 1);
+                    Ust[col * LDC + i] = __float2bfloat16_rn(acc[nn][e]);
+                }
+        }
+        __syncthreads();
+        for (int e = tid; e < C * (DK / 8); e += 128) {
+            const int r = e >> 4, cc = (e & 15) * 8;
+            *reinterpret_cast<uint4*>(Wo + (bh * Tp + t0 + r) * DK + cc) =
+                *reinterpret_cast<const uint4*>(Wst + r * LDK + cc);
+        }
+    } else {
+        for (int e = tid; e < C * DV; e += 128) {
+            const int i = e / DV, col = e % DV;
+            Ust[col * LDC + i] = Vs[i * LDV + col];
+        }
+        __syncthreads();
+    }
+    bf16* Utg = Uto + ((size_t)bh * s.NC + c) * DV * C;
+    for (int e = tid; e < DV * (C / 8); e += 128) {
+        const int r = e >> 3, cc = (e & 7) * 8;
+        *reinterpret_cast<uint4*>(Utg + r * C + cc) = *reinterpret_cast<const uint4*>(Ust + r * LDC + cc);
+    }
+
+    if (BWD) {
+        bf16* Ps = Tw;  // Tw is no longer read (all warps passed the barrier above)
+        {
+            float acc[8][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                uint32_t a[4];
+                ldA(a, Qs, LDK, 16 * w, 16 * kk, lane);
+#pragma unroll
+                for (int nn = 0; nn < 8; nn += 2) {
+                    uint32_t b[4];
+                    ldBnk(b, Ks, LDK, 8 * nn, 16 * kk, lane);
+                    mma(acc[nn], a, b[0], b[1]);
+                    mma(acc[nn + 1], a, b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int nn = 0; nn < 8; ++nn)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 16 * w + gq + 8 * (e >> 1), j = 8 * nn + 2 * tq + (e & 1);
+                    const float p = (j <= i) ? s.scale * expf(Gs[i] - Gs[j]) * acc[nn][e] : 0.f;
+                    Ps[i * LDC + j] = __float2bfloat16_rn(p);
+                }
+        }
+        __syncthreads();
+        // dVi^T[v][j] = sum_i dO[i][v] P[i][j]
+        constexpr int MT = DV / 64;  // 16-row m-tiles per warp
+        bf16* dst = dVito + ((size_t)bh * s.NC + c) * DV * C;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int m0 = (w * MT + mt) * 16;
+            float acc[8][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                uint32_t a[4];
+                ldAt(a, dOs, LDV, m0, 16 * kk, lane);
+#pragma unroll
+                for (int nn = 0; nn < 8; nn += 2) {
+                    uint32_t b[4];
+                    ldBkn(b, Ps, LDC, 8 * nn, 16 * kk, lane);
+                    mma(acc[nn], a, b[0], b[1]);
+                    mma(acc[nn + 1], a, b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int nn = 0; nn < 8; ++nn) {
+                const int r = m0 + gq, j = 8 * nn + 2 * tq;
+                *reinterpret_cast<uint32_t*>(dst + r * C + j) = pack(acc[nn][0], acc[nn][1]);
+                *reinterpret_cast<uint32_t*>(dst + (r + 8) * C + j) = pack(acc[nn][2], acc[nn][3]);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------ state scans ---
+template <bool BETA>
+constexpr size_t fwd_stage_bytes() {
+    return (size_t)C * LDK * 2 * (BETA ? 2 : 1) + (size_t)64 * LDC * 2 + C * 4;
+}
+template <bool BETA>
+constexpr size_t bwd_stage_bytes() {
+    return (size_t)C * LDK * 2 * (BETA ? 3 : 2) + (size_t)C * LDC * 2 * 2 + C * 4;
+}
+
+// Forward chain for one (head, 64 state columns) on 4 warps of 16 columns:
+// per chunk V_new^T = U^T - S^T W^T, S^T <- gamma_C S^T + V_new^T Khat.
+// Optional outputs: V_new^T and S0^T per chunk (bf16), S_out (fp32).
+template <int DV, bool BETA>
+__device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, const float* __restrict__ Gc,
+                                             const bf16* __restrict__ W, const bf16* __restrict__ Kh,
+                                             const bf16* __restrict__ Ut, const float* __restrict__ S_in,
+                                             bf16* __restrict__ Vnt, bf16* __restrict__ S0t,
+                                             float* __restrict__ S_out, unsigned char* smem) {
+    constexpr size_t STAGE = fwd_stage_bytes<BETA>();
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, gq = lane >> 2, tq = lane & 3;
+    const int vl = 16 * w;            // first state column of this warp inside the block
+    const int v0 = vb * 64 + vl;      // ... and inside the head
+    const size_t Tp = (size_t)s.NC * C;
+
+    auto ptrs = [&](int buf, bf16*& Khs, bf16*& Ws, bf16*& Uts, float*& Gs) {
+        unsigned char* p = smem + buf * STAGE;
+        Khs = reinterpret_cast<bf16*>(p);
+        p += C * LDK * 2;
+        Ws = reinterpret_cast<bf16*>(p);
+        if (BETA) p += C * LDK * 2;
+        Uts = reinterpret_cast<bf16*>(p);
+        p += 64 * LDC * 2;
+        Gs = reinterpret_cast<float*>(p);
+    };
+    auto load = [&](int cc, int buf) {
+        bf16 *Khs, *Ws, *Uts;
+        float* Gs;
+        ptrs(buf, Khs, Ws, Uts, Gs);
+        const size_t row0 = (size_t)bh * Tp + (size_t)cc * C;
+        load_tile<C, DK, 128>(Khs, LDK, Kh + row0 * DK, DK, C, tid);
+        if (BETA) load_tile<C, DK, 128>(Ws, LDK, W + row0 * DK, DK, C, tid);
+        load_tile<64, C, 128>(Uts, LDC, Ut + (((size_t)bh * s.NC + cc) * DV + vb * 64) * C, C, 64, tid);
+        if (tid < 16) cp_async16(Gs + tid * 4, Gc + row0 + tid * 4, true);
+    };
+
+    float st[16][4];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int vv = v0 + gq + 8 * (e >> 1), d = 8 * j + 2 * tq + (e & 1);
+            st[j][e] = S_in ? S_in[((size_t)bh * DK + d) * DV + vv] : 0.f;
+        }
+
+    load(0, 0);
+    cp_async_commit();
+    for (int cc = 0; cc < s.NC; ++cc) {
+        if (cc + 1 < s.NC) load(cc + 1, (cc + 1) & 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        bf16 *Khs, *Ws, *Uts;
+        float* Gs;
+        ptrs(cc & 1, Khs, Ws, Uts, Gs);
+        const float gamC = expf(Gs[C - 1]);
+        if (S0t) {
+            bf16* dst = S0t + ((size_t)bh * s.NC + cc) * DV * DK;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int d = 8 * j + 2 * tq;
+                *reinterpret_cast<uint32_t*>(dst + (size_t)(v0 + gq) * DK + d) = pack(st[j][0], st[j][1]);
+                *reinterpret_cast<uint32_t*>(dst + (size_t)(v0 + gq + 8) * DK + d) = pack(st[j][2], st[j][3]);
+            }
+        }
+        float vn[8][4];
+#pragma unroll
+        for (int nn = 0; nn < 8; ++nn) {
+            const int tk = 8 * nn + 2 * tq;
+            const float2 u0 = unpack(*reinterpret_cast<const uint32_t*>(Uts + (vl + gq) * LDC + tk));
+            const float2 u1 = unpack(*reinterpret_cast<const uint32_t*>(Uts + (vl + gq + 8) * LDC + tk));
+            vn[nn][0] = u0.x;
+            vn[nn][1] = u0.y;
+            vn[nn][2] = u1.x;
+            vn[nn][3] = u1.y;
+        }
+        if (BETA) {
+            uint32_t sa[8][4];
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                sa[kk][0] = pack(-st[2 * kk][0], -st[2 * kk][1]);
+                sa[kk][1] = pack(-st[2 * kk][2], -st[2 * kk][3]);
+                sa[kk][2] = pack(-st[2 * kk + 1][0], -st[2 * kk + 1][1]);
+                sa[kk][3] = pack(-st[2 * kk + 1][2], -st[2 * kk + 1][3]);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+#pragma unroll
+                for (int nn = 0; nn < 8; nn += 2) {
+                    uint32_t b[4];
+                    ldBnk(b, Ws, LDK, 8 * nn, 16 * kk, lane);
+                    mma(vn[nn], sa[kk], b[0], b[1]);
+                    mma(vn[nn + 1], sa[kk], b[2], b[3]);
+                }
+        }
+        if (Vnt) {
+            bf16* dst = Vnt + ((size_t)bh * s.NC + cc) * DV * C;
+#pragma unroll
+            for (int nn = 0; nn < 8; ++nn) {
+                const int tk = 8 * nn + 2 * tq;
+                *reinterpret_cast<uint32_t*>(dst + (v0 + gq) * C + tk) = pack(vn[nn][0], vn[nn][1]);
+                *reinterpret_cast<uint32_t*>(dst + (v0 + gq + 8) * C + tk) = pack(vn[nn][2], vn[nn][3]);
+            }
+        }
+        uint32_t va[4][4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) c2a(va[kk], vn[2 * kk], vn[2 * kk + 1]);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) st[j][e] *= gamC;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+            for (int nn = 0; nn < 16; nn += 2) {
+                uint32_t b[4];
+                ldBkn(b, Khs, LDK, 8 * nn, 16 * kk, lane);
+                mma(st[nn], va[kk], b[0], b[1]);
+                mma(st[nn + 1], va[kk], b[2], b[3]);
+            }
+        __syncthreads();
+    }
+    if (S_out) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int vv = v0 + gq + 8 * (e >> 1), d = 8 * j + 2 * tq + (e & 1);
+                S_out[((size_t)bh * DK + d) * DV + vv] = st[j][e];
+            }
+    }
+}
+
+// Reverse chain of the state gradient for one (head, 64 state columns):
+// per chunk, from the last, dV_new^T = dVi^T + dS^T Khat^T and
+// dS^T <- gamma_C dS^T + dO^T (scale gamma * Q) - dV_new^T W.
+// Outputs dV_new^T and dS_C^T per chunk (bf16), dS_in (fp32).
+template <int DV, bool BETA>
+__device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, const bf16* __restrict__ q,
+                                             const bf16* __restrict__ dO, const float* __restrict__ Gc,
+                                             const bf16* __restrict__ W, const bf16* __restrict__ Kh,
+                                             const bf16* __restrict__ dVit, const float* __restrict__ dS_out,
+                                             bf16* __restrict__ dVnt, bf16* __restrict__ dSCt,
+                                             float* __restrict__ dS_in, unsigned char* smem) {
+    constexpr size_t STAGE = bwd_stage_bytes<BETA>();
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, gq = lane >> 2, tq = lane & 3;
+    const int vl = 16 * w;
+    const int v0 = vb * 64 + vl;
+    const size_t Tp = (size_t)s.NC * C;
+
+    auto ptrs = [&](int buf, bf16*& Khs, bf16*& Qs, bf16*& Ws, bf16*& dOs, bf16*& dVis, float*& Gs) {
+        unsigned char* p = smem + buf * STAGE;
+        Khs = reinterpret_cast<bf16*>(p);
+        p += C * LDK * 2;
+        Qs = reinterpret_cast<bf16*>(p);
+        p += C * LDK * 2;
+        Ws = reinterpret_cast<bf16*>(p);
+        if (BETA) p += C * LDK * 2;
+        dOs = reinterpret_cast<bf16*>(p);
+        p += C * LDC * 2;
+        dVis = reinterpret_cast<bf16*>(p);
+        p += C * LDC * 2;
+        Gs = reinterpret_cast<float*>(p);
+    };
+    auto load = [&](int cc, int buf) {
+        bf16 *Khs, *Qs, *Ws, *dOs, *dVis;
+        float* Gs;
+        ptrs(buf, Khs, Qs, Ws, dOs, dVis, Gs);
+        const size_t row0 = (size_t)bh * Tp + (size_t)cc * C;
+        const int nval = min(C, s.T - cc * C);
+        load_tile<C, DK, 128>(Khs, LDK, Kh + row0 * DK, DK, C, tid);
+        load_tile<C, DK, 128>(Qs, LDK, q + bh * s.hs_k + (size_t)cc * C * DK, DK, nval, tid);
+        if (BETA) load_tile<C, DK, 128>(Ws, LDK, W + row0 * DK, DK, C, tid);
+        load_tile<C, 64, 128>(dOs, LDC, dO + bh * s.hs_v + (size_t)cc * C * DV + vb * 64, DV, nval, tid);
+        load_tile<64, C, 128>(dVis, LDC, dVit + (((size_t)bh * s.NC + cc) * DV + vb * 64) * C, C, 64, tid);
+        if (tid < 16) cp_async16(Gs + tid * 4, Gc + row0 + tid * 4, true);
+    };
+
+    float ds[16][4];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int vv = v0 + gq + 8 * (e >> 1), d = 8 * j + 2 * tq + (e & 1);
+            ds[j][e] = dS_out ? dS_out[((size_t)bh * DK + d) * DV + vv] : 0.f;
+        }
+
+    load(s.NC - 1, (s.NC - 1) & 1);
+    cp_async_commit();
+    for (int cc = s.NC - 1; cc >= 0; --cc) {
+        if (cc > 0) load(cc - 1, (cc - 1) & 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        bf16 *Khs, *Qs, *Ws, *dOs, *dVis;
+        float* Gs;
+        ptrs(cc & 1, Khs, Qs, Ws, dOs, dVis, Gs);
+        const float gamC = expf(Gs[C - 1]);
+        if (dSCt) {
+            bf16* dst = dSCt + ((size_t)bh * s.NC + cc) * DV * DK;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int d = 8 * j + 2 * tq;
+                *reinterpret_cast<uint32_t*>(dst + (size_t)(v0 + gq) * DK + d) = pack(ds[j][0], ds[j][1]);
+                *reinterpret_cast<uint32_t*>(dst + (size_t)(v0 + gq + 8) * DK + d) = pack(ds[j][2], ds[j][3]);
+            }
+        }
+        float dvn[8][4];
+#pragma unroll
+        for (int nn = 0; nn < 8; ++nn) {
+            const int tk = 8 * nn + 2 * tq;
+            const float2 u0 = unpack(*reinterpret_cast<const uint32_t*>(dVis + (vl + gq) * LDC + tk));
+            const float2 u1 = unpack(*reinterpret_cast<const uint32_t*>(dVis + (vl + gq + 8) * LDC + tk));
+            dvn[nn][0] = u0.x;
+            dvn[nn][1] = u0.y;
+            dvn[nn][2] = u1.x;
+            dvn[nn][3] = u1.y;
+        }
+        {
+            uint32_t da[8][4];
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) c2a(da[kk], ds[2 * kk], ds[2 * kk + 1]);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+#pragma unroll
+                for (int nn = 0; nn < 8; nn += 2) {
+                    uint32_t b[4];
+                    ldBnk(b, Khs, LDK, 8 * nn, 16 * kk, lane);
+                    mma(dvn[nn], da[kk], b[0], b[1]);
+                    mma(dvn[nn + 1], da[kk], b[2], b[3]);
+                }
+        }
+        if (dVnt) {
+            bf16* dst = dVnt + ((size_t)bh * s.NC + cc) * DV * C;
+#pragma unroll
+            for (int nn = 0; nn < 8; ++nn) {
+                const int tk = 8 * nn + 2 * tq;
+                *reinterpret_cast<uint32_t*>(dst + (v0 + gq) * C + tk) = pack(dvn[nn][0], dvn[nn][1]);
+                *reinterpret_cast<uint32_t*>(dst + (v0 + gq + 8) * C + tk) = pack(dvn[nn][2], dvn[nn][3]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) ds[j][e] *= gamC;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t a[4];
+            ldAt(a, dOs, LDC, vl, 16 * kk, lane);
+            const int tk = 16 * kk + 2 * tq;
+            const float g0 = s.scale * expf(Gs[tk]), g1 = s.scale * expf(Gs[tk + 1]);
+            const float g2 = s.scale * expf(Gs[tk + 8]), g3 = s.scale * expf(Gs[tk + 9]);
+            a[0] = scale2(a[0], g0, g1);
+            a[1] = scale2(a[1], g0, g1);
+            a[2] = scale2(a[2], g2, g3);
+            a[3] = scale2(a[3], g2, g3);
+#pragma unroll
+            for (int nn = 0; nn < 16; nn += 2) {
+                uint32_t b[4];
+                ldBkn(b, Qs, LDK, 8 * nn, 16 * kk, lane);
+                mma(ds[nn], a, b[0], b[1]);
+                mma(ds[nn + 1], a, b[2], b[3]);
+            }
+        }
+        if (BETA) {
+            uint32_t na[4][4];
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                na[kk][0] = pack(-dvn[2 * kk][0], -dvn[2 * kk][1]);
+                na[kk][1] = pack(-dvn[2 * kk][2], -dvn[2 * kk][3]);
+                na[kk][2] = pack(-dvn[2 * kk + 1][0], -dvn[2 * kk + 1][1]);
+                na[kk][3] = pack(-dvn[2 * kk + 1][2], -dvn[2 * kk + 1][3]);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                for (int nn = 0; nn < 16; nn += 2) {
+                    uint32_t b[4];
+                    ldBkn(b, Ws, LDK, 8 * nn, 16 * kk, lane);
+                    mma(ds[nn], na[kk], b[0], b[1]);
+                    mma(ds[nn + 1], na[kk], b[2], b[3]);
+                }
+        }
+        __syncthreads();
+    }
+    if (dS_in) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int vv = v0 + gq + 8 * (e >> 1), d = 8 * j + 2 * tq + (e & 1);
+                dS_in[((size_t)bh * DK + d) * DV + vv] = ds[j][e];
+            }
+    }
+}
+
+template <int DV, bool BETA>
+__global__ void __launch_bounds__(128, 1)
+tc_scan_fwd_kernel(SeqView s, const float* __restrict__ Gc, const bf16* __restrict__ W,
+                   const bf16* __restrict__ Kh, const bf16* __restrict__ Ut,
+                   const float* __restrict__ S_in, bf16* __restrict__ Vnt, bf16* __restrict__ S0t,
+                   float* __restrict__ S_out) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    constexpr int NVB = DV / 64;
+    scan_fwd_cta<DV, BETA>(s, blockIdx.x / NVB, blockIdx.x % NVB, Gc, W, Kh, Ut, S_in, Vnt, S0t, S_out, smem);
+}
+
+// Backward chains in one launch: blocks [0, BH*DV/64) recompute the forward
+// states (V_new and the chunk-entry states), the rest run the reverse
+// state-gradient scan.  The two groups share no data.
+template <int DV, bool BETA>
+__global__ void __launch_bounds__(128, 1)
+tc_scan_bwd_dual_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ dO,
+                        const float* __restrict__ Gc, const bf16* __restrict__ W,
+                        const bf16* __restrict__ Kh, const bf16* __restrict__ Ut,
+                        const bf16* __restrict__ dVit, const float* __restrict__ S_in,
+                        const float* __restrict__ dS_out, bf16* __restrict__ Vnt, bf16* __restrict__ S0t,
+                        bf16* __restrict__ dVnt, bf16* __restrict__ dSCt, float* __restrict__ dS_in) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    constexpr int NVB = DV / 64;
+    const int nsr = s.BH * NVB;
+    int id = blockIdx.x;
+    if (id < nsr) {
+        scan_fwd_cta<DV, BETA>(s, id / NVB, id % NVB, Gc, W, Kh, Ut, S_in, Vnt, S0t, nullptr, smem);
+    } else {
+        id -= nsr;
+        scan_bwd_cta<DV, BETA>(s, id / NVB, id % NVB, q, dO, Gc, W, Kh, dVit, dS_out, dVnt, dSCt, dS_in, smem);
+    }
+}
+
+// ------------------------------------------------------------------- out ---
+template <int DV>
+constexpr size_t out_smem() {
+    return (size_t)C * LDK * 2 * 2 + (size_t)DV * LDK * 2 + (size_t)DV * LDC * 2 + C * 4;
+}
+
+// O = scale (gamma * Q) S0 + (scale (Q K^T) * Gamma) V_new; 4 warps x 16 rows.
+template <int DV>
+__global__ void __launch_bounds__(128)
+tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
+              const float* __restrict__ Gc, const bf16* __restrict__ Vnt,
+              const bf16* __restrict__ S0t, bf16* __restrict__ o) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    bf16* Qs = reinterpret_cast<bf16*>(smem);
+    bf16* Ks = Qs + C * LDK;
+    bf16* S0s = Ks + C * LDK;   // [DV][LDK]
+    bf16* Vns = S0s + DV * LDK;  // [DV][LDC]
+    float* Gs = reinterpret_cast<float*>(Vns + DV * LDC);
+    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int gq = lane >> 2, tq = lane & 3;
+    const int t0 = c * C;
+    const int nval = min(C, s.T - t0);
+    const size_t Tp = (size_t)s.NC * C;
+    load_tile<C, DK, 128>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+    load_tile<C, DK, 128>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+    load_tile<DV, DK, 128>(S0s, LDK, S0t + ((size_t)bh * s.NC + c) * DV * DK, DK, DV, tid);
+    load_tile<DV, C, 128>(Vns, LDC, Vnt + ((size_t)bh * s.NC + c) * DV * C, C, DV, tid);
+    if (tid < 16) cp_async16(Gs + tid * 4, Gc + bh * Tp + t0 + tid * 4, true);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+
+    float p[8][4] = {};
+    float acc[DV / 8][4] = {};
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        uint32_t a[4];
+        ldA(a, Qs, LDK, 16 * w, 16 * kk, lane);
+#pragma unroll
+        for (int nn = 0; nn < 8; nn += 2) {
+            uint32_t b[4];
+            ldBnk(b, Ks, LDK, 8 * nn, 16 * kk, lane);
+            mma(p[nn], a, b[0], b[1]);
+            mma(p[nn + 1], a, b[2], b[3]);
+        }
+#pragma unroll
+        for (int nn = 0; nn < DV / 8; nn += 2) {
+            uint32_t b[4];
+            ldBnk(b, S0s, LDK, 8 * nn, 16 * kk, lane);
+            mma(acc[nn], a, b[0], b[1]);
+            mma(acc[nn + 1], a, b[2], b[3]);
+        }
+    }
+    const int i0 = 16 * w + gq, i1 = i0 + 8;
+    const float G0 = Gs[i0], G1 = Gs[i1];
+    const float sg0 = s.scale * expf(G0), sg1 = s.scale * expf(G1);
+#pragma unroll
+    for (int nn = 0; nn < DV / 8; ++nn) {
+        acc[nn][0] *= sg0;
+        acc[nn][1] *= sg0;
+        acc[nn][2] *= sg1;
+        acc[nn][3] *= sg1;
+    }
+#pragma unroll
+    for (int nn = 0; nn < 8; ++nn)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int i = (e >> 1) ? i1 : i0, j = 8 * nn + 2 * tq + (e & 1);
+            p[nn][e] = (j <= i) ? s.scale * expf(((e >> 1) ? G1 : G0) - Gs[j]) * p[nn][e] : 0.f;
+        }
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        uint32_t a[4];
+        c2a(a, p[2 * kk], p[2 * kk + 1]);
+#pragma unroll
+        for (int nn = 0; nn < DV / 8; nn += 2) {
+            uint32_t b[4];
+            ldBnk(b, Vns, LDC, 8 * nn, 16 * kk, lane);
+            mma(acc[nn], a, b[0], b[1]);
+            mma(acc[nn + 1], a, b[2], b[3]);
+        }
+    }
+    bf16* ob = o + bh * s.hs_v + (size_t)t0 * DV;
+#pragma unroll
+    for (int nn = 0; nn < DV / 8; ++nn) {
+        const int col = 8 * nn + 2 * tq;
+        if (i0 < nval) *reinterpret_cast<uint32_t*>(ob + (size_t)i0 * DV + col) = pack(acc[nn][0], acc[nn][1]);
+        if (i1 < nval) *reinterpret_cast<uint32_t*>(ob + (size_t)i1 * DV + col) = pack(acc[nn][2], acc[nn][3]);
+    }
+}
+
+// ------------------------------------------------------------------ grad ---
+// Partial-sum rows (each [64] fp32) of the gradient kernel's reductions.
+enum GradPart {
+    P_INTER = 0,   // [2]  sum_k Q_ik dq_inter_ik
+    P_Z = 2,       // [2]  sum_k K_jk dK_state_jk
+    P_ROWP = 4,    // [2]  row sums of M * (Qs K^T)
+    P_COLP = 6,    // [4]  column sums of the same
+    P_KT = 10,     // [2]  gamma_j k_j . dKt_j
+    P_DBC = 12,    // [4]  column sums of dT * L
+    P_DBR = 16,    // [2]  row sums of dA * Gamma * KK
+    P_ROWA = 18,   // [2]  row sums of Z * KK
+    P_COLA = 20,   // [4]  column sums of Z * KK
+    P_DG = 24,     // [1]  dG
+    P_ROWS = 25
+};
+
+template <int DV>
+constexpr size_t grad_region_bytes() {
+    const size_t sa = (size_t)DV * LDK * 2 * 2;                                     // S0^T, dS_C^T
+    const size_t sb = (size_t)C * LDK * 2 + (size_t)C * LDF * 4 * 2 + (size_t)C * LDC * 2 * 4;  // dW, A, L, T/L/M/dL
+    return sa > sb ? sa : sb;
+}
+template <int DV>
+constexpr size_t grad_smem() {
+    return (size_t)C * LDK * 2 * 2 + (size_t)C * (DV + 8) * 2 * 2 + (size_t)DV * LDC * 2 * 2 +
+           grad_region_bytes<DV>() + (size_t)P_ROWS * C * 4 + 256 * 4 + 2 * C * 4;
+}
+
+// Every input gradient of one chunk (8 warps: rows 16*(w%4), column half w/4).
+template <int DV, bool BETA>
+__global__ void __launch_bounds__(256, 1)
+tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
+               const bf16* __restrict__ v, const float* __restrict__ beta,
+               const bf16* __restrict__ dO, const float* __restrict__ Gc,
+               const bf16* __restrict__ Vnt, const bf16* __restrict__ dVnt,
+               const bf16* __restrict__ S0t, const bf16* __restrict__ dSCt, bf16* __restrict__ dq,
+               bf16* __restrict__ dk, bf16* __restrict__ dv, float* __restrict__ dg,
+               float* __restrict__ dbeta) {
+    constexpr int LDV = DV + 8;
+    extern __shared__ __align__(16) unsigned char smem[];
+    bf16* Qs = reinterpret_cast<bf16*>(smem);
+    bf16* Ks = Qs + C * LDK;
+    bf16* Vs = Ks + C * LDK;     // [C][LDV]
+    bf16* dOs = Vs + C * LDV;    // [C][LDV]
+    bf16* Vns = dOs + C * LDV;   // [DV][LDC]  V_new^T
+    bf16* dVns = Vns + DV * LDC;  // [DV][LDC] dV_new^T
+    unsigned char* R = reinterpret_cast<unsigned char*>(dVns + DV * LDC);
+    bf16* S0s = reinterpret_cast<bf16*>(R);       // [DV][LDK]  (phase S)
+    bf16* dSs = S0s + DV * LDK;                   // [DV][LDK]  (phase S)
+    bf16* dWs = reinterpret_cast<bf16*>(R);       // [C][LDK]   (after phase S)
+    float* Af = reinterpret_cast<float*>(R + C * LDK * 2);  // [C][LDF]; later Xs, Zs
+    float* Lf = Af + C * LDF;                     // [C][LDF]
+    bf16* Ts = reinterpret_cast<bf16*>(Lf + C * LDF);  // [C][LDC]; Y scratch during the inverse
+    bf16* Ls = Ts + C * LDC;
+    bf16* Ms = Ls + C * LDC;
+    bf16* dLs = Ms + C * LDC;
+    bf16* Xs = reinterpret_cast<bf16*>(Af);
+    bf16* Zs = Xs + C * LDC;
+    float* part = reinterpret_cast<float*>(R + grad_region_bytes<DV>());  // [P_ROWS][C]
+    float* red = part + P_ROWS * C;                                        // [256]
+    float* Gs = red + 256;
+    float* Bs = Gs + C;
+
+    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int gq = lane >> 2, tq = lane & 3;
+    const int mw = w & 3, nw = w >> 2;
+    const int t0 = c * C;
+    const int nval = min(C, s.T - t0);
+    const size_t Tp = (size_t)s.NC * C;
+    const size_t ci = (size_t)bh * s.NC + c;
+    load_tile<C, DK, 256>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+    load_tile<C, DK, 256>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+    load_tile<C, DV, 256>(Vs, LDV, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+    load_tile<C, DV, 256>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+    load_tile<DV, C, 256>(Vns, LDC, Vnt + ci * DV * C, C, DV, tid);
+    load_tile<DV, C, 256>(dVns, LDC, dVnt + ci * DV * C, C, DV, tid);
+    load_tile<DV, DK, 256>(S0s, LDK, S0t + ci * DV * DK, DK, DV, tid);
+    load_tile<DV, DK, 256>(dSs, LDK, dSCt + ci * DV * DK, DK, DV, tid);
+    if (tid < 16) cp_async16(Gs + tid * 4, Gc + bh * Tp + t0 + tid * 4, true);
+    cp_async_commit();
+    for (int i = tid; i < C; i += 256) Bs[i] = (BETA && i < nval) ? beta[bh * s.hs_g + t0 + i] : 0.f;
+    for (int e = tid; e < P_ROWS * C; e += 256) part[e] = 0.f;
+    cp_async_wait<0>();
+    __syncthreads();
+
+    const int r0 = 16 * mw + gq, r1 = r0 + 8;  // the two rows this thread holds
+    const float gam0 = expf(Gs[r0]), gam1 = expf(Gs[r1]);
+    const float gC = Gs[C - 1];
+    const float dec0 = expf(gC - Gs[r0]), dec1 = expf(gC - Gs[r1]);
+
+    // ---- phase S: products with the chunk-entry state and the state gradient
+    float accQ[8][4] = {}, accK[8][4] = {};
+    {
+        float accW[8][4] = {};
+#pragma unroll
+        for (int kv = 0; kv < DV / 16; ++kv) {
+            uint32_t aO[4], aN[4], aV[4];
+            ldA(aO, dOs, LDV, 16 * mw, 16 * kv, lane);
+            ldAt(aN, dVns, LDC, 16 * mw, 16 * kv, lane);
+            ldAt(aV, Vns, LDC, 16 * mw, 16 * kv, lane);
+#pragma unroll
+            for (int nn = 0; nn < 8; nn += 2) {
+                uint32_t b[4];
+                ldBkn(b, S0s, LDK, 64 * nw + 8 * nn, 16 * kv, lane);
+                mma(accQ[nn], aO, b[0], b[1]);
+                mma(accQ[nn + 1], aO, b[2], b[3]);
+                mma(accW[nn], aN, b[0], b[1]);
+                mma(accW[nn + 1], aN, b[2], b[3]);
+                ldBkn(b, dSs, LDK, 64 * nw + 8 * nn, 16 * kv, lane);
+                mma(accK[nn], aV, b[0], b[1]);
+                mma(accK[nn + 1], aV, b[2], b[3]);
+            }
+        }
+        float pd = 0.f;  // <S0, dS_C>
+        for (int e = tid; e < DV * DK; e += 256) {
+            const int r = e / DK, cc = e % DK;
+            pd += __bfloat162float(S0s[r * LDK + cc]) * __bfloat162float(dSs[r * LDK + cc]);
+        }
+        red[tid] = pd;
+        // dq_inter = scale gamma (dO S0^T); dK_state = dec (V_new dS_C^T)
+        const float sq0 = s.scale * gam0, sq1 = s.scale * gam1;
+        float pi0 = 0.f, pi1 = 0.f, pz0 = 0.f, pz1 = 0.f;
+#pragma unroll
+        for (int nn = 0; nn < 8; ++nn) {
+            const int col = 64 * nw + 8 * nn + 2 * tq;
+            const float2 q0 = unpack(*reinterpret_cast<const uint32_t*>(Qs + r0 * LDK + col));
+            const float2 q1 = unpack(*reinterpret_cast<const uint32_t*>(Qs + r1 * LDK + col));
+            const float2 k0 = unpack(*reinterpret_cast<const uint32_t*>(Ks + r0 * LDK + col));
+            const float2 k1 = unpack(*reinterpret_cast<const uint32_t*>(Ks + r1 * LDK + col));
+            accQ[nn][0] *= sq0;
+            accQ[nn][1] *= sq0;
+            accQ[nn][2] *= sq1;
+            accQ[nn][3] *= sq1;
+            accK[nn][0] *= dec0;
+            accK[nn][1] *= dec0;
+            accK[nn][2] *= dec1;
+            accK[nn][3] *= dec1;
+            pi0 += q0.x * accQ[nn][0] + q0.y * accQ[nn][1];
+            pi1 += q1.x * accQ[nn][2] + q1.y * accQ[nn][3];
+            pz0 += k0.x * accK[nn][0] + k0.y * accK[nn][1];
+            pz1 += k1.x * accK[nn][2] + k1.y * accK[nn][3];
+        }
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+            pi0 += __shfl_xor_sync(0xffffffffu, pi0, o);
+            pi1 += __shfl_xor_sync(0xffffffffu, pi1, o);
+            pz0 += __shfl_xor_sync(0xffffffffu, pz0, o);
+            pz1 += __shfl_xor_sync(0xffffffffu, pz1, o);
+        }
+        if (tq == 0) {
+            part[(P_INTER + nw) * C + r0] = pi0;
+            part[(P_INTER + nw) * C + r1] = pi1;
+            part[(P_Z + nw) * C + r0] = pz0;
+            part[(P_Z + nw) * C + r1] = pz1;
+        }
+        __syncthreads();  // everyone is done with S0^T and dS_C^T
+        // dW = -dV_new S0^T into the freed region
+#pragma unroll
+        for (int nn = 0; nn < 8; ++nn) {
+            const int col = 64 * nw + 8 * nn + 2 * tq;
+            *reinterpret_cast<uint32_t*>(dWs + r0 * LDK + col) = pack(-accW[nn][0], -accW[nn][1]);
+            *reinterpret_cast<uint32_t*>(dWs + r1 * LDK + col) = pack(-accW[nn][2], -accW[nn][3]);
+        }
+    }
+    for (int o = 128; o > 0; o >>= 1) {
+        if (tid < o) red[tid] += red[tid + o];
+        __syncthreads();
+    }
+    const float sdot = red[0];
+
+    // ---- phase C1: C x C products (rows 16mw.., columns 32nw..)
+    float kkr[4][4] = {};
+    {
+        float qk[4][4] = {}, dp[4][4] = {};
+#pragma unroll
+        for (int kd = 0; kd < 8; ++kd) {
+            uint32_t aQ[4], aK[4];
+            ldA(aQ, Qs, LDK, 16 * mw, 16 * kd, lane);
+            ldA(aK, Ks, LDK, 16 * mw, 16 * kd, lane);
+#pragma unroll
+            for (int nn = 0; nn < 4; nn += 2) {
+                uint32_t b[4];
+                ldBnk(b, Ks, LDK, 32 * nw + 8 * nn, 16 * kd, lane);
+                mma(qk[nn], aQ, b[0], b[1]);
+                mma(qk[nn + 1], aQ, b[2], b[3]);
+                mma(kkr[nn], aK, b[0], b[1]);
+                mma(kkr[nn + 1], aK, b[2], b[3]);
+            }
+        }
+#pragma unroll
+        for (int kv = 0; kv < DV / 16; ++kv) {
+            uint32_t aO[4];
+            ldA(aO, dOs, LDV, 16 * mw, 16 * kv, lane);
+#pragma unroll
+            for (int nn = 0; nn < 4; nn += 2) {
+                uint32_t b[4];
+                ldBkn(b, Vns, LDC, 32 * nw + 8 * nn, 16 * kv, lane);
+                mma(dp[nn], aO, b[0], b[1]);
+                mma(dp[nn + 1], aO, b[2], b[3]);
+            }
+        }
+        float row0 = 0.f, row1 = 0.f;
+#pragma unroll
+        for (int nn = 0; nn < 4; ++nn) {
+            float col[2] = {0.f, 0.f};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = (e >> 1) ? r1 : r0, j = 32 * nw + 8 * nn + 2 * tq + (e & 1);
+                const float gm = (j <= i) ? expf(Gs[i] - Gs[j]) : 0.f;
+                const float m = s.scale * dp[nn][e] * gm;
+                Ms[i * LDC + j] = __float2bfloat16_rn(m);
+                const float zp = m * qk[nn][e];
+                if (e >> 1) row1 += zp; else row0 += zp;
+                col[e & 1] += zp;
+                if (BETA) Af[i * LDF + j] = (j < i) ? Bs[i] * gm * kkr[nn][e] : 0.f;
+            }
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                col[0] += __shfl_xor_sync(0xffffffffu, col[0], o);
+                col[1] += __shfl_xor_sync(0xffffffffu, col[1], o);
+            }
+            if (gq == 0) {
+                const int j = 32 * nw + 8 * nn + 2 * tq;
+                part[(P_COLP + mw) * C + j] = col[0];
+                part[(P_COLP + mw) * C + j + 1] = col[1];
+            }
+        }
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+            row0 += __shfl_xor_sync(0xffffffffu, row0, o);
+            row1 += __shfl_xor_sync(0xffffffffu, row1, o);
+        }
+        if (tq == 0) {
+            part[(P_ROWP + nw) * C + r0] = row0;
+            part[(P_ROWP + nw) * C + r1] = row1;
+        }
+        if (BETA)
+            for (int e = tid; e < C * LDF; e += 256) Lf[e] = 0.f;
+    }
+    __syncthreads();
+
+    // ---- phase C2: L = (I + A)^{-1}; T = L diag(beta)
+    if (BETA) {
+        block_inverse(Af, LDF, Lf, LDF, reinterpret_cast<float*>(Ts), tid, 256);
+        for (int e = tid; e < C * C; e += 256) {
+            const int i = e >> 6, j = e & 63;
+            const float l = Lf[i * LDF + j];
+            Ts[i * LDC + j] = __float2bfloat16_rn(l * Bs[j]);
+            Ls[i * LDC + j] = __float2bfloat16_rn(l);
+        }
+        __syncthreads();
+    }
+
+    // ---- phase C3: dKt = T^T dW (into dK), dV = T^T dV_new
+    if (BETA) {
+        float acc[8][4] = {};
+#pragma unroll
+        for (int kr = 0; kr < 4; ++kr) {
+            uint32_t a[4];
+            ldAt(a, Ts, LDC, 16 * mw, 16 * kr, lane);
+#pragma unroll
+            for (int nn = 0; nn < 8; nn += 2) {
+                uint32_t b[4];
+                ldBkn(b, dWs, LDK, 64 * nw + 8 * nn, 16 * kr, lane);
+                mma(acc[nn], a, b[0], b[1]);
+                mma(acc[nn + 1], a, b[2], b[3]);
+            }
+        }
+        float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+        for (int nn = 0; nn < 8; ++nn) {
+            const int col = 64 * nw + 8 * nn + 2 * tq;
+            const float2 k0 = unpack(*reinterpret_cast<const uint32_t*>(Ks + r0 * LDK + col));
+            const float2 k1 = unpack(*reinterpret_cast<const uint32_t*>(Ks + r1 * LDK + col));
+            const float a0 = gam0 * acc[nn][0], a1 = gam0 * acc[nn][1];
+            const float a2 = gam1 * acc[nn][2], a3 = gam1 * acc[nn][3];
+            accK[nn][0] += a0;
+            accK[nn][1] += a1;
+            accK[nn][2] += a2;
+            accK[nn][3] += a3;
+            p0 += k0.x * a0 + k0.y * a1;
+            p1 += k1.x * a2 + k1.y * a3;
+        }
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+            p0 += __shfl_xor_sync(0xffffffffu, p0, o);
+            p1 += __shfl_xor_sync(0xffffffffu, p1, o);
+        }
+        if (tq == 0) {
+            part[(P_KT + nw) * C + r0] = p0;
+            part[(P_KT + nw) * C + r1] = p1;
+        }
+    }
+    {
+        constexpr int NT = DV / 16;  // n-tiles of this warp's half of the value columns
+        bf16* dvb = dv + bh * s.hs_v + (size_t)t0 * DV;
+        if (BETA) {
+            float acc[NT][4] = {};
+#pragma unroll
+            for (int kr = 0; kr < 4; ++kr) {
+                uint32_t a[4];
+                ldAt(a, Ts, LDC, 16 * mw, 16 * kr, lane);
+#pragma unroll
+                for (int nn = 0; nn < NT; nn += 2) {
+                    uint32_t b[4];
+                    ldBnk(b, dVns, LDC, (DV / 2) * nw + 8 * nn, 16 * kr, lane);
+                    mma(acc[nn], a, b[0], b[1]);
+                    mma(acc[nn + 1], a, b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int nn = 0; nn < NT; ++nn) {
+                const int col = (DV / 2) * nw + 8 * nn + 2 * tq;
+                if (r0 < nval) *reinterpret_cast<uint32_t*>(dvb + (size_t)r0 * DV + col) = pack(acc[nn][0], acc[nn][1]);
+                if (r1 < nval) *reinterpret_cast<uint32_t*>(dvb + (size_t)r1 * DV + col) = pack(acc[nn][2], acc[nn][3]);
+            }
+        } else {
+            for (int e = tid; e < nval * DV; e += 256) {
+                const int j = e / DV, col = e % DV;
+                dvb[(size_t)j * DV + col] = dVns[col * LDC + j];
+            }
+        }
+    }
+
+    // ---- phase C4: dT = dW (gamma K)^T + dV_new V^T; dbeta (column part); dL = dT diag(beta)
+    if (BETA) {
+        float dt[4][4] = {};
+#pragma unroll
+        for (int kd = 0; kd < 8; ++kd) {
+            uint32_t a[4];
+            ldA(a, dWs, LDK, 16 * mw, 16 * kd, lane);
+#pragma unroll
+            for (int nn = 0; nn < 4; nn += 2) {
+                uint32_t b[4];
+                ldBnk(b, Ks, LDK, 32 * nw + 8 * nn, 16 * kd, lane);
+                mma(dt[nn], a, b[0], b[1]);
+                mma(dt[nn + 1], a, b[2], b[3]);
+            }
+        }
+#pragma unroll
+        for (int nn = 0; nn < 4; ++nn)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dt[nn][e] *= expf(Gs[32 * nw + 8 * nn + 2 * tq + (e & 1)]);
+#pragma unroll
+        for (int kv = 0; kv < DV / 16; ++kv) {
+            uint32_t a[4];
+            ldAt(a, dVns, LDC, 16 * mw, 16 * kv, lane);
+#pragma unroll
+            for (int nn = 0; nn < 4; nn += 2) {
+                uint32_t b[4];
+                ldBnk(b, Vs, LDV, 32 * nw + 8 * nn, 16 * kv, lane);
+                mma(dt[nn], a, b[0], b[1]);
+                mma(dt[nn + 1], a, b[2], b[3]);
+            }
+        }
+#pragma unroll
+        for (int nn = 0; nn < 4; ++nn) {
+            float col[2] = {0.f, 0.f};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = (e >> 1) ? r1 : r0, j = 32 * nw + 8 * nn + 2 * tq + (e & 1);
+                col[e & 1] += dt[nn][e] * Lf[r * LDF + j];
+                dLs[r * LDC + j] = __float2bfloat16_rn(dt[nn][e] * Bs[j]);
+            }
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                col[0] += __shfl_xor_sync(0xffffffffu, col[0], o);
+                col[1] += __shfl_xor_sync(0xffffffffu, col[1], o);
+            }
+            if (gq == 0) {
+                const int j = 32 * nw + 8 * nn + 2 * tq;
+                part[(P_DBC + mw) * C + j] = col[0];
+                part[(P_DBC + mw) * C + j + 1] = col[1];
+            }
+        }
+        __syncthreads();
+        // ---- phase C5: X = L^T dL
+        {
+            float x[4][4] = {};
+#pragma unroll
+            for (int kr = 0; kr < 4; ++kr) {
+                uint32_t a[4];
+                ldAt(a, Ls, LDC, 16 * mw, 16 * kr, lane);
+#pragma unroll
+                for (int nn = 0; nn < 4; nn += 2) {
+                    uint32_t b[4];
+                    ldBkn(b, dLs, LDC, 32 * nw + 8 * nn, 16 * kr, lane);
+                    mma(x[nn], a, b[0], b[1]);
+                    mma(x[nn + 1], a, b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int nn = 0; nn < 4; ++nn) {
+                const int j = 32 * nw + 8 * nn + 2 * tq;
+                *reinterpret_cast<uint32_t*>(Xs + r0 * LDC + j) = pack(x[nn][0], x[nn][1]);
+                *reinterpret_cast<uint32_t*>(Xs + r1 * LDC + j) = pack(x[nn][2], x[nn][3]);
+            }
+        }
+        __syncthreads();
+        // ---- phase C6: dA = strictly-lower(-X L^T); Z = dA beta_i Gamma; dbeta (row part)
+        {
+            float da[4][4] = {};
+#pragma unroll
+            for (int km = 0; km < 4; ++km) {
+                uint32_t a[4];
+                ldA(a, Xs, LDC, 16 * mw, 16 * km, lane);
+#pragma unroll
+                for (int nn = 0; nn < 4; nn += 2) {
+                    uint32_t b[4];
+                    ldBnk(b, Ls, LDC, 32 * nw + 8 * nn, 16 * km, lane);
+                    mma(da[nn], a, b[0], b[1]);
+                    mma(da[nn + 1], a, b[2], b[3]);
+                }
+            }
+            float rz0 = 0.f, rz1 = 0.f, rb0 = 0.f, rb1 = 0.f;
+#pragma unroll
+            for (int nn = 0; nn < 4; ++nn) {
+                float col[2] = {0.f, 0.f};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = (e >> 1) ? r1 : r0, j = 32 * nw + 8 * nn + 2 * tq + (e & 1);
+                    float z = 0.f, bterm = 0.f;
+                    if (j < i) {
+                        const float gm = expf(Gs[i] - Gs[j]);
+                        const float dav = -da[nn][e];
+                        bterm = dav * gm * kkr[nn][e];
+                        z = dav * Bs[i] * gm;
+                    }
+                    Zs[i * LDC + j] = __float2bfloat16_rn(z);
+                    const float za = z * kkr[nn][e];
+                    if (e >> 1) {
+                        rz1 += za;
+                        rb1 += bterm;
+                    } else {
+                        rz0 += za;
+                        rb0 += bterm;
+                    }
+                    col[e & 1] += za;
+                }
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) {
+                    col[0] += __shfl_xor_sync(0xffffffffu, col[0], o);
+                    col[1] += __shfl_xor_sync(0xffffffffu, col[1], o);
+                }
+                if (gq == 0) {
+                    const int j = 32 * nw + 8 * nn + 2 * tq;
+                    part[(P_COLA + mw) * C + j] = col[0];
+                    part[(P_COLA + mw) * C + j + 1] = col[1];
+                }
+            }
+#pragma unroll
+            for (int o = 1; o < 4; o <<= 1) {
+                rz0 += __shfl_xor_sync(0xffffffffu, rz0, o);
+                rz1 += __shfl_xor_sync(0xffffffffu, rz1, o);
+                rb0 += __shfl_xor_sync(0xffffffffu, rb0, o);
+                rb1 += __shfl_xor_sync(0xffffffffu, rb1, o);
+            }
+            if (tq == 0) {
+                part[(P_ROWA + nw) * C + r0] = rz0;
+                part[(P_ROWA + nw) * C + r1] = rz1;
+                part[(P_DBR + nw) * C + r0] = rb0;
+                part[(P_DBR + nw) * C + r1] = rb1;
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- phase C7: dK += (Z + Z^T) K + Ms^T Q ; dq += Ms K
+#pragma unroll
+    for (int ki = 0; ki < 4; ++ki) {
+        uint32_t aM[4], aMt[4];
+        ldA(aM, Ms, LDC, 16 * mw, 16 * ki, lane);
+        ldAt(aMt, Ms, LDC, 16 * mw, 16 * ki, lane);
+        uint32_t aZ[4], aZt[4];
+        if (BETA) {
+            ldA(aZ, Zs, LDC, 16 * mw, 16 * ki, lane);
+            ldAt(aZt, Zs, LDC, 16 * mw, 16 * ki, lane);
+        }
+#pragma unroll
+        for (int nn = 0; nn < 8; nn += 2) {
+            uint32_t bk[4], bq[4];
+            ldBkn(bk, Ks, LDK, 64 * nw + 8 * nn, 16 * ki, lane);
+            ldBkn(bq, Qs, LDK, 64 * nw + 8 * nn, 16 * ki, lane);
+            mma(accQ[nn], aM, bk[0], bk[1]);
+            mma(accQ[nn + 1], aM, bk[2], bk[3]);
+            mma(accK[nn], aMt, bq[0], bq[1]);
+            mma(accK[nn + 1], aMt, bq[2], bq[3]);
+            if (BETA) {
+                mma(accK[nn], aZ, bk[0], bk[1]);
+                mma(accK[nn + 1], aZ, bk[2], bk[3]);
+                mma(accK[nn], aZt, bk[0], bk[1]);
+                mma(accK[nn + 1], aZt, bk[2], bk[3]);
+            }
+        }
+    }
+    {
+        bf16* dqb = dq + bh * s.hs_k + (size_t)t0 * DK;
+        bf16* dkb = dk + bh * s.hs_k + (size_t)t0 * DK;
+#pragma unroll
+        for (int nn = 0; nn < 8; ++nn) {
+            const int col = 64 * nw + 8 * nn + 2 * tq;
+            if (r0 < nval) {
+                *reinterpret_cast<uint32_t*>(dqb + (size_t)r0 * DK + col) = pack(accQ[nn][0], accQ[nn][1]);
+                *reinterpret_cast<uint32_t*>(dkb + (size_t)r0 * DK + col) = pack(accK[nn][0], accK[nn][1]);
+            }
+            if (r1 < nval) {
+                *reinterpret_cast<uint32_t*>(dqb + (size_t)r1 * DK + col) = pack(accQ[nn][2], accQ[nn][3]);
+                *reinterpret_cast<uint32_t*>(dkb + (size_t)r1 * DK + col) = pack(accK[nn][2], accK[nn][3]);
+            }
+        }
+    }
+
+    // ---- phase C8: dG, dg (reverse cumsum), dbeta
+    float* dG = part + P_DG * C;
+    if (tid < C) {
+        const int i = tid;
+        auto P = [&](int row) { return part[row * C + i]; };
+        float x = P(P_INTER) + P(P_INTER + 1) + P(P_ROWP) + P(P_ROWP + 1) -
+                  (P(P_COLP) + P(P_COLP + 1) + P(P_COLP + 2) + P(P_COLP + 3)) - (P(P_Z) + P(P_Z + 1));
+        if (BETA) {
+            x += P(P_ROWA) + P(P_ROWA + 1) - (P(P_COLA) + P(P_COLA + 1) + P(P_COLA + 2) + P(P_COLA + 3)) +
+                 P(P_KT) + P(P_KT + 1);
+            const float db = P(P_DBC) + P(P_DBC + 1) + P(P_DBC + 2) + P(P_DBC + 3) + P(P_DBR) + P(P_DBR + 1);
+            if (i < nval) dbeta[bh * s.hs_g + t0 + i] = db;
+        }
+        dG[i] = x;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float zs = 0.f;
+        for (int j = 0; j < C; ++j) zs += part[P_Z * C + j] + part[(P_Z + 1) * C + j];
+        dG[C - 1] += expf(gC) * sdot + zs;
+        float acc = 0.f;
+        for (int i = C - 1; i >= 0; --i) {
+            acc += dG[i];
+            if (i < nval) dg[bh * s.hs_g + t0 + i] = acc;
+        }
+    }
+}
+
+template <typename K>
+cudaError_t smem_attr(K* kern, size_t bytes) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+#define TC_TRY(x)                          \
+    do {                                   \
+        cudaError_t e_ = (x);              \
+        if (e_ != cudaSuccess) return e_;  \
+    } while (0)
+
+template <int DV, bool BETA>
+cudaError_t fwd_impl(const SeqView& s, const FwdArgs& a, void* ws, cudaStream_t st) {
+    char* base = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), 256));
+    TcWs w = tc_layout(s, false, base);
+    const bf16* q = static_cast<const bf16*>(a.q);
+    const bf16* k = static_cast<const bf16*>(a.k);
+    const bf16* v = static_cast<const bf16*>(a.v);
+    constexpr size_t sm_prep = prep_smem<DV, false>();
+    constexpr size_t sm_scan = 2 * fwd_stage_bytes<BETA>();
+    constexpr size_t sm_out = out_smem<DV>();
+    TC_TRY(smem_attr(tc_prep_kernel<DV, BETA, false>, sm_prep));
+    TC_TRY(smem_attr(tc_scan_fwd_kernel<DV, BETA>, sm_scan));
+    TC_TRY(smem_attr(tc_out_kernel<DV>, sm_out));
+    const dim3 gc(s.NC, s.BH);
+    SF_LAUNCH("tc_prep", st, tc_prep_kernel<DV, BETA, false><<<gc, 128, sm_prep, st>>>(
+                                 s, q, k, v, a.g, a.beta, nullptr, w.Gc, w.W, w.Kh, w.Ut, nullptr));
+    TC_TRY(cudaGetLastError());
+    SF_LAUNCH("tc_scan_fwd", st, tc_scan_fwd_kernel<DV, BETA><<<s.BH * (DV / 64), 128, sm_scan, st>>>(
+                                     s, w.Gc, w.W, w.Kh, w.Ut, a.S_in, w.Vnt, w.S0t, a.S_out));
+    TC_TRY(cudaGetLastError());
+    SF_LAUNCH("tc_out", st, tc_out_kernel<DV><<<gc, 128, sm_out, st>>>(s, q, k, w.Gc, w.Vnt, w.S0t,
+                                                                         static_cast<bf16*>(a.o)));
+    return cudaGetLastError();
+}
+
+template <int DV, bool BETA>
+cudaError_t bwd_impl(const SeqView& s, const BwdArgs& a, void* ws, cudaStream_t st) {
+    char* base = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), 256));
+    TcWs w = tc_layout(s, true, base);
+    const bf16* q = static_cast<const bf16*>(a.q);
+    const bf16* k = static_cast<const bf16*>(a.k);
+    const bf16* v = static_cast<const bf16*>(a.v);
+    const bf16* dO = static_cast<const bf16*>(a.dO);
+    constexpr size_t sm_prep = prep_smem<DV, true>();
+    constexpr size_t sm_f = 2 * fwd_stage_bytes<BETA>(), sm_b = 2 * bwd_stage_bytes<BETA>();
+    constexpr size_t sm_scan = sm_f > sm_b ? sm_f : sm_b;
+    constexpr size_t sm_grad = grad_smem<DV>();
+    TC_TRY(smem_attr(tc_prep_kernel<DV, BETA, true>, sm_prep));
+    TC_TRY(smem_attr(tc_scan_bwd_dual_kernel<DV, BETA>, sm_scan));
+    TC_TRY(smem_attr(tc_grad_kernel<DV, BETA>, sm_grad));
+    const dim3 gc(s.NC, s.BH);
+    SF_LAUNCH("tc_prep_bwd", st, tc_prep_kernel<DV, BETA, true><<<gc, 128, sm_prep, st>>>(
+                                     s, q, k, v, a.g, a.beta, dO, w.Gc, w.W, w.Kh, w.Ut, w.dVit));
+    TC_TRY(cudaGetLastError());
+    SF_LAUNCH("tc_scan_bwd", st, tc_scan_bwd_dual_kernel<DV, BETA><<<2 * s.BH * (DV / 64), 128, sm_scan, st>>>(
+                                     s, q, dO, w.Gc, w.W, w.Kh, w.Ut, w.dVit, a.S_in, a.dS_out, w.Vnt, w.S0t,
+                                     w.dVnt, w.dSCt, a.dS_in));
+    TC_TRY(cudaGetLastError());
+    SF_LAUNCH("tc_grad", st, tc_grad_kernel<DV, BETA><<<gc, 256, sm_grad, st>>>(
+                                 s, q, k, v, a.beta, dO, w.Gc, w.Vnt, w.dVnt, w.S0t, w.dSCt,
+                                 static_cast<bf16*>(a.dq), static_cast<bf16*>(a.dk), static_cast<bf16*>(a.dv),
+                                 a.dg, a.dbeta));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_supports(bool bf16_io, int dk, int dv, int Cc, bool) {
+    return bf16_io && dk == DK && (dv == 64 || dv == 128) && Cc == C;
+}
+
+size_t tc_workspace_bytes(const SeqView& s, bool backward) { return tc_layout(s, backward, nullptr).total; }
+
+cudaError_t tc_fwd(const SeqView& s, const FwdArgs& a, void* ws, cudaStream_t st) {
+    if (s.dv == 128) return s.use_beta ? fwd_impl<128, true>(s, a, ws, st) : fwd_impl<128, false>(s, a, ws, st);
+    return s.use_beta ? fwd_impl<64, true>(s, a, ws, st) : fwd_impl<64, false>(s, a, ws, st);
+}
+
+cudaError_t tc_bwd(const SeqView& s, const BwdArgs& a, void* ws, cudaStream_t st) {
+    if (s.dv == 128) return s.use_beta ? bwd_impl<128, true>(s, a, ws, st) : bwd_impl<128, false>(s, a, ws, st);
+    return s.use_beta ? bwd_impl<64, true>(s, a, ws, st) : bwd_impl<64, false>(s, a, ws, st);
+}
+
+int tc_launches(bool) { return 3; }
 
 }  // namespace sf

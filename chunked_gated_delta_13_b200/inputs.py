@@ -63,6 +63,9 @@ CONFIGS = {
                         S_in_std=0.0, dS_out_std=0.0, N=1),
     "headline_h16_t64k": Workload("headline_h16_t64k", B=1, H=16, T=65536, dk=128, dv=128,
                                   C=64, S_in_std=0.0, dS_out_std=0.1, N=1),
+    # a small case of the headline shape for profiler captures (inputs still larger than L2)
+    "profile_h16_t8k": Workload("profile_h16_t8k", B=1, H=16, T=8192, dk=128, dv=128, C=64,
+                                S_in_std=0.0, dS_out_std=0.1, N=1),
 }
 
 
