@@ -35,15 +35,16 @@ constexpr int LDC = C + 8;   // shared row stride of [*][C] tiles
 constexpr int LDF = 72;      // shared row stride of fp32 [C][C] tiles
 
 struct TcWs {
-    float* Gc;   // [BH][Tp]           chunk-local cumulative log-decay
-    bf16* W;     // [BH][Tp][DK]
+    float* Gc;   // [BH][Tp]           chunk-local cumulative log-decay G
+    float* Gm;   // [BH][Tp]           exp(G)
+    bf16* W;     // [BH][Tp][DK]       -W (stored negated: the scans only ever subtract W products)
     bf16* Kh;    // [BH][Tp][DK]       K * exp(G_C - G)
     bf16* Ut;    // [BH][NC][DV][C]    U transposed per chunk (V^T without the beta path)
-    bf16* Vnt;   // [BH][NC][DV][C]    V_new transposed per chunk
-    bf16* S0t;   // [BH][NC][DV][DK]   state entering each chunk, transposed
+    bf16* Vnt;   // [BH][NC][DV][C]    V_new transposed per chunk (pieces permuted, see swz)
+    bf16* S0t;   // [BH][NC][DV][DK]   state entering each chunk, transposed (permuted)
     bf16* dVit;  // [BH][NC][DV][C]    intra-chunk part of dV_new, transposed
-    bf16* dVnt;  // [BH][NC][DV][C]    dV_new transposed
-    bf16* dSCt;  // [BH][NC][DV][DK]   gradient of the state leaving each chunk, transposed
+    bf16* dVnt;  // [BH][NC][DV][C]    dV_new transposed (permuted)
+    bf16* dSCt;  // [BH][NC][DV][DK]   gradient of the state leaving each chunk, transposed (permuted)
     size_t total;
 };
 
@@ -57,6 +58,7 @@ TcWs tc_layout(const SeqView& s, bool backward, char* base) {
         return p;
     };
     w.Gc = reinterpret_cast<float*>(take(BH * Tp * 4));
+    w.Gm = reinterpret_cast<float*>(take(BH * Tp * 4));
     w.W = reinterpret_cast<bf16*>(take(s.use_beta ? BH * Tp * DK * 2 : 0));
     w.Kh = reinterpret_cast<bf16*>(take(BH * Tp * DK * 2));
     w.Ut = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
@@ -91,36 +93,49 @@ __device__ __forceinline__ void chunk_cumsum(const float* g, int nval, float* Gs
 }
 
 // (I + A)^{-1} of a strictly lower-triangular 64x64 fp32 matrix A (row stride
-// la) into L (row stride ll; its strictly upper part must be zero on entry).
-// Forward substitution inside the four 16x16 diagonal blocks (warps 0-3, one
-// column per lane), then the off-diagonal blocks one block row at a time:
-// L_IJ = -L_II * sum_{m=J}^{I-1} A_Im L_mJ.  Y: 768 floats of scratch.
+// la) into L (row stride ll; the blocks strictly above the block diagonal must
+// be zero on entry).  Each 16x16 diagonal block is inverted by forward
+// substitution with one column per thread held in registers (threads 0-63);
+// the off-diagonal blocks follow in three rounds by distance from the
+// diagonal: L_IJ = -L_II * sum_{m=J}^{I-1} A_Im L_mJ.  Y: 768 floats of scratch.
 __device__ void block_inverse(const float* A, int la, float* L, int ll, float* Y, int tid, int nthr) {
-    const int lane = tid & 31, w = tid >> 5;
-    if (w < 4 && lane < 16) {
-        const int o = 16 * w, cc = lane;
-        for (int r = cc; r < 16; ++r) {
-            float x = (r == cc) ? 1.f : 0.f;
-            for (int j = cc; j < r; ++j) x -= A[(o + r) * la + o + j] * L[(o + j) * ll + o + cc];
-            L[(o + r) * ll + o + cc] = x;
+    if (tid < 64) {
+        const int o = 16 * (tid >> 4), c = tid & 15;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc = (r == c) ? 1.f : 0.f;
+#pragma unroll
+            for (int j = 0; j < r; ++j) acc = fmaf(-A[(o + r) * la + o + j], x[j], acc);
+            x[r] = acc;
         }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) L[(o + r) * ll + o + c] = x[r];
     }
     __syncthreads();
-    for (int I = 1; I < 4; ++I) {
-        for (int e = tid; e < I * 256; e += nthr) {
-            const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+#pragma unroll 1
+    for (int d = 1; d < 4; ++d) {
+        const int nb = 4 - d;
+        for (int e = tid; e < nb * 256; e += nthr) {
+            const int J = e >> 8, I = J + d, r = (e >> 4) & 15, c = e & 15;
             float y = 0.f;
-            for (int m = J; m < I; ++m)
-                for (int p = 0; p < 16; ++p)
-                    y += A[(16 * I + r) * la + 16 * m + p] * L[(16 * m + p) * ll + 16 * J + cc];
+            for (int m = J; m < I; ++m) {
+                const float* Ar = A + (16 * I + r) * la + 16 * m;
+                const float* Lc = L + (16 * m) * ll + 16 * J + c;
+#pragma unroll
+                for (int p = 0; p < 16; ++p) y = fmaf(Ar[p], Lc[p * ll], y);
+            }
             Y[e] = y;
         }
         __syncthreads();
-        for (int e = tid; e < I * 256; e += nthr) {
-            const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+        for (int e = tid; e < nb * 256; e += nthr) {
+            const int J = e >> 8, I = J + d, r = (e >> 4) & 15, c = e & 15;
+            const float* Lr = L + (16 * I + r) * ll + 16 * I;
+            const float* Yc = Y + (J << 8) + c;
             float x = 0.f;
-            for (int p = 0; p <= r; ++p) x += L[(16 * I + r) * ll + 16 * I + p] * Y[(J << 8) + p * 16 + cc];
-            L[(16 * I + r) * ll + 16 * J + cc] = -x;
+#pragma unroll
+            for (int p = 0; p < 16; ++p) x = fmaf(Lr[p], Yc[p * 16], x);
+            L[(16 * I + r) * ll + 16 * J + c] = -x;
         }
         __syncthreads();
     }
@@ -140,7 +155,7 @@ __global__ void __launch_bounds__(128)
 tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
                const bf16* __restrict__ v, const float* __restrict__ g,
                const float* __restrict__ beta, const bf16* __restrict__ dO, float* __restrict__ Gc,
-               bf16* __restrict__ Wo, bf16* __restrict__ Kho, bf16* __restrict__ Uto,
+               float* __restrict__ Gmo, bf16* __restrict__ Wo, bf16* __restrict__ Kho, bf16* __restrict__ Uto,
                bf16* __restrict__ dVito) {
     constexpr int LDV = DV + 8;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -175,7 +190,10 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     cp_async_wait<0>();
     __syncthreads();
 
-    for (int i = tid; i < C; i += 128) Gc[bh * Tp + t0 + i] = Gs[i];
+    for (int i = tid; i < C; i += 128) {
+        Gc[bh * Tp + t0 + i] = Gs[i];
+        Gmo[bh * Tp + t0 + i] = expf(Gs[i]);
+    }
     const float gC = Gs[C - 1];
     for (int e = tid; e < C * (DK / 8); e += 128) {
         const int r = e >> 4, cc = (e & 15) * 8;
@@ -222,7 +240,7 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         }
         __syncthreads();
         bf16* Wst = reinterpret_cast<bf16*>(Af);  // [C][LDK]
-        {  // W = T (gamma * K)
+        {  // W = T (gamma * K), staged negated
             float acc[16][4] = {};
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -239,8 +257,8 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 #pragma unroll
             for (int nn = 0; nn < 16; ++nn) {
                 const int i = 16 * w + gq, col = 8 * nn + 2 * tq;
-                *reinterpret_cast<uint32_t*>(Wst + i * LDK + col) = pack(acc[nn][0], acc[nn][1]);
-                *reinterpret_cast<uint32_t*>(Wst + (i + 8) * LDK + col) = pack(acc[nn][2], acc[nn][3]);
+                *reinterpret_cast<uint32_t*>(Wst + i * LDK + col) = pack(-acc[nn][0], -acc[nn][1]);
+                *reinterpret_cast<uint32_t*>(Wst + (i + 8) * LDK + col) = pack(-acc[nn][2], -acc[nn][3]);
             }
         }
         {  // U = T V, staged transposed
@@ -348,13 +366,32 @@ template <bool BETA>
 constexpr size_t bwd_stage_bytes() {
     return (size_t)C * LDK * 2 * (BETA ? 3 : 2) + (size_t)C * LDC * 2 * 2 + C * 4;
 }
+// Output staging of one chunk step of a 64-column block: the state tile
+// (64 x DK) and the value tile (64 x C), in the permuted layout of swz().
+constexpr size_t out_stage_bytes() { return (size_t)64 * DK * 2 + (size_t)64 * C * 2; }
+template <bool BETA>
+constexpr size_t fwd_scan_smem() { return 2 * fwd_stage_bytes<BETA>() + 2 * out_stage_bytes(); }
+template <bool BETA>
+constexpr size_t bwd_scan_smem() { return 2 * bwd_stage_bytes<BETA>() + 2 * out_stage_bytes(); }
+
+// Write a bf16 A-fragment of a [16 x 16] block (rows r0.., cols c0..) into a
+// permuted staging tile of row length `cols`.
+__device__ __forceinline__ void stage_afrag(bf16* t, int cols, int r0, int c0, const uint32_t (&a)[4], int gq,
+                                            int tq) {
+    const int ra = r0 + gq, rb = ra + 8, ca = c0 + 2 * tq, cb = ca + 8;
+    *reinterpret_cast<uint32_t*>(t + swz(ra, ca, cols)) = a[0];
+    *reinterpret_cast<uint32_t*>(t + swz(rb, ca, cols)) = a[1];
+    *reinterpret_cast<uint32_t*>(t + swz(ra, cb, cols)) = a[2];
+    *reinterpret_cast<uint32_t*>(t + swz(rb, cb, cols)) = a[3];
+}
 
 // Forward chain for one (head, 64 state columns) on 4 warps of 16 columns:
-// per chunk V_new^T = U^T - S^T W^T, S^T <- gamma_C S^T + V_new^T Khat.
-// Optional outputs: V_new^T and S0^T per chunk (bf16), S_out (fp32).
+// per chunk V_new^T = U^T + S^T (-W)^T, S^T <- gamma_C S^T + V_new^T Khat.
+// Optional outputs: V_new^T and S0^T per chunk (bf16, bulk-stored from a
+// double-buffered staging area by one thread), S_out (fp32).
 template <int DV, bool BETA>
-__device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, const float* __restrict__ Gc,
-                                             const bf16* __restrict__ W, const bf16* __restrict__ Kh,
+__device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, const float* __restrict__ Gm,
+                                             const bf16* __restrict__ Wn, const bf16* __restrict__ Kh,
                                              const bf16* __restrict__ Ut, const float* __restrict__ S_in,
                                              bf16* __restrict__ Vnt, bf16* __restrict__ S0t,
                                              float* __restrict__ S_out, unsigned char* smem) {
@@ -363,6 +400,7 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
     const int vl = 16 * w;            // first state column of this warp inside the block
     const int v0 = vb * 64 + vl;      // ... and inside the head
     const size_t Tp = (size_t)s.NC * C;
+    unsigned char* outs = smem + 2 * STAGE;
 
     auto ptrs = [&](int buf, bf16*& Khs, bf16*& Ws, bf16*& Uts, float*& Gs) {
         unsigned char* p = smem + buf * STAGE;
@@ -380,9 +418,16 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
         ptrs(buf, Khs, Ws, Uts, Gs);
         const size_t row0 = (size_t)bh * Tp + (size_t)cc * C;
         load_tile<C, DK, 128>(Khs, LDK, Kh + row0 * DK, DK, C, tid);
-        if (BETA) load_tile<C, DK, 128>(Ws, LDK, W + row0 * DK, DK, C, tid);
+        if (BETA) load_tile<C, DK, 128>(Ws, LDK, Wn + row0 * DK, DK, C, tid);
         load_tile<64, C, 128>(Uts, LDC, Ut + (((size_t)bh * s.NC + cc) * DV + vb * 64) * C, C, 64, tid);
-        if (tid < 16) cp_async16(Gs + tid * 4, Gc + row0 + tid * 4, true);
+        if (tid < 16) cp_async16(Gs + tid * 4, Gm + row0 + tid * 4, true);
+    };
+    auto flush = [&](int cc) {  // one thread: bulk-store the staged outputs of chunk cc
+        unsigned char* o = outs + (cc & 1) * out_stage_bytes();
+        const size_t blk = ((size_t)bh * s.NC + cc) * DV + vb * 64;
+        if (S0t) bulk_store(S0t + blk * DK, o, 64 * DK * 2);
+        if (Vnt) bulk_store(Vnt + blk * C, o + 64 * DK * 2, 64 * C * 2);
+        bulk_commit();
     };
 
     float st[16][4];
@@ -399,20 +444,24 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
     for (int cc = 0; cc < s.NC; ++cc) {
         if (cc + 1 < s.NC) load(cc + 1, (cc + 1) & 1);
         cp_async_commit();
+        if (tid == 0 && cc > 0) {
+            flush(cc - 1);
+            bulk_wait_read<1>();  // the staging buffer of chunk cc (last used by cc-2) is free
+        }
         cp_async_wait<1>();
         __syncthreads();
         bf16 *Khs, *Ws, *Uts;
         float* Gs;
         ptrs(cc & 1, Khs, Ws, Uts, Gs);
-        const float gamC = expf(Gs[C - 1]);
-        if (S0t) {
-            bf16* dst = S0t + ((size_t)bh * s.NC + cc) * DV * DK;
+        bf16* S0s = reinterpret_cast<bf16*>(outs + (cc & 1) * out_stage_bytes());
+        bf16* Vns = S0s + 64 * DK;
+        const float gamC = Gs[C - 1];
+        uint32_t sa[8][4];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int d = 8 * j + 2 * tq;
-                *reinterpret_cast<uint32_t*>(dst + (size_t)(v0 + gq) * DK + d) = pack(st[j][0], st[j][1]);
-                *reinterpret_cast<uint32_t*>(dst + (size_t)(v0 + gq + 8) * DK + d) = pack(st[j][2], st[j][3]);
-            }
+        for (int kk = 0; kk < 8; ++kk) c2a(sa[kk], st[2 * kk], st[2 * kk + 1]);
+        if (S0t) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) stage_afrag(S0s, DK, vl, 16 * kk, sa[kk], gq, tq);
         }
         float vn[8][4];
 #pragma unroll
@@ -426,14 +475,6 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
             vn[nn][3] = u1.y;
         }
         if (BETA) {
-            uint32_t sa[8][4];
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                sa[kk][0] = pack(-st[2 * kk][0], -st[2 * kk][1]);
-                sa[kk][1] = pack(-st[2 * kk][2], -st[2 * kk][3]);
-                sa[kk][2] = pack(-st[2 * kk + 1][0], -st[2 * kk + 1][1]);
-                sa[kk][3] = pack(-st[2 * kk + 1][2], -st[2 * kk + 1][3]);
-            }
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
 #pragma unroll
@@ -444,18 +485,14 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
                     mma(vn[nn + 1], sa[kk], b[2], b[3]);
                 }
         }
-        if (Vnt) {
-            bf16* dst = Vnt + ((size_t)bh * s.NC + cc) * DV * C;
-#pragma unroll
-            for (int nn = 0; nn < 8; ++nn) {
-                const int tk = 8 * nn + 2 * tq;
-                *reinterpret_cast<uint32_t*>(dst + (v0 + gq) * C + tk) = pack(vn[nn][0], vn[nn][1]);
-                *reinterpret_cast<uint32_t*>(dst + (v0 + gq + 8) * C + tk) = pack(vn[nn][2], vn[nn][3]);
-            }
-        }
         uint32_t va[4][4];
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) c2a(va[kk], vn[2 * kk], vn[2 * kk + 1]);
+        if (Vnt) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) stage_afrag(Vns, C, vl, 16 * kk, va[kk], gq, tq);
+        }
+        if (S0t || Vnt) fence_proxy_async_smem();
 #pragma unroll
         for (int j = 0; j < 16; ++j)
 #pragma unroll
@@ -471,6 +508,10 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
             }
         __syncthreads();
     }
+    if (tid == 0) {
+        if (s.NC > 0 && (S0t || Vnt)) flush(s.NC - 1);
+        bulk_wait<0>();
+    }
     if (S_out) {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
@@ -484,12 +525,12 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
 
 // Reverse chain of the state gradient for one (head, 64 state columns):
 // per chunk, from the last, dV_new^T = dVi^T + dS^T Khat^T and
-// dS^T <- gamma_C dS^T + dO^T (scale gamma * Q) - dV_new^T W.
-// Outputs dV_new^T and dS_C^T per chunk (bf16), dS_in (fp32).
+// dS^T <- gamma_C dS^T + dO^T (scale gamma * Q) + dV_new^T (-W).
+// Outputs dV_new^T and dS_C^T per chunk (bf16, staged and bulk-stored), dS_in (fp32).
 template <int DV, bool BETA>
 __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, const bf16* __restrict__ q,
-                                             const bf16* __restrict__ dO, const float* __restrict__ Gc,
-                                             const bf16* __restrict__ W, const bf16* __restrict__ Kh,
+                                             const bf16* __restrict__ dO, const float* __restrict__ Gm,
+                                             const bf16* __restrict__ Wn, const bf16* __restrict__ Kh,
                                              const bf16* __restrict__ dVit, const float* __restrict__ dS_out,
                                              bf16* __restrict__ dVnt, bf16* __restrict__ dSCt,
                                              float* __restrict__ dS_in, unsigned char* smem) {
@@ -498,6 +539,7 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
     const int vl = 16 * w;
     const int v0 = vb * 64 + vl;
     const size_t Tp = (size_t)s.NC * C;
+    unsigned char* outs = smem + 2 * STAGE;
 
     auto ptrs = [&](int buf, bf16*& Khs, bf16*& Qs, bf16*& Ws, bf16*& dOs, bf16*& dVis, float*& Gs) {
         unsigned char* p = smem + buf * STAGE;
@@ -521,10 +563,17 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
         const int nval = min(C, s.T - cc * C);
         load_tile<C, DK, 128>(Khs, LDK, Kh + row0 * DK, DK, C, tid);
         load_tile<C, DK, 128>(Qs, LDK, q + bh * s.hs_k + (size_t)cc * C * DK, DK, nval, tid);
-        if (BETA) load_tile<C, DK, 128>(Ws, LDK, W + row0 * DK, DK, C, tid);
+        if (BETA) load_tile<C, DK, 128>(Ws, LDK, Wn + row0 * DK, DK, C, tid);
         load_tile<C, 64, 128>(dOs, LDC, dO + bh * s.hs_v + (size_t)cc * C * DV + vb * 64, DV, nval, tid);
         load_tile<64, C, 128>(dVis, LDC, dVit + (((size_t)bh * s.NC + cc) * DV + vb * 64) * C, C, 64, tid);
-        if (tid < 16) cp_async16(Gs + tid * 4, Gc + row0 + tid * 4, true);
+        if (tid < 16) cp_async16(Gs + tid * 4, Gm + row0 + tid * 4, true);
+    };
+    auto flush = [&](int cc) {
+        unsigned char* o = outs + (cc & 1) * out_stage_bytes();
+        const size_t blk = ((size_t)bh * s.NC + cc) * DV + vb * 64;
+        if (dSCt) bulk_store(dSCt + blk * DK, o, 64 * DK * 2);
+        if (dVnt) bulk_store(dVnt + blk * C, o + 64 * DK * 2, 64 * C * 2);
+        bulk_commit();
     };
 
     float ds[16][4];
@@ -541,20 +590,24 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
     for (int cc = s.NC - 1; cc >= 0; --cc) {
         if (cc > 0) load(cc - 1, (cc - 1) & 1);
         cp_async_commit();
+        if (tid == 0 && cc < s.NC - 1) {
+            flush(cc + 1);
+            bulk_wait_read<1>();
+        }
         cp_async_wait<1>();
         __syncthreads();
         bf16 *Khs, *Qs, *Ws, *dOs, *dVis;
         float* Gs;
         ptrs(cc & 1, Khs, Qs, Ws, dOs, dVis, Gs);
-        const float gamC = expf(Gs[C - 1]);
-        if (dSCt) {
-            bf16* dst = dSCt + ((size_t)bh * s.NC + cc) * DV * DK;
+        bf16* dSs = reinterpret_cast<bf16*>(outs + (cc & 1) * out_stage_bytes());
+        bf16* dVns = dSs + 64 * DK;
+        const float gamC = Gs[C - 1];
+        uint32_t da[8][4];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int d = 8 * j + 2 * tq;
-                *reinterpret_cast<uint32_t*>(dst + (size_t)(v0 + gq) * DK + d) = pack(ds[j][0], ds[j][1]);
-                *reinterpret_cast<uint32_t*>(dst + (size_t)(v0 + gq + 8) * DK + d) = pack(ds[j][2], ds[j][3]);
-            }
+        for (int kk = 0; kk < 8; ++kk) c2a(da[kk], ds[2 * kk], ds[2 * kk + 1]);
+        if (dSCt) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) stage_afrag(dSs, DK, vl, 16 * kk, da[kk], gq, tq);
         }
         float dvn[8][4];
 #pragma unroll
@@ -567,29 +620,23 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
             dvn[nn][2] = u1.x;
             dvn[nn][3] = u1.y;
         }
-        {
-            uint32_t da[8][4];
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) c2a(da[kk], ds[2 * kk], ds[2 * kk + 1]);
+        for (int kk = 0; kk < 8; ++kk)
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-#pragma unroll
-                for (int nn = 0; nn < 8; nn += 2) {
-                    uint32_t b[4];
-                    ldBnk(b, Khs, LDK, 8 * nn, 16 * kk, lane);
-                    mma(dvn[nn], da[kk], b[0], b[1]);
-                    mma(dvn[nn + 1], da[kk], b[2], b[3]);
-                }
-        }
-        if (dVnt) {
-            bf16* dst = dVnt + ((size_t)bh * s.NC + cc) * DV * C;
-#pragma unroll
-            for (int nn = 0; nn < 8; ++nn) {
-                const int tk = 8 * nn + 2 * tq;
-                *reinterpret_cast<uint32_t*>(dst + (v0 + gq) * C + tk) = pack(dvn[nn][0], dvn[nn][1]);
-                *reinterpret_cast<uint32_t*>(dst + (v0 + gq + 8) * C + tk) = pack(dvn[nn][2], dvn[nn][3]);
+            for (int nn = 0; nn < 8; nn += 2) {
+                uint32_t b[4];
+                ldBnk(b, Khs, LDK, 8 * nn, 16 * kk, lane);
+                mma(dvn[nn], da[kk], b[0], b[1]);
+                mma(dvn[nn + 1], da[kk], b[2], b[3]);
             }
+        uint32_t va[4][4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) c2a(va[kk], dvn[2 * kk], dvn[2 * kk + 1]);
+        if (dVnt) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) stage_afrag(dVns, C, vl, 16 * kk, va[kk], gq, tq);
         }
+        if (dSCt || dVnt) fence_proxy_async_smem();
 #pragma unroll
         for (int j = 0; j < 16; ++j)
 #pragma unroll
@@ -599,8 +646,8 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
             uint32_t a[4];
             ldAt(a, dOs, LDC, vl, 16 * kk, lane);
             const int tk = 16 * kk + 2 * tq;
-            const float g0 = s.scale * expf(Gs[tk]), g1 = s.scale * expf(Gs[tk + 1]);
-            const float g2 = s.scale * expf(Gs[tk + 8]), g3 = s.scale * expf(Gs[tk + 9]);
+            const float g0 = s.scale * Gs[tk], g1 = s.scale * Gs[tk + 1];
+            const float g2 = s.scale * Gs[tk + 8], g3 = s.scale * Gs[tk + 9];
             a[0] = scale2(a[0], g0, g1);
             a[1] = scale2(a[1], g0, g1);
             a[2] = scale2(a[2], g2, g3);
@@ -614,25 +661,21 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
             }
         }
         if (BETA) {
-            uint32_t na[4][4];
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                na[kk][0] = pack(-dvn[2 * kk][0], -dvn[2 * kk][1]);
-                na[kk][1] = pack(-dvn[2 * kk][2], -dvn[2 * kk][3]);
-                na[kk][2] = pack(-dvn[2 * kk + 1][0], -dvn[2 * kk + 1][1]);
-                na[kk][3] = pack(-dvn[2 * kk + 1][2], -dvn[2 * kk + 1][3]);
-            }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
                 for (int nn = 0; nn < 16; nn += 2) {
                     uint32_t b[4];
                     ldBkn(b, Ws, LDK, 8 * nn, 16 * kk, lane);
-                    mma(ds[nn], na[kk], b[0], b[1]);
-                    mma(ds[nn + 1], na[kk], b[2], b[3]);
+                    mma(ds[nn], va[kk], b[0], b[1]);
+                    mma(ds[nn + 1], va[kk], b[2], b[3]);
                 }
         }
         __syncthreads();
+    }
+    if (tid == 0) {
+        if (s.NC > 0 && (dSCt || dVnt)) flush(0);
+        bulk_wait<0>();
     }
     if (dS_in) {
 #pragma unroll
@@ -647,13 +690,13 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
 
 template <int DV, bool BETA>
 __global__ void __launch_bounds__(128, 1)
-tc_scan_fwd_kernel(SeqView s, const float* __restrict__ Gc, const bf16* __restrict__ W,
+tc_scan_fwd_kernel(SeqView s, const float* __restrict__ Gm, const bf16* __restrict__ Wn,
                    const bf16* __restrict__ Kh, const bf16* __restrict__ Ut,
                    const float* __restrict__ S_in, bf16* __restrict__ Vnt, bf16* __restrict__ S0t,
                    float* __restrict__ S_out) {
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int NVB = DV / 64;
-    scan_fwd_cta<DV, BETA>(s, blockIdx.x / NVB, blockIdx.x % NVB, Gc, W, Kh, Ut, S_in, Vnt, S0t, S_out, smem);
+    scan_fwd_cta<DV, BETA>(s, blockIdx.x / NVB, blockIdx.x % NVB, Gm, Wn, Kh, Ut, S_in, Vnt, S0t, S_out, smem);
 }
 
 // Backward chains in one launch: blocks [0, BH*DV/64) recompute the forward
@@ -662,7 +705,7 @@ tc_scan_fwd_kernel(SeqView s, const float* __restrict__ Gc, const bf16* __restri
 template <int DV, bool BETA>
 __global__ void __launch_bounds__(128, 1)
 tc_scan_bwd_dual_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ dO,
-                        const float* __restrict__ Gc, const bf16* __restrict__ W,
+                        const float* __restrict__ Gm, const bf16* __restrict__ Wn,
                         const bf16* __restrict__ Kh, const bf16* __restrict__ Ut,
                         const bf16* __restrict__ dVit, const float* __restrict__ S_in,
                         const float* __restrict__ dS_out, bf16* __restrict__ Vnt, bf16* __restrict__ S0t,
@@ -672,10 +715,10 @@ tc_scan_bwd_dual_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __res
     const int nsr = s.BH * NVB;
     int id = blockIdx.x;
     if (id < nsr) {
-        scan_fwd_cta<DV, BETA>(s, id / NVB, id % NVB, Gc, W, Kh, Ut, S_in, Vnt, S0t, nullptr, smem);
+        scan_fwd_cta<DV, BETA>(s, id / NVB, id % NVB, Gm, Wn, Kh, Ut, S_in, Vnt, S0t, nullptr, smem);
     } else {
         id -= nsr;
-        scan_bwd_cta<DV, BETA>(s, id / NVB, id % NVB, q, dO, Gc, W, Kh, dVit, dS_out, dVnt, dSCt, dS_in, smem);
+        scan_bwd_cta<DV, BETA>(s, id / NVB, id % NVB, q, dO, Gm, Wn, Kh, dVit, dS_out, dVnt, dSCt, dS_in, smem);
     }
 }
 
@@ -704,8 +747,8 @@ tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
     const size_t Tp = (size_t)s.NC * C;
     load_tile<C, DK, 128>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
     load_tile<C, DK, 128>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
-    load_tile<DV, DK, 128>(S0s, LDK, S0t + ((size_t)bh * s.NC + c) * DV * DK, DK, DV, tid);
-    load_tile<DV, C, 128>(Vns, LDC, Vnt + ((size_t)bh * s.NC + c) * DV * C, C, DV, tid);
+    load_tile_swz<DV, DK, 128>(S0s, LDK, S0t + ((size_t)bh * s.NC + c) * DV * DK, tid);
+    load_tile_swz<DV, C, 128>(Vns, LDC, Vnt + ((size_t)bh * s.NC + c) * DV * C, tid);
     if (tid < 16) cp_async16(Gs + tid * 4, Gc + bh * Tp + t0 + tid * 4, true);
     cp_async_commit();
     cp_async_wait<0>();
@@ -844,10 +887,10 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     load_tile<C, DK, 256>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
     load_tile<C, DV, 256>(Vs, LDV, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
     load_tile<C, DV, 256>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
-    load_tile<DV, C, 256>(Vns, LDC, Vnt + ci * DV * C, C, DV, tid);
-    load_tile<DV, C, 256>(dVns, LDC, dVnt + ci * DV * C, C, DV, tid);
-    load_tile<DV, DK, 256>(S0s, LDK, S0t + ci * DV * DK, DK, DV, tid);
-    load_tile<DV, DK, 256>(dSs, LDK, dSCt + ci * DV * DK, DK, DV, tid);
+    load_tile_swz<DV, C, 256>(Vns, LDC, Vnt + ci * DV * C, tid);
+    load_tile_swz<DV, C, 256>(dVns, LDC, dVnt + ci * DV * C, tid);
+    load_tile_swz<DV, DK, 256>(S0s, LDK, S0t + ci * DV * DK, tid);
+    load_tile_swz<DV, DK, 256>(dSs, LDK, dSCt + ci * DV * DK, tid);
     if (tid < 16) cp_async16(Gs + tid * 4, Gc + bh * Tp + t0 + tid * 4, true);
     cp_async_commit();
     for (int i = tid; i < C; i += 256) Bs[i] = (BETA && i < nval) ? beta[bh * s.hs_g + t0 + i] : 0.f;
@@ -1329,17 +1372,17 @@ cudaError_t fwd_impl(const SeqView& s, const FwdArgs& a, void* ws, cudaStream_t 
     const bf16* k = static_cast<const bf16*>(a.k);
     const bf16* v = static_cast<const bf16*>(a.v);
     constexpr size_t sm_prep = prep_smem<DV, false>();
-    constexpr size_t sm_scan = 2 * fwd_stage_bytes<BETA>();
+    constexpr size_t sm_scan = fwd_scan_smem<BETA>();
     constexpr size_t sm_out = out_smem<DV>();
     TC_TRY(smem_attr(tc_prep_kernel<DV, BETA, false>, sm_prep));
     TC_TRY(smem_attr(tc_scan_fwd_kernel<DV, BETA>, sm_scan));
     TC_TRY(smem_attr(tc_out_kernel<DV>, sm_out));
     const dim3 gc(s.NC, s.BH);
     SF_LAUNCH("tc_prep", st, tc_prep_kernel<DV, BETA, false><<<gc, 128, sm_prep, st>>>(
-                                 s, q, k, v, a.g, a.beta, nullptr, w.Gc, w.W, w.Kh, w.Ut, nullptr));
+                                 s, q, k, v, a.g, a.beta, nullptr, w.Gc, w.Gm, w.W, w.Kh, w.Ut, nullptr));
     TC_TRY(cudaGetLastError());
     SF_LAUNCH("tc_scan_fwd", st, tc_scan_fwd_kernel<DV, BETA><<<s.BH * (DV / 64), 128, sm_scan, st>>>(
-                                     s, w.Gc, w.W, w.Kh, w.Ut, a.S_in, w.Vnt, w.S0t, a.S_out));
+                                     s, w.Gm, w.W, w.Kh, w.Ut, a.S_in, w.Vnt, w.S0t, a.S_out));
     TC_TRY(cudaGetLastError());
     SF_LAUNCH("tc_out", st, tc_out_kernel<DV><<<gc, 128, sm_out, st>>>(s, q, k, w.Gc, w.Vnt, w.S0t,
                                                                          static_cast<bf16*>(a.o)));
@@ -1355,7 +1398,7 @@ cudaError_t bwd_impl(const SeqView& s, const BwdArgs& a, void* ws, cudaStream_t 
     const bf16* v = static_cast<const bf16*>(a.v);
     const bf16* dO = static_cast<const bf16*>(a.dO);
     constexpr size_t sm_prep = prep_smem<DV, true>();
-    constexpr size_t sm_f = 2 * fwd_stage_bytes<BETA>(), sm_b = 2 * bwd_stage_bytes<BETA>();
+    constexpr size_t sm_f = fwd_scan_smem<BETA>(), sm_b = bwd_scan_smem<BETA>();
     constexpr size_t sm_scan = sm_f > sm_b ? sm_f : sm_b;
     constexpr size_t sm_grad = grad_smem<DV>();
     TC_TRY(smem_attr(tc_prep_kernel<DV, BETA, true>, sm_prep));
@@ -1363,10 +1406,10 @@ cudaError_t bwd_impl(const SeqView& s, const BwdArgs& a, void* ws, cudaStream_t 
     TC_TRY(smem_attr(tc_grad_kernel<DV, BETA>, sm_grad));
     const dim3 gc(s.NC, s.BH);
     SF_LAUNCH("tc_prep_bwd", st, tc_prep_kernel<DV, BETA, true><<<gc, 128, sm_prep, st>>>(
-                                     s, q, k, v, a.g, a.beta, dO, w.Gc, w.W, w.Kh, w.Ut, w.dVit));
+                                     s, q, k, v, a.g, a.beta, dO, w.Gc, w.Gm, w.W, w.Kh, w.Ut, w.dVit));
     TC_TRY(cudaGetLastError());
     SF_LAUNCH("tc_scan_bwd", st, tc_scan_bwd_dual_kernel<DV, BETA><<<2 * s.BH * (DV / 64), 128, sm_scan, st>>>(
-                                     s, q, dO, w.Gc, w.W, w.Kh, w.Ut, w.dVit, a.S_in, a.dS_out, w.Vnt, w.S0t,
+                                     s, q, dO, w.Gm, w.W, w.Kh, w.Ut, w.dVit, a.S_in, a.dS_out, w.Vnt, w.S0t,
                                      w.dVnt, w.dSCt, a.dS_in));
     TC_TRY(cudaGetLastError());
     SF_LAUNCH("tc_grad", st, tc_grad_kernel<DV, BETA><<<gc, 256, sm_grad, st>>>(

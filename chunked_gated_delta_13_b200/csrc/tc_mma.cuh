@@ -97,6 +97,36 @@ __device__ __forceinline__ void c2a(uint32_t (&a)[4], const float (&c0)[4], cons
     a[3] = pack(c1[2], c1[3]);
 }
 
+// Bulk asynchronous shared -> global copy (one thread issues it; 16-byte
+// aligned addresses, size a multiple of 16), its group commit and waits.
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(gdst),
+                 "r"(smem_u32(ssrc)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;\n" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+    asm volatile("cp.async.bulk.wait_group %0;\n" ::"n"(N) : "memory");
+}
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+// Tiles written by the state scans are stored with the 16-byte pieces of every
+// row permuted, piece p of row r at position p ^ (r & 7), so that the scan can
+// stage them in shared memory without bank conflicts and write them out with
+// one linear bulk copy.  Element offset of (r, col) in such a tile of row
+// length `cols` (a multiple of 64):
+__device__ __forceinline__ int swz(int r, int col, int cols) {
+    return r * cols + ((((col >> 3) ^ (r & 7))) << 3) + (col & 7);
+}
+
 // Copy a [rows][cols] bf16 global tile (row stride gld elements) into shared
 // memory (row stride sld), 16 bytes per request, rows >= nrows zero-filled.
 template <int ROWS, int COLS, int NT>
@@ -107,6 +137,16 @@ __device__ __forceinline__ void load_tile(__nv_bfloat16* s, int sld, const __nv_
         const int r = e / CPR, c = (e % CPR) * 8;
         const bool ok = r < nrows;
         cp_async16(s + r * sld + c, g + (ok ? (long long)r * gld : 0) + c, ok);
+    }
+}
+
+// As load_tile, for a global tile stored with the piece permutation of swz().
+template <int ROWS, int COLS, int NT>
+__device__ __forceinline__ void load_tile_swz(__nv_bfloat16* s, int sld, const __nv_bfloat16* g, int tid) {
+    constexpr int CPR = COLS / 8;
+    for (int e = tid; e < ROWS * CPR; e += NT) {
+        const int r = e / CPR, c = e % CPR;
+        cp_async16(s + r * sld + c * 8, g + (long long)r * COLS + ((c ^ (r & 7)) << 3), true);
     }
 }
 
