@@ -34,7 +34,7 @@ STATUS_NAMES = ["SF_OK", "SF_ERR_INVALID_ARG", "SF_ERR_UNSUPPORTED", "SF_ERR_ALI
 EXPORTED_SYMBOLS = [
     "sf_status_str", "sf_last_cuda_error", "sf_gdn_fwd_workspace_bytes",
     "sf_gdn_bwd_workspace_bytes", "sf_gdn_fwd", "sf_gdn_bwd", "sf_segment_workspace_bytes",
-    "sf_segment_run", "sf_gdn_path", "sf_gdn_launches", "sf_set_launch_hook",
+    "sf_segment_run", "sf_gdn_path", "sf_gdn_launches", "sf_set_launch_hook", "sf_gdn_fwd_noalloc",
 ]
 
 HOOK_T = ctypes.CFUNCTYPE(None, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p)
@@ -95,6 +95,8 @@ def lib():
         L.sf_gdn_path.restype = ctypes.c_char_p
         L.sf_gdn_launches.argtypes = [SP, ctypes.c_int]
         L.sf_gdn_launches.restype = ctypes.c_int
+        L.sf_gdn_fwd_noalloc.argtypes = [SP] + [P] * 8 + [P]
+        L.sf_gdn_fwd_noalloc.restype = ctypes.c_int
         L.sf_set_launch_hook.argtypes = [HOOK_T, ctypes.c_void_p]
         L.sf_set_launch_hook.restype = None
         _lib = L

@@ -129,6 +129,24 @@ sf_status sf_segment_run(const sf_gdn_shape* full, int N, const int* seg_len, co
                          float* S_out, void* dq, void* dk, void* dv, float* dg, float* dbeta,
                          float* dS_in, void* ws, size_t ws_bytes, void* stream);
 
+/* Forward of one segment for callers that cannot allocate device memory (an
+ * engine or plugin whose memory is planned up front and gives no allocation
+ * hook, or code that must not call cudaMalloc on its hot path).  The paper has
+ * no counterpart: this is a packaging of sf_gdn_fwd, which it runs unchanged,
+ * with the workspace taken from a fixed array of SF_NOALLOC_SCRATCH_BYTES that
+ * the library keeps in each GPU's memory for the life of the process.
+ *   - Shapes whose forward workspace (sf_gdn_fwd_workspace_bytes) exceeds the
+ *     array return SF_ERR_WORKSPACE before anything is enqueued.
+ *   - All calls share the array: calls whose work overlaps on the GPU race on
+ *     it, so issue them on one stream or order them with events.
+ *   - The first call on a device looks up the array's address with that device
+ *     current; make it outside any stream capture.
+ * Other arguments, errors and results are those of sf_gdn_fwd. */
+#define SF_NOALLOC_SCRATCH_BYTES (32u << 20)
+sf_status sf_gdn_fwd_noalloc(const sf_gdn_shape* shape, const void* q, const void* k, const void* v,
+                             const float* g, const float* beta, const float* S_in, void* o,
+                             float* S_out, void* stream);
+
 /* Optional launch observer, for profiling.  When set, every kernel this
  * library launches is bracketed by hook(name, 0, stream, user) just before the
  * launch and hook(name, 1, stream, user) just after it, on the calling thread,
