@@ -22,7 +22,7 @@ import threading
 
 from ._build import LIB, build, needs_build
 
-__all__ = ["Shape", "SFError", "lib", "fwd", "bwd", "segment_run", "make_shape", "path",
+__all__ = ["Shape", "SFError", "lib", "fwd", "bwd", "segment_run", "make_shape", "path", "device_check",
            "launches", "set_launch_hook", "fwd_workspace_bytes", "bwd_workspace_bytes", "segment_workspace_bytes",
            "EXPORTED_SYMBOLS"]
 
@@ -35,6 +35,7 @@ EXPORTED_SYMBOLS = [
     "sf_status_str", "sf_last_cuda_error", "sf_gdn_fwd_workspace_bytes",
     "sf_gdn_bwd_workspace_bytes", "sf_gdn_fwd", "sf_gdn_bwd", "sf_segment_workspace_bytes",
     "sf_segment_run", "sf_gdn_path", "sf_gdn_launches", "sf_set_launch_hook", "sf_gdn_fwd_noalloc",
+    "sf_device_check",
 ]
 
 HOOK_T = ctypes.CFUNCTYPE(None, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p)
@@ -95,6 +96,8 @@ def lib():
         L.sf_gdn_path.restype = ctypes.c_char_p
         L.sf_gdn_launches.argtypes = [SP, ctypes.c_int]
         L.sf_gdn_launches.restype = ctypes.c_int
+        L.sf_device_check.argtypes = []
+        L.sf_device_check.restype = ctypes.c_int
         L.sf_gdn_fwd_noalloc.argtypes = [SP] + [P] * 8 + [P]
         L.sf_gdn_fwd_noalloc.restype = ctypes.c_int
         L.sf_set_launch_hook.argtypes = [HOOK_T, ctypes.c_void_p]
@@ -106,6 +109,12 @@ def lib():
 def _check(status: int):
     if status != 0:
         raise SFError(status, lib().sf_last_cuda_error().decode() if status == 5 else "")
+
+
+def device_check():
+    """Synchronise and raise SFError(SF_ERR_TIMEOUT) if a kernel gave up one of its
+    bounded waits since the last check."""
+    _check(lib().sf_device_check())
 
 
 def make_shape(B, H, T, dk, dv, C=64, io="bf16", use_beta=True, scale=1.0) -> Shape:

@@ -344,6 +344,13 @@ sf_status sf_segment_run(const sf_gdn_shape* s, int N, const int* seg_len, const
     return SF_OK;
 }
 
+sf_status sf_device_check(void) {
+    int status = 0;
+    cudaError_t e = sf::tc_device_status(&status, true);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return status ? SF_ERR_TIMEOUT : SF_OK;
+}
+
 const char* sf_gdn_path(const sf_gdn_shape* s) {
     if (check_shape(s) != SF_OK) return nullptr;
     return pick_path(*s) == Path::Tc ? "tc" : "simt";

@@ -34,15 +34,19 @@ constexpr int LDK = DK + 8;  // shared row stride of [*][DK] tiles
 constexpr int LDC = C + 8;   // shared row stride of [*][C] tiles
 constexpr int LDF = 72;      // shared row stride of fp32 [C][C] tiles
 
+// Set (bit 0) by a kernel that gave up waiting for one of its own bulk copies;
+// read and cleared by sf_device_check().
+__device__ int g_tc_status = 0;
+
 struct TcWs {
     float* Gc;   // [BH][Tp]           chunk-local cumulative log-decay G
     float* Gm;   // [BH][Tp]           exp(G)
-    bf16* W;     // [BH][Tp][DK]       -W (stored negated: the scans only ever subtract W products)
-    bf16* Kh;    // [BH][Tp][DK]       K * exp(G_C - G)
-    bf16* Ut;    // [BH][NC][DV][C]    U transposed per chunk (V^T without the beta path)
+    bf16* W;     // [BH][Tp][DK]       -W (negated: the scans only ever subtract W products; permuted, see swz)
+    bf16* Kh;    // [BH][Tp][DK]       K * exp(G_C - G) (permuted)
+    bf16* Ut;    // [BH][NC][DV][C]    U transposed per chunk, V^T without the beta path (permuted)
     bf16* Vnt;   // [BH][NC][DV][C]    V_new transposed per chunk (pieces permuted, see swz)
     bf16* S0t;   // [BH][NC][DV][DK]   state entering each chunk, transposed (permuted)
-    bf16* dVit;  // [BH][NC][DV][C]    intra-chunk part of dV_new, transposed
+    bf16* dVit;  // [BH][NC][DV][C]    intra-chunk part of dV_new, transposed (permuted)
     bf16* dVnt;  // [BH][NC][DV][C]    dV_new transposed (permuted)
     bf16* dSCt;  // [BH][NC][DV][DK]   gradient of the state leaving each chunk, transposed (permuted)
     size_t total;
@@ -115,27 +119,41 @@ __device__ void block_inverse(const float* A, int la, float* L, int ll, float* Y
     __syncthreads();
 #pragma unroll 1
     for (int d = 1; d < 4; ++d) {
-        const int nb = 4 - d;
-        for (int e = tid; e < nb * 256; e += nthr) {
-            const int J = e >> 8, I = J + d, r = (e >> 4) & 15, c = e & 15;
-            float y = 0.f;
+        const int nb = 4 - d;  // blocks (I, J = I - d) of this round; one item = a row and 4 columns
+        for (int e = tid; e < nb * 64; e += nthr) {
+            const int J = e >> 6, I = J + d, r = (e >> 2) & 15, c4 = (e & 3) * 4;
+            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int m = J; m < I; ++m) {
                 const float* Ar = A + (16 * I + r) * la + 16 * m;
-                const float* Lc = L + (16 * m) * ll + 16 * J + c;
+                const float* Lc = L + (16 * m) * ll + 16 * J + c4;
 #pragma unroll
-                for (int p = 0; p < 16; ++p) y = fmaf(Ar[p], Lc[p * ll], y);
+                for (int p = 0; p < 16; ++p) {
+                    const float a = Ar[p];
+                    const float4 l = *reinterpret_cast<const float4*>(Lc + p * ll);
+                    y.x = fmaf(a, l.x, y.x);
+                    y.y = fmaf(a, l.y, y.y);
+                    y.z = fmaf(a, l.z, y.z);
+                    y.w = fmaf(a, l.w, y.w);
+                }
             }
-            Y[e] = y;
+            *reinterpret_cast<float4*>(Y + (J << 8) + r * 16 + c4) = y;
         }
         __syncthreads();
-        for (int e = tid; e < nb * 256; e += nthr) {
-            const int J = e >> 8, I = J + d, r = (e >> 4) & 15, c = e & 15;
+        for (int e = tid; e < nb * 64; e += nthr) {
+            const int J = e >> 6, I = J + d, r = (e >> 2) & 15, c4 = (e & 3) * 4;
             const float* Lr = L + (16 * I + r) * ll + 16 * I;
-            const float* Yc = Y + (J << 8) + c;
-            float x = 0.f;
+            const float* Yc = Y + (J << 8) + c4;
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int p = 0; p < 16; ++p) x = fmaf(Lr[p], Yc[p * 16], x);
-            L[(16 * I + r) * ll + 16 * J + c] = -x;
+            for (int p = 0; p < 16; ++p) {
+                const float a = Lr[p];
+                const float4 yy = *reinterpret_cast<const float4*>(Yc + p * 16);
+                x.x = fmaf(a, yy.x, x.x);
+                x.y = fmaf(a, yy.y, x.y);
+                x.z = fmaf(a, yy.z, x.z);
+                x.w = fmaf(a, yy.w, x.w);
+            }
+            *reinterpret_cast<float4*>(L + (16 * I + r) * ll + 16 * J + c4) = make_float4(-x.x, -x.y, -x.z, -x.w);
         }
         __syncthreads();
     }
@@ -192,18 +210,18 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 
     for (int i = tid; i < C; i += 128) {
         Gc[bh * Tp + t0 + i] = Gs[i];
-        Gmo[bh * Tp + t0 + i] = expf(Gs[i]);
+        Gmo[bh * Tp + t0 + i] = __expf(Gs[i]);
     }
     const float gC = Gs[C - 1];
     for (int e = tid; e < C * (DK / 8); e += 128) {
         const int r = e >> 4, cc = (e & 15) * 8;
-        const float d = expf(gC - Gs[r]);
+        const float d = __expf(gC - Gs[r]);
         uint4 x = *reinterpret_cast<const uint4*>(Ks + r * LDK + cc);
         x.x = scale2(x.x, d, d);
         x.y = scale2(x.y, d, d);
         x.z = scale2(x.z, d, d);
         x.w = scale2(x.w, d, d);
-        *reinterpret_cast<uint4*>(Kho + (bh * Tp + t0 + r) * DK + cc) = x;
+        *reinterpret_cast<uint4*>(Kho + (bh * Tp + t0) * DK + swz(r, cc, DK)) = x;
     }
 
     bf16* Ust = reinterpret_cast<bf16*>(Lf);  // [DV][LDC]
@@ -227,7 +245,7 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int i = 16 * w + gq + 8 * (e >> 1), j = 8 * nn + 2 * tq + (e & 1);
-                    Af[i * LDF + j] = (j < i) ? Bs[i] * expf(Gs[i] - Gs[j]) * acc[nn][e] : 0.f;
+                    Af[i * LDF + j] = (j < i) ? Bs[i] * __expf(Gs[i] - Gs[j]) * acc[nn][e] : 0.f;
                 }
         }
         __syncthreads();
@@ -235,7 +253,7 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         for (int e = tid; e < C * C; e += 128) {
             const int i = e >> 6, j = e & 63;
             const float l = Lf[i * LDF + j];
-            Tw[i * LDC + j] = __float2bfloat16_rn(l * Bs[j] * expf(Gs[j]));
+            Tw[i * LDC + j] = __float2bfloat16_rn(l * Bs[j] * __expf(Gs[j]));
             Tu[i * LDC + j] = __float2bfloat16_rn(l * Bs[j]);
         }
         __syncthreads();
@@ -286,7 +304,7 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         __syncthreads();
         for (int e = tid; e < C * (DK / 8); e += 128) {
             const int r = e >> 4, cc = (e & 15) * 8;
-            *reinterpret_cast<uint4*>(Wo + (bh * Tp + t0 + r) * DK + cc) =
+            *reinterpret_cast<uint4*>(Wo + (bh * Tp + t0) * DK + swz(r, cc, DK)) =
                 *reinterpret_cast<const uint4*>(Wst + r * LDK + cc);
         }
     } else {
@@ -299,7 +317,7 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     bf16* Utg = Uto + ((size_t)bh * s.NC + c) * DV * C;
     for (int e = tid; e < DV * (C / 8); e += 128) {
         const int r = e >> 3, cc = (e & 7) * 8;
-        *reinterpret_cast<uint4*>(Utg + r * C + cc) = *reinterpret_cast<const uint4*>(Ust + r * LDC + cc);
+        *reinterpret_cast<uint4*>(Utg + swz(r, cc, C)) = *reinterpret_cast<const uint4*>(Ust + r * LDC + cc);
     }
 
     if (BWD) {
@@ -323,7 +341,7 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int i = 16 * w + gq + 8 * (e >> 1), j = 8 * nn + 2 * tq + (e & 1);
-                    const float p = (j <= i) ? s.scale * expf(Gs[i] - Gs[j]) * acc[nn][e] : 0.f;
+                    const float p = (j <= i) ? s.scale * __expf(Gs[i] - Gs[j]) * acc[nn][e] : 0.f;
                     Ps[i * LDC + j] = __float2bfloat16_rn(p);
                 }
         }
@@ -350,39 +368,64 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 #pragma unroll
             for (int nn = 0; nn < 8; ++nn) {
                 const int r = m0 + gq, j = 8 * nn + 2 * tq;
-                *reinterpret_cast<uint32_t*>(dst + r * C + j) = pack(acc[nn][0], acc[nn][1]);
-                *reinterpret_cast<uint32_t*>(dst + (r + 8) * C + j) = pack(acc[nn][2], acc[nn][3]);
+                *reinterpret_cast<uint32_t*>(dst + swz(r, j, C)) = pack(acc[nn][0], acc[nn][1]);
+                *reinterpret_cast<uint32_t*>(dst + swz(r + 8, j, C)) = pack(acc[nn][2], acc[nn][3]);
             }
         }
     }
 }
 
 // ------------------------------------------------------------ state scans ---
+// Operand stages of the chains are filled by one thread with bulk copies that
+// complete on an mbarrier per stage; tiles produced by the prep kernel are
+// stored permuted (swz), so the linear copies land bank-conflict-free.
+constexpr uint32_t kTileK = C * DK * 2;   // a [C][DK] bf16 tile
+constexpr uint32_t kTileV = 64 * C * 2;   // 64 rows of a [DV][C] bf16 tile
 template <bool BETA>
 constexpr size_t fwd_stage_bytes() {
-    return (size_t)C * LDK * 2 * (BETA ? 2 : 1) + (size_t)64 * LDC * 2 + C * 4;
+    return (size_t)kTileK * (BETA ? 2 : 1) + kTileV + C * 4;
 }
 template <bool BETA>
-constexpr size_t bwd_stage_bytes() {
-    return (size_t)C * LDK * 2 * (BETA ? 3 : 2) + (size_t)C * LDC * 2 * 2 + C * 4;
+constexpr size_t bwd_stage_bytes() {  // + Q and dO tiles copied per thread (padded rows)
+    return (size_t)kTileK * (BETA ? 2 : 1) + kTileV + C * 4 + (size_t)C * LDK * 2 + (size_t)C * LDC * 2;
 }
 // Output staging of one chunk step of a 64-column block: the state tile
 // (64 x DK) and the value tile (64 x C), in the permuted layout of swz().
 constexpr size_t out_stage_bytes() { return (size_t)64 * DK * 2 + (size_t)64 * C * 2; }
+constexpr int kOutBufs = 3;  // staged outputs of chunk c are flushed during step c+1 and must be read by step c+3
 template <bool BETA>
-constexpr size_t fwd_scan_smem() { return 2 * fwd_stage_bytes<BETA>() + 2 * out_stage_bytes(); }
+constexpr size_t fwd_scan_smem() { return 2 * fwd_stage_bytes<BETA>() + kOutBufs * out_stage_bytes() + 16; }
 template <bool BETA>
-constexpr size_t bwd_scan_smem() { return 2 * bwd_stage_bytes<BETA>() + 2 * out_stage_bytes(); }
+constexpr size_t bwd_scan_smem() { return 2 * bwd_stage_bytes<BETA>() + kOutBufs * out_stage_bytes() + 16; }
 
-// Write a bf16 A-fragment of a [16 x 16] block (rows r0.., cols c0..) into a
-// permuted staging tile of row length `cols`.
-__device__ __forceinline__ void stage_afrag(bf16* t, int cols, int r0, int c0, const uint32_t (&a)[4], int gq,
-                                            int tq) {
-    const int ra = r0 + gq, rb = ra + 8, ca = c0 + 2 * tq, cb = ca + 8;
-    *reinterpret_cast<uint32_t*>(t + swz(ra, ca, cols)) = a[0];
-    *reinterpret_cast<uint32_t*>(t + swz(rb, ca, cols)) = a[1];
-    *reinterpret_cast<uint32_t*>(t + swz(ra, cb, cols)) = a[2];
-    *reinterpret_cast<uint32_t*>(t + swz(rb, cb, cols)) = a[3];
+// Per-lane parts of the addresses into permuted [rows][128] tiles.
+//   B fragments (stored [n][k], k = 16kk..): row = n0 + lr, piece 2kk + pb
+//   B fragments (stored [k][n], trans):      row = k0 + lr, piece nn + pb (nn even)
+// with lr, pb the lane's row/piece offsets; the piece is XOR-ed with lr & 7.
+struct SwLane {
+    int row;   // lane row offset inside a 16-row group (times the row length is added by callers)
+    int lo;    // (pb ^ (lr & 1)) * 8   element offset of the low bit of the permuted piece
+    int hi8;   // (lr & 6) * 8          XOR mask for the even part of the piece
+};
+__device__ __forceinline__ SwLane sw_lane_nk(int lane) {  // ldmatrix non-trans, row = n, piece from k
+    const int lr = (lane & 7) + ((lane >> 4) << 3), pb = (lane >> 3) & 1;
+    return {lr, (pb ^ (lr & 1)) * 8, (lr & 6) * 8};
+}
+__device__ __forceinline__ SwLane sw_lane_kn(int lane) {  // ldmatrix trans, row = k, piece from n
+    const int lr = (lane & 7) + (((lane >> 3) & 1) << 3), pb = lane >> 4;
+    return {lr, (pb ^ (lr & 1)) * 8, (lr & 6) * 8};
+}
+// Element offset of the fragment row/piece for an even logical piece `pe`.
+__device__ __forceinline__ int sw_off(const SwLane& L, int rowbase, int pe, int rowlen) {
+    return (rowbase + L.row) * rowlen + ((pe * 8) ^ L.hi8) + L.lo;
+}
+
+// Write a bf16 A-fragment block (16 rows x 16 cols at [r0, c0]) into a permuted
+// staging tile of row length `cols` with one stmatrix.
+__device__ __forceinline__ void stage_afrag(bf16* t, int cols, int r0, int c0, const uint32_t (&a)[4], int lane) {
+    const int lr = (lane & 7) + (((lane >> 3) & 1) << 3), pb = lane >> 4;
+    const int piece = ((c0 >> 3) + pb) ^ (lr & 7);
+    stsm_x4(t + (r0 + lr) * cols + piece * 8, a);
 }
 
 // Forward chain for one (head, 64 state columns) on 4 warps of 16 columns:
@@ -396,34 +439,39 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
                                              bf16* __restrict__ Vnt, bf16* __restrict__ S0t,
                                              float* __restrict__ S_out, unsigned char* smem) {
     constexpr size_t STAGE = fwd_stage_bytes<BETA>();
+    constexpr uint32_t TX = (BETA ? 2 : 1) * kTileK + kTileV + C * 4;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, gq = lane >> 2, tq = lane & 3;
     const int vl = 16 * w;            // first state column of this warp inside the block
     const int v0 = vb * 64 + vl;      // ... and inside the head
     const size_t Tp = (size_t)s.NC * C;
     unsigned char* outs = smem + 2 * STAGE;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(outs + kOutBufs * out_stage_bytes());
+    bool failed = false;
 
-    auto ptrs = [&](int buf, bf16*& Khs, bf16*& Ws, bf16*& Uts, float*& Gs) {
+    auto stage = [&](int buf, bf16*& Khs, bf16*& Ws, bf16*& Uts, float*& Gs) {
         unsigned char* p = smem + buf * STAGE;
         Khs = reinterpret_cast<bf16*>(p);
-        p += C * LDK * 2;
+        p += kTileK;
         Ws = reinterpret_cast<bf16*>(p);
-        if (BETA) p += C * LDK * 2;
+        if (BETA) p += kTileK;
         Uts = reinterpret_cast<bf16*>(p);
-        p += 64 * LDC * 2;
+        p += kTileV;
         Gs = reinterpret_cast<float*>(p);
     };
-    auto load = [&](int cc, int buf) {
+    auto load = [&](int cc) {  // thread 0 only
         bf16 *Khs, *Ws, *Uts;
         float* Gs;
-        ptrs(buf, Khs, Ws, Uts, Gs);
+        const int buf = cc & 1;
+        stage(buf, Khs, Ws, Uts, Gs);
         const size_t row0 = (size_t)bh * Tp + (size_t)cc * C;
-        load_tile<C, DK, 128>(Khs, LDK, Kh + row0 * DK, DK, C, tid);
-        if (BETA) load_tile<C, DK, 128>(Ws, LDK, Wn + row0 * DK, DK, C, tid);
-        load_tile<64, C, 128>(Uts, LDC, Ut + (((size_t)bh * s.NC + cc) * DV + vb * 64) * C, C, 64, tid);
-        if (tid < 16) cp_async16(Gs + tid * 4, Gm + row0 + tid * 4, true);
+        mbar_expect_tx(&bars[buf], TX);
+        bulk_load(Khs, Kh + row0 * DK, kTileK, &bars[buf]);
+        if (BETA) bulk_load(Ws, Wn + row0 * DK, kTileK, &bars[buf]);
+        bulk_load(Uts, Ut + (((size_t)bh * s.NC + cc) * DV + vb * 64) * C, kTileV, &bars[buf]);
+        bulk_load(Gs, Gm + row0, C * 4, &bars[buf]);
     };
-    auto flush = [&](int cc) {  // one thread: bulk-store the staged outputs of chunk cc
-        unsigned char* o = outs + (cc & 1) * out_stage_bytes();
+    auto flush = [&](int cc) {  // thread 0 only: bulk-store the staged outputs of chunk cc
+        unsigned char* o = outs + (cc % kOutBufs) * out_stage_bytes();
         const size_t blk = ((size_t)bh * s.NC + cc) * DV + vb * 64;
         if (S0t) bulk_store(S0t + blk * DK, o, 64 * DK * 2);
         if (Vnt) bulk_store(Vnt + blk * C, o + 64 * DK * 2, 64 * C * 2);
@@ -438,37 +486,37 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
             const int vv = v0 + gq + 8 * (e >> 1), d = 8 * j + 2 * tq + (e & 1);
             st[j][e] = S_in ? S_in[((size_t)bh * DK + d) * DV + vv] : 0.f;
         }
+    const SwLane Lnk = sw_lane_nk(lane), Lkn = sw_lane_kn(lane);
+    const bool outputs = S0t || Vnt;
 
-    load(0, 0);
-    cp_async_commit();
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    if (tid == 0) load(0);
     for (int cc = 0; cc < s.NC; ++cc) {
-        if (cc + 1 < s.NC) load(cc + 1, (cc + 1) & 1);
-        cp_async_commit();
-        if (tid == 0 && cc > 0) {
-            flush(cc - 1);
-            bulk_wait_read<1>();  // the staging buffer of chunk cc (last used by cc-2) is free
+        if (tid == 0) {
+            if (cc + 1 < s.NC) load(cc + 1);  // its buffer was released by the barrier ending step cc-1
+            if (outputs && cc > 0) flush(cc - 1);
         }
-        cp_async_wait<1>();
-        __syncthreads();
         bf16 *Khs, *Ws, *Uts;
         float* Gs;
-        ptrs(cc & 1, Khs, Ws, Uts, Gs);
-        bf16* S0s = reinterpret_cast<bf16*>(outs + (cc & 1) * out_stage_bytes());
+        stage(cc & 1, Khs, Ws, Uts, Gs);
+        mbar_wait(&bars[cc & 1], (cc >> 1) & 1, &g_tc_status, failed);
+        bf16* S0s = reinterpret_cast<bf16*>(outs + (cc % kOutBufs) * out_stage_bytes());
         bf16* Vns = S0s + 64 * DK;
         const float gamC = Gs[C - 1];
         uint32_t sa[8][4];
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) c2a(sa[kk], st[2 * kk], st[2 * kk + 1]);
-        if (S0t) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) stage_afrag(S0s, DK, vl, 16 * kk, sa[kk], gq, tq);
-        }
         float vn[8][4];
 #pragma unroll
         for (int nn = 0; nn < 8; ++nn) {
-            const int tk = 8 * nn + 2 * tq;
-            const float2 u0 = unpack(*reinterpret_cast<const uint32_t*>(Uts + (vl + gq) * LDC + tk));
-            const float2 u1 = unpack(*reinterpret_cast<const uint32_t*>(Uts + (vl + gq + 8) * LDC + tk));
+            const int po = ((nn ^ gq) << 3) + 2 * tq;
+            const float2 u0 = unpack(*reinterpret_cast<const uint32_t*>(Uts + (vl + gq) * C + po));
+            const float2 u1 = unpack(*reinterpret_cast<const uint32_t*>(Uts + (vl + gq + 8) * C + po));
             vn[nn][0] = u0.x;
             vn[nn][1] = u0.y;
             vn[nn][2] = u1.x;
@@ -480,7 +528,7 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
 #pragma unroll
                 for (int nn = 0; nn < 8; nn += 2) {
                     uint32_t b[4];
-                    ldBnk(b, Ws, LDK, 8 * nn, 16 * kk, lane);
+                    ldsm_x4(b, Ws + sw_off(Lnk, 8 * nn, 2 * kk, DK));
                     mma(vn[nn], sa[kk], b[0], b[1]);
                     mma(vn[nn + 1], sa[kk], b[2], b[3]);
                 }
@@ -488,11 +536,6 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
         uint32_t va[4][4];
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) c2a(va[kk], vn[2 * kk], vn[2 * kk + 1]);
-        if (Vnt) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) stage_afrag(Vns, C, vl, 16 * kk, va[kk], gq, tq);
-        }
-        if (S0t || Vnt) fence_proxy_async_smem();
 #pragma unroll
         for (int j = 0; j < 16; ++j)
 #pragma unroll
@@ -502,14 +545,25 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
 #pragma unroll
             for (int nn = 0; nn < 16; nn += 2) {
                 uint32_t b[4];
-                ldBkn(b, Khs, LDK, 8 * nn, 16 * kk, lane);
+                ldsm_x4_t(b, Khs + sw_off(Lkn, 16 * kk, nn, DK));
                 mma(st[nn], va[kk], b[0], b[1]);
                 mma(st[nn + 1], va[kk], b[2], b[3]);
             }
+        // stage this chunk's outputs while the state update is in flight
+        if (S0t) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) stage_afrag(S0s, DK, vl, 16 * kk, sa[kk], lane);
+        }
+        if (Vnt) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) stage_afrag(Vns, C, vl, 16 * kk, va[kk], lane);
+        }
+        if (outputs) fence_proxy_async_smem();
+        if (tid == 0 && outputs) bulk_wait_read<1>();  // chunk cc-2's outputs left their buffer
         __syncthreads();
     }
     if (tid == 0) {
-        if (s.NC > 0 && (S0t || Vnt)) flush(s.NC - 1);
+        if (outputs && s.NC > 0) flush(s.NC - 1);
         bulk_wait<0>();
     }
     if (S_out) {
@@ -535,41 +589,49 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
                                              bf16* __restrict__ dVnt, bf16* __restrict__ dSCt,
                                              float* __restrict__ dS_in, unsigned char* smem) {
     constexpr size_t STAGE = bwd_stage_bytes<BETA>();
+    constexpr uint32_t TX = (BETA ? 2 : 1) * kTileK + kTileV + C * 4;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, gq = lane >> 2, tq = lane & 3;
     const int vl = 16 * w;
     const int v0 = vb * 64 + vl;
     const size_t Tp = (size_t)s.NC * C;
     unsigned char* outs = smem + 2 * STAGE;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(outs + kOutBufs * out_stage_bytes());
+    bool failed = false;
 
-    auto ptrs = [&](int buf, bf16*& Khs, bf16*& Qs, bf16*& Ws, bf16*& dOs, bf16*& dVis, float*& Gs) {
+    auto stage = [&](int buf, bf16*& Khs, bf16*& Ws, bf16*& dVis, float*& Gs, bf16*& Qs, bf16*& dOs) {
         unsigned char* p = smem + buf * STAGE;
         Khs = reinterpret_cast<bf16*>(p);
-        p += C * LDK * 2;
+        p += kTileK;
+        Ws = reinterpret_cast<bf16*>(p);
+        if (BETA) p += kTileK;
+        dVis = reinterpret_cast<bf16*>(p);
+        p += kTileV;
+        Gs = reinterpret_cast<float*>(p);
+        p += C * 4;
         Qs = reinterpret_cast<bf16*>(p);
         p += C * LDK * 2;
-        Ws = reinterpret_cast<bf16*>(p);
-        if (BETA) p += C * LDK * 2;
         dOs = reinterpret_cast<bf16*>(p);
-        p += C * LDC * 2;
-        dVis = reinterpret_cast<bf16*>(p);
-        p += C * LDC * 2;
-        Gs = reinterpret_cast<float*>(p);
     };
-    auto load = [&](int cc, int buf) {
-        bf16 *Khs, *Qs, *Ws, *dOs, *dVis;
+    auto load = [&](int cc) {  // all threads: Q and dO per thread; thread 0: bulk copies
+        bf16 *Khs, *Ws, *dVis, *Qs, *dOs;
         float* Gs;
-        ptrs(buf, Khs, Qs, Ws, dOs, dVis, Gs);
+        const int buf = cc & 1;
+        stage(buf, Khs, Ws, dVis, Gs, Qs, dOs);
         const size_t row0 = (size_t)bh * Tp + (size_t)cc * C;
         const int nval = min(C, s.T - cc * C);
-        load_tile<C, DK, 128>(Khs, LDK, Kh + row0 * DK, DK, C, tid);
+        if (tid == 0) {
+            mbar_expect_tx(&bars[buf], TX);
+            bulk_load(Khs, Kh + row0 * DK, kTileK, &bars[buf]);
+            if (BETA) bulk_load(Ws, Wn + row0 * DK, kTileK, &bars[buf]);
+            bulk_load(dVis, dVit + (((size_t)bh * s.NC + cc) * DV + vb * 64) * C, kTileV, &bars[buf]);
+            bulk_load(Gs, Gm + row0, C * 4, &bars[buf]);
+        }
         load_tile<C, DK, 128>(Qs, LDK, q + bh * s.hs_k + (size_t)cc * C * DK, DK, nval, tid);
-        if (BETA) load_tile<C, DK, 128>(Ws, LDK, Wn + row0 * DK, DK, C, tid);
         load_tile<C, 64, 128>(dOs, LDC, dO + bh * s.hs_v + (size_t)cc * C * DV + vb * 64, DV, nval, tid);
-        load_tile<64, C, 128>(dVis, LDC, dVit + (((size_t)bh * s.NC + cc) * DV + vb * 64) * C, C, 64, tid);
-        if (tid < 16) cp_async16(Gs + tid * 4, Gm + row0 + tid * 4, true);
+        cp_async_commit();
     };
     auto flush = [&](int cc) {
-        unsigned char* o = outs + (cc & 1) * out_stage_bytes();
+        unsigned char* o = outs + (cc % kOutBufs) * out_stage_bytes();
         const size_t blk = ((size_t)bh * s.NC + cc) * DV + vb * 64;
         if (dSCt) bulk_store(dSCt + blk * DK, o, 64 * DK * 2);
         if (dVnt) bulk_store(dVnt + blk * C, o + 64 * DK * 2, 64 * C * 2);
@@ -584,37 +646,39 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
             const int vv = v0 + gq + 8 * (e >> 1), d = 8 * j + 2 * tq + (e & 1);
             ds[j][e] = dS_out ? dS_out[((size_t)bh * DK + d) * DV + vv] : 0.f;
         }
+    const SwLane Lnk = sw_lane_nk(lane), Lkn = sw_lane_kn(lane);
+    const bool outputs = dSCt || dVnt;
 
-    load(s.NC - 1, (s.NC - 1) & 1);
-    cp_async_commit();
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    load(s.NC - 1);
     for (int cc = s.NC - 1; cc >= 0; --cc) {
-        if (cc > 0) load(cc - 1, (cc - 1) & 1);
-        cp_async_commit();
-        if (tid == 0 && cc < s.NC - 1) {
-            flush(cc + 1);
-            bulk_wait_read<1>();
-        }
+        const int use = s.NC - 1 - cc;  // how many chunks were processed before this one
+        if (cc > 0) load(cc - 1);
+        else cp_async_commit();
+        if (tid == 0 && outputs && cc < s.NC - 1) flush(cc + 1);
+        bf16 *Khs, *Ws, *dVis, *Qs, *dOs;
+        float* Gs;
+        stage(cc & 1, Khs, Ws, dVis, Gs, Qs, dOs);
         cp_async_wait<1>();
         __syncthreads();
-        bf16 *Khs, *Qs, *Ws, *dOs, *dVis;
-        float* Gs;
-        ptrs(cc & 1, Khs, Qs, Ws, dOs, dVis, Gs);
-        bf16* dSs = reinterpret_cast<bf16*>(outs + (cc & 1) * out_stage_bytes());
+        mbar_wait(&bars[cc & 1], (use >> 1) & 1, &g_tc_status, failed);
+        bf16* dSs = reinterpret_cast<bf16*>(outs + (cc % kOutBufs) * out_stage_bytes());
         bf16* dVns = dSs + 64 * DK;
         const float gamC = Gs[C - 1];
         uint32_t da[8][4];
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) c2a(da[kk], ds[2 * kk], ds[2 * kk + 1]);
-        if (dSCt) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) stage_afrag(dSs, DK, vl, 16 * kk, da[kk], gq, tq);
-        }
         float dvn[8][4];
 #pragma unroll
         for (int nn = 0; nn < 8; ++nn) {
-            const int tk = 8 * nn + 2 * tq;
-            const float2 u0 = unpack(*reinterpret_cast<const uint32_t*>(dVis + (vl + gq) * LDC + tk));
-            const float2 u1 = unpack(*reinterpret_cast<const uint32_t*>(dVis + (vl + gq + 8) * LDC + tk));
+            const int po = ((nn ^ gq) << 3) + 2 * tq;
+            const float2 u0 = unpack(*reinterpret_cast<const uint32_t*>(dVis + (vl + gq) * C + po));
+            const float2 u1 = unpack(*reinterpret_cast<const uint32_t*>(dVis + (vl + gq + 8) * C + po));
             dvn[nn][0] = u0.x;
             dvn[nn][1] = u0.y;
             dvn[nn][2] = u1.x;
@@ -625,18 +689,13 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
 #pragma unroll
             for (int nn = 0; nn < 8; nn += 2) {
                 uint32_t b[4];
-                ldBnk(b, Khs, LDK, 8 * nn, 16 * kk, lane);
+                ldsm_x4(b, Khs + sw_off(Lnk, 8 * nn, 2 * kk, DK));
                 mma(dvn[nn], da[kk], b[0], b[1]);
                 mma(dvn[nn + 1], da[kk], b[2], b[3]);
             }
         uint32_t va[4][4];
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) c2a(va[kk], dvn[2 * kk], dvn[2 * kk + 1]);
-        if (dVnt) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) stage_afrag(dVns, C, vl, 16 * kk, va[kk], gq, tq);
-        }
-        if (dSCt || dVnt) fence_proxy_async_smem();
 #pragma unroll
         for (int j = 0; j < 16; ++j)
 #pragma unroll
@@ -666,15 +725,25 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
 #pragma unroll
                 for (int nn = 0; nn < 16; nn += 2) {
                     uint32_t b[4];
-                    ldBkn(b, Ws, LDK, 8 * nn, 16 * kk, lane);
+                    ldsm_x4_t(b, Ws + sw_off(Lkn, 16 * kk, nn, DK));
                     mma(ds[nn], va[kk], b[0], b[1]);
                     mma(ds[nn + 1], va[kk], b[2], b[3]);
                 }
         }
+        if (dSCt) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) stage_afrag(dSs, DK, vl, 16 * kk, da[kk], lane);
+        }
+        if (dVnt) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) stage_afrag(dVns, C, vl, 16 * kk, va[kk], lane);
+        }
+        if (outputs) fence_proxy_async_smem();
+        if (tid == 0 && outputs) bulk_wait_read<1>();
         __syncthreads();
     }
     if (tid == 0) {
-        if (s.NC > 0 && (dSCt || dVnt)) flush(0);
+        if (outputs && s.NC > 0) flush(0);
         bulk_wait<0>();
     }
     if (dS_in) {
@@ -777,7 +846,7 @@ tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
     }
     const int i0 = 16 * w + gq, i1 = i0 + 8;
     const float G0 = Gs[i0], G1 = Gs[i1];
-    const float sg0 = s.scale * expf(G0), sg1 = s.scale * expf(G1);
+    const float sg0 = s.scale * __expf(G0), sg1 = s.scale * __expf(G1);
 #pragma unroll
     for (int nn = 0; nn < DV / 8; ++nn) {
         acc[nn][0] *= sg0;
@@ -790,7 +859,7 @@ tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int i = (e >> 1) ? i1 : i0, j = 8 * nn + 2 * tq + (e & 1);
-            p[nn][e] = (j <= i) ? s.scale * expf(((e >> 1) ? G1 : G0) - Gs[j]) * p[nn][e] : 0.f;
+            p[nn][e] = (j <= i) ? s.scale * __expf(((e >> 1) ? G1 : G0) - Gs[j]) * p[nn][e] : 0.f;
         }
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
@@ -899,9 +968,9 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     __syncthreads();
 
     const int r0 = 16 * mw + gq, r1 = r0 + 8;  // the two rows this thread holds
-    const float gam0 = expf(Gs[r0]), gam1 = expf(Gs[r1]);
+    const float gam0 = __expf(Gs[r0]), gam1 = __expf(Gs[r1]);
     const float gC = Gs[C - 1];
-    const float dec0 = expf(gC - Gs[r0]), dec1 = expf(gC - Gs[r1]);
+    const float dec0 = __expf(gC - Gs[r0]), dec1 = __expf(gC - Gs[r1]);
 
     // ---- phase S: products with the chunk-entry state and the state gradient
     float accQ[8][4] = {}, accK[8][4] = {};
@@ -1021,7 +1090,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int i = (e >> 1) ? r1 : r0, j = 32 * nw + 8 * nn + 2 * tq + (e & 1);
-                const float gm = (j <= i) ? expf(Gs[i] - Gs[j]) : 0.f;
+                const float gm = (j <= i) ? __expf(Gs[i] - Gs[j]) : 0.f;
                 const float m = s.scale * dp[nn][e] * gm;
                 Ms[i * LDC + j] = __float2bfloat16_rn(m);
                 const float zp = m * qk[nn][e];
@@ -1155,7 +1224,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 #pragma unroll
         for (int nn = 0; nn < 4; ++nn)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dt[nn][e] *= expf(Gs[32 * nw + 8 * nn + 2 * tq + (e & 1)]);
+            for (int e = 0; e < 4; ++e) dt[nn][e] *= __expf(Gs[32 * nw + 8 * nn + 2 * tq + (e & 1)]);
 #pragma unroll
         for (int kv = 0; kv < DV / 16; ++kv) {
             uint32_t a[4];
@@ -1236,7 +1305,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
                     const int i = (e >> 1) ? r1 : r0, j = 32 * nw + 8 * nn + 2 * tq + (e & 1);
                     float z = 0.f, bterm = 0.f;
                     if (j < i) {
-                        const float gm = expf(Gs[i] - Gs[j]);
+                        const float gm = __expf(Gs[i] - Gs[j]);
                         const float dav = -da[nn][e];
                         bterm = dav * gm * kkr[nn][e];
                         z = dav * Bs[i] * gm;
@@ -1344,7 +1413,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     if (tid == 0) {
         float zs = 0.f;
         for (int j = 0; j < C; ++j) zs += part[P_Z * C + j] + part[(P_Z + 1) * C + j];
-        dG[C - 1] += expf(gC) * sdot + zs;
+        dG[C - 1] += __expf(gC) * sdot + zs;
         float acc = 0.f;
         for (int i = C - 1; i >= 0; --i) {
             acc += dG[i];
@@ -1438,5 +1507,12 @@ cudaError_t tc_bwd(const SeqView& s, const BwdArgs& a, void* ws, cudaStream_t st
 }
 
 int tc_launches(bool) { return 3; }
+
+cudaError_t tc_device_status(int* status, bool clear) {
+    cudaError_t e = cudaMemcpyFromSymbol(status, g_tc_status, sizeof(int));
+    if (e != cudaSuccess || !clear || *status == 0) return e;
+    const int zero = 0;
+    return cudaMemcpyToSymbol(g_tc_status, &zero, sizeof(int));
+}
 
 }  // namespace sf

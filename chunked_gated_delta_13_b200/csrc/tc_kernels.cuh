@@ -10,5 +10,8 @@ size_t tc_workspace_bytes(const SeqView& s, bool backward);
 cudaError_t tc_fwd(const SeqView& s, const FwdArgs& a, void* ws, cudaStream_t st);
 cudaError_t tc_bwd(const SeqView& s, const BwdArgs& a, void* ws, cudaStream_t st);
 int tc_launches(bool backward);
+// Status word of the current device (bit 0: a kernel gave up waiting for one
+// of its own bulk copies); synchronising; optionally cleared.
+cudaError_t tc_device_status(int* status, bool clear);
 
 }  // namespace sf

@@ -58,7 +58,8 @@ typedef enum {
     SF_ERR_ALIGNMENT = 3,     /* a device pointer is not 16-byte aligned */
     SF_ERR_WORKSPACE = 4,     /* workspace missing or smaller than the *_workspace_bytes query */
     SF_ERR_CUDA = 5,          /* a CUDA launch or copy failed */
-    SF_ERR_TIMEOUT = 6        /* reserved: no kernel of this build waits on another */
+    SF_ERR_TIMEOUT = 6        /* a kernel gave up waiting for one of its own asynchronous copies
+                                 (reported by sf_device_check; that call's results are undefined) */
 } sf_status;
 
 typedef enum { SF_F32 = 0, SF_BF16 = 1 } sf_dtype;
@@ -128,6 +129,13 @@ sf_status sf_segment_run(const sf_gdn_shape* full, int N, const int* seg_len, co
                          const float* S_in, const void* dO, const float* dS_out, void* o,
                          float* S_out, void* dq, void* dk, void* dv, float* dg, float* dbeta,
                          float* dS_in, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises the current device and reports whether any kernel of this
+ * library gave up a bounded wait for its own asynchronous copies since the last
+ * check (SF_ERR_TIMEOUT), then clears the flag.  No kernel waits on another
+ * CTA or another launch, so this only fires if the memory system failed to
+ * deliver a copy within about two seconds. */
+sf_status sf_device_check(void);
 
 /* Forward of one segment for callers that cannot allocate device memory (an
  * engine or plugin whose memory is planned up front and gives no allocation

@@ -36,6 +36,7 @@ def gpu_fwd_bwd(d: dict, C: int, scale=1.0) -> dict:
     gr = sf.bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S_in"], d["dO"], d["dS_out"],
                 C=C, scale=scale)
     torch.cuda.synchronize()
+    sf.device_check()
     out = {"o": host(o), "S_out": host(S_out)}
     out.update({k: host(v) for k, v in gr.items()})
     return out
@@ -45,6 +46,7 @@ def gpu_segments(d: dict, C: int, N: int, seg_len=None, scale=1.0) -> dict:
     o, S_out, gr = sf.segment_run(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S_in"], d["dO"],
                                   d["dS_out"], N=N, seg_len=seg_len, C=C, scale=scale)
     torch.cuda.synchronize()
+    sf.device_check()
     out = {"o": o.clone(), "S_out": S_out.clone()}
     out.update({k: None if v is None else v.clone() for k, v in gr.items()})
     return out
