@@ -386,17 +386,18 @@ constexpr size_t fwd_stage_bytes() {
     return (size_t)kTileK * (BETA ? 2 : 1) + kTileV + C * 4;
 }
 template <bool BETA>
-constexpr size_t bwd_stage_bytes() {  // + Q and dO tiles copied per thread (padded rows)
-    return (size_t)kTileK * (BETA ? 2 : 1) + kTileV + C * 4 + (size_t)C * LDK * 2 + (size_t)C * LDC * 2;
+constexpr size_t bwd_stage_bytes() {  // + Q and dO tiles copied per thread (permuted, see swz)
+    return (size_t)kTileK * (BETA ? 2 : 1) + kTileV + C * 4 + kTileK + (size_t)C * 64 * 2;
 }
 // Output staging of one chunk step of a 64-column block: the state tile
 // (64 x DK) and the value tile (64 x C), in the permuted layout of swz().
 constexpr size_t out_stage_bytes() { return (size_t)64 * DK * 2 + (size_t)64 * C * 2; }
 constexpr int kOutBufs = 3;  // staged outputs of chunk c are flushed during step c+1 and must be read by step c+3
+constexpr size_t xch_bytes();
 template <bool BETA>
-constexpr size_t fwd_scan_smem() { return 2 * fwd_stage_bytes<BETA>() + kOutBufs * out_stage_bytes() + 16; }
+constexpr size_t fwd_scan_smem() { return 2 * fwd_stage_bytes<BETA>() + kOutBufs * out_stage_bytes() + xch_bytes() + 16; }
 template <bool BETA>
-constexpr size_t bwd_scan_smem() { return 2 * bwd_stage_bytes<BETA>() + kOutBufs * out_stage_bytes() + 16; }
+constexpr size_t bwd_scan_smem() { return 2 * bwd_stage_bytes<BETA>() + kOutBufs * out_stage_bytes() + xch_bytes() + 16; }
 
 // Per-lane parts of the addresses into permuted [rows][128] tiles.
 //   B fragments (stored [n][k], k = 16kk..): row = n0 + lr, piece 2kk + pb
@@ -428,10 +429,42 @@ __device__ __forceinline__ void stage_afrag(bf16* t, int cols, int r0, int c0, c
     stsm_x4(t + (r0 + lr) * cols + piece * 8, a);
 }
 
-// Forward chain for one (head, 64 state columns) on 4 warps of 16 columns:
-// per chunk V_new^T = U^T + S^T (-W)^T, S^T <- gamma_C S^T + V_new^T Khat.
+// The chains use 8 warps per 64-column block: warps w and w+4 (which share an
+// SM sub-partition) own the same 16 state columns and split every chunk step,
+// the first warp taking tokens 0-31 of V_new and state rows 0-63 (of d_k),
+// the second tokens 32-63 and rows 64-127.  Each product needs the partner's
+// half of its left operand, which the pair swaps as bf16 fragments through
+// shared memory.  One warp alone can issue a warp-level MMA only every ~18
+// cycles, so two warps per sub-partition halve the step's issue time.
+constexpr size_t xch_bytes() { return (size_t)4 * 2 * (4 + 2) * 32 * 16; }  // per pair: 4 state + 2 value fragments
+
+// Pair barrier of the two warps that share a column group.
+__device__ __forceinline__ void pair_sync(int cg) { asm volatile("bar.sync %0, 64;\n" ::"r"(cg + 1) : "memory"); }
+
+// Fragment exchange slots (16 bytes per lane): [cg][half][slot 0-5][lane].
+__device__ __forceinline__ uint4* xslot(unsigned char* xch, int cg, int half, int slot, int lane) {
+    return reinterpret_cast<uint4*>(xch) + (((cg * 2 + half) * 6 + slot) * 32 + lane);
+}
+__device__ __forceinline__ void put_frag(uint4* p, const uint32_t (&a)[4]) { *p = make_uint4(a[0], a[1], a[2], a[3]); }
+__device__ __forceinline__ void get_frag(const uint4* p, uint32_t (&a)[4]) {
+    const uint4 v = *p;
+    a[0] = v.x;
+    a[1] = v.y;
+    a[2] = v.z;
+    a[3] = v.w;
+}
+
+// A^T fragment (ldmatrix.trans) from a permuted tile of row length `rowlen`
+// stored [k][m] (see swz): rows k0.., columns m0.. (m0, k0 multiples of 16).
+__device__ __forceinline__ int swz_at_off(int k0, int m0, int lane, int rowlen) {
+    const int lr = (lane & 7) + ((lane >> 4) << 3), pb = (lane >> 3) & 1;
+    return (k0 + lr) * rowlen + ((((m0 >> 3) + pb) ^ (lr & 7)) << 3);
+}
+
+// Forward chain for one (head, 64 state columns): per chunk
+// V_new^T = U^T + S^T (-W)^T, S^T <- gamma_C S^T + V_new^T Khat.
 // Optional outputs: V_new^T and S0^T per chunk (bf16, bulk-stored from a
-// double-buffered staging area by one thread), S_out (fp32).
+// staging area by one thread), S_out (fp32).
 template <int DV, bool BETA>
 __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, const float* __restrict__ Gm,
                                              const bf16* __restrict__ Wn, const bf16* __restrict__ Kh,
@@ -441,11 +474,13 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
     constexpr size_t STAGE = fwd_stage_bytes<BETA>();
     constexpr uint32_t TX = (BETA ? 2 : 1) * kTileK + kTileV + C * 4;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, gq = lane >> 2, tq = lane & 3;
-    const int vl = 16 * w;            // first state column of this warp inside the block
+    const int cg = w & 3, half = w >> 2, oth = half ^ 1;
+    const int vl = 16 * cg;           // first state column of this warp pair inside the block
     const int v0 = vb * 64 + vl;      // ... and inside the head
     const size_t Tp = (size_t)s.NC * C;
     unsigned char* outs = smem + 2 * STAGE;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(outs + kOutBufs * out_stage_bytes());
+    unsigned char* xch = outs + kOutBufs * out_stage_bytes();
+    uint64_t* bars = reinterpret_cast<uint64_t*>(xch + xch_bytes());
     bool failed = false;
 
     auto stage = [&](int buf, bf16*& Khs, bf16*& Ws, bf16*& Uts, float*& Gs) {
@@ -478,12 +513,12 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
         bulk_commit();
     };
 
-    float st[16][4];
+    float st[8][4];  // S^T rows vl.., state rows 64*half + 8j..
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
+    for (int j = 0; j < 8; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const int vv = v0 + gq + 8 * (e >> 1), d = 8 * j + 2 * tq + (e & 1);
+            const int vv = v0 + gq + 8 * (e >> 1), d = 64 * half + 8 * j + 2 * tq + (e & 1);
             st[j][e] = S_in ? S_in[((size_t)bh * DK + d) * DV + vv] : 0.f;
         }
     const SwLane Lnk = sw_lane_nk(lane), Lkn = sw_lane_kn(lane);
@@ -504,17 +539,21 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
         bf16 *Khs, *Ws, *Uts;
         float* Gs;
         stage(cc & 1, Khs, Ws, Uts, Gs);
-        mbar_wait(&bars[cc & 1], (cc >> 1) & 1, &g_tc_status, failed);
         bf16* S0s = reinterpret_cast<bf16*>(outs + (cc % kOutBufs) * out_stage_bytes());
         bf16* Vns = S0s + 64 * DK;
+        // own half of S^T as bf16 fragments, swapped with the partner
+        uint32_t sa[4][4], sp[4][4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            c2a(sa[kk], st[2 * kk], st[2 * kk + 1]);
+            put_frag(xslot(xch, cg, half, kk, lane), sa[kk]);
+        }
+        mbar_wait(&bars[cc & 1], (cc >> 1) & 1, &g_tc_status, failed);
         const float gamC = Gs[C - 1];
-        uint32_t sa[8][4];
+        float vn[4][4];  // V_new^T, tokens 32*half + 8nn..
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) c2a(sa[kk], st[2 * kk], st[2 * kk + 1]);
-        float vn[8][4];
-#pragma unroll
-        for (int nn = 0; nn < 8; ++nn) {
-            const int po = ((nn ^ gq) << 3) + 2 * tq;
+        for (int nn = 0; nn < 4; ++nn) {
+            const int po = (((4 * half + nn) ^ gq) << 3) + 2 * tq;
             const float2 u0 = unpack(*reinterpret_cast<const uint32_t*>(Uts + (vl + gq) * C + po));
             const float2 u1 = unpack(*reinterpret_cast<const uint32_t*>(Uts + (vl + gq + 8) * C + po));
             vn[nn][0] = u0.x;
@@ -522,41 +561,64 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
             vn[nn][2] = u1.x;
             vn[nn][3] = u1.y;
         }
+        pair_sync(cg);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) get_frag(xslot(xch, cg, oth, kk, lane), sp[kk]);
         if (BETA) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
+            for (int j = 0; j < 8; ++j) {  // own state rows first, then the partner's
+                const int kt = (j < 4) ? 4 * half + j : 4 * oth + (j - 4);
 #pragma unroll
-                for (int nn = 0; nn < 8; nn += 2) {
+                for (int nn = 0; nn < 4; nn += 2) {
                     uint32_t b[4];
-                    ldsm_x4(b, Ws + sw_off(Lnk, 8 * nn, 2 * kk, DK));
-                    mma(vn[nn], sa[kk], b[0], b[1]);
-                    mma(vn[nn + 1], sa[kk], b[2], b[3]);
+                    ldsm_x4(b, Ws + sw_off(Lnk, 8 * (4 * half + nn), 2 * kt, DK));
+                    if (j < 4) {
+                        mma(vn[nn], sa[j], b[0], b[1]);
+                        mma(vn[nn + 1], sa[j], b[2], b[3]);
+                    } else {
+                        mma(vn[nn], sp[j - 4], b[0], b[1]);
+                        mma(vn[nn + 1], sp[j - 4], b[2], b[3]);
+                    }
                 }
+            }
         }
-        uint32_t va[4][4];
+        uint32_t va[2][4], vp[2][4];
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) c2a(va[kk], vn[2 * kk], vn[2 * kk + 1]);
+        for (int kk = 0; kk < 2; ++kk) {
+            c2a(va[kk], vn[2 * kk], vn[2 * kk + 1]);
+            put_frag(xslot(xch, cg, half, 4 + kk, lane), va[kk]);
+        }
+        pair_sync(cg);
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
+        for (int kk = 0; kk < 2; ++kk) get_frag(xslot(xch, cg, oth, 4 + kk, lane), vp[kk]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) st[j][e] *= gamC;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
+        for (int j = 0; j < 4; ++j) {  // token tiles: own first, then the partner's
+            const int kt = (j < 2) ? 2 * half + j : 2 * oth + (j - 2);
 #pragma unroll
-            for (int nn = 0; nn < 16; nn += 2) {
+            for (int nn = 0; nn < 8; nn += 2) {
                 uint32_t b[4];
-                ldsm_x4_t(b, Khs + sw_off(Lkn, 16 * kk, nn, DK));
-                mma(st[nn], va[kk], b[0], b[1]);
-                mma(st[nn + 1], va[kk], b[2], b[3]);
+                ldsm_x4_t(b, Khs + sw_off(Lkn, 16 * kt, 8 * half + nn, DK));
+                if (j < 2) {
+                    mma(st[nn], va[j], b[0], b[1]);
+                    mma(st[nn + 1], va[j], b[2], b[3]);
+                } else {
+                    mma(st[nn], vp[j - 2], b[0], b[1]);
+                    mma(st[nn + 1], vp[j - 2], b[2], b[3]);
+                }
             }
-        // stage this chunk's outputs while the state update is in flight
+        }
+        // stage this chunk's outputs (own halves) while the state update is in flight
         if (S0t) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) stage_afrag(S0s, DK, vl, 16 * kk, sa[kk], lane);
+            for (int kk = 0; kk < 4; ++kk) stage_afrag(S0s, DK, vl, 64 * half + 16 * kk, sa[kk], lane);
         }
         if (Vnt) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) stage_afrag(Vns, C, vl, 16 * kk, va[kk], lane);
+            for (int kk = 0; kk < 2; ++kk) stage_afrag(Vns, C, vl, 32 * half + 16 * kk, va[kk], lane);
         }
         if (outputs) fence_proxy_async_smem();
         if (tid == 0 && outputs) bulk_wait_read<1>();  // chunk cc-2's outputs left their buffer
@@ -568,10 +630,10 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
     }
     if (S_out) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int vv = v0 + gq + 8 * (e >> 1), d = 8 * j + 2 * tq + (e & 1);
+                const int vv = v0 + gq + 8 * (e >> 1), d = 64 * half + 8 * j + 2 * tq + (e & 1);
                 S_out[((size_t)bh * DK + d) * DV + vv] = st[j][e];
             }
     }
@@ -591,11 +653,13 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
     constexpr size_t STAGE = bwd_stage_bytes<BETA>();
     constexpr uint32_t TX = (BETA ? 2 : 1) * kTileK + kTileV + C * 4;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, gq = lane >> 2, tq = lane & 3;
-    const int vl = 16 * w;
+    const int cg = w & 3, half = w >> 2, oth = half ^ 1;
+    const int vl = 16 * cg;
     const int v0 = vb * 64 + vl;
     const size_t Tp = (size_t)s.NC * C;
     unsigned char* outs = smem + 2 * STAGE;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(outs + kOutBufs * out_stage_bytes());
+    unsigned char* xch = outs + kOutBufs * out_stage_bytes();
+    uint64_t* bars = reinterpret_cast<uint64_t*>(xch + xch_bytes());
     bool failed = false;
 
     auto stage = [&](int buf, bf16*& Khs, bf16*& Ws, bf16*& dVis, float*& Gs, bf16*& Qs, bf16*& dOs) {
@@ -609,10 +673,10 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
         Gs = reinterpret_cast<float*>(p);
         p += C * 4;
         Qs = reinterpret_cast<bf16*>(p);
-        p += C * LDK * 2;
+        p += kTileK;
         dOs = reinterpret_cast<bf16*>(p);
     };
-    auto load = [&](int cc) {  // all threads: Q and dO per thread; thread 0: bulk copies
+    auto load = [&](int cc) {  // all threads: Q and dO pieces (permuted); thread 0: bulk copies
         bf16 *Khs, *Ws, *dVis, *Qs, *dOs;
         float* Gs;
         const int buf = cc & 1;
@@ -626,8 +690,18 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
             bulk_load(dVis, dVit + (((size_t)bh * s.NC + cc) * DV + vb * 64) * C, kTileV, &bars[buf]);
             bulk_load(Gs, Gm + row0, C * 4, &bars[buf]);
         }
-        load_tile<C, DK, 128>(Qs, LDK, q + bh * s.hs_k + (size_t)cc * C * DK, DK, nval, tid);
-        load_tile<C, 64, 128>(dOs, LDC, dO + bh * s.hs_v + (size_t)cc * C * DV + vb * 64, DV, nval, tid);
+        const bf16* qg = q + bh * s.hs_k + (size_t)cc * C * DK;
+        for (int e = tid; e < C * (DK / 8); e += 256) {
+            const int t = e >> 4, pc = e & 15;
+            const bool ok = t < nval;
+            cp_async16(Qs + swz(t, 8 * pc, DK), qg + (ok ? (size_t)t * DK : 0) + 8 * pc, ok);
+        }
+        const bf16* og = dO + bh * s.hs_v + (size_t)cc * C * DV + vb * 64;
+        for (int e = tid; e < C * 8; e += 256) {
+            const int t = e >> 3, pc = e & 7;
+            const bool ok = t < nval;
+            cp_async16(dOs + swz(t, 8 * pc, 64), og + (ok ? (size_t)t * DV : 0) + 8 * pc, ok);
+        }
         cp_async_commit();
     };
     auto flush = [&](int cc) {
@@ -638,12 +712,12 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
         bulk_commit();
     };
 
-    float ds[16][4];
+    float ds[8][4];
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
+    for (int j = 0; j < 8; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const int vv = v0 + gq + 8 * (e >> 1), d = 8 * j + 2 * tq + (e & 1);
+            const int vv = v0 + gq + 8 * (e >> 1), d = 64 * half + 8 * j + 2 * tq + (e & 1);
             ds[j][e] = dS_out ? dS_out[((size_t)bh * DK + d) * DV + vv] : 0.f;
         }
     const SwLane Lnk = sw_lane_nk(lane), Lkn = sw_lane_kn(lane);
@@ -664,19 +738,24 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
         bf16 *Khs, *Ws, *dVis, *Qs, *dOs;
         float* Gs;
         stage(cc & 1, Khs, Ws, dVis, Gs, Qs, dOs);
-        cp_async_wait<1>();
-        __syncthreads();
-        mbar_wait(&bars[cc & 1], (use >> 1) & 1, &g_tc_status, failed);
         bf16* dSs = reinterpret_cast<bf16*>(outs + (cc % kOutBufs) * out_stage_bytes());
         bf16* dVns = dSs + 64 * DK;
+        uint32_t da[4][4], dp[4][4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            c2a(da[kk], ds[2 * kk], ds[2 * kk + 1]);
+            put_frag(xslot(xch, cg, half, kk, lane), da[kk]);
+        }
+        cp_async_wait<1>();
+        __syncthreads();  // Q / dO pieces of this chunk and the exchanged fragments are visible
+        mbar_wait(&bars[cc & 1], (use >> 1) & 1, &g_tc_status, failed);
         const float gamC = Gs[C - 1];
-        uint32_t da[8][4];
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) c2a(da[kk], ds[2 * kk], ds[2 * kk + 1]);
-        float dvn[8][4];
+        for (int kk = 0; kk < 4; ++kk) get_frag(xslot(xch, cg, oth, kk, lane), dp[kk]);
+        float dvn[4][4];  // dV_new^T, tokens 32*half + 8nn..
 #pragma unroll
-        for (int nn = 0; nn < 8; ++nn) {
-            const int po = ((nn ^ gq) << 3) + 2 * tq;
+        for (int nn = 0; nn < 4; ++nn) {
+            const int po = (((4 * half + nn) ^ gq) << 3) + 2 * tq;
             const float2 u0 = unpack(*reinterpret_cast<const uint32_t*>(dVis + (vl + gq) * C + po));
             const float2 u1 = unpack(*reinterpret_cast<const uint32_t*>(dVis + (vl + gq + 8) * C + po));
             dvn[nn][0] = u0.x;
@@ -685,25 +764,36 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
             dvn[nn][3] = u1.y;
         }
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        for (int j = 0; j < 8; ++j) {
+            const int kt = (j < 4) ? 4 * half + j : 4 * oth + (j - 4);
 #pragma unroll
-            for (int nn = 0; nn < 8; nn += 2) {
+            for (int nn = 0; nn < 4; nn += 2) {
                 uint32_t b[4];
-                ldsm_x4(b, Khs + sw_off(Lnk, 8 * nn, 2 * kk, DK));
-                mma(dvn[nn], da[kk], b[0], b[1]);
-                mma(dvn[nn + 1], da[kk], b[2], b[3]);
+                ldsm_x4(b, Khs + sw_off(Lnk, 8 * (4 * half + nn), 2 * kt, DK));
+                if (j < 4) {
+                    mma(dvn[nn], da[j], b[0], b[1]);
+                    mma(dvn[nn + 1], da[j], b[2], b[3]);
+                } else {
+                    mma(dvn[nn], dp[j - 4], b[0], b[1]);
+                    mma(dvn[nn + 1], dp[j - 4], b[2], b[3]);
+                }
             }
-        uint32_t va[4][4];
+        }
+        uint32_t va[2][4], vp[2][4];
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) c2a(va[kk], dvn[2 * kk], dvn[2 * kk + 1]);
+        for (int kk = 0; kk < 2; ++kk) {
+            c2a(va[kk], dvn[2 * kk], dvn[2 * kk + 1]);
+            put_frag(xslot(xch, cg, half, 4 + kk, lane), va[kk]);
+        }
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) ds[j][e] *= gamC;
+        // (scale gamma * dO)^T Q for this warp's state rows; independent of the chain
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             uint32_t a[4];
-            ldAt(a, dOs, LDC, vl, 16 * kk, lane);
+            ldsm_x4_t(a, dOs + swz_at_off(16 * kk, vl, lane, 64));
             const int tk = 16 * kk + 2 * tq;
             const float g0 = s.scale * Gs[tk], g1 = s.scale * Gs[tk + 1];
             const float g2 = s.scale * Gs[tk + 8], g3 = s.scale * Gs[tk + 9];
@@ -712,31 +802,41 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
             a[2] = scale2(a[2], g2, g3);
             a[3] = scale2(a[3], g2, g3);
 #pragma unroll
-            for (int nn = 0; nn < 16; nn += 2) {
+            for (int nn = 0; nn < 8; nn += 2) {
                 uint32_t b[4];
-                ldBkn(b, Qs, LDK, 8 * nn, 16 * kk, lane);
+                ldsm_x4_t(b, Qs + sw_off(Lkn, 16 * kk, 8 * half + nn, DK));
                 mma(ds[nn], a, b[0], b[1]);
                 mma(ds[nn + 1], a, b[2], b[3]);
             }
         }
+        pair_sync(cg);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) get_frag(xslot(xch, cg, oth, 4 + kk, lane), vp[kk]);
         if (BETA) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
+            for (int j = 0; j < 4; ++j) {
+                const int kt = (j < 2) ? 2 * half + j : 2 * oth + (j - 2);
 #pragma unroll
-                for (int nn = 0; nn < 16; nn += 2) {
+                for (int nn = 0; nn < 8; nn += 2) {
                     uint32_t b[4];
-                    ldsm_x4_t(b, Ws + sw_off(Lkn, 16 * kk, nn, DK));
-                    mma(ds[nn], va[kk], b[0], b[1]);
-                    mma(ds[nn + 1], va[kk], b[2], b[3]);
+                    ldsm_x4_t(b, Ws + sw_off(Lkn, 16 * kt, 8 * half + nn, DK));
+                    if (j < 2) {
+                        mma(ds[nn], va[j], b[0], b[1]);
+                        mma(ds[nn + 1], va[j], b[2], b[3]);
+                    } else {
+                        mma(ds[nn], vp[j - 2], b[0], b[1]);
+                        mma(ds[nn + 1], vp[j - 2], b[2], b[3]);
+                    }
                 }
+            }
         }
         if (dSCt) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) stage_afrag(dSs, DK, vl, 16 * kk, da[kk], lane);
+            for (int kk = 0; kk < 4; ++kk) stage_afrag(dSs, DK, vl, 64 * half + 16 * kk, da[kk], lane);
         }
         if (dVnt) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) stage_afrag(dVns, C, vl, 16 * kk, va[kk], lane);
+            for (int kk = 0; kk < 2; ++kk) stage_afrag(dVns, C, vl, 32 * half + 16 * kk, va[kk], lane);
         }
         if (outputs) fence_proxy_async_smem();
         if (tid == 0 && outputs) bulk_wait_read<1>();
@@ -748,17 +848,17 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
     }
     if (dS_in) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int vv = v0 + gq + 8 * (e >> 1), d = 8 * j + 2 * tq + (e & 1);
+                const int vv = v0 + gq + 8 * (e >> 1), d = 64 * half + 8 * j + 2 * tq + (e & 1);
                 dS_in[((size_t)bh * DK + d) * DV + vv] = ds[j][e];
             }
     }
 }
 
 template <int DV, bool BETA>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
 tc_scan_fwd_kernel(SeqView s, const float* __restrict__ Gm, const bf16* __restrict__ Wn,
                    const bf16* __restrict__ Kh, const bf16* __restrict__ Ut,
                    const float* __restrict__ S_in, bf16* __restrict__ Vnt, bf16* __restrict__ S0t,
@@ -772,7 +872,7 @@ tc_scan_fwd_kernel(SeqView s, const float* __restrict__ Gm, const bf16* __restri
 // states (V_new and the chunk-entry states), the rest run the reverse
 // state-gradient scan.  The two groups share no data.
 template <int DV, bool BETA>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
 tc_scan_bwd_dual_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ dO,
                         const float* __restrict__ Gm, const bf16* __restrict__ Wn,
                         const bf16* __restrict__ Kh, const bf16* __restrict__ Ut,
@@ -1450,7 +1550,7 @@ cudaError_t fwd_impl(const SeqView& s, const FwdArgs& a, void* ws, cudaStream_t 
     SF_LAUNCH("tc_prep", st, tc_prep_kernel<DV, BETA, false><<<gc, 128, sm_prep, st>>>(
                                  s, q, k, v, a.g, a.beta, nullptr, w.Gc, w.Gm, w.W, w.Kh, w.Ut, nullptr));
     TC_TRY(cudaGetLastError());
-    SF_LAUNCH("tc_scan_fwd", st, tc_scan_fwd_kernel<DV, BETA><<<s.BH * (DV / 64), 128, sm_scan, st>>>(
+    SF_LAUNCH("tc_scan_fwd", st, tc_scan_fwd_kernel<DV, BETA><<<s.BH * (DV / 64), 256, sm_scan, st>>>(
                                      s, w.Gm, w.W, w.Kh, w.Ut, a.S_in, w.Vnt, w.S0t, a.S_out));
     TC_TRY(cudaGetLastError());
     SF_LAUNCH("tc_out", st, tc_out_kernel<DV><<<gc, 128, sm_out, st>>>(s, q, k, w.Gc, w.Vnt, w.S0t,
@@ -1477,7 +1577,7 @@ cudaError_t bwd_impl(const SeqView& s, const BwdArgs& a, void* ws, cudaStream_t 
     SF_LAUNCH("tc_prep_bwd", st, tc_prep_kernel<DV, BETA, true><<<gc, 128, sm_prep, st>>>(
                                      s, q, k, v, a.g, a.beta, dO, w.Gc, w.Gm, w.W, w.Kh, w.Ut, w.dVit));
     TC_TRY(cudaGetLastError());
-    SF_LAUNCH("tc_scan_bwd", st, tc_scan_bwd_dual_kernel<DV, BETA><<<2 * s.BH * (DV / 64), 128, sm_scan, st>>>(
+    SF_LAUNCH("tc_scan_bwd", st, tc_scan_bwd_dual_kernel<DV, BETA><<<2 * s.BH * (DV / 64), 256, sm_scan, st>>>(
                                      s, q, dO, w.Gm, w.W, w.Kh, w.Ut, w.dVit, a.S_in, a.dS_out, w.Vnt, w.S0t,
                                      w.dVnt, w.dSCt, a.dS_in));
     TC_TRY(cudaGetLastError());
