@@ -319,58 +319,87 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         const int r = e >> 3, cc = (e & 7) * 8;
         *reinterpret_cast<uint4*>(Utg + swz(r, cc, C)) = *reinterpret_cast<const uint4*>(Ust + r * LDC + cc);
     }
+}
 
-    if (BWD) {
-        bf16* Ps = Tw;  // Tw is no longer read (all warps passed the barrier above)
-        {
-            float acc[8][4] = {};
+// ----------------------------------------------------------------- intra ---
+template <int DV>
+constexpr size_t intra_smem() {
+    return (size_t)C * LDK * 2 * 2 + (size_t)C * (DV + 8) * 2 + (size_t)C * LDC * 2 + C * 4;
+}
+
+// Intra-chunk output gradient (OG): dVi^T = (P^T dO)^T with
+// P = scale (Q K^T) * Gamma, one CTA (4 warps) per (chunk, head).
+template <int DV>
+__global__ void __launch_bounds__(128)
+tc_intra_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ dO,
+                const float* __restrict__ Gc, bf16* __restrict__ dVito) {
+    constexpr int LDV = DV + 8;
+    extern __shared__ __align__(16) unsigned char smem[];
+    bf16* Qs = reinterpret_cast<bf16*>(smem);
+    bf16* Ks = Qs + C * LDK;
+    bf16* dOs = Ks + C * LDK;
+    bf16* Ps = dOs + C * LDV;
+    float* Gs = reinterpret_cast<float*>(Ps + C * LDC);
+    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int gq = lane >> 2, tq = lane & 3;
+    const int t0 = c * C;
+    const int nval = min(C, s.T - t0);
+    const size_t Tp = (size_t)s.NC * C;
+    load_tile<C, DK, 128>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+    load_tile<C, DK, 128>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+    load_tile<C, DV, 128>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+    if (tid < 16) cp_async16(Gs + tid * 4, Gc + bh * Tp + t0 + tid * 4, true);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    {
+        float acc[8][4] = {};
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                uint32_t a[4];
-                ldA(a, Qs, LDK, 16 * w, 16 * kk, lane);
+        for (int kk = 0; kk < 8; ++kk) {
+            uint32_t a[4];
+            ldA(a, Qs, LDK, 16 * w, 16 * kk, lane);
 #pragma unroll
-                for (int nn = 0; nn < 8; nn += 2) {
-                    uint32_t b[4];
-                    ldBnk(b, Ks, LDK, 8 * nn, 16 * kk, lane);
-                    mma(acc[nn], a, b[0], b[1]);
-                    mma(acc[nn + 1], a, b[2], b[3]);
-                }
+            for (int nn = 0; nn < 8; nn += 2) {
+                uint32_t b[4];
+                ldBnk(b, Ks, LDK, 8 * nn, 16 * kk, lane);
+                mma(acc[nn], a, b[0], b[1]);
+                mma(acc[nn + 1], a, b[2], b[3]);
             }
-#pragma unroll
-            for (int nn = 0; nn < 8; ++nn)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = 16 * w + gq + 8 * (e >> 1), j = 8 * nn + 2 * tq + (e & 1);
-                    const float p = (j <= i) ? s.scale * __expf(Gs[i] - Gs[j]) * acc[nn][e] : 0.f;
-                    Ps[i * LDC + j] = __float2bfloat16_rn(p);
-                }
         }
-        __syncthreads();
-        // dVi^T[v][j] = sum_i dO[i][v] P[i][j]
-        constexpr int MT = DV / 64;  // 16-row m-tiles per warp
-        bf16* dst = dVito + ((size_t)bh * s.NC + c) * DV * C;
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            const int m0 = (w * MT + mt) * 16;
-            float acc[8][4] = {};
+        for (int nn = 0; nn < 8; ++nn)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                uint32_t a[4];
-                ldAt(a, dOs, LDV, m0, 16 * kk, lane);
-#pragma unroll
-                for (int nn = 0; nn < 8; nn += 2) {
-                    uint32_t b[4];
-                    ldBkn(b, Ps, LDC, 8 * nn, 16 * kk, lane);
-                    mma(acc[nn], a, b[0], b[1]);
-                    mma(acc[nn + 1], a, b[2], b[3]);
-                }
+            for (int e = 0; e < 4; ++e) {
+                const int i = 16 * w + gq + 8 * (e >> 1), j = 8 * nn + 2 * tq + (e & 1);
+                const float p = (j <= i) ? s.scale * __expf(Gs[i] - Gs[j]) * acc[nn][e] : 0.f;
+                Ps[i * LDC + j] = __float2bfloat16_rn(p);
             }
+    }
+    __syncthreads();
+    // dVi^T[v][j] = sum_i dO[i][v] P[i][j]
+    constexpr int MT = DV / 64;  // 16-row m-tiles per warp
+    bf16* dst = dVito + ((size_t)bh * s.NC + c) * DV * C;
 #pragma unroll
-            for (int nn = 0; nn < 8; ++nn) {
-                const int r = m0 + gq, j = 8 * nn + 2 * tq;
-                *reinterpret_cast<uint32_t*>(dst + swz(r, j, C)) = pack(acc[nn][0], acc[nn][1]);
-                *reinterpret_cast<uint32_t*>(dst + swz(r + 8, j, C)) = pack(acc[nn][2], acc[nn][3]);
+    for (int mt = 0; mt < MT; ++mt) {
+        const int m0 = (w * MT + mt) * 16;
+        float acc[8][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t a[4];
+            ldAt(a, dOs, LDV, m0, 16 * kk, lane);
+#pragma unroll
+            for (int nn = 0; nn < 8; nn += 2) {
+                uint32_t b[4];
+                ldBkn(b, Ps, LDC, 8 * nn, 16 * kk, lane);
+                mma(acc[nn], a, b[0], b[1]);
+                mma(acc[nn + 1], a, b[2], b[3]);
             }
+        }
+#pragma unroll
+        for (int nn = 0; nn < 8; ++nn) {
+            const int r = m0 + gq, j = 8 * nn + 2 * tq;
+            *reinterpret_cast<uint32_t*>(dst + swz(r, j, C)) = pack(acc[nn][0], acc[nn][1]);
+            *reinterpret_cast<uint32_t*>(dst + swz(r + 8, j, C)) = pack(acc[nn][2], acc[nn][3]);
         }
     }
 }
@@ -1566,16 +1595,20 @@ cudaError_t bwd_impl(const SeqView& s, const BwdArgs& a, void* ws, cudaStream_t 
     const bf16* k = static_cast<const bf16*>(a.k);
     const bf16* v = static_cast<const bf16*>(a.v);
     const bf16* dO = static_cast<const bf16*>(a.dO);
-    constexpr size_t sm_prep = prep_smem<DV, true>();
+    constexpr size_t sm_prep = prep_smem<DV, false>();
+    constexpr size_t sm_intra = intra_smem<DV>();
     constexpr size_t sm_f = fwd_scan_smem<BETA>(), sm_b = bwd_scan_smem<BETA>();
     constexpr size_t sm_scan = sm_f > sm_b ? sm_f : sm_b;
     constexpr size_t sm_grad = grad_smem<DV>();
-    TC_TRY(smem_attr(tc_prep_kernel<DV, BETA, true>, sm_prep));
+    TC_TRY(smem_attr(tc_prep_kernel<DV, BETA, false>, sm_prep));
+    TC_TRY(smem_attr(tc_intra_kernel<DV>, sm_intra));
     TC_TRY(smem_attr(tc_scan_bwd_dual_kernel<DV, BETA>, sm_scan));
     TC_TRY(smem_attr(tc_grad_kernel<DV, BETA>, sm_grad));
     const dim3 gc(s.NC, s.BH);
-    SF_LAUNCH("tc_prep_bwd", st, tc_prep_kernel<DV, BETA, true><<<gc, 128, sm_prep, st>>>(
-                                     s, q, k, v, a.g, a.beta, dO, w.Gc, w.Gm, w.W, w.Kh, w.Ut, w.dVit));
+    SF_LAUNCH("tc_prep_bwd", st, tc_prep_kernel<DV, BETA, false><<<gc, 128, sm_prep, st>>>(
+                                     s, q, k, v, a.g, a.beta, nullptr, w.Gc, w.Gm, w.W, w.Kh, w.Ut, nullptr));
+    TC_TRY(cudaGetLastError());
+    SF_LAUNCH("tc_intra", st, tc_intra_kernel<DV><<<gc, 128, sm_intra, st>>>(s, q, k, dO, w.Gc, w.dVit));
     TC_TRY(cudaGetLastError());
     SF_LAUNCH("tc_scan_bwd", st, tc_scan_bwd_dual_kernel<DV, BETA><<<2 * s.BH * (DV / 64), 256, sm_scan, st>>>(
                                      s, q, dO, w.Gm, w.W, w.Kh, w.Ut, w.dVit, a.S_in, a.dS_out, w.Vnt, w.S0t,
@@ -1606,7 +1639,7 @@ cudaError_t tc_bwd(const SeqView& s, const BwdArgs& a, void* ws, cudaStream_t st
     return s.use_beta ? bwd_impl<64, true>(s, a, ws, st) : bwd_impl<64, false>(s, a, ws, st);
 }
 
-int tc_launches(bool) { return 3; }
+int tc_launches(bool backward) { return backward ? 4 : 3; }
 
 cudaError_t tc_device_status(int* status, bool clear) {
     cudaError_t e = cudaMemcpyFromSymbol(status, g_tc_status, sizeof(int));
