@@ -594,19 +594,24 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) get_frag(xslot(xch, cg, oth, kk, lane), sp[kk]);
         if (BETA) {
+            uint32_t bw[8][2][4];  // all B fragments of this phase, loaded before the first MMA
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {  // own state rows first, then the partner's
+            for (int j = 0; j < 8; ++j) {
                 const int kt = (j < 4) ? 4 * half + j : 4 * oth + (j - 4);
 #pragma unroll
-                for (int nn = 0; nn < 4; nn += 2) {
-                    uint32_t b[4];
-                    ldsm_x4(b, Ws + sw_off(Lnk, 8 * (4 * half + nn), 2 * kt, DK));
+                for (int n2 = 0; n2 < 2; ++n2) ldsm_x4(bw[j][n2], Ws + sw_off(Lnk, 8 * (4 * half + 2 * n2), 2 * kt, DK));
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {  // own state rows first, then the partner's
+#pragma unroll
+                for (int n2 = 0; n2 < 2; ++n2) {
+                    const uint32_t(&b)[4] = bw[j][n2];
                     if (j < 4) {
-                        mma(vn[nn], sa[j], b[0], b[1]);
-                        mma(vn[nn + 1], sa[j], b[2], b[3]);
+                        mma(vn[2 * n2], sa[j], b[0], b[1]);
+                        mma(vn[2 * n2 + 1], sa[j], b[2], b[3]);
                     } else {
-                        mma(vn[nn], sp[j - 4], b[0], b[1]);
-                        mma(vn[nn + 1], sp[j - 4], b[2], b[3]);
+                        mma(vn[2 * n2], sp[j - 4], b[0], b[1]);
+                        mma(vn[2 * n2 + 1], sp[j - 4], b[2], b[3]);
                     }
                 }
             }
@@ -624,19 +629,26 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
         for (int j = 0; j < 8; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) st[j][e] *= gamC;
+        {
+            uint32_t bk[4][4][4];  // all B fragments of Khat for this phase
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {  // token tiles: own first, then the partner's
-            const int kt = (j < 2) ? 2 * half + j : 2 * oth + (j - 2);
+            for (int j = 0; j < 4; ++j) {
+                const int kt = (j < 2) ? 2 * half + j : 2 * oth + (j - 2);
 #pragma unroll
-            for (int nn = 0; nn < 8; nn += 2) {
-                uint32_t b[4];
-                ldsm_x4_t(b, Khs + sw_off(Lkn, 16 * kt, 8 * half + nn, DK));
-                if (j < 2) {
-                    mma(st[nn], va[j], b[0], b[1]);
-                    mma(st[nn + 1], va[j], b[2], b[3]);
-                } else {
-                    mma(st[nn], vp[j - 2], b[0], b[1]);
-                    mma(st[nn + 1], vp[j - 2], b[2], b[3]);
+                for (int n2 = 0; n2 < 4; ++n2) ldsm_x4_t(bk[j][n2], Khs + sw_off(Lkn, 16 * kt, 8 * half + 2 * n2, DK));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {  // token tiles: own first, then the partner's
+#pragma unroll
+                for (int n2 = 0; n2 < 4; ++n2) {
+                    const uint32_t(&b)[4] = bk[j][n2];
+                    if (j < 2) {
+                        mma(st[2 * n2], va[j], b[0], b[1]);
+                        mma(st[2 * n2 + 1], va[j], b[2], b[3]);
+                    } else {
+                        mma(st[2 * n2], vp[j - 2], b[0], b[1]);
+                        mma(st[2 * n2 + 1], vp[j - 2], b[2], b[3]);
+                    }
                 }
             }
         }
@@ -792,19 +804,26 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
             dvn[nn][2] = u1.x;
             dvn[nn][3] = u1.y;
         }
+        {
+            uint32_t bk[8][2][4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int kt = (j < 4) ? 4 * half + j : 4 * oth + (j - 4);
+            for (int j = 0; j < 8; ++j) {
+                const int kt = (j < 4) ? 4 * half + j : 4 * oth + (j - 4);
 #pragma unroll
-            for (int nn = 0; nn < 4; nn += 2) {
-                uint32_t b[4];
-                ldsm_x4(b, Khs + sw_off(Lnk, 8 * (4 * half + nn), 2 * kt, DK));
-                if (j < 4) {
-                    mma(dvn[nn], da[j], b[0], b[1]);
-                    mma(dvn[nn + 1], da[j], b[2], b[3]);
-                } else {
-                    mma(dvn[nn], dp[j - 4], b[0], b[1]);
-                    mma(dvn[nn + 1], dp[j - 4], b[2], b[3]);
+                for (int n2 = 0; n2 < 2; ++n2) ldsm_x4(bk[j][n2], Khs + sw_off(Lnk, 8 * (4 * half + 2 * n2), 2 * kt, DK));
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+#pragma unroll
+                for (int n2 = 0; n2 < 2; ++n2) {
+                    const uint32_t(&b)[4] = bk[j][n2];
+                    if (j < 4) {
+                        mma(dvn[2 * n2], da[j], b[0], b[1]);
+                        mma(dvn[2 * n2 + 1], da[j], b[2], b[3]);
+                    } else {
+                        mma(dvn[2 * n2], dp[j - 4], b[0], b[1]);
+                        mma(dvn[2 * n2 + 1], dp[j - 4], b[2], b[3]);
+                    }
                 }
             }
         }
@@ -819,42 +838,53 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
 #pragma unroll
             for (int e = 0; e < 4; ++e) ds[j][e] *= gamC;
         // (scale gamma * dO)^T Q for this warp's state rows; independent of the chain
+        {
+            uint32_t ad[4][4], bq[4][4][4];
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            uint32_t a[4];
-            ldsm_x4_t(a, dOs + swz_at_off(16 * kk, vl, lane, 64));
-            const int tk = 16 * kk + 2 * tq;
-            const float g0 = s.scale * Gs[tk], g1 = s.scale * Gs[tk + 1];
-            const float g2 = s.scale * Gs[tk + 8], g3 = s.scale * Gs[tk + 9];
-            a[0] = scale2(a[0], g0, g1);
-            a[1] = scale2(a[1], g0, g1);
-            a[2] = scale2(a[2], g2, g3);
-            a[3] = scale2(a[3], g2, g3);
+            for (int kk = 0; kk < 4; ++kk) {
+                ldsm_x4_t(ad[kk], dOs + swz_at_off(16 * kk, vl, lane, 64));
 #pragma unroll
-            for (int nn = 0; nn < 8; nn += 2) {
-                uint32_t b[4];
-                ldsm_x4_t(b, Qs + sw_off(Lkn, 16 * kk, 8 * half + nn, DK));
-                mma(ds[nn], a, b[0], b[1]);
-                mma(ds[nn + 1], a, b[2], b[3]);
+                for (int n2 = 0; n2 < 4; ++n2) ldsm_x4_t(bq[kk][n2], Qs + sw_off(Lkn, 16 * kk, 8 * half + 2 * n2, DK));
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const int tk = 16 * kk + 2 * tq;
+                const float g0 = s.scale * Gs[tk], g1 = s.scale * Gs[tk + 1];
+                const float g2 = s.scale * Gs[tk + 8], g3 = s.scale * Gs[tk + 9];
+                uint32_t a[4];
+                a[0] = scale2(ad[kk][0], g0, g1);
+                a[1] = scale2(ad[kk][1], g0, g1);
+                a[2] = scale2(ad[kk][2], g2, g3);
+                a[3] = scale2(ad[kk][3], g2, g3);
+#pragma unroll
+                for (int n2 = 0; n2 < 4; ++n2) {
+                    mma(ds[2 * n2], a, bq[kk][n2][0], bq[kk][n2][1]);
+                    mma(ds[2 * n2 + 1], a, bq[kk][n2][2], bq[kk][n2][3]);
+                }
             }
         }
         pair_sync(cg);
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) get_frag(xslot(xch, cg, oth, 4 + kk, lane), vp[kk]);
         if (BETA) {
+            uint32_t bw[4][4][4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int kt = (j < 2) ? 2 * half + j : 2 * oth + (j - 2);
 #pragma unroll
-                for (int nn = 0; nn < 8; nn += 2) {
-                    uint32_t b[4];
-                    ldsm_x4_t(b, Ws + sw_off(Lkn, 16 * kt, 8 * half + nn, DK));
+                for (int n2 = 0; n2 < 4; ++n2) ldsm_x4_t(bw[j][n2], Ws + sw_off(Lkn, 16 * kt, 8 * half + 2 * n2, DK));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                for (int n2 = 0; n2 < 4; ++n2) {
+                    const uint32_t(&b)[4] = bw[j][n2];
                     if (j < 2) {
-                        mma(ds[nn], va[j], b[0], b[1]);
-                        mma(ds[nn + 1], va[j], b[2], b[3]);
+                        mma(ds[2 * n2], va[j], b[0], b[1]);
+                        mma(ds[2 * n2 + 1], va[j], b[2], b[3]);
                     } else {
-                        mma(ds[nn], vp[j - 2], b[0], b[1]);
-                        mma(ds[nn + 1], vp[j - 2], b[2], b[3]);
+                        mma(ds[2 * n2], vp[j - 2], b[0], b[1]);
+                        mma(ds[2 * n2 + 1], vp[j - 2], b[2], b[3]);
                     }
                 }
             }
