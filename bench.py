@@ -81,7 +81,7 @@ def kernel_work(name, w, T_seg):
         flops = nch * (2 * C * dk * dv + 2 * C * C * dk + 2 * C * C * dv)
         byts = n * (es * (2 * dk + dv)) + nch * dk * dv * 4
         return "hbm", flops, byts
-    if name.endswith("bwd_intra"):
+    if name.endswith("intra"):
         flops = nch * (2 * C * C * dk + 2 * C * C * dv)
         byts = n * (es * (2 * dk + dv) + wu * dv)
         return "hbm", flops, byts
@@ -307,9 +307,10 @@ def run_ours(args):
     rec = []
 
     def hook(name, after, stream_handle):
-        # every launch of this step goes to `stream` (the handle passed to the library)
+        # the library launches on its own streams (forked from `stream`); the
+        # events go on the stream the kernel is launched on
         ev = torch.cuda.Event(enable_timing=True)
-        ev.record(stream)
+        ev.record(torch.cuda.ExternalStream(stream_handle, device=dev))
         rec.append((name, after, ev))
 
     sf.set_launch_hook(hook)

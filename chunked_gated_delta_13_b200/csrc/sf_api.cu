@@ -194,6 +194,201 @@ bool segment_lengths(const sf_gdn_shape& s, int N, const int* seg_len, std::vect
     return true;
 }
 
+// Workspace of the pipelined segment chain (tensor-core path): N+1 boundary
+// states, two boundary state gradients (ping-pong), one keep region per
+// segment (the forward's intermediates, read again by that segment's
+// backward) and two slot regions (the backward's per-chunk tiles, used by
+// alternate segments).  Offsets from a 256-byte aligned base.
+struct PipeLayout {
+    size_t sstride, keep0, kstride, slot0, slstride, total;
+};
+
+PipeLayout pipe_layout(const sf_gdn_shape& s, const std::vector<int>& lens) {
+    PipeLayout L{};
+    const int N = (int)lens.size();
+    int lmax = 0;
+    for (int l : lens) lmax = l > lmax ? l : lmax;
+    const sf::SeqView v = make_view(s, lmax, s.T);
+    const size_t nstate = (size_t)s.B * s.H * s.dk * s.dv;
+    L.sstride = sf::align_up(nstate * sizeof(float), 256);
+    L.kstride = sf::tc_keep_bytes(v);
+    L.slstride = sf::tc_slot_bytes(v);
+    L.keep0 = L.sstride * (size_t)(N + 3);
+    L.slot0 = L.keep0 + L.kstride * (size_t)N;
+    L.total = L.slot0 + 2 * L.slstride;
+    return L;
+}
+
+// Two streams of one call, forked from and joined back to the caller's stream:
+// `chain` (highest priority) runs the state chains in order, `side` (lowest
+// priority) the chunk-parallel kernels, which fill the SMs the chains leave
+// idle.  Created per call and released asynchronously at its end, so nothing
+// outlives the call.
+struct Pipe {
+    cudaStream_t user = nullptr, chain = nullptr, side = nullptr;
+    enum { kFork, kPrep, kScan, kIntra, kBwdScan, kJoinChain, kJoinSide, kNumEv };
+    cudaEvent_t ev[kNumEv] = {};
+    cudaError_t open(cudaStream_t u) {
+        user = u;
+        int least = 0, greatest = 0;
+        cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+        if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&chain, cudaStreamNonBlocking, greatest);
+        if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&side, cudaStreamNonBlocking, least);
+        for (int i = 0; i < kNumEv && e == cudaSuccess; ++i)
+            e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventRecord(ev[kFork], user);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(chain, ev[kFork], 0);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev[kFork], 0);
+        return e;
+    }
+    // Stream dst waits for all work enqueued so far on src (through event i).
+    cudaError_t after(cudaStream_t dst, cudaStream_t src, int i) {
+        cudaError_t e = cudaEventRecord(ev[i], src);
+        return e == cudaSuccess ? cudaStreamWaitEvent(dst, ev[i], 0) : e;
+    }
+    cudaError_t join() {
+        cudaError_t e = after(user, chain, kJoinChain);
+        cudaError_t e2 = after(user, side, kJoinSide);
+        return e != cudaSuccess ? e : e2;
+    }
+    ~Pipe() {
+        for (cudaEvent_t x : ev)
+            if (x) cudaEventDestroy(x);
+        if (chain) cudaStreamDestroy(chain);
+        if (side) cudaStreamDestroy(side);
+    }
+};
+
+// The segment chain of the tensor-core path, pipelined: while the forward scan
+// of segment i runs on the chain stream, Pre of segment i+1 and Out of segment
+// i-1 run on the side stream; in the backward, OG of segment i-1 and PG of
+// segment i+1 run beside the reverse scan of segment i.  Each segment keeps its
+// forward intermediates, so the backward repeats neither Pre nor the forward
+// state recompute.  The kernels and their order within a segment are those of
+// sf_gdn_fwd / sf_gdn_bwd, so every result is bit-identical to the sequential
+// chain.
+sf_status segment_run_pipelined(const sf_gdn_shape& s, const std::vector<int>& lens, const sf::FwdArgs& F,
+                                const sf::BwdArgs* B, char* base, cudaStream_t user) {
+    const int N = (int)lens.size();
+    const size_t es = elem_size(s);
+    const size_t nstate = (size_t)s.B * s.H * s.dk * s.dv;
+    const PipeLayout L = pipe_layout(s, lens);
+    auto state = [&](int i) { return reinterpret_cast<float*>(base + L.sstride * (size_t)i); };
+    auto keep = [&](int i) { return static_cast<void*>(base + L.keep0 + L.kstride * (size_t)i); };
+    auto slot = [&](int i) { return static_cast<void*>(base + L.slot0 + L.slstride * (size_t)(i & 1)); };
+    std::vector<long long> t0(N);
+    long long t = 0;
+    for (int i = 0; i < N; ++i) {
+        t0[i] = t;
+        t += lens[i];
+    }
+    auto fargs = [&](int i) {
+        sf::FwdArgs a = F;
+        a.q = at_token(F.q, t0[i], s.dk, es);
+        a.k = at_token(F.k, t0[i], s.dk, es);
+        a.v = at_token(F.v, t0[i], s.dv, es);
+        a.o = at_token(F.o, t0[i], s.dv, es);
+        a.g = at_token(F.g, t0[i], 1, 4);
+        a.beta = at_token(F.beta, t0[i], 1, 4);
+        a.S_in = state(i);
+        a.S_out = state(i + 1);
+        return a;
+    };
+
+    Pipe p;
+    cudaError_t e = p.open(user);
+    const bool opened = e == cudaSuccess;
+    auto run = [&](sf::TcStage st, int i, const sf::FwdArgs* f, const sf::BwdArgs* b, cudaStream_t str) {
+        if (e != cudaSuccess) return;
+        const sf::SeqView v = make_view(s, lens[i], s.T);
+        e = sf::tc_stage(st, v, f, b, keep(i), slot(i), str);
+    };
+    auto chk = [&](cudaError_t x) {
+        if (e == cudaSuccess) e = x;
+    };
+    // Forward.  Side stream order: Pre 0, Pre 1, Out 0, Pre 2, Out 1, ...
+    if (e == cudaSuccess) chk(copy_state(state(0), F.S_in, nstate, p.chain));
+    std::vector<sf::FwdArgs> fa(N);
+    for (int i = 0; i < N; ++i) fa[i] = fargs(i);
+    auto issue_prep = [&](int i) {
+        if (lens[i] == 0) return;
+        run(sf::TcStage::Prep, i, &fa[i], nullptr, p.side);
+        if (e == cudaSuccess) chk(p.after(p.chain, p.side, Pipe::kPrep));
+    };
+    issue_prep(0);
+    for (int i = 0; i < N && e == cudaSuccess; ++i) {
+        if (lens[i] > 0) {
+            run(sf::TcStage::Scan, i, &fa[i], nullptr, p.chain);
+            if (e == cudaSuccess) chk(cudaEventRecord(p.ev[Pipe::kScan], p.chain));
+        } else {
+            chk(copy_state(state(i + 1), state(i), nstate, p.chain));
+        }
+        if (i + 1 < N) issue_prep(i + 1);
+        if (lens[i] > 0 && e == cudaSuccess) {
+            chk(cudaStreamWaitEvent(p.side, p.ev[Pipe::kScan], 0));
+            run(sf::TcStage::Out, i, &fa[i], nullptr, p.side);
+        }
+    }
+    if (F.S_out && e == cudaSuccess) chk(copy_state(F.S_out, state(N), nstate, p.chain));
+
+    // Backward.  Side stream order: OG N-1, OG N-2, PG N-1, OG N-3, PG N-2, ...
+    // The slot of segment i (dVi, dV_new, dS_C) is reused by segment i-2: OG of
+    // i-2 follows PG of i on the side stream, and the reverse scan of i-2
+    // waits for that OG, so nothing is overwritten while still being read.
+    if (B && e == cudaSuccess) {
+        float* cur = state(N + 1);
+        float* nxt = state(N + 2);
+        chk(copy_state(cur, B->dS_out, nstate, p.chain));
+        std::vector<sf::BwdArgs> ba(N);
+        for (int i = 0; i < N; ++i) {
+            sf::BwdArgs a = *B;
+            a.q = at_token(B->q, t0[i], s.dk, es);
+            a.k = at_token(B->k, t0[i], s.dk, es);
+            a.v = at_token(B->v, t0[i], s.dv, es);
+            a.dO = at_token(B->dO, t0[i], s.dv, es);
+            a.dq = at_token(B->dq, t0[i], s.dk, es);
+            a.dk = at_token(B->dk, t0[i], s.dk, es);
+            a.dv = at_token(B->dv, t0[i], s.dv, es);
+            a.g = at_token(B->g, t0[i], 1, 4);
+            a.beta = at_token(B->beta, t0[i], 1, 4);
+            a.dg = at_token(B->dg, t0[i], 1, 4);
+            a.dbeta = at_token(B->dbeta, t0[i], 1, 4);
+            a.S_in = state(i);
+            ba[i] = a;
+        }
+        auto issue_intra = [&](int i) {
+            if (lens[i] == 0) return;
+            run(sf::TcStage::Intra, i, nullptr, &ba[i], p.side);
+            if (e == cudaSuccess) chk(p.after(p.chain, p.side, Pipe::kIntra));
+        };
+        issue_intra(N - 1);
+        for (int i = N - 1; i >= 0 && e == cudaSuccess; --i) {
+            ba[i].dS_out = cur;
+            ba[i].dS_in = nxt;
+            if (lens[i] > 0) {
+                run(sf::TcStage::ScanBwd, i, nullptr, &ba[i], p.chain);
+                if (e == cudaSuccess) chk(cudaEventRecord(p.ev[Pipe::kBwdScan], p.chain));
+            } else {
+                chk(copy_state(nxt, cur, nstate, p.chain));
+            }
+            float* tmp = cur;
+            cur = nxt;
+            nxt = tmp;
+            if (i > 0) issue_intra(i - 1);
+            if (lens[i] > 0 && e == cudaSuccess) {
+                chk(cudaStreamWaitEvent(p.side, p.ev[Pipe::kBwdScan], 0));
+                run(sf::TcStage::Grad, i, nullptr, &ba[i], p.side);
+            }
+        }
+        if (B->dS_in && e == cudaSuccess) chk(copy_state(B->dS_in, cur, nstate, p.chain));
+    }
+    if (opened) {
+        const cudaError_t ej = p.join();
+        if (e == cudaSuccess) e = ej;
+    }
+    return e == cudaSuccess ? SF_OK : cuda_fail(e);
+}
+
 }  // namespace
 
 namespace sf {
@@ -266,6 +461,10 @@ size_t sf_segment_workspace_bytes(const sf_gdn_shape* s, int N, const int* seg_l
     if (check_shape(s) != SF_OK) return 0;
     std::vector<int> lens;
     if (!segment_lengths(*s, N, seg_len, lens)) return 0;
+    if (pick_path(*s) == Path::Tc) {
+        const PipeLayout L = pipe_layout(*s, lens);
+        return L.total + 256;
+    }
     size_t per = 0;
     for (int L : lens) {
         const size_t f = call_ws(*s, L, false), b = call_ws(*s, L, true);
@@ -298,6 +497,12 @@ sf_status sf_segment_run(const sf_gdn_shape* s, int N, const int* seg_len, const
     if (st != SF_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (s->B * s->H == 0) return SF_OK;
+    if (pick_path(*s) == Path::Tc) {
+        char* b = reinterpret_cast<char*>(sf::align_up(reinterpret_cast<uintptr_t>(ws), 256));
+        const sf::FwdArgs F{q, k, v, g, beta, S_in, o, S_out};
+        const sf::BwdArgs B{q, k, v, g, beta, S_in, dO, dS_out, dq, dk, dv, dg, dbeta, dS_in};
+        return segment_run_pipelined(*s, lens, F, dO ? &B : nullptr, b, cs);
+    }
 
     const size_t nstate = (size_t)s->B * s->H * s->dk * s->dv;
     const size_t sstride = sf::align_up(nstate * sizeof(float), 256);

@@ -52,9 +52,14 @@ struct TcWs {
     size_t total;
 };
 
-TcWs tc_layout(const SeqView& s, bool backward, char* base) {
+// The buffers fall in two parts: what the forward produces and the backward
+// reads again (Gc .. S0t, "keep"), and the backward's own tiles (dVit .. dSCt,
+// "slot").  Either base may be null to size the part.  Returns the bytes of
+// each part (multiples of 256; the bases must be 256-byte aligned).
+TcWs tc_parts(const SeqView& s, char* keep, char* slot, size_t* keep_bytes, size_t* slot_bytes) {
     TcWs w{};
     const size_t BH = s.BH, NC = s.NC, Tp = NC * C, DV = s.dv;
+    char* base = keep;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         char* p = base ? base + off : nullptr;
@@ -68,12 +73,23 @@ TcWs tc_layout(const SeqView& s, bool backward, char* base) {
     w.Ut = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
     w.Vnt = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
     w.S0t = reinterpret_cast<bf16*>(take(BH * NC * DV * DK * 2));
-    if (backward) {
-        w.dVit = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
-        w.dVnt = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
-        w.dSCt = reinterpret_cast<bf16*>(take(BH * NC * DV * DK * 2));
-    }
-    w.total = off + 256;
+    if (keep_bytes) *keep_bytes = off;
+    base = slot;
+    off = 0;
+    w.dVit = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
+    w.dVnt = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
+    w.dSCt = reinterpret_cast<bf16*>(take(BH * NC * DV * DK * 2));
+    if (slot_bytes) *slot_bytes = off;
+    return w;
+}
+
+// One call's workspace: the keep part, then (backward) the slot part.
+TcWs tc_layout(const SeqView& s, bool backward, char* base) {
+    size_t kb = 0, sb = 0;
+    tc_parts(s, nullptr, nullptr, &kb, &sb);
+    TcWs w = tc_parts(s, base, base ? base + kb : nullptr, nullptr, nullptr);
+    if (!backward) w.dVit = w.dVnt = w.dSCt = nullptr;
+    w.total = kb + (backward ? sb : 0) + 256;
     return w;
 }
 
@@ -927,9 +943,10 @@ tc_scan_fwd_kernel(SeqView s, const float* __restrict__ Gm, const bf16* __restri
     scan_fwd_cta<DV, BETA>(s, blockIdx.x / NVB, blockIdx.x % NVB, Gm, Wn, Kh, Ut, S_in, Vnt, S0t, S_out, smem);
 }
 
-// Backward chains in one launch: blocks [0, BH*DV/64) recompute the forward
-// states (V_new and the chunk-entry states), the rest run the reverse
-// state-gradient scan.  The two groups share no data.
+// Backward chains in one launch: with with_sr, blocks [0, BH*DV/64) recompute
+// the forward states (V_new and the chunk-entry states) and the rest run the
+// reverse state-gradient scan; the two groups share no data.  Without it (the
+// forward's states are kept), every block runs the reverse scan.
 template <int DV, bool BETA>
 __global__ void __launch_bounds__(256, 1)
 tc_scan_bwd_dual_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ dO,
@@ -937,10 +954,11 @@ tc_scan_bwd_dual_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __res
                         const bf16* __restrict__ Kh, const bf16* __restrict__ Ut,
                         const bf16* __restrict__ dVit, const float* __restrict__ S_in,
                         const float* __restrict__ dS_out, bf16* __restrict__ Vnt, bf16* __restrict__ S0t,
-                        bf16* __restrict__ dVnt, bf16* __restrict__ dSCt, float* __restrict__ dS_in) {
+                        bf16* __restrict__ dVnt, bf16* __restrict__ dSCt, float* __restrict__ dS_in,
+                        int with_sr) {
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int NVB = DV / 64;
-    const int nsr = s.BH * NVB;
+    const int nsr = with_sr ? s.BH * NVB : 0;
     int id = blockIdx.x;
     if (id < nsr) {
         scan_fwd_cta<DV, BETA>(s, id / NVB, id % NVB, Gm, Wn, Kh, Ut, S_in, Vnt, S0t, nullptr, smem);
@@ -1592,63 +1610,110 @@ cudaError_t smem_attr(K* kern, size_t bytes) {
         if (e_ != cudaSuccess) return e_;  \
     } while (0)
 
+// Launches of the stages.  `w` carries the buffers of one segment.
+template <int DV, bool BETA>
+cudaError_t launch_prep(const char* name, const SeqView& s, const bf16* k, const bf16* v, const float* g,
+                        const float* beta, const TcWs& w, cudaStream_t st) {
+    constexpr size_t sm = prep_smem<DV, false>();
+    TC_TRY(smem_attr(tc_prep_kernel<DV, BETA, false>, sm));
+    SF_LAUNCH(name, st, tc_prep_kernel<DV, BETA, false><<<dim3(s.NC, s.BH), 128, sm, st>>>(
+                            s, nullptr, k, v, g, beta, nullptr, w.Gc, w.Gm, w.W, w.Kh, w.Ut, nullptr));
+    return cudaGetLastError();
+}
+
+template <int DV, bool BETA>
+cudaError_t launch_scan_fwd(const SeqView& s, const float* S_in, float* S_out, const TcWs& w, cudaStream_t st) {
+    constexpr size_t sm = fwd_scan_smem<BETA>();
+    TC_TRY(smem_attr(tc_scan_fwd_kernel<DV, BETA>, sm));
+    SF_LAUNCH("tc_scan_fwd", st, tc_scan_fwd_kernel<DV, BETA><<<s.BH * (DV / 64), 256, sm, st>>>(
+                                     s, w.Gm, w.W, w.Kh, w.Ut, S_in, w.Vnt, w.S0t, S_out));
+    return cudaGetLastError();
+}
+
+template <int DV>
+cudaError_t launch_out(const SeqView& s, const bf16* q, const bf16* k, bf16* o, const TcWs& w, cudaStream_t st) {
+    constexpr size_t sm = out_smem<DV>();
+    TC_TRY(smem_attr(tc_out_kernel<DV>, sm));
+    SF_LAUNCH("tc_out", st, tc_out_kernel<DV><<<dim3(s.NC, s.BH), 128, sm, st>>>(s, q, k, w.Gc, w.Vnt, w.S0t, o));
+    return cudaGetLastError();
+}
+
+template <int DV>
+cudaError_t launch_intra(const SeqView& s, const bf16* q, const bf16* k, const bf16* dO, const TcWs& w,
+                         cudaStream_t st) {
+    constexpr size_t sm = intra_smem<DV>();
+    TC_TRY(smem_attr(tc_intra_kernel<DV>, sm));
+    SF_LAUNCH("tc_intra", st, tc_intra_kernel<DV><<<dim3(s.NC, s.BH), 128, sm, st>>>(s, q, k, dO, w.Gc, w.dVit));
+    return cudaGetLastError();
+}
+
+template <int DV, bool BETA>
+cudaError_t launch_scan_bwd(const SeqView& s, const BwdArgs& a, bool with_sr, const TcWs& w, cudaStream_t st) {
+    constexpr size_t sm_f = fwd_scan_smem<BETA>(), sm_b = bwd_scan_smem<BETA>();
+    constexpr size_t sm = sm_f > sm_b ? sm_f : sm_b;
+    TC_TRY(smem_attr(tc_scan_bwd_dual_kernel<DV, BETA>, sm));
+    const int nb = (with_sr ? 2 : 1) * s.BH * (DV / 64);
+    SF_LAUNCH("tc_scan_bwd", st, tc_scan_bwd_dual_kernel<DV, BETA><<<nb, 256, sm, st>>>(
+                                     s, static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.dO), w.Gm,
+                                     w.W, w.Kh, w.Ut, w.dVit, a.S_in, a.dS_out, w.Vnt, w.S0t, w.dVnt, w.dSCt,
+                                     a.dS_in, with_sr ? 1 : 0));
+    return cudaGetLastError();
+}
+
+template <int DV, bool BETA>
+cudaError_t launch_grad(const SeqView& s, const BwdArgs& a, const TcWs& w, cudaStream_t st) {
+    constexpr size_t sm = grad_smem<DV>();
+    TC_TRY(smem_attr(tc_grad_kernel<DV, BETA>, sm));
+    SF_LAUNCH("tc_grad", st, tc_grad_kernel<DV, BETA><<<dim3(s.NC, s.BH), 256, sm, st>>>(
+                                 s, static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k),
+                                 static_cast<const bf16*>(a.v), a.beta, static_cast<const bf16*>(a.dO), w.Gc,
+                                 w.Vnt, w.dVnt, w.S0t, w.dSCt, static_cast<bf16*>(a.dq), static_cast<bf16*>(a.dk),
+                                 static_cast<bf16*>(a.dv), a.dg, a.dbeta));
+    return cudaGetLastError();
+}
+
 template <int DV, bool BETA>
 cudaError_t fwd_impl(const SeqView& s, const FwdArgs& a, void* ws, cudaStream_t st) {
     char* base = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), 256));
-    TcWs w = tc_layout(s, false, base);
+    const TcWs w = tc_layout(s, false, base);
     const bf16* q = static_cast<const bf16*>(a.q);
     const bf16* k = static_cast<const bf16*>(a.k);
-    const bf16* v = static_cast<const bf16*>(a.v);
-    constexpr size_t sm_prep = prep_smem<DV, false>();
-    constexpr size_t sm_scan = fwd_scan_smem<BETA>();
-    constexpr size_t sm_out = out_smem<DV>();
-    TC_TRY(smem_attr(tc_prep_kernel<DV, BETA, false>, sm_prep));
-    TC_TRY(smem_attr(tc_scan_fwd_kernel<DV, BETA>, sm_scan));
-    TC_TRY(smem_attr(tc_out_kernel<DV>, sm_out));
-    const dim3 gc(s.NC, s.BH);
-    SF_LAUNCH("tc_prep", st, tc_prep_kernel<DV, BETA, false><<<gc, 128, sm_prep, st>>>(
-                                 s, q, k, v, a.g, a.beta, nullptr, w.Gc, w.Gm, w.W, w.Kh, w.Ut, nullptr));
-    TC_TRY(cudaGetLastError());
-    SF_LAUNCH("tc_scan_fwd", st, tc_scan_fwd_kernel<DV, BETA><<<s.BH * (DV / 64), 256, sm_scan, st>>>(
-                                     s, w.Gm, w.W, w.Kh, w.Ut, a.S_in, w.Vnt, w.S0t, a.S_out));
-    TC_TRY(cudaGetLastError());
-    SF_LAUNCH("tc_out", st, tc_out_kernel<DV><<<gc, 128, sm_out, st>>>(s, q, k, w.Gc, w.Vnt, w.S0t,
-                                                                         static_cast<bf16*>(a.o)));
-    return cudaGetLastError();
+    TC_TRY((launch_prep<DV, BETA>("tc_prep", s, k, static_cast<const bf16*>(a.v), a.g, a.beta, w, st)));
+    TC_TRY((launch_scan_fwd<DV, BETA>(s, a.S_in, a.S_out, w, st)));
+    return launch_out<DV>(s, q, k, static_cast<bf16*>(a.o), w, st);
 }
 
 template <int DV, bool BETA>
 cudaError_t bwd_impl(const SeqView& s, const BwdArgs& a, void* ws, cudaStream_t st) {
     char* base = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), 256));
-    TcWs w = tc_layout(s, true, base);
+    const TcWs w = tc_layout(s, true, base);
     const bf16* q = static_cast<const bf16*>(a.q);
     const bf16* k = static_cast<const bf16*>(a.k);
-    const bf16* v = static_cast<const bf16*>(a.v);
-    const bf16* dO = static_cast<const bf16*>(a.dO);
-    constexpr size_t sm_prep = prep_smem<DV, false>();
-    constexpr size_t sm_intra = intra_smem<DV>();
-    constexpr size_t sm_f = fwd_scan_smem<BETA>(), sm_b = bwd_scan_smem<BETA>();
-    constexpr size_t sm_scan = sm_f > sm_b ? sm_f : sm_b;
-    constexpr size_t sm_grad = grad_smem<DV>();
-    TC_TRY(smem_attr(tc_prep_kernel<DV, BETA, false>, sm_prep));
-    TC_TRY(smem_attr(tc_intra_kernel<DV>, sm_intra));
-    TC_TRY(smem_attr(tc_scan_bwd_dual_kernel<DV, BETA>, sm_scan));
-    TC_TRY(smem_attr(tc_grad_kernel<DV, BETA>, sm_grad));
-    const dim3 gc(s.NC, s.BH);
-    SF_LAUNCH("tc_prep_bwd", st, tc_prep_kernel<DV, BETA, false><<<gc, 128, sm_prep, st>>>(
-                                     s, q, k, v, a.g, a.beta, nullptr, w.Gc, w.Gm, w.W, w.Kh, w.Ut, nullptr));
-    TC_TRY(cudaGetLastError());
-    SF_LAUNCH("tc_intra", st, tc_intra_kernel<DV><<<gc, 128, sm_intra, st>>>(s, q, k, dO, w.Gc, w.dVit));
-    TC_TRY(cudaGetLastError());
-    SF_LAUNCH("tc_scan_bwd", st, tc_scan_bwd_dual_kernel<DV, BETA><<<2 * s.BH * (DV / 64), 256, sm_scan, st>>>(
-                                     s, q, dO, w.Gm, w.W, w.Kh, w.Ut, w.dVit, a.S_in, a.dS_out, w.Vnt, w.S0t,
-                                     w.dVnt, w.dSCt, a.dS_in));
-    TC_TRY(cudaGetLastError());
-    SF_LAUNCH("tc_grad", st, tc_grad_kernel<DV, BETA><<<gc, 256, sm_grad, st>>>(
-                                 s, q, k, v, a.beta, dO, w.Gc, w.Vnt, w.dVnt, w.S0t, w.dSCt,
-                                 static_cast<bf16*>(a.dq), static_cast<bf16*>(a.dk), static_cast<bf16*>(a.dv),
-                                 a.dg, a.dbeta));
-    return cudaGetLastError();
+    TC_TRY((launch_prep<DV, BETA>("tc_prep_bwd", s, k, static_cast<const bf16*>(a.v), a.g, a.beta, w, st)));
+    TC_TRY((launch_intra<DV>(s, q, k, static_cast<const bf16*>(a.dO), w, st)));
+    TC_TRY((launch_scan_bwd<DV, BETA>(s, a, true, w, st)));
+    return launch_grad<DV, BETA>(s, a, w, st);
+}
+
+template <int DV, bool BETA>
+cudaError_t stage_impl(TcStage stage, const SeqView& s, const FwdArgs* f, const BwdArgs* b, void* keep, void* slot,
+                       cudaStream_t st) {
+    const TcWs w = tc_parts(s, static_cast<char*>(keep), static_cast<char*>(slot), nullptr, nullptr);
+    switch (stage) {
+        case TcStage::Prep:
+            return launch_prep<DV, BETA>("tc_prep", s, static_cast<const bf16*>(f->k),
+                                         static_cast<const bf16*>(f->v), f->g, f->beta, w, st);
+        case TcStage::Scan: return launch_scan_fwd<DV, BETA>(s, f->S_in, f->S_out, w, st);
+        case TcStage::Out:
+            return launch_out<DV>(s, static_cast<const bf16*>(f->q), static_cast<const bf16*>(f->k),
+                                  static_cast<bf16*>(f->o), w, st);
+        case TcStage::Intra:
+            return launch_intra<DV>(s, static_cast<const bf16*>(b->q), static_cast<const bf16*>(b->k),
+                                    static_cast<const bf16*>(b->dO), w, st);
+        case TcStage::ScanBwd: return launch_scan_bwd<DV, BETA>(s, *b, false, w, st);
+        case TcStage::Grad: return launch_grad<DV, BETA>(s, *b, w, st);
+    }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -1658,6 +1723,27 @@ bool tc_supports(bool bf16_io, int dk, int dv, int Cc, bool) {
 }
 
 size_t tc_workspace_bytes(const SeqView& s, bool backward) { return tc_layout(s, backward, nullptr).total; }
+
+size_t tc_keep_bytes(const SeqView& s) {
+    size_t kb = 0;
+    tc_parts(s, nullptr, nullptr, &kb, nullptr);
+    return kb;
+}
+
+size_t tc_slot_bytes(const SeqView& s) {
+    size_t sb = 0;
+    tc_parts(s, nullptr, nullptr, nullptr, &sb);
+    return sb;
+}
+
+cudaError_t tc_stage(TcStage stage, const SeqView& s, const FwdArgs* f, const BwdArgs* b, void* keep, void* slot,
+                     cudaStream_t st) {
+    if (s.dv == 128)
+        return s.use_beta ? stage_impl<128, true>(stage, s, f, b, keep, slot, st)
+                          : stage_impl<128, false>(stage, s, f, b, keep, slot, st);
+    return s.use_beta ? stage_impl<64, true>(stage, s, f, b, keep, slot, st)
+                      : stage_impl<64, false>(stage, s, f, b, keep, slot, st);
+}
 
 cudaError_t tc_fwd(const SeqView& s, const FwdArgs& a, void* ws, cudaStream_t st) {
     if (s.dv == 128) return s.use_beta ? fwd_impl<128, true>(s, a, ws, st) : fwd_impl<128, false>(s, a, ws, st);
