@@ -196,9 +196,11 @@ bool segment_lengths(const sf_gdn_shape& s, int N, const int* seg_len, std::vect
 
 // Workspace of the pipelined segment chain (tensor-core path): N+1 boundary
 // states, two boundary state gradients (ping-pong), one keep region per
-// segment (the forward's intermediates, read again by that segment's
-// backward) and two slot regions (the backward's per-chunk tiles, used by
-// alternate segments).  Offsets from a 256-byte aligned base.
+// segment (what its forward and intra stages produce for its later stages)
+// and kSlots slot regions (the reverse scan's per-chunk tiles, used by
+// segments in turn).  Offsets from a 256-byte aligned base.
+constexpr int kSlots = 3;
+
 struct PipeLayout {
     size_t sstride, keep0, kstride, slot0, slstride, total;
 };
@@ -215,7 +217,7 @@ PipeLayout pipe_layout(const sf_gdn_shape& s, const std::vector<int>& lens) {
     L.slstride = sf::tc_slot_bytes(v);
     L.keep0 = L.sstride * (size_t)(N + 3);
     L.slot0 = L.keep0 + L.kstride * (size_t)N;
-    L.total = L.slot0 + 2 * L.slstride;
+    L.total = L.slot0 + kSlots * L.slstride;
     return L;
 }
 
@@ -226,7 +228,7 @@ PipeLayout pipe_layout(const sf_gdn_shape& s, const std::vector<int>& lens) {
 // outlives the call.
 struct Pipe {
     cudaStream_t user = nullptr, chain = nullptr, side = nullptr;
-    enum { kFork, kPrep, kScan, kIntra, kBwdScan, kJoinChain, kJoinSide, kNumEv };
+    enum { kFork, kPrep, kScan, kIntra, kBwdScan, kGrad0, kJoinChain = kGrad0 + kSlots, kJoinSide, kNumEv };
     cudaEvent_t ev[kNumEv] = {};
     cudaError_t open(cudaStream_t u) {
         user = u;
@@ -259,14 +261,14 @@ struct Pipe {
     }
 };
 
-// The segment chain of the tensor-core path, pipelined: while the forward scan
-// of segment i runs on the chain stream, Pre of segment i+1 and Out of segment
-// i-1 run on the side stream; in the backward, OG of segment i-1 and PG of
-// segment i+1 run beside the reverse scan of segment i.  Each segment keeps its
-// forward intermediates, so the backward repeats neither Pre nor the forward
-// state recompute.  The kernels and their order within a segment are those of
-// sf_gdn_fwd / sf_gdn_bwd, so every result is bit-identical to the sequential
-// chain.
+// The segment chain of the tensor-core path, pipelined.  Forward: while the
+// forward scan of segment i runs on the chain stream, Pre and the intra-chunk
+// output gradient (OG) of segment i+1 and Out of segment i-1 run on the side
+// stream.  Backward: the parallel gradients (PG) of segment i+1 run beside the
+// reverse scan of segment i.  Each segment keeps its forward intermediates, so
+// the backward repeats neither Pre nor the forward state recompute.  Every
+// kernel computes exactly what it computes in sf_gdn_fwd / sf_gdn_bwd, so the
+// results are bit-identical to the sequential chain.
 sf_status segment_run_pipelined(const sf_gdn_shape& s, const std::vector<int>& lens, const sf::FwdArgs& F,
                                 const sf::BwdArgs* B, char* base, cudaStream_t user) {
     const int N = (int)lens.size();
@@ -275,14 +277,16 @@ sf_status segment_run_pipelined(const sf_gdn_shape& s, const std::vector<int>& l
     const PipeLayout L = pipe_layout(s, lens);
     auto state = [&](int i) { return reinterpret_cast<float*>(base + L.sstride * (size_t)i); };
     auto keep = [&](int i) { return static_cast<void*>(base + L.keep0 + L.kstride * (size_t)i); };
-    auto slot = [&](int i) { return static_cast<void*>(base + L.slot0 + L.slstride * (size_t)(i & 1)); };
+    auto slot = [&](int i) { return static_cast<void*>(base + L.slot0 + L.slstride * (size_t)(i % kSlots)); };
     std::vector<long long> t0(N);
     long long t = 0;
     for (int i = 0; i < N; ++i) {
         t0[i] = t;
         t += lens[i];
     }
-    auto fargs = [&](int i) {
+    std::vector<sf::FwdArgs> fa(N);
+    std::vector<sf::BwdArgs> ba(B ? N : 0);
+    for (int i = 0; i < N; ++i) {
         sf::FwdArgs a = F;
         a.q = at_token(F.q, t0[i], s.dk, es);
         a.k = at_token(F.k, t0[i], s.dk, es);
@@ -292,95 +296,101 @@ sf_status segment_run_pipelined(const sf_gdn_shape& s, const std::vector<int>& l
         a.beta = at_token(F.beta, t0[i], 1, 4);
         a.S_in = state(i);
         a.S_out = state(i + 1);
-        return a;
-    };
+        fa[i] = a;
+        if (!B) continue;
+        sf::BwdArgs b = *B;
+        b.q = a.q;
+        b.k = a.k;
+        b.v = a.v;
+        b.g = a.g;
+        b.beta = a.beta;
+        b.dO = at_token(B->dO, t0[i], s.dv, es);
+        b.dq = at_token(B->dq, t0[i], s.dk, es);
+        b.dk = at_token(B->dk, t0[i], s.dk, es);
+        b.dv = at_token(B->dv, t0[i], s.dv, es);
+        b.dg = at_token(B->dg, t0[i], 1, 4);
+        b.dbeta = at_token(B->dbeta, t0[i], 1, 4);
+        b.S_in = state(i);
+        ba[i] = b;
+    }
 
     Pipe p;
     cudaError_t e = p.open(user);
     const bool opened = e == cudaSuccess;
-    auto run = [&](sf::TcStage st, int i, const sf::FwdArgs* f, const sf::BwdArgs* b, cudaStream_t str) {
-        if (e != cudaSuccess) return;
-        const sf::SeqView v = make_view(s, lens[i], s.T);
-        e = sf::tc_stage(st, v, f, b, keep(i), slot(i), str);
-    };
     auto chk = [&](cudaError_t x) {
         if (e == cudaSuccess) e = x;
     };
-    // Forward.  Side stream order: Pre 0, Pre 1, Out 0, Pre 2, Out 1, ...
-    if (e == cudaSuccess) chk(copy_state(state(0), F.S_in, nstate, p.chain));
-    std::vector<sf::FwdArgs> fa(N);
-    for (int i = 0; i < N; ++i) fa[i] = fargs(i);
+    auto run = [&](sf::TcStage st, int i, cudaStream_t str) {
+        if (e != cudaSuccess) return;
+        const sf::SeqView v = make_view(s, lens[i], s.T);
+        e = sf::tc_stage(st, v, &fa[i], B ? &ba[i] : nullptr, keep(i), slot(i), str);
+    };
+    auto wait = [&](cudaStream_t dst, int i) {
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(dst, p.ev[i], 0);
+    };
+    auto record = [&](cudaStream_t src, int i) {
+        if (e == cudaSuccess) e = cudaEventRecord(p.ev[i], src);
+    };
+
+    // Forward.  Side stream order: Pre 0, OG 0, Pre 1, OG 1, Out 0, Pre 2, OG 2, Out 1, ...
+    bool any_intra = false;
     auto issue_prep = [&](int i) {
         if (lens[i] == 0) return;
-        run(sf::TcStage::Prep, i, &fa[i], nullptr, p.side);
-        if (e == cudaSuccess) chk(p.after(p.chain, p.side, Pipe::kPrep));
+        run(sf::TcStage::Prep, i, p.side);
+        record(p.side, Pipe::kPrep);
+        wait(p.chain, Pipe::kPrep);
+        if (B) {
+            run(sf::TcStage::Intra, i, p.side);
+            record(p.side, Pipe::kIntra);
+            any_intra = true;
+        }
     };
+    chk(copy_state(state(0), F.S_in, nstate, p.chain));
     issue_prep(0);
     for (int i = 0; i < N && e == cudaSuccess; ++i) {
         if (lens[i] > 0) {
-            run(sf::TcStage::Scan, i, &fa[i], nullptr, p.chain);
-            if (e == cudaSuccess) chk(cudaEventRecord(p.ev[Pipe::kScan], p.chain));
+            run(sf::TcStage::Scan, i, p.chain);
+            record(p.chain, Pipe::kScan);
         } else {
             chk(copy_state(state(i + 1), state(i), nstate, p.chain));
         }
         if (i + 1 < N) issue_prep(i + 1);
-        if (lens[i] > 0 && e == cudaSuccess) {
-            chk(cudaStreamWaitEvent(p.side, p.ev[Pipe::kScan], 0));
-            run(sf::TcStage::Out, i, &fa[i], nullptr, p.side);
+        if (lens[i] > 0) {
+            wait(p.side, Pipe::kScan);
+            run(sf::TcStage::Out, i, p.side);
         }
     }
-    if (F.S_out && e == cudaSuccess) chk(copy_state(F.S_out, state(N), nstate, p.chain));
+    if (F.S_out) chk(copy_state(F.S_out, state(N), nstate, p.chain));
 
-    // Backward.  Side stream order: OG N-1, OG N-2, PG N-1, OG N-3, PG N-2, ...
-    // The slot of segment i (dVi, dV_new, dS_C) is reused by segment i-2: OG of
-    // i-2 follows PG of i on the side stream, and the reverse scan of i-2
-    // waits for that OG, so nothing is overwritten while still being read.
+    // Backward.  The reverse scans wait once for the last OG (the side stream
+    // ran every OG before it).  The slot of segment i (dV_new, dS_C) is next
+    // written by the reverse scan of segment i - kSlots, which waits for the
+    // PG that last read it.
     if (B && e == cudaSuccess) {
         float* cur = state(N + 1);
         float* nxt = state(N + 2);
         chk(copy_state(cur, B->dS_out, nstate, p.chain));
-        std::vector<sf::BwdArgs> ba(N);
-        for (int i = 0; i < N; ++i) {
-            sf::BwdArgs a = *B;
-            a.q = at_token(B->q, t0[i], s.dk, es);
-            a.k = at_token(B->k, t0[i], s.dk, es);
-            a.v = at_token(B->v, t0[i], s.dv, es);
-            a.dO = at_token(B->dO, t0[i], s.dv, es);
-            a.dq = at_token(B->dq, t0[i], s.dk, es);
-            a.dk = at_token(B->dk, t0[i], s.dk, es);
-            a.dv = at_token(B->dv, t0[i], s.dv, es);
-            a.g = at_token(B->g, t0[i], 1, 4);
-            a.beta = at_token(B->beta, t0[i], 1, 4);
-            a.dg = at_token(B->dg, t0[i], 1, 4);
-            a.dbeta = at_token(B->dbeta, t0[i], 1, 4);
-            a.S_in = state(i);
-            ba[i] = a;
-        }
-        auto issue_intra = [&](int i) {
-            if (lens[i] == 0) return;
-            run(sf::TcStage::Intra, i, nullptr, &ba[i], p.side);
-            if (e == cudaSuccess) chk(p.after(p.chain, p.side, Pipe::kIntra));
-        };
-        issue_intra(N - 1);
+        if (any_intra) wait(p.chain, Pipe::kIntra);
+        bool slot_read[kSlots] = {};
         for (int i = N - 1; i >= 0 && e == cudaSuccess; --i) {
             ba[i].dS_out = cur;
             ba[i].dS_in = nxt;
             if (lens[i] > 0) {
-                run(sf::TcStage::ScanBwd, i, nullptr, &ba[i], p.chain);
-                if (e == cudaSuccess) chk(cudaEventRecord(p.ev[Pipe::kBwdScan], p.chain));
+                if (slot_read[i % kSlots]) wait(p.chain, Pipe::kGrad0 + i % kSlots);
+                run(sf::TcStage::ScanBwd, i, p.chain);
+                record(p.chain, Pipe::kBwdScan);
+                wait(p.side, Pipe::kBwdScan);
+                run(sf::TcStage::Grad, i, p.side);
+                record(p.side, Pipe::kGrad0 + i % kSlots);
+                slot_read[i % kSlots] = true;
             } else {
                 chk(copy_state(nxt, cur, nstate, p.chain));
             }
             float* tmp = cur;
             cur = nxt;
             nxt = tmp;
-            if (i > 0) issue_intra(i - 1);
-            if (lens[i] > 0 && e == cudaSuccess) {
-                chk(cudaStreamWaitEvent(p.side, p.ev[Pipe::kBwdScan], 0));
-                run(sf::TcStage::Grad, i, nullptr, &ba[i], p.side);
-            }
         }
-        if (B->dS_in && e == cudaSuccess) chk(copy_state(B->dS_in, cur, nstate, p.chain));
+        if (B->dS_in) chk(copy_state(B->dS_in, cur, nstate, p.chain));
     }
     if (opened) {
         const cudaError_t ej = p.join();

@@ -42,6 +42,7 @@ struct TcWs {
     float* Gc;   // [BH][Tp]           chunk-local cumulative log-decay G
     float* Gm;   // [BH][Tp]           exp(G)
     bf16* W;     // [BH][Tp][DK]       -W (negated: the scans only ever subtract W products; permuted, see swz)
+    float* Lm;   // [BH][NC][C][C]     L = (I + A)^{-1} per chunk (delta path), for the gradient kernel
     bf16* Kh;    // [BH][Tp][DK]       K * exp(G_C - G) (permuted)
     bf16* Ut;    // [BH][NC][DV][C]    U transposed per chunk, V^T without the beta path (permuted)
     bf16* Vnt;   // [BH][NC][DV][C]    V_new transposed per chunk (pieces permuted, see swz)
@@ -49,14 +50,17 @@ struct TcWs {
     bf16* dVit;  // [BH][NC][DV][C]    intra-chunk part of dV_new, transposed (permuted)
     bf16* dVnt;  // [BH][NC][DV][C]    dV_new transposed (permuted)
     bf16* dSCt;  // [BH][NC][DV][DK]   gradient of the state leaving each chunk, transposed (permuted)
+    bf16* Dt;    // [BH][NC][DV][DK]   scale (gamma * dO)^T Q per chunk, transposed (permuted)
     size_t total;
 };
 
-// The buffers fall in two parts: what the forward produces and the backward
-// reads again (Gc .. S0t, "keep"), and the backward's own tiles (dVit .. dSCt,
-// "slot").  Either base may be null to size the part.  Returns the bytes of
-// each part (multiples of 256; the bases must be 256-byte aligned).
-TcWs tc_parts(const SeqView& s, char* keep, char* slot, size_t* keep_bytes, size_t* slot_bytes) {
+// The buffers fall in three parts: what the forward produces and the
+// backward reads again (Gc .. S0t, "keep"), what the intra-chunk kernel of the
+// backward produces for the reverse scan (dVit, Dt, "og"), and the reverse
+// scan's own tiles (dVnt, dSCt, "slot").  A base may be null to size its part.
+// Returns the bytes of each part (multiples of 256; bases 256-byte aligned).
+TcWs tc_parts(const SeqView& s, char* keep, char* og, char* slot, size_t* keep_bytes, size_t* og_bytes,
+              size_t* slot_bytes) {
     TcWs w{};
     const size_t BH = s.BH, NC = s.NC, Tp = NC * C, DV = s.dv;
     char* base = keep;
@@ -69,27 +73,33 @@ TcWs tc_parts(const SeqView& s, char* keep, char* slot, size_t* keep_bytes, size
     w.Gc = reinterpret_cast<float*>(take(BH * Tp * 4));
     w.Gm = reinterpret_cast<float*>(take(BH * Tp * 4));
     w.W = reinterpret_cast<bf16*>(take(s.use_beta ? BH * Tp * DK * 2 : 0));
+    w.Lm = reinterpret_cast<float*>(take(s.use_beta ? BH * NC * C * C * 4 : 0));
     w.Kh = reinterpret_cast<bf16*>(take(BH * Tp * DK * 2));
     w.Ut = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
     w.Vnt = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
     w.S0t = reinterpret_cast<bf16*>(take(BH * NC * DV * DK * 2));
     if (keep_bytes) *keep_bytes = off;
-    base = slot;
+    base = og;
     off = 0;
     w.dVit = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
+    w.Dt = reinterpret_cast<bf16*>(take(BH * NC * DV * DK * 2));
+    if (og_bytes) *og_bytes = off;
+    base = slot;
+    off = 0;
     w.dVnt = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
     w.dSCt = reinterpret_cast<bf16*>(take(BH * NC * DV * DK * 2));
     if (slot_bytes) *slot_bytes = off;
     return w;
 }
 
-// One call's workspace: the keep part, then (backward) the slot part.
+// One call's workspace: the keep part, then (backward) the og and slot parts.
 TcWs tc_layout(const SeqView& s, bool backward, char* base) {
-    size_t kb = 0, sb = 0;
-    tc_parts(s, nullptr, nullptr, &kb, &sb);
-    TcWs w = tc_parts(s, base, base ? base + kb : nullptr, nullptr, nullptr);
-    if (!backward) w.dVit = w.dVnt = w.dSCt = nullptr;
-    w.total = kb + (backward ? sb : 0) + 256;
+    size_t kb = 0, ob = 0, sb = 0;
+    tc_parts(s, nullptr, nullptr, nullptr, &kb, &ob, &sb);
+    TcWs w = tc_parts(s, base, base ? base + kb : nullptr, base ? base + kb + ob : nullptr, nullptr, nullptr,
+                      nullptr);
+    if (!backward) w.dVit = w.dVnt = w.dSCt = w.Dt = nullptr;
+    w.total = kb + (backward ? ob + sb : 0) + 256;
     return w;
 }
 
@@ -182,15 +192,15 @@ constexpr size_t prep_smem() {
            (size_t)C * LDF * 4 * 2 + (size_t)C * LDC * 2 * 2 + 768 * 4 + 2 * C * 4;
 }
 
-// One CTA (4 warps) per (chunk, head).  Writes G, Khat, W, U^T; in backward
+// One CTA (8 warps: rows 16*(w%4), column half w/4) per (chunk, head).  Writes G, Khat, W, U^T; in backward
 // mode also dVi^T = (P^T dO)^T with P = scale (Q K^T) * Gamma.
 template <int DV, bool BETA, bool BWD>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
 tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
                const bf16* __restrict__ v, const float* __restrict__ g,
                const float* __restrict__ beta, const bf16* __restrict__ dO, float* __restrict__ Gc,
-               float* __restrict__ Gmo, bf16* __restrict__ Wo, bf16* __restrict__ Kho, bf16* __restrict__ Uto,
-               bf16* __restrict__ dVito) {
+               float* __restrict__ Gmo, bf16* __restrict__ Wo, float* __restrict__ Lmo, bf16* __restrict__ Kho,
+               bf16* __restrict__ Uto, bf16* __restrict__ dVito) {
     constexpr int LDV = DV + 8;
     extern __shared__ __align__(16) unsigned char smem[];
     bf16* Ks = reinterpret_cast<bf16*>(smem);
@@ -207,29 +217,30 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 
     const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int gq = lane >> 2, tq = lane & 3;
+    const int mw = w & 3, nw = w >> 2;
     const int t0 = c * C;
     const int nval = min(C, s.T - t0);
     const size_t Tp = (size_t)s.NC * C;
-    load_tile<C, DK, 128>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
-    load_tile<C, DV, 128>(Vs, LDV, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+    load_tile<C, DK, 256>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+    load_tile<C, DV, 256>(Vs, LDV, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
     if (BWD) {
-        load_tile<C, DK, 128>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
-        load_tile<C, DV, 128>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+        load_tile<C, DK, 256>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+        load_tile<C, DV, 256>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
     }
     cp_async_commit();
     if (w == 0) chunk_cumsum(g + bh * s.hs_g + t0, nval, Gs, lane);
-    for (int i = tid; i < C; i += 128) Bs[i] = (BETA && i < nval) ? beta[bh * s.hs_g + t0 + i] : 0.f;
+    for (int i = tid; i < C; i += 256) Bs[i] = (BETA && i < nval) ? beta[bh * s.hs_g + t0 + i] : 0.f;
     if (BETA)
-        for (int e = tid; e < C * LDF; e += 128) Lf[e] = 0.f;
+        for (int e = tid; e < C * LDF; e += 256) Lf[e] = 0.f;
     cp_async_wait<0>();
     __syncthreads();
 
-    for (int i = tid; i < C; i += 128) {
+    for (int i = tid; i < C; i += 256) {
         Gc[bh * Tp + t0 + i] = Gs[i];
         Gmo[bh * Tp + t0 + i] = __expf(Gs[i]);
     }
     const float gC = Gs[C - 1];
-    for (int e = tid; e < C * (DK / 8); e += 128) {
+    for (int e = tid; e < C * (DK / 8); e += 256) {
         const int r = e >> 4, cc = (e & 15) * 8;
         const float d = __expf(gC - Gs[r]);
         uint4 x = *reinterpret_cast<const uint4*>(Ks + r * LDK + cc);
@@ -243,30 +254,35 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     bf16* Ust = reinterpret_cast<bf16*>(Lf);  // [DV][LDC]
     if (BETA) {
         {  // A = strictly-lower(diag(beta) (K K^T * Gamma))
-            float acc[8][4] = {};
+            float acc[4][4] = {};
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 uint32_t a[4];
-                ldA(a, Ks, LDK, 16 * w, 16 * kk, lane);
+                ldA(a, Ks, LDK, 16 * mw, 16 * kk, lane);
 #pragma unroll
-                for (int nn = 0; nn < 8; nn += 2) {
+                for (int nn = 0; nn < 4; nn += 2) {
                     uint32_t b[4];
-                    ldBnk(b, Ks, LDK, 8 * nn, 16 * kk, lane);
+                    ldBnk(b, Ks, LDK, 32 * nw + 8 * nn, 16 * kk, lane);
                     mma(acc[nn], a, b[0], b[1]);
                     mma(acc[nn + 1], a, b[2], b[3]);
                 }
             }
 #pragma unroll
-            for (int nn = 0; nn < 8; ++nn)
+            for (int nn = 0; nn < 4; ++nn)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int i = 16 * w + gq + 8 * (e >> 1), j = 8 * nn + 2 * tq + (e & 1);
+                    const int i = 16 * mw + gq + 8 * (e >> 1), j = 32 * nw + 8 * nn + 2 * tq + (e & 1);
                     Af[i * LDF + j] = (j < i) ? Bs[i] * __expf(Gs[i] - Gs[j]) * acc[nn][e] : 0.f;
                 }
         }
         __syncthreads();
-        block_inverse(Af, LDF, Lf, LDF, Yb, tid, 128);
-        for (int e = tid; e < C * C; e += 128) {
+        block_inverse(Af, LDF, Lf, LDF, Yb, tid, 256);
+        float* Lg = Lmo + ((size_t)bh * s.NC + c) * C * C;
+        for (int e = tid; e < C * C / 4; e += 256) {
+            const int i = e >> 4, j = (e & 15) * 4;
+            *reinterpret_cast<float4*>(Lg + i * C + j) = *reinterpret_cast<const float4*>(Lf + i * LDF + j);
+        }
+        for (int e = tid; e < C * C; e += 256) {
             const int i = e >> 6, j = e & 63;
             const float l = Lf[i * LDF + j];
             Tw[i * LDC + j] = __float2bfloat16_rn(l * Bs[j] * __expf(Gs[j]));
@@ -275,63 +291,63 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         __syncthreads();
         bf16* Wst = reinterpret_cast<bf16*>(Af);  // [C][LDK]
         {  // W = T (gamma * K), staged negated
-            float acc[16][4] = {};
+            float acc[8][4] = {};
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 uint32_t a[4];
-                ldA(a, Tw, LDC, 16 * w, 16 * kk, lane);
+                ldA(a, Tw, LDC, 16 * mw, 16 * kk, lane);
 #pragma unroll
-                for (int nn = 0; nn < 16; nn += 2) {
+                for (int nn = 0; nn < 8; nn += 2) {
                     uint32_t b[4];
-                    ldBkn(b, Ks, LDK, 8 * nn, 16 * kk, lane);
+                    ldBkn(b, Ks, LDK, 64 * nw + 8 * nn, 16 * kk, lane);
                     mma(acc[nn], a, b[0], b[1]);
                     mma(acc[nn + 1], a, b[2], b[3]);
                 }
             }
 #pragma unroll
-            for (int nn = 0; nn < 16; ++nn) {
-                const int i = 16 * w + gq, col = 8 * nn + 2 * tq;
+            for (int nn = 0; nn < 8; ++nn) {
+                const int i = 16 * mw + gq, col = 64 * nw + 8 * nn + 2 * tq;
                 *reinterpret_cast<uint32_t*>(Wst + i * LDK + col) = pack(-acc[nn][0], -acc[nn][1]);
                 *reinterpret_cast<uint32_t*>(Wst + (i + 8) * LDK + col) = pack(-acc[nn][2], -acc[nn][3]);
             }
         }
         {  // U = T V, staged transposed
-            float acc[DV / 8][4] = {};
+            float acc[DV / 16][4] = {};
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 uint32_t a[4];
-                ldA(a, Tu, LDC, 16 * w, 16 * kk, lane);
+                ldA(a, Tu, LDC, 16 * mw, 16 * kk, lane);
 #pragma unroll
-                for (int nn = 0; nn < DV / 8; nn += 2) {
+                for (int nn = 0; nn < DV / 16; nn += 2) {
                     uint32_t b[4];
-                    ldBkn(b, Vs, LDV, 8 * nn, 16 * kk, lane);
+                    ldBkn(b, Vs, LDV, (DV / 2) * nw + 8 * nn, 16 * kk, lane);
                     mma(acc[nn], a, b[0], b[1]);
                     mma(acc[nn + 1], a, b[2], b[3]);
                 }
             }
 #pragma unroll
-            for (int nn = 0; nn < DV / 8; ++nn)
+            for (int nn = 0; nn < DV / 16; ++nn)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int i = 16 * w + gq + 8 * (e >> 1), col = 8 * nn + 2 * tq + (e & 1);
+                    const int i = 16 * mw + gq + 8 * (e >> 1), col = (DV / 2) * nw + 8 * nn + 2 * tq + (e & 1);
                     Ust[col * LDC + i] = __float2bfloat16_rn(acc[nn][e]);
                 }
         }
         __syncthreads();
-        for (int e = tid; e < C * (DK / 8); e += 128) {
+        for (int e = tid; e < C * (DK / 8); e += 256) {
             const int r = e >> 4, cc = (e & 15) * 8;
             *reinterpret_cast<uint4*>(Wo + (bh * Tp + t0) * DK + swz(r, cc, DK)) =
                 *reinterpret_cast<const uint4*>(Wst + r * LDK + cc);
         }
     } else {
-        for (int e = tid; e < C * DV; e += 128) {
+        for (int e = tid; e < C * DV; e += 256) {
             const int i = e / DV, col = e % DV;
             Ust[col * LDC + i] = Vs[i * LDV + col];
         }
         __syncthreads();
     }
     bf16* Utg = Uto + ((size_t)bh * s.NC + c) * DV * C;
-    for (int e = tid; e < DV * (C / 8); e += 128) {
+    for (int e = tid; e < DV * (C / 8); e += 256) {
         const int r = e >> 3, cc = (e & 7) * 8;
         *reinterpret_cast<uint4*>(Utg + swz(r, cc, C)) = *reinterpret_cast<const uint4*>(Ust + r * LDC + cc);
     }
@@ -344,11 +360,12 @@ constexpr size_t intra_smem() {
 }
 
 // Intra-chunk output gradient (OG): dVi^T = (P^T dO)^T with
-// P = scale (Q K^T) * Gamma, one CTA (4 warps) per (chunk, head).
+// P = scale (Q K^T) * Gamma, and the chain-independent term of the reverse
+// state scan, D^T = (scale (gamma * dO)^T Q)^T; one CTA (4 warps) per (chunk, head).
 template <int DV>
 __global__ void __launch_bounds__(128)
 tc_intra_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ dO,
-                const float* __restrict__ Gc, bf16* __restrict__ dVito) {
+                const float* __restrict__ Gc, bf16* __restrict__ dVito, bf16* __restrict__ Dto) {
     constexpr int LDV = DV + 8;
     extern __shared__ __align__(16) unsigned char smem[];
     bf16* Qs = reinterpret_cast<bf16*>(smem);
@@ -418,6 +435,44 @@ tc_intra_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
             *reinterpret_cast<uint32_t*>(dst + swz(r + 8, j, C)) = pack(acc[nn][2], acc[nn][3]);
         }
     }
+    // D^T[v][d] = sum_t scale gamma_t dO[t][v] Q[t][d]
+    bf16* dd = Dto + ((size_t)bh * s.NC + c) * DV * DK;
+#pragma unroll 1
+    for (int mt = 0; mt < MT; ++mt) {
+        const int m0 = (w * MT + mt) * 16;
+        uint32_t a[4][4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            ldAt(a[kk], dOs, LDV, m0, 16 * kk, lane);
+            const int tk = 16 * kk + 2 * tq;
+            const float g0 = s.scale * __expf(Gs[tk]), g1 = s.scale * __expf(Gs[tk + 1]);
+            const float g2 = s.scale * __expf(Gs[tk + 8]), g3 = s.scale * __expf(Gs[tk + 9]);
+            a[kk][0] = scale2(a[kk][0], g0, g1);
+            a[kk][1] = scale2(a[kk][1], g0, g1);
+            a[kk][2] = scale2(a[kk][2], g2, g3);
+            a[kk][3] = scale2(a[kk][3], g2, g3);
+        }
+#pragma unroll 1
+        for (int nh = 0; nh < 2; ++nh) {
+            float acc[8][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                for (int nn = 0; nn < 8; nn += 2) {
+                    uint32_t b[4];
+                    ldBkn(b, Qs, LDK, 64 * nh + 8 * nn, 16 * kk, lane);
+                    mma(acc[nn], a[kk], b[0], b[1]);
+                    mma(acc[nn + 1], a[kk], b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int nn = 0; nn < 8; ++nn) {
+                const int r = m0 + gq, d = 64 * nh + 8 * nn + 2 * tq;
+                *reinterpret_cast<uint32_t*>(dd + swz(r, d, DK)) = pack(acc[nn][0], acc[nn][1]);
+                *reinterpret_cast<uint32_t*>(dd + swz(r + 8, d, DK)) = pack(acc[nn][2], acc[nn][3]);
+            }
+        }
+    }
 }
 
 // ------------------------------------------------------------ state scans ---
@@ -431,8 +486,8 @@ constexpr size_t fwd_stage_bytes() {
     return (size_t)kTileK * (BETA ? 2 : 1) + kTileV + C * 4;
 }
 template <bool BETA>
-constexpr size_t bwd_stage_bytes() {  // + Q and dO tiles copied per thread (permuted, see swz)
-    return (size_t)kTileK * (BETA ? 2 : 1) + kTileV + C * 4 + kTileK + (size_t)C * 64 * 2;
+constexpr size_t bwd_stage_bytes() {  // + the 64 rows of D^T of this block
+    return (size_t)kTileK * (BETA ? 2 : 1) + kTileV + C * 4 + kTileK;
 }
 // Output staging of one chunk step of a 64-column block: the state tile
 // (64 x DK) and the value tile (64 x C), in the permuted layout of swz().
@@ -701,14 +756,14 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
 // dS^T <- gamma_C dS^T + dO^T (scale gamma * Q) + dV_new^T (-W).
 // Outputs dV_new^T and dS_C^T per chunk (bf16, staged and bulk-stored), dS_in (fp32).
 template <int DV, bool BETA>
-__device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, const bf16* __restrict__ q,
-                                             const bf16* __restrict__ dO, const float* __restrict__ Gm,
+__device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, const bf16* __restrict__ Dt,
+                                             const float* __restrict__ Gm,
                                              const bf16* __restrict__ Wn, const bf16* __restrict__ Kh,
                                              const bf16* __restrict__ dVit, const float* __restrict__ dS_out,
                                              bf16* __restrict__ dVnt, bf16* __restrict__ dSCt,
                                              float* __restrict__ dS_in, unsigned char* smem) {
     constexpr size_t STAGE = bwd_stage_bytes<BETA>();
-    constexpr uint32_t TX = (BETA ? 2 : 1) * kTileK + kTileV + C * 4;
+    constexpr uint32_t TX = (BETA ? 2 : 1) * kTileK + kTileV + C * 4 + kTileK;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, gq = lane >> 2, tq = lane & 3;
     const int cg = w & 3, half = w >> 2, oth = half ^ 1;
     const int vl = 16 * cg;
@@ -719,7 +774,7 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
     uint64_t* bars = reinterpret_cast<uint64_t*>(xch + xch_bytes());
     bool failed = false;
 
-    auto stage = [&](int buf, bf16*& Khs, bf16*& Ws, bf16*& dVis, float*& Gs, bf16*& Qs, bf16*& dOs) {
+    auto stage = [&](int buf, bf16*& Khs, bf16*& Ws, bf16*& dVis, float*& Gs, bf16*& Dts) {
         unsigned char* p = smem + buf * STAGE;
         Khs = reinterpret_cast<bf16*>(p);
         p += kTileK;
@@ -729,37 +784,23 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
         p += kTileV;
         Gs = reinterpret_cast<float*>(p);
         p += C * 4;
-        Qs = reinterpret_cast<bf16*>(p);
-        p += kTileK;
-        dOs = reinterpret_cast<bf16*>(p);
+        Dts = reinterpret_cast<bf16*>(p);
     };
-    auto load = [&](int cc) {  // all threads: Q and dO pieces (permuted); thread 0: bulk copies
-        bf16 *Khs, *Ws, *dVis, *Qs, *dOs;
+    auto load = [&](int cc) {  // thread 0: bulk copies of one chunk's operands
+        bf16 *Khs, *Ws, *dVis, *Dts;
         float* Gs;
         const int buf = cc & 1;
-        stage(buf, Khs, Ws, dVis, Gs, Qs, dOs);
+        stage(buf, Khs, Ws, dVis, Gs, Dts);
         const size_t row0 = (size_t)bh * Tp + (size_t)cc * C;
-        const int nval = min(C, s.T - cc * C);
+        const size_t blk = ((size_t)bh * s.NC + cc) * DV + vb * 64;
         if (tid == 0) {
             mbar_expect_tx(&bars[buf], TX);
             bulk_load(Khs, Kh + row0 * DK, kTileK, &bars[buf]);
             if (BETA) bulk_load(Ws, Wn + row0 * DK, kTileK, &bars[buf]);
-            bulk_load(dVis, dVit + (((size_t)bh * s.NC + cc) * DV + vb * 64) * C, kTileV, &bars[buf]);
+            bulk_load(dVis, dVit + blk * C, kTileV, &bars[buf]);
             bulk_load(Gs, Gm + row0, C * 4, &bars[buf]);
+            bulk_load(Dts, Dt + blk * DK, kTileK, &bars[buf]);
         }
-        const bf16* qg = q + bh * s.hs_k + (size_t)cc * C * DK;
-        for (int e = tid; e < C * (DK / 8); e += 256) {
-            const int t = e >> 4, pc = e & 15;
-            const bool ok = t < nval;
-            cp_async16(Qs + swz(t, 8 * pc, DK), qg + (ok ? (size_t)t * DK : 0) + 8 * pc, ok);
-        }
-        const bf16* og = dO + bh * s.hs_v + (size_t)cc * C * DV + vb * 64;
-        for (int e = tid; e < C * 8; e += 256) {
-            const int t = e >> 3, pc = e & 7;
-            const bool ok = t < nval;
-            cp_async16(dOs + swz(t, 8 * pc, 64), og + (ok ? (size_t)t * DV : 0) + 8 * pc, ok);
-        }
-        cp_async_commit();
     };
     auto flush = [&](int cc) {
         unsigned char* o = outs + (cc % kOutBufs) * out_stage_bytes();
@@ -790,11 +831,10 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
     for (int cc = s.NC - 1; cc >= 0; --cc) {
         const int use = s.NC - 1 - cc;  // how many chunks were processed before this one
         if (cc > 0) load(cc - 1);
-        else cp_async_commit();
         if (tid == 0 && outputs && cc < s.NC - 1) flush(cc + 1);
-        bf16 *Khs, *Ws, *dVis, *Qs, *dOs;
+        bf16 *Khs, *Ws, *dVis, *Dts;
         float* Gs;
-        stage(cc & 1, Khs, Ws, dVis, Gs, Qs, dOs);
+        stage(cc & 1, Khs, Ws, dVis, Gs, Dts);
         bf16* dSs = reinterpret_cast<bf16*>(outs + (cc % kOutBufs) * out_stage_bytes());
         bf16* dVns = dSs + 64 * DK;
         uint32_t da[4][4], dp[4][4];
@@ -803,8 +843,7 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
             c2a(da[kk], ds[2 * kk], ds[2 * kk + 1]);
             put_frag(xslot(xch, cg, half, kk, lane), da[kk]);
         }
-        cp_async_wait<1>();
-        __syncthreads();  // Q / dO pieces of this chunk and the exchanged fragments are visible
+        __syncthreads();  // the exchanged fragments are visible
         mbar_wait(&bars[cc & 1], (use >> 1) & 1, &g_tc_status, failed);
         const float gamC = Gs[C - 1];
 #pragma unroll
@@ -849,35 +888,16 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
             c2a(va[kk], dvn[2 * kk], dvn[2 * kk + 1]);
             put_frag(xslot(xch, cg, half, 4 + kk, lane), va[kk]);
         }
+        // dS <- gamma_C dS + D (D from the intra kernel, independent of the chain)
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) ds[j][e] *= gamC;
-        // (scale gamma * dO)^T Q for this warp's state rows; independent of the chain
-        {
-            uint32_t ad[4][4], bq[4][4][4];
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                ldsm_x4_t(ad[kk], dOs + swz_at_off(16 * kk, vl, lane, 64));
-#pragma unroll
-                for (int n2 = 0; n2 < 4; ++n2) ldsm_x4_t(bq[kk][n2], Qs + sw_off(Lkn, 16 * kk, 8 * half + 2 * n2, DK));
-            }
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const int tk = 16 * kk + 2 * tq;
-                const float g0 = s.scale * Gs[tk], g1 = s.scale * Gs[tk + 1];
-                const float g2 = s.scale * Gs[tk + 8], g3 = s.scale * Gs[tk + 9];
-                uint32_t a[4];
-                a[0] = scale2(ad[kk][0], g0, g1);
-                a[1] = scale2(ad[kk][1], g0, g1);
-                a[2] = scale2(ad[kk][2], g2, g3);
-                a[3] = scale2(ad[kk][3], g2, g3);
-#pragma unroll
-                for (int n2 = 0; n2 < 4; ++n2) {
-                    mma(ds[2 * n2], a, bq[kk][n2][0], bq[kk][n2][1]);
-                    mma(ds[2 * n2 + 1], a, bq[kk][n2][2], bq[kk][n2][3]);
-                }
-            }
+        for (int j = 0; j < 8; ++j) {
+            const int col = 64 * half + 8 * j + 2 * tq;
+            const float2 d0 = unpack(*reinterpret_cast<const uint32_t*>(Dts + swz(vl + gq, col, DK)));
+            const float2 d1 = unpack(*reinterpret_cast<const uint32_t*>(Dts + swz(vl + gq + 8, col, DK)));
+            ds[j][0] = fmaf(ds[j][0], gamC, d0.x);
+            ds[j][1] = fmaf(ds[j][1], gamC, d0.y);
+            ds[j][2] = fmaf(ds[j][2], gamC, d1.x);
+            ds[j][3] = fmaf(ds[j][3], gamC, d1.y);
         }
         pair_sync(cg);
 #pragma unroll
@@ -949,7 +969,7 @@ tc_scan_fwd_kernel(SeqView s, const float* __restrict__ Gm, const bf16* __restri
 // forward's states are kept), every block runs the reverse scan.
 template <int DV, bool BETA>
 __global__ void __launch_bounds__(256, 1)
-tc_scan_bwd_dual_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ dO,
+tc_scan_bwd_dual_kernel(SeqView s, const bf16* __restrict__ Dt,
                         const float* __restrict__ Gm, const bf16* __restrict__ Wn,
                         const bf16* __restrict__ Kh, const bf16* __restrict__ Ut,
                         const bf16* __restrict__ dVit, const float* __restrict__ S_in,
@@ -964,7 +984,7 @@ tc_scan_bwd_dual_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __res
         scan_fwd_cta<DV, BETA>(s, id / NVB, id % NVB, Gm, Wn, Kh, Ut, S_in, Vnt, S0t, nullptr, smem);
     } else {
         id -= nsr;
-        scan_bwd_cta<DV, BETA>(s, id / NVB, id % NVB, q, dO, Gm, Wn, Kh, dVit, dS_out, dVnt, dSCt, dS_in, smem);
+        scan_bwd_cta<DV, BETA>(s, id / NVB, id % NVB, Dt, Gm, Wn, Kh, dVit, dS_out, dVnt, dSCt, dS_in, smem);
     }
 }
 
@@ -1060,39 +1080,43 @@ tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
 }
 
 // ------------------------------------------------------------------ grad ---
+// Warps of the gradient kernel: 4 row blocks of 16 x GW column groups.
+constexpr int GW = 4;
+constexpr int GTH = 128 * GW;
+constexpr int DKW = DK / GW;  // key columns of one column group
+constexpr int CW = C / GW;    // chunk columns of one column group
 // Partial-sum rows (each [64] fp32) of the gradient kernel's reductions.
 enum GradPart {
-    P_INTER = 0,   // [2]  sum_k Q_ik dq_inter_ik
-    P_Z = 2,       // [2]  sum_k K_jk dK_state_jk
-    P_ROWP = 4,    // [2]  row sums of M * (Qs K^T)
-    P_COLP = 6,    // [4]  column sums of the same
-    P_KT = 10,     // [2]  gamma_j k_j . dKt_j
-    P_DBC = 12,    // [4]  column sums of dT * L
-    P_DBR = 16,    // [2]  row sums of dA * Gamma * KK
-    P_ROWA = 18,   // [2]  row sums of Z * KK
-    P_COLA = 20,   // [4]  column sums of Z * KK
-    P_DG = 24,     // [1]  dG
-    P_ROWS = 25
+    P_INTER = 0,             // [GW] sum_k Q_ik dq_inter_ik
+    P_Z = GW,                // [GW] sum_k K_jk dK_state_jk
+    P_ROWP = 2 * GW,         // [GW] row sums of M * (Qs K^T)
+    P_COLP = 3 * GW,         // [4]  column sums of the same
+    P_KT = 3 * GW + 4,       // [GW] gamma_j k_j . dKt_j
+    P_DBC = 4 * GW + 4,      // [4]  column sums of dT * L
+    P_DBR = 4 * GW + 8,      // [GW] row sums of dA * Gamma * KK
+    P_ROWA = 5 * GW + 8,     // [GW] row sums of Z * KK
+    P_COLA = 6 * GW + 8,     // [4]  column sums of Z * KK
+    P_ROWS = 6 * GW + 12
 };
 
 template <int DV>
 constexpr size_t grad_region_bytes() {
     const size_t sa = (size_t)DV * LDK * 2 * 2;                                     // S0^T, dS_C^T
-    const size_t sb = (size_t)C * LDK * 2 + (size_t)C * LDF * 4 * 2 + (size_t)C * LDC * 2 * 4;  // dW, A, L, T/L/M/dL
+    const size_t sb = (size_t)C * LDK * 2 + (size_t)C * LDF * 4 * 2 + (size_t)C * LDC * 2 * 4;  // dW, X/Z, L, T/L/M/dL
     return sa > sb ? sa : sb;
 }
 template <int DV>
 constexpr size_t grad_smem() {
     return (size_t)C * LDK * 2 * 2 + (size_t)C * (DV + 8) * 2 * 2 + (size_t)DV * LDC * 2 * 2 +
-           grad_region_bytes<DV>() + (size_t)P_ROWS * C * 4 + 256 * 4 + 2 * C * 4;
+           grad_region_bytes<DV>() + (size_t)P_ROWS * C * 4 + GTH * 4 + 2 * C * 4;
 }
 
-// Every input gradient of one chunk (8 warps: rows 16*(w%4), column half w/4).
+// Every input gradient of one chunk (4 x GW warps: rows 16*(w%4), column group w/4).
 template <int DV, bool BETA>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(GTH, 1)
 tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
                const bf16* __restrict__ v, const float* __restrict__ beta,
-               const bf16* __restrict__ dO, const float* __restrict__ Gc,
+               const bf16* __restrict__ dO, const float* __restrict__ Gc, const float* __restrict__ Lm,
                const bf16* __restrict__ Vnt, const bf16* __restrict__ dVnt,
                const bf16* __restrict__ S0t, const bf16* __restrict__ dSCt, bf16* __restrict__ dq,
                bf16* __restrict__ dk, bf16* __restrict__ dv, float* __restrict__ dg,
@@ -1109,17 +1133,17 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     bf16* S0s = reinterpret_cast<bf16*>(R);       // [DV][LDK]  (phase S)
     bf16* dSs = S0s + DV * LDK;                   // [DV][LDK]  (phase S)
     bf16* dWs = reinterpret_cast<bf16*>(R);       // [C][LDK]   (after phase S)
-    float* Af = reinterpret_cast<float*>(R + C * LDK * 2);  // [C][LDF]; later Xs, Zs
-    float* Lf = Af + C * LDF;                     // [C][LDF]
+    float* XZ = reinterpret_cast<float*>(R + C * LDK * 2);  // X, Z (bf16 [C][LDC] each)
+    float* Lf = XZ + C * LDF;                     // [C][LDF] L (fp32)
     bf16* Ts = reinterpret_cast<bf16*>(Lf + C * LDF);  // [C][LDC]; Y scratch during the inverse
     bf16* Ls = Ts + C * LDC;
     bf16* Ms = Ls + C * LDC;
     bf16* dLs = Ms + C * LDC;
-    bf16* Xs = reinterpret_cast<bf16*>(Af);
+    bf16* Xs = reinterpret_cast<bf16*>(XZ);
     bf16* Zs = Xs + C * LDC;
     float* part = reinterpret_cast<float*>(R + grad_region_bytes<DV>());  // [P_ROWS][C]
-    float* red = part + P_ROWS * C;                                        // [256]
-    float* Gs = red + 256;
+    float* red = part + P_ROWS * C;                                        // [GTH]
+    float* Gs = red + GTH;
     float* Bs = Gs + C;
 
     const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -1129,19 +1153,21 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     const int nval = min(C, s.T - t0);
     const size_t Tp = (size_t)s.NC * C;
     const size_t ci = (size_t)bh * s.NC + c;
-    load_tile<C, DK, 256>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
-    load_tile<C, DK, 256>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
-    load_tile<C, DV, 256>(Vs, LDV, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
-    load_tile<C, DV, 256>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
-    load_tile_swz<DV, C, 256>(Vns, LDC, Vnt + ci * DV * C, tid);
-    load_tile_swz<DV, C, 256>(dVns, LDC, dVnt + ci * DV * C, tid);
-    load_tile_swz<DV, DK, 256>(S0s, LDK, S0t + ci * DV * DK, tid);
-    load_tile_swz<DV, DK, 256>(dSs, LDK, dSCt + ci * DV * DK, tid);
+    // Two copy groups: what the state products of phase S read, then Q, K, V.
+    load_tile<C, DV, GTH>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+    load_tile_swz<DV, C, GTH>(Vns, LDC, Vnt + ci * DV * C, tid);
+    load_tile_swz<DV, C, GTH>(dVns, LDC, dVnt + ci * DV * C, tid);
+    load_tile_swz<DV, DK, GTH>(S0s, LDK, S0t + ci * DV * DK, tid);
+    load_tile_swz<DV, DK, GTH>(dSs, LDK, dSCt + ci * DV * DK, tid);
     if (tid < 16) cp_async16(Gs + tid * 4, Gc + bh * Tp + t0 + tid * 4, true);
     cp_async_commit();
-    for (int i = tid; i < C; i += 256) Bs[i] = (BETA && i < nval) ? beta[bh * s.hs_g + t0 + i] : 0.f;
-    for (int e = tid; e < P_ROWS * C; e += 256) part[e] = 0.f;
-    cp_async_wait<0>();
+    load_tile<C, DK, GTH>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+    load_tile<C, DK, GTH>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+    load_tile<C, DV, GTH>(Vs, LDV, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+    cp_async_commit();
+    for (int i = tid; i < C; i += GTH) Bs[i] = (BETA && i < nval) ? beta[bh * s.hs_g + t0 + i] : 0.f;
+    for (int e = tid; e < P_ROWS * C; e += GTH) part[e] = 0.f;
+    cp_async_wait<1>();
     __syncthreads();
 
     const int r0 = 16 * mw + gq, r1 = r0 + 8;  // the two rows this thread holds
@@ -1150,9 +1176,9 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     const float dec0 = __expf(gC - Gs[r0]), dec1 = __expf(gC - Gs[r1]);
 
     // ---- phase S: products with the chunk-entry state and the state gradient
-    float accQ[8][4] = {}, accK[8][4] = {};
+    float accQ[DKW / 8][4] = {}, accK[DKW / 8][4] = {};
     {
-        float accW[8][4] = {};
+        float accW[DKW / 8][4] = {};
 #pragma unroll
         for (int kv = 0; kv < DV / 16; ++kv) {
             uint32_t aO[4], aN[4], aV[4];
@@ -1160,20 +1186,22 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
             ldAt(aN, dVns, LDC, 16 * mw, 16 * kv, lane);
             ldAt(aV, Vns, LDC, 16 * mw, 16 * kv, lane);
 #pragma unroll
-            for (int nn = 0; nn < 8; nn += 2) {
+            for (int nn = 0; nn < DKW / 8; nn += 2) {
                 uint32_t b[4];
-                ldBkn(b, S0s, LDK, 64 * nw + 8 * nn, 16 * kv, lane);
+                ldBkn(b, S0s, LDK, DKW * nw + 8 * nn, 16 * kv, lane);
                 mma(accQ[nn], aO, b[0], b[1]);
                 mma(accQ[nn + 1], aO, b[2], b[3]);
                 mma(accW[nn], aN, b[0], b[1]);
                 mma(accW[nn + 1], aN, b[2], b[3]);
-                ldBkn(b, dSs, LDK, 64 * nw + 8 * nn, 16 * kv, lane);
+                ldBkn(b, dSs, LDK, DKW * nw + 8 * nn, 16 * kv, lane);
                 mma(accK[nn], aV, b[0], b[1]);
                 mma(accK[nn + 1], aV, b[2], b[3]);
             }
         }
+        cp_async_wait<0>();
+        __syncthreads();  // Q, K, V have landed
         float pd = 0.f;  // <S0, dS_C>
-        for (int e = tid; e < DV * DK; e += 256) {
+        for (int e = tid; e < DV * DK; e += GTH) {
             const int r = e / DK, cc = e % DK;
             pd += __bfloat162float(S0s[r * LDK + cc]) * __bfloat162float(dSs[r * LDK + cc]);
         }
@@ -1182,8 +1210,8 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         const float sq0 = s.scale * gam0, sq1 = s.scale * gam1;
         float pi0 = 0.f, pi1 = 0.f, pz0 = 0.f, pz1 = 0.f;
 #pragma unroll
-        for (int nn = 0; nn < 8; ++nn) {
-            const int col = 64 * nw + 8 * nn + 2 * tq;
+        for (int nn = 0; nn < DKW / 8; ++nn) {
+            const int col = DKW * nw + 8 * nn + 2 * tq;
             const float2 q0 = unpack(*reinterpret_cast<const uint32_t*>(Qs + r0 * LDK + col));
             const float2 q1 = unpack(*reinterpret_cast<const uint32_t*>(Qs + r1 * LDK + col));
             const float2 k0 = unpack(*reinterpret_cast<const uint32_t*>(Ks + r0 * LDK + col));
@@ -1215,33 +1243,41 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
             part[(P_Z + nw) * C + r1] = pz1;
         }
         __syncthreads();  // everyone is done with S0^T and dS_C^T
+        if (BETA) {  // L of this chunk (from the prep kernel) into Lf; waited for before phase C2
+            const float* Lg = Lm + ci * C * C;
+            for (int e = tid; e < C * C / 4; e += GTH) {
+                const int i = e >> 4, j = (e & 15) * 4;
+                cp_async16(Lf + i * LDF + j, Lg + i * C + j, true);
+            }
+            cp_async_commit();
+        }
         // dW = -dV_new S0^T into the freed region
 #pragma unroll
-        for (int nn = 0; nn < 8; ++nn) {
-            const int col = 64 * nw + 8 * nn + 2 * tq;
+        for (int nn = 0; nn < DKW / 8; ++nn) {
+            const int col = DKW * nw + 8 * nn + 2 * tq;
             *reinterpret_cast<uint32_t*>(dWs + r0 * LDK + col) = pack(-accW[nn][0], -accW[nn][1]);
             *reinterpret_cast<uint32_t*>(dWs + r1 * LDK + col) = pack(-accW[nn][2], -accW[nn][3]);
         }
     }
-    for (int o = 128; o > 0; o >>= 1) {
+    for (int o = GTH / 2; o > 0; o >>= 1) {
         if (tid < o) red[tid] += red[tid + o];
         __syncthreads();
     }
     const float sdot = red[0];
 
     // ---- phase C1: C x C products (rows 16mw.., columns 32nw..)
-    float kkr[4][4] = {};
+    float kkr[CW / 8][4] = {};
     {
-        float qk[4][4] = {}, dp[4][4] = {};
+        float qk[CW / 8][4] = {}, dp[CW / 8][4] = {};
 #pragma unroll
         for (int kd = 0; kd < 8; ++kd) {
             uint32_t aQ[4], aK[4];
             ldA(aQ, Qs, LDK, 16 * mw, 16 * kd, lane);
             ldA(aK, Ks, LDK, 16 * mw, 16 * kd, lane);
 #pragma unroll
-            for (int nn = 0; nn < 4; nn += 2) {
+            for (int nn = 0; nn < CW / 8; nn += 2) {
                 uint32_t b[4];
-                ldBnk(b, Ks, LDK, 32 * nw + 8 * nn, 16 * kd, lane);
+                ldBnk(b, Ks, LDK, CW * nw + 8 * nn, 16 * kd, lane);
                 mma(qk[nn], aQ, b[0], b[1]);
                 mma(qk[nn + 1], aQ, b[2], b[3]);
                 mma(kkr[nn], aK, b[0], b[1]);
@@ -1253,27 +1289,26 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
             uint32_t aO[4];
             ldA(aO, dOs, LDV, 16 * mw, 16 * kv, lane);
 #pragma unroll
-            for (int nn = 0; nn < 4; nn += 2) {
+            for (int nn = 0; nn < CW / 8; nn += 2) {
                 uint32_t b[4];
-                ldBkn(b, Vns, LDC, 32 * nw + 8 * nn, 16 * kv, lane);
+                ldBkn(b, Vns, LDC, CW * nw + 8 * nn, 16 * kv, lane);
                 mma(dp[nn], aO, b[0], b[1]);
                 mma(dp[nn + 1], aO, b[2], b[3]);
             }
         }
         float row0 = 0.f, row1 = 0.f;
 #pragma unroll
-        for (int nn = 0; nn < 4; ++nn) {
+        for (int nn = 0; nn < CW / 8; ++nn) {
             float col[2] = {0.f, 0.f};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int i = (e >> 1) ? r1 : r0, j = 32 * nw + 8 * nn + 2 * tq + (e & 1);
+                const int i = (e >> 1) ? r1 : r0, j = CW * nw + 8 * nn + 2 * tq + (e & 1);
                 const float gm = (j <= i) ? __expf(Gs[i] - Gs[j]) : 0.f;
                 const float m = s.scale * dp[nn][e] * gm;
                 Ms[i * LDC + j] = __float2bfloat16_rn(m);
                 const float zp = m * qk[nn][e];
                 if (e >> 1) row1 += zp; else row0 += zp;
                 col[e & 1] += zp;
-                if (BETA) Af[i * LDF + j] = (j < i) ? Bs[i] * gm * kkr[nn][e] : 0.f;
             }
 #pragma unroll
             for (int o = 4; o < 32; o <<= 1) {
@@ -1281,7 +1316,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
                 col[1] += __shfl_xor_sync(0xffffffffu, col[1], o);
             }
             if (gq == 0) {
-                const int j = 32 * nw + 8 * nn + 2 * tq;
+                const int j = CW * nw + 8 * nn + 2 * tq;
                 part[(P_COLP + mw) * C + j] = col[0];
                 part[(P_COLP + mw) * C + j + 1] = col[1];
             }
@@ -1295,15 +1330,13 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
             part[(P_ROWP + nw) * C + r0] = row0;
             part[(P_ROWP + nw) * C + r1] = row1;
         }
-        if (BETA)
-            for (int e = tid; e < C * LDF; e += 256) Lf[e] = 0.f;
     }
+    if (BETA) cp_async_wait<0>();
     __syncthreads();
 
-    // ---- phase C2: L = (I + A)^{-1}; T = L diag(beta)
+    // ---- phase C2: T = L diag(beta), L = (I + A)^{-1} as computed by the prep kernel
     if (BETA) {
-        block_inverse(Af, LDF, Lf, LDF, reinterpret_cast<float*>(Ts), tid, 256);
-        for (int e = tid; e < C * C; e += 256) {
+        for (int e = tid; e < C * C; e += GTH) {
             const int i = e >> 6, j = e & 63;
             const float l = Lf[i * LDF + j];
             Ts[i * LDC + j] = __float2bfloat16_rn(l * Bs[j]);
@@ -1314,23 +1347,23 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 
     // ---- phase C3: dKt = T^T dW (into dK), dV = T^T dV_new
     if (BETA) {
-        float acc[8][4] = {};
+        float acc[DKW / 8][4] = {};
 #pragma unroll
         for (int kr = 0; kr < 4; ++kr) {
             uint32_t a[4];
             ldAt(a, Ts, LDC, 16 * mw, 16 * kr, lane);
 #pragma unroll
-            for (int nn = 0; nn < 8; nn += 2) {
+            for (int nn = 0; nn < DKW / 8; nn += 2) {
                 uint32_t b[4];
-                ldBkn(b, dWs, LDK, 64 * nw + 8 * nn, 16 * kr, lane);
+                ldBkn(b, dWs, LDK, DKW * nw + 8 * nn, 16 * kr, lane);
                 mma(acc[nn], a, b[0], b[1]);
                 mma(acc[nn + 1], a, b[2], b[3]);
             }
         }
         float p0 = 0.f, p1 = 0.f;
 #pragma unroll
-        for (int nn = 0; nn < 8; ++nn) {
-            const int col = 64 * nw + 8 * nn + 2 * tq;
+        for (int nn = 0; nn < DKW / 8; ++nn) {
+            const int col = DKW * nw + 8 * nn + 2 * tq;
             const float2 k0 = unpack(*reinterpret_cast<const uint32_t*>(Ks + r0 * LDK + col));
             const float2 k1 = unpack(*reinterpret_cast<const uint32_t*>(Ks + r1 * LDK + col));
             const float a0 = gam0 * acc[nn][0], a1 = gam0 * acc[nn][1];
@@ -1353,7 +1386,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         }
     }
     {
-        constexpr int NT = DV / 16;  // n-tiles of this warp's half of the value columns
+        constexpr int NT = DV / (8 * GW);  // n-tiles of this warp's group of value columns
         bf16* dvb = dv + bh * s.hs_v + (size_t)t0 * DV;
         if (BETA) {
             float acc[NT][4] = {};
@@ -1364,19 +1397,19 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 #pragma unroll
                 for (int nn = 0; nn < NT; nn += 2) {
                     uint32_t b[4];
-                    ldBnk(b, dVns, LDC, (DV / 2) * nw + 8 * nn, 16 * kr, lane);
+                    ldBnk(b, dVns, LDC, (DV / GW) * nw + 8 * nn, 16 * kr, lane);
                     mma(acc[nn], a, b[0], b[1]);
                     mma(acc[nn + 1], a, b[2], b[3]);
                 }
             }
 #pragma unroll
             for (int nn = 0; nn < NT; ++nn) {
-                const int col = (DV / 2) * nw + 8 * nn + 2 * tq;
+                const int col = (DV / GW) * nw + 8 * nn + 2 * tq;
                 if (r0 < nval) *reinterpret_cast<uint32_t*>(dvb + (size_t)r0 * DV + col) = pack(acc[nn][0], acc[nn][1]);
                 if (r1 < nval) *reinterpret_cast<uint32_t*>(dvb + (size_t)r1 * DV + col) = pack(acc[nn][2], acc[nn][3]);
             }
         } else {
-            for (int e = tid; e < nval * DV; e += 256) {
+            for (int e = tid; e < nval * DV; e += GTH) {
                 const int j = e / DV, col = e % DV;
                 dvb[(size_t)j * DV + col] = dVns[col * LDC + j];
             }
@@ -1385,41 +1418,41 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 
     // ---- phase C4: dT = dW (gamma K)^T + dV_new V^T; dbeta (column part); dL = dT diag(beta)
     if (BETA) {
-        float dt[4][4] = {};
+        float dt[CW / 8][4] = {};
 #pragma unroll
         for (int kd = 0; kd < 8; ++kd) {
             uint32_t a[4];
             ldA(a, dWs, LDK, 16 * mw, 16 * kd, lane);
 #pragma unroll
-            for (int nn = 0; nn < 4; nn += 2) {
+            for (int nn = 0; nn < CW / 8; nn += 2) {
                 uint32_t b[4];
-                ldBnk(b, Ks, LDK, 32 * nw + 8 * nn, 16 * kd, lane);
+                ldBnk(b, Ks, LDK, CW * nw + 8 * nn, 16 * kd, lane);
                 mma(dt[nn], a, b[0], b[1]);
                 mma(dt[nn + 1], a, b[2], b[3]);
             }
         }
 #pragma unroll
-        for (int nn = 0; nn < 4; ++nn)
+        for (int nn = 0; nn < CW / 8; ++nn)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dt[nn][e] *= __expf(Gs[32 * nw + 8 * nn + 2 * tq + (e & 1)]);
+            for (int e = 0; e < 4; ++e) dt[nn][e] *= __expf(Gs[CW * nw + 8 * nn + 2 * tq + (e & 1)]);
 #pragma unroll
         for (int kv = 0; kv < DV / 16; ++kv) {
             uint32_t a[4];
             ldAt(a, dVns, LDC, 16 * mw, 16 * kv, lane);
 #pragma unroll
-            for (int nn = 0; nn < 4; nn += 2) {
+            for (int nn = 0; nn < CW / 8; nn += 2) {
                 uint32_t b[4];
-                ldBnk(b, Vs, LDV, 32 * nw + 8 * nn, 16 * kv, lane);
+                ldBnk(b, Vs, LDV, CW * nw + 8 * nn, 16 * kv, lane);
                 mma(dt[nn], a, b[0], b[1]);
                 mma(dt[nn + 1], a, b[2], b[3]);
             }
         }
 #pragma unroll
-        for (int nn = 0; nn < 4; ++nn) {
+        for (int nn = 0; nn < CW / 8; ++nn) {
             float col[2] = {0.f, 0.f};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int r = (e >> 1) ? r1 : r0, j = 32 * nw + 8 * nn + 2 * tq + (e & 1);
+                const int r = (e >> 1) ? r1 : r0, j = CW * nw + 8 * nn + 2 * tq + (e & 1);
                 col[e & 1] += dt[nn][e] * Lf[r * LDF + j];
                 dLs[r * LDC + j] = __float2bfloat16_rn(dt[nn][e] * Bs[j]);
             }
@@ -1429,7 +1462,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
                 col[1] += __shfl_xor_sync(0xffffffffu, col[1], o);
             }
             if (gq == 0) {
-                const int j = 32 * nw + 8 * nn + 2 * tq;
+                const int j = CW * nw + 8 * nn + 2 * tq;
                 part[(P_DBC + mw) * C + j] = col[0];
                 part[(P_DBC + mw) * C + j + 1] = col[1];
             }
@@ -1437,22 +1470,22 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         __syncthreads();
         // ---- phase C5: X = L^T dL
         {
-            float x[4][4] = {};
+            float x[CW / 8][4] = {};
 #pragma unroll
             for (int kr = 0; kr < 4; ++kr) {
                 uint32_t a[4];
                 ldAt(a, Ls, LDC, 16 * mw, 16 * kr, lane);
 #pragma unroll
-                for (int nn = 0; nn < 4; nn += 2) {
+                for (int nn = 0; nn < CW / 8; nn += 2) {
                     uint32_t b[4];
-                    ldBkn(b, dLs, LDC, 32 * nw + 8 * nn, 16 * kr, lane);
+                    ldBkn(b, dLs, LDC, CW * nw + 8 * nn, 16 * kr, lane);
                     mma(x[nn], a, b[0], b[1]);
                     mma(x[nn + 1], a, b[2], b[3]);
                 }
             }
 #pragma unroll
-            for (int nn = 0; nn < 4; ++nn) {
-                const int j = 32 * nw + 8 * nn + 2 * tq;
+            for (int nn = 0; nn < CW / 8; ++nn) {
+                const int j = CW * nw + 8 * nn + 2 * tq;
                 *reinterpret_cast<uint32_t*>(Xs + r0 * LDC + j) = pack(x[nn][0], x[nn][1]);
                 *reinterpret_cast<uint32_t*>(Xs + r1 * LDC + j) = pack(x[nn][2], x[nn][3]);
             }
@@ -1460,26 +1493,26 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         __syncthreads();
         // ---- phase C6: dA = strictly-lower(-X L^T); Z = dA beta_i Gamma; dbeta (row part)
         {
-            float da[4][4] = {};
+            float da[CW / 8][4] = {};
 #pragma unroll
             for (int km = 0; km < 4; ++km) {
                 uint32_t a[4];
                 ldA(a, Xs, LDC, 16 * mw, 16 * km, lane);
 #pragma unroll
-                for (int nn = 0; nn < 4; nn += 2) {
+                for (int nn = 0; nn < CW / 8; nn += 2) {
                     uint32_t b[4];
-                    ldBnk(b, Ls, LDC, 32 * nw + 8 * nn, 16 * km, lane);
+                    ldBnk(b, Ls, LDC, CW * nw + 8 * nn, 16 * km, lane);
                     mma(da[nn], a, b[0], b[1]);
                     mma(da[nn + 1], a, b[2], b[3]);
                 }
             }
             float rz0 = 0.f, rz1 = 0.f, rb0 = 0.f, rb1 = 0.f;
 #pragma unroll
-            for (int nn = 0; nn < 4; ++nn) {
+            for (int nn = 0; nn < CW / 8; ++nn) {
                 float col[2] = {0.f, 0.f};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int i = (e >> 1) ? r1 : r0, j = 32 * nw + 8 * nn + 2 * tq + (e & 1);
+                    const int i = (e >> 1) ? r1 : r0, j = CW * nw + 8 * nn + 2 * tq + (e & 1);
                     float z = 0.f, bterm = 0.f;
                     if (j < i) {
                         const float gm = __expf(Gs[i] - Gs[j]);
@@ -1504,7 +1537,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
                     col[1] += __shfl_xor_sync(0xffffffffu, col[1], o);
                 }
                 if (gq == 0) {
-                    const int j = 32 * nw + 8 * nn + 2 * tq;
+                    const int j = CW * nw + 8 * nn + 2 * tq;
                     part[(P_COLA + mw) * C + j] = col[0];
                     part[(P_COLA + mw) * C + j + 1] = col[1];
                 }
@@ -1538,10 +1571,10 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
             ldAt(aZt, Zs, LDC, 16 * mw, 16 * ki, lane);
         }
 #pragma unroll
-        for (int nn = 0; nn < 8; nn += 2) {
+        for (int nn = 0; nn < DKW / 8; nn += 2) {
             uint32_t bk[4], bq[4];
-            ldBkn(bk, Ks, LDK, 64 * nw + 8 * nn, 16 * ki, lane);
-            ldBkn(bq, Qs, LDK, 64 * nw + 8 * nn, 16 * ki, lane);
+            ldBkn(bk, Ks, LDK, DKW * nw + 8 * nn, 16 * ki, lane);
+            ldBkn(bq, Qs, LDK, DKW * nw + 8 * nn, 16 * ki, lane);
             mma(accQ[nn], aM, bk[0], bk[1]);
             mma(accQ[nn + 1], aM, bk[2], bk[3]);
             mma(accK[nn], aMt, bq[0], bq[1]);
@@ -1558,8 +1591,8 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         bf16* dqb = dq + bh * s.hs_k + (size_t)t0 * DK;
         bf16* dkb = dk + bh * s.hs_k + (size_t)t0 * DK;
 #pragma unroll
-        for (int nn = 0; nn < 8; ++nn) {
-            const int col = 64 * nw + 8 * nn + 2 * tq;
+        for (int nn = 0; nn < DKW / 8; ++nn) {
+            const int col = DKW * nw + 8 * nn + 2 * tq;
             if (r0 < nval) {
                 *reinterpret_cast<uint32_t*>(dqb + (size_t)r0 * DK + col) = pack(accQ[nn][0], accQ[nn][1]);
                 *reinterpret_cast<uint32_t*>(dkb + (size_t)r0 * DK + col) = pack(accK[nn][0], accK[nn][1]);
@@ -1571,31 +1604,37 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         }
     }
 
-    // ---- phase C8: dG, dg (reverse cumsum), dbeta
-    float* dG = part + P_DG * C;
-    if (tid < C) {
-        const int i = tid;
-        auto P = [&](int row) { return part[row * C + i]; };
-        float x = P(P_INTER) + P(P_INTER + 1) + P(P_ROWP) + P(P_ROWP + 1) -
-                  (P(P_COLP) + P(P_COLP + 1) + P(P_COLP + 2) + P(P_COLP + 3)) - (P(P_Z) + P(P_Z + 1));
-        if (BETA) {
-            x += P(P_ROWA) + P(P_ROWA + 1) - (P(P_COLA) + P(P_COLA + 1) + P(P_COLA + 2) + P(P_COLA + 3)) +
-                 P(P_KT) + P(P_KT + 1);
-            const float db = P(P_DBC) + P(P_DBC + 1) + P(P_DBC + 2) + P(P_DBC + 3) + P(P_DBR) + P(P_DBR + 1);
-            if (i < nval) dbeta[bh * s.hs_g + t0 + i] = db;
+    // ---- phase C8: dG, dg (reverse cumsum), dbeta; warp 0, two tokens per lane
+    if (w == 0) {
+        auto P = [&](int row, int n, int i) {
+            float x = 0.f;
+            for (int u = 0; u < n; ++u) x += part[(row + u) * C + i];
+            return x;
+        };
+        float x[2], zs = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int i = 2 * lane + h;
+            x[h] = P(P_INTER, GW, i) + P(P_ROWP, GW, i) - P(P_COLP, 4, i) - P(P_Z, GW, i);
+            zs += P(P_Z, GW, i);
+            if (BETA) {
+                x[h] += P(P_ROWA, GW, i) - P(P_COLA, 4, i) + P(P_KT, GW, i);
+                if (i < nval) dbeta[bh * s.hs_g + t0 + i] = P(P_DBC, 4, i) + P(P_DBR, GW, i);
+            }
         }
-        dG[i] = x;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        float zs = 0.f;
-        for (int j = 0; j < C; ++j) zs += part[P_Z * C + j] + part[(P_Z + 1) * C + j];
-        dG[C - 1] += __expf(gC) * sdot + zs;
-        float acc = 0.f;
-        for (int i = C - 1; i >= 0; --i) {
-            acc += dG[i];
-            if (i < nval) dg[bh * s.hs_g + t0 + i] = acc;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
+        if (lane == 31) x[1] += __expf(gC) * sdot + zs;
+        // suffix sums over the lanes' pairs: dg_i = sum_{m >= i} dG_m
+        float suf = x[0] + x[1];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_down_sync(0xffffffffu, suf, o);
+            if (lane + o < 32) suf += y;
         }
+        float* dgb = dg + bh * s.hs_g + t0;
+        if (2 * lane < nval) dgb[2 * lane] = suf;
+        if (2 * lane + 1 < nval) dgb[2 * lane + 1] = suf - x[0];
     }
 }
 
@@ -1616,8 +1655,8 @@ cudaError_t launch_prep(const char* name, const SeqView& s, const bf16* k, const
                         const float* beta, const TcWs& w, cudaStream_t st) {
     constexpr size_t sm = prep_smem<DV, false>();
     TC_TRY(smem_attr(tc_prep_kernel<DV, BETA, false>, sm));
-    SF_LAUNCH(name, st, tc_prep_kernel<DV, BETA, false><<<dim3(s.NC, s.BH), 128, sm, st>>>(
-                            s, nullptr, k, v, g, beta, nullptr, w.Gc, w.Gm, w.W, w.Kh, w.Ut, nullptr));
+    SF_LAUNCH(name, st, tc_prep_kernel<DV, BETA, false><<<dim3(s.NC, s.BH), 256, sm, st>>>(
+                            s, nullptr, k, v, g, beta, nullptr, w.Gc, w.Gm, w.W, w.Lm, w.Kh, w.Ut, nullptr));
     return cudaGetLastError();
 }
 
@@ -1643,7 +1682,7 @@ cudaError_t launch_intra(const SeqView& s, const bf16* q, const bf16* k, const b
                          cudaStream_t st) {
     constexpr size_t sm = intra_smem<DV>();
     TC_TRY(smem_attr(tc_intra_kernel<DV>, sm));
-    SF_LAUNCH("tc_intra", st, tc_intra_kernel<DV><<<dim3(s.NC, s.BH), 128, sm, st>>>(s, q, k, dO, w.Gc, w.dVit));
+    SF_LAUNCH("tc_intra", st, tc_intra_kernel<DV><<<dim3(s.NC, s.BH), 128, sm, st>>>(s, q, k, dO, w.Gc, w.dVit, w.Dt));
     return cudaGetLastError();
 }
 
@@ -1654,8 +1693,7 @@ cudaError_t launch_scan_bwd(const SeqView& s, const BwdArgs& a, bool with_sr, co
     TC_TRY(smem_attr(tc_scan_bwd_dual_kernel<DV, BETA>, sm));
     const int nb = (with_sr ? 2 : 1) * s.BH * (DV / 64);
     SF_LAUNCH("tc_scan_bwd", st, tc_scan_bwd_dual_kernel<DV, BETA><<<nb, 256, sm, st>>>(
-                                     s, static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.dO), w.Gm,
-                                     w.W, w.Kh, w.Ut, w.dVit, a.S_in, a.dS_out, w.Vnt, w.S0t, w.dVnt, w.dSCt,
+                                     s, w.Dt, w.Gm, w.W, w.Kh, w.Ut, w.dVit, a.S_in, a.dS_out, w.Vnt, w.S0t, w.dVnt, w.dSCt,
                                      a.dS_in, with_sr ? 1 : 0));
     return cudaGetLastError();
 }
@@ -1664,10 +1702,10 @@ template <int DV, bool BETA>
 cudaError_t launch_grad(const SeqView& s, const BwdArgs& a, const TcWs& w, cudaStream_t st) {
     constexpr size_t sm = grad_smem<DV>();
     TC_TRY(smem_attr(tc_grad_kernel<DV, BETA>, sm));
-    SF_LAUNCH("tc_grad", st, tc_grad_kernel<DV, BETA><<<dim3(s.NC, s.BH), 256, sm, st>>>(
+    SF_LAUNCH("tc_grad", st, tc_grad_kernel<DV, BETA><<<dim3(s.NC, s.BH), GTH, sm, st>>>(
                                  s, static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k),
                                  static_cast<const bf16*>(a.v), a.beta, static_cast<const bf16*>(a.dO), w.Gc,
-                                 w.Vnt, w.dVnt, w.S0t, w.dSCt, static_cast<bf16*>(a.dq), static_cast<bf16*>(a.dk),
+                                 w.Lm, w.Vnt, w.dVnt, w.S0t, w.dSCt, static_cast<bf16*>(a.dq), static_cast<bf16*>(a.dk),
                                  static_cast<bf16*>(a.dv), a.dg, a.dbeta));
     return cudaGetLastError();
 }
@@ -1698,7 +1736,10 @@ cudaError_t bwd_impl(const SeqView& s, const BwdArgs& a, void* ws, cudaStream_t 
 template <int DV, bool BETA>
 cudaError_t stage_impl(TcStage stage, const SeqView& s, const FwdArgs* f, const BwdArgs* b, void* keep, void* slot,
                        cudaStream_t st) {
-    const TcWs w = tc_parts(s, static_cast<char*>(keep), static_cast<char*>(slot), nullptr, nullptr);
+    size_t kb = 0;
+    tc_parts(s, nullptr, nullptr, nullptr, &kb, nullptr, nullptr);
+    const TcWs w = tc_parts(s, static_cast<char*>(keep), static_cast<char*>(keep) + kb, static_cast<char*>(slot),
+                            nullptr, nullptr, nullptr);
     switch (stage) {
         case TcStage::Prep:
             return launch_prep<DV, BETA>("tc_prep", s, static_cast<const bf16*>(f->k),
@@ -1725,14 +1766,14 @@ bool tc_supports(bool bf16_io, int dk, int dv, int Cc, bool) {
 size_t tc_workspace_bytes(const SeqView& s, bool backward) { return tc_layout(s, backward, nullptr).total; }
 
 size_t tc_keep_bytes(const SeqView& s) {
-    size_t kb = 0;
-    tc_parts(s, nullptr, nullptr, &kb, nullptr);
-    return kb;
+    size_t kb = 0, ob = 0;
+    tc_parts(s, nullptr, nullptr, nullptr, &kb, &ob, nullptr);
+    return kb + ob;
 }
 
 size_t tc_slot_bytes(const SeqView& s) {
     size_t sb = 0;
-    tc_parts(s, nullptr, nullptr, nullptr, &sb);
+    tc_parts(s, nullptr, nullptr, nullptr, nullptr, nullptr, &sb);
     return sb;
 }
 

@@ -12,13 +12,13 @@ cudaError_t tc_bwd(const SeqView& s, const BwdArgs& a, void* ws, cudaStream_t st
 int tc_launches(bool backward);
 
 // Single stages of the path, for the pipelined segment chain.  A segment's
-// "keep" region (tc_keep_bytes) holds what its forward stages produce and its
-// backward stages read again: G, exp(G), -W, Khat, U^T, V_new^T and the
-// chunk-entry states.  A "slot" region (tc_slot_bytes) holds the backward's
-// per-chunk tiles dVi^T, dV_new^T, dS_C^T.  Both 256-byte aligned.
+// "keep" region (tc_keep_bytes) holds what its forward stages and its intra
+// stage produce for its later stages: G, exp(G), -W, L, Khat, U^T, V_new^T, the
+// chunk-entry states, dVi^T and D^T.  A "slot" region (tc_slot_bytes) holds
+// the reverse scan's per-chunk tiles dV_new^T, dS_C^T.  Both 256-byte aligned.
 //   Prep    (f): k, v, g, beta -> keep            Scan    (f): keep, S_in -> keep, S_out
-//   Out     (f): q, k, keep -> o                  Intra   (b): q, k, dO, keep -> slot
-//   ScanBwd (b): q, dO, keep, slot, dS_out -> slot, dS_in (no forward recompute)
+//   Out     (f): q, k, keep -> o                  Intra   (b): q, k, dO, keep (G) -> keep
+//   ScanBwd (b): keep, dS_out -> slot, dS_in (no forward recompute)
 //   Grad    (b): q, k, v, beta, dO, keep, slot -> dq, dk, dv, dg, dbeta
 enum class TcStage { Prep, Scan, Out, Intra, ScanBwd, Grad };
 size_t tc_keep_bytes(const SeqView& s);
