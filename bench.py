@@ -77,6 +77,12 @@ def kernel_work(name, w, T_seg):
         flops = nch * 2 * (2 * C * dk * dv) + nch * 2 * C * dk * dv
         byts = n * (es * (2 * dk + dv) + wu * dv * 2)
         return "tensor", flops, byts
+    if name.endswith("out_og"):
+        # Out plus the intra-chunk backward products: O, dVi = P^T dO, D = (gamma dO)^T Q
+        flops = nch * (2 * C * dk * dv + 2 * C * C * dk + 2 * C * C * dv) + nch * (2 * C * C * dv + 2 * C * dk * dv)
+        byts = (n * (es * (2 * dk + dv) + wu * dv + es * dv + es * dv + wu * dv)
+                + nch * dk * dv * wu * 2)
+        return "hbm", flops, byts
     if name.endswith("out"):
         flops = nch * (2 * C * dk * dv + 2 * C * C * dk + 2 * C * C * dv)
         byts = n * (es * (2 * dk + dv)) + nch * dk * dv * 4

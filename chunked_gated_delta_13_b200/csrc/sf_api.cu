@@ -228,7 +228,7 @@ PipeLayout pipe_layout(const sf_gdn_shape& s, const std::vector<int>& lens) {
 // outlives the call.
 struct Pipe {
     cudaStream_t user = nullptr, chain = nullptr, side = nullptr;
-    enum { kFork, kPrep, kScan, kIntra, kBwdScan, kGrad0, kJoinChain = kGrad0 + kSlots, kJoinSide, kNumEv };
+    enum { kFork, kPrep, kScan, kOut, kBwdScan, kGrad0, kJoinChain = kGrad0 + kSlots, kJoinSide, kNumEv };
     cudaEvent_t ev[kNumEv] = {};
     cudaError_t open(cudaStream_t u) {
         user = u;
@@ -262,9 +262,9 @@ struct Pipe {
 };
 
 // The segment chain of the tensor-core path, pipelined.  Forward: while the
-// forward scan of segment i runs on the chain stream, Pre and the intra-chunk
-// output gradient (OG) of segment i+1 and Out of segment i-1 run on the side
-// stream.  Backward: the parallel gradients (PG) of segment i+1 run beside the
+// forward scan of segment i runs on the chain stream, Pre of segment i+1 and
+// Out of segment i-1 (with the intra-chunk output gradient OG of that segment
+// when the backward follows) run on the side stream.  Backward: the parallel gradients (PG) of segment i+1 run beside the
 // reverse scan of segment i.  Each segment keeps its forward intermediates, so
 // the backward repeats neither Pre nor the forward state recompute.  Every
 // kernel computes exactly what it computes in sf_gdn_fwd / sf_gdn_bwd, so the
@@ -332,18 +332,13 @@ sf_status segment_run_pipelined(const sf_gdn_shape& s, const std::vector<int>& l
         if (e == cudaSuccess) e = cudaEventRecord(p.ev[i], src);
     };
 
-    // Forward.  Side stream order: Pre 0, OG 0, Pre 1, OG 1, Out 0, Pre 2, OG 2, Out 1, ...
-    bool any_intra = false;
+    // Forward.  Side stream order: Pre 0, Pre 1, Out 0, Pre 2, Out 1, ...
+    bool any_out = false;
     auto issue_prep = [&](int i) {
         if (lens[i] == 0) return;
         run(sf::TcStage::Prep, i, p.side);
         record(p.side, Pipe::kPrep);
         wait(p.chain, Pipe::kPrep);
-        if (B) {
-            run(sf::TcStage::Intra, i, p.side);
-            record(p.side, Pipe::kIntra);
-            any_intra = true;
-        }
     };
     chk(copy_state(state(0), F.S_in, nstate, p.chain));
     issue_prep(0);
@@ -357,20 +352,22 @@ sf_status segment_run_pipelined(const sf_gdn_shape& s, const std::vector<int>& l
         if (i + 1 < N) issue_prep(i + 1);
         if (lens[i] > 0) {
             wait(p.side, Pipe::kScan);
-            run(sf::TcStage::Out, i, p.side);
+            run(B ? sf::TcStage::OutOg : sf::TcStage::Out, i, p.side);
+            record(p.side, Pipe::kOut);
+            any_out = true;
         }
     }
     if (F.S_out) chk(copy_state(F.S_out, state(N), nstate, p.chain));
 
-    // Backward.  The reverse scans wait once for the last OG (the side stream
-    // ran every OG before it).  The slot of segment i (dV_new, dS_C) is next
+    // Backward.  The reverse scans wait once for the last Out/OG (the side
+    // stream ran every other one before it).  The slot of segment i (dV_new, dS_C) is next
     // written by the reverse scan of segment i - kSlots, which waits for the
     // PG that last read it.
     if (B && e == cudaSuccess) {
         float* cur = state(N + 1);
         float* nxt = state(N + 2);
         chk(copy_state(cur, B->dS_out, nstate, p.chain));
-        if (any_intra) wait(p.chain, Pipe::kIntra);
+        if (any_out) wait(p.chain, Pipe::kOut);
         bool slot_read[kSlots] = {};
         for (int i = N - 1; i >= 0 && e == cudaSuccess; --i) {
             ba[i].dS_out = cur;

@@ -354,6 +354,77 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 }
 
 // ----------------------------------------------------------------- intra ---
+// Intra-chunk parts of the backward that only read inputs: dVi^T = (P^T dO)^T
+// and D^T = (scale (gamma * dO)^T Q)^T, 4 warps, P in shared memory.
+template <int DV>
+__device__ __forceinline__ void og_products(const SeqView& s, const bf16* Qs, const bf16* dOs, const bf16* Ps,
+                                            const float* Gs, bf16* dVi, bf16* Dg, int w, int lane) {
+    constexpr int LDV = DV + 8;
+    constexpr int MT = DV / 64;  // 16-row m-tiles per warp
+    const int gq = lane >> 2, tq = lane & 3;
+    // dVi^T[v][j] = sum_i dO[i][v] P[i][j]
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int m0 = (w * MT + mt) * 16;
+        float acc[8][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t a[4];
+            ldAt(a, dOs, LDV, m0, 16 * kk, lane);
+#pragma unroll
+            for (int nn = 0; nn < 8; nn += 2) {
+                uint32_t b[4];
+                ldBkn(b, Ps, LDC, 8 * nn, 16 * kk, lane);
+                mma(acc[nn], a, b[0], b[1]);
+                mma(acc[nn + 1], a, b[2], b[3]);
+            }
+        }
+#pragma unroll
+        for (int nn = 0; nn < 8; ++nn) {
+            const int r = m0 + gq, j = 8 * nn + 2 * tq;
+            *reinterpret_cast<uint32_t*>(dVi + swz(r, j, C)) = pack(acc[nn][0], acc[nn][1]);
+            *reinterpret_cast<uint32_t*>(dVi + swz(r + 8, j, C)) = pack(acc[nn][2], acc[nn][3]);
+        }
+    }
+    // D^T[v][d] = sum_t scale gamma_t dO[t][v] Q[t][d]
+#pragma unroll 1
+    for (int mt = 0; mt < MT; ++mt) {
+        const int m0 = (w * MT + mt) * 16;
+        uint32_t a[4][4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            ldAt(a[kk], dOs, LDV, m0, 16 * kk, lane);
+            const int tk = 16 * kk + 2 * tq;
+            const float g0 = s.scale * __expf(Gs[tk]), g1 = s.scale * __expf(Gs[tk + 1]);
+            const float g2 = s.scale * __expf(Gs[tk + 8]), g3 = s.scale * __expf(Gs[tk + 9]);
+            a[kk][0] = scale2(a[kk][0], g0, g1);
+            a[kk][1] = scale2(a[kk][1], g0, g1);
+            a[kk][2] = scale2(a[kk][2], g2, g3);
+            a[kk][3] = scale2(a[kk][3], g2, g3);
+        }
+#pragma unroll 1
+        for (int nh = 0; nh < 2; ++nh) {
+            float acc[8][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                for (int nn = 0; nn < 8; nn += 2) {
+                    uint32_t b[4];
+                    ldBkn(b, Qs, LDK, 64 * nh + 8 * nn, 16 * kk, lane);
+                    mma(acc[nn], a[kk], b[0], b[1]);
+                    mma(acc[nn + 1], a[kk], b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int nn = 0; nn < 8; ++nn) {
+                const int r = m0 + gq, d = 64 * nh + 8 * nn + 2 * tq;
+                *reinterpret_cast<uint32_t*>(Dg + swz(r, d, DK)) = pack(acc[nn][0], acc[nn][1]);
+                *reinterpret_cast<uint32_t*>(Dg + swz(r + 8, d, DK)) = pack(acc[nn][2], acc[nn][3]);
+            }
+        }
+    }
+}
+
 template <int DV>
 constexpr size_t intra_smem() {
     return (size_t)C * LDK * 2 * 2 + (size_t)C * (DV + 8) * 2 + (size_t)C * LDC * 2 + C * 4;
@@ -409,70 +480,8 @@ tc_intra_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
             }
     }
     __syncthreads();
-    // dVi^T[v][j] = sum_i dO[i][v] P[i][j]
-    constexpr int MT = DV / 64;  // 16-row m-tiles per warp
-    bf16* dst = dVito + ((size_t)bh * s.NC + c) * DV * C;
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-        const int m0 = (w * MT + mt) * 16;
-        float acc[8][4] = {};
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            uint32_t a[4];
-            ldAt(a, dOs, LDV, m0, 16 * kk, lane);
-#pragma unroll
-            for (int nn = 0; nn < 8; nn += 2) {
-                uint32_t b[4];
-                ldBkn(b, Ps, LDC, 8 * nn, 16 * kk, lane);
-                mma(acc[nn], a, b[0], b[1]);
-                mma(acc[nn + 1], a, b[2], b[3]);
-            }
-        }
-#pragma unroll
-        for (int nn = 0; nn < 8; ++nn) {
-            const int r = m0 + gq, j = 8 * nn + 2 * tq;
-            *reinterpret_cast<uint32_t*>(dst + swz(r, j, C)) = pack(acc[nn][0], acc[nn][1]);
-            *reinterpret_cast<uint32_t*>(dst + swz(r + 8, j, C)) = pack(acc[nn][2], acc[nn][3]);
-        }
-    }
-    // D^T[v][d] = sum_t scale gamma_t dO[t][v] Q[t][d]
-    bf16* dd = Dto + ((size_t)bh * s.NC + c) * DV * DK;
-#pragma unroll 1
-    for (int mt = 0; mt < MT; ++mt) {
-        const int m0 = (w * MT + mt) * 16;
-        uint32_t a[4][4];
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            ldAt(a[kk], dOs, LDV, m0, 16 * kk, lane);
-            const int tk = 16 * kk + 2 * tq;
-            const float g0 = s.scale * __expf(Gs[tk]), g1 = s.scale * __expf(Gs[tk + 1]);
-            const float g2 = s.scale * __expf(Gs[tk + 8]), g3 = s.scale * __expf(Gs[tk + 9]);
-            a[kk][0] = scale2(a[kk][0], g0, g1);
-            a[kk][1] = scale2(a[kk][1], g0, g1);
-            a[kk][2] = scale2(a[kk][2], g2, g3);
-            a[kk][3] = scale2(a[kk][3], g2, g3);
-        }
-#pragma unroll 1
-        for (int nh = 0; nh < 2; ++nh) {
-            float acc[8][4] = {};
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-                for (int nn = 0; nn < 8; nn += 2) {
-                    uint32_t b[4];
-                    ldBkn(b, Qs, LDK, 64 * nh + 8 * nn, 16 * kk, lane);
-                    mma(acc[nn], a[kk], b[0], b[1]);
-                    mma(acc[nn + 1], a[kk], b[2], b[3]);
-                }
-            }
-#pragma unroll
-            for (int nn = 0; nn < 8; ++nn) {
-                const int r = m0 + gq, d = 64 * nh + 8 * nn + 2 * tq;
-                *reinterpret_cast<uint32_t*>(dd + swz(r, d, DK)) = pack(acc[nn][0], acc[nn][1]);
-                *reinterpret_cast<uint32_t*>(dd + swz(r + 8, d, DK)) = pack(acc[nn][2], acc[nn][3]);
-            }
-        }
-    }
+    const size_t ci = (size_t)bh * s.NC + c;
+    og_products<DV>(s, Qs, dOs, Ps, Gs, dVito + ci * DV * C, Dto + ci * DV * DK, w, lane);
 }
 
 // ------------------------------------------------------------ state scans ---
@@ -989,23 +998,29 @@ tc_scan_bwd_dual_kernel(SeqView s, const bf16* __restrict__ Dt,
 }
 
 // ------------------------------------------------------------------- out ---
-template <int DV>
+template <int DV, bool OG>
 constexpr size_t out_smem() {
-    return (size_t)C * LDK * 2 * 2 + (size_t)DV * LDK * 2 + (size_t)DV * LDC * 2 + C * 4;
+    return (size_t)C * LDK * 2 * 2 + (size_t)DV * LDK * 2 + (size_t)DV * LDC * 2 + C * 4 +
+           (OG ? (size_t)C * (DV + 8) * 2 : 0);
 }
 
 // O = scale (gamma * Q) S0 + (scale (Q K^T) * Gamma) V_new; 4 warps x 16 rows.
-template <int DV>
+// With OG (the forward of a segment whose backward follows), the same CTA also
+// writes the intra-chunk backward products of og_products, reusing Q and P.
+template <int DV, bool OG>
 __global__ void __launch_bounds__(128)
 tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
               const float* __restrict__ Gc, const bf16* __restrict__ Vnt,
-              const bf16* __restrict__ S0t, bf16* __restrict__ o) {
+              const bf16* __restrict__ S0t, bf16* __restrict__ o, const bf16* __restrict__ dO,
+              bf16* __restrict__ dVito, bf16* __restrict__ Dto) {
+    constexpr int LDV = DV + 8;
     extern __shared__ __align__(16) unsigned char smem[];
     bf16* Qs = reinterpret_cast<bf16*>(smem);
-    bf16* Ks = Qs + C * LDK;
+    bf16* Ks = Qs + C * LDK;     // later (OG): P [C][LDC]
     bf16* S0s = Ks + C * LDK;   // [DV][LDK]
     bf16* Vns = S0s + DV * LDK;  // [DV][LDC]
     float* Gs = reinterpret_cast<float*>(Vns + DV * LDC);
+    bf16* dOs = reinterpret_cast<bf16*>(Gs + C);  // [C][LDV] (OG)
     const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int gq = lane >> 2, tq = lane & 3;
     const int t0 = c * C;
@@ -1017,7 +1032,13 @@ tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
     load_tile_swz<DV, C, 128>(Vns, LDC, Vnt + ((size_t)bh * s.NC + c) * DV * C, tid);
     if (tid < 16) cp_async16(Gs + tid * 4, Gc + bh * Tp + t0 + tid * 4, true);
     cp_async_commit();
-    cp_async_wait<0>();
+    if (OG) {
+        load_tile<C, DV, 128>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+        cp_async_commit();
+        cp_async_wait<1>();
+    } else {
+        cp_async_wait<0>();
+    }
     __syncthreads();
 
     float p[8][4] = {};
@@ -1058,6 +1079,16 @@ tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
             const int i = (e >> 1) ? i1 : i0, j = 8 * nn + 2 * tq + (e & 1);
             p[nn][e] = (j <= i) ? s.scale * __expf(((e >> 1) ? G1 : G0) - Gs[j]) * p[nn][e] : 0.f;
         }
+    bf16* Ps = Ks;
+    if (OG) {
+        __syncthreads();  // every warp is done reading K
+#pragma unroll
+        for (int nn = 0; nn < 8; ++nn) {
+            const int j = 8 * nn + 2 * tq;
+            *reinterpret_cast<uint32_t*>(Ps + i0 * LDC + j) = pack(p[nn][0], p[nn][1]);
+            *reinterpret_cast<uint32_t*>(Ps + i1 * LDC + j) = pack(p[nn][2], p[nn][3]);
+        }
+    }
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
         uint32_t a[4];
@@ -1076,6 +1107,12 @@ tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
         const int col = 8 * nn + 2 * tq;
         if (i0 < nval) *reinterpret_cast<uint32_t*>(ob + (size_t)i0 * DV + col) = pack(acc[nn][0], acc[nn][1]);
         if (i1 < nval) *reinterpret_cast<uint32_t*>(ob + (size_t)i1 * DV + col) = pack(acc[nn][2], acc[nn][3]);
+    }
+    if (OG) {
+        cp_async_wait<0>();
+        __syncthreads();  // P and dO are visible
+        const size_t ci = (size_t)bh * s.NC + c;
+        og_products<DV>(s, Qs, dOs, Ps, Gs, dVito + ci * DV * C, Dto + ci * DV * DK, w, lane);
     }
 }
 
@@ -1671,9 +1708,20 @@ cudaError_t launch_scan_fwd(const SeqView& s, const float* S_in, float* S_out, c
 
 template <int DV>
 cudaError_t launch_out(const SeqView& s, const bf16* q, const bf16* k, bf16* o, const TcWs& w, cudaStream_t st) {
-    constexpr size_t sm = out_smem<DV>();
-    TC_TRY(smem_attr(tc_out_kernel<DV>, sm));
-    SF_LAUNCH("tc_out", st, tc_out_kernel<DV><<<dim3(s.NC, s.BH), 128, sm, st>>>(s, q, k, w.Gc, w.Vnt, w.S0t, o));
+    constexpr size_t sm = out_smem<DV, false>();
+    TC_TRY(smem_attr(tc_out_kernel<DV, false>, sm));
+    SF_LAUNCH("tc_out", st, tc_out_kernel<DV, false><<<dim3(s.NC, s.BH), 128, sm, st>>>(
+                                s, q, k, w.Gc, w.Vnt, w.S0t, o, nullptr, nullptr, nullptr));
+    return cudaGetLastError();
+}
+
+template <int DV>
+cudaError_t launch_out_og(const SeqView& s, const bf16* q, const bf16* k, bf16* o, const bf16* dO, const TcWs& w,
+                          cudaStream_t st) {
+    constexpr size_t sm = out_smem<DV, true>();
+    TC_TRY(smem_attr(tc_out_kernel<DV, true>, sm));
+    SF_LAUNCH("tc_out_og", st, tc_out_kernel<DV, true><<<dim3(s.NC, s.BH), 128, sm, st>>>(
+                                   s, q, k, w.Gc, w.Vnt, w.S0t, o, dO, w.dVit, w.Dt));
     return cudaGetLastError();
 }
 
@@ -1748,6 +1796,9 @@ cudaError_t stage_impl(TcStage stage, const SeqView& s, const FwdArgs* f, const 
         case TcStage::Out:
             return launch_out<DV>(s, static_cast<const bf16*>(f->q), static_cast<const bf16*>(f->k),
                                   static_cast<bf16*>(f->o), w, st);
+        case TcStage::OutOg:
+            return launch_out_og<DV>(s, static_cast<const bf16*>(f->q), static_cast<const bf16*>(f->k),
+                                     static_cast<bf16*>(f->o), static_cast<const bf16*>(b->dO), w, st);
         case TcStage::Intra:
             return launch_intra<DV>(s, static_cast<const bf16*>(b->q), static_cast<const bf16*>(b->k),
                                     static_cast<const bf16*>(b->dO), w, st);

@@ -18,9 +18,10 @@ int tc_launches(bool backward);
 // the reverse scan's per-chunk tiles dV_new^T, dS_C^T.  Both 256-byte aligned.
 //   Prep    (f): k, v, g, beta -> keep            Scan    (f): keep, S_in -> keep, S_out
 //   Out     (f): q, k, keep -> o                  Intra   (b): q, k, dO, keep (G) -> keep
+//   OutOg (f, b): Out and Intra of one segment in one launch
 //   ScanBwd (b): keep, dS_out -> slot, dS_in (no forward recompute)
 //   Grad    (b): q, k, v, beta, dO, keep, slot -> dq, dk, dv, dg, dbeta
-enum class TcStage { Prep, Scan, Out, Intra, ScanBwd, Grad };
+enum class TcStage { Prep, Scan, Out, OutOg, Intra, ScanBwd, Grad };
 size_t tc_keep_bytes(const SeqView& s);
 size_t tc_slot_bytes(const SeqView& s);
 cudaError_t tc_stage(TcStage stage, const SeqView& s, const FwdArgs* f, const BwdArgs* b, void* keep, void* slot,
