@@ -221,50 +221,62 @@ PipeLayout pipe_layout(const sf_gdn_shape& s, const std::vector<int>& lens) {
     return L;
 }
 
-// Two streams of one call, forked from and joined back to the caller's stream:
-// `chain` (highest priority) runs the state chains in order, `side` (lowest
-// priority) the chunk-parallel kernels, which fill the SMs the chains leave
-// idle.  Created per call and released asynchronously at its end, so nothing
+// Three streams of one call, forked from and joined back to the caller's
+// stream: `chain` (highest priority) runs the state chains in order; `pre`
+// (middle priority) runs Pre of every segment ahead of the chain; `side`
+// (lowest priority) runs Out.  In the backward, PG alternates between `side`
+// and `pre`, so one segment's kernel fills the last wave of the previous
+// one.  Created per call and released asynchronously at its end, so nothing
 // outlives the call.
 struct Pipe {
-    cudaStream_t user = nullptr, chain = nullptr, side = nullptr;
-    enum { kFork, kPrep, kScan, kOut, kBwdScan, kGrad0, kJoinChain = kGrad0 + kSlots, kJoinSide, kNumEv };
+    cudaStream_t user = nullptr, chain = nullptr, pre = nullptr, side = nullptr;
+    enum { kFork, kScan, kOut, kBwdScan, kGrad0, kJoin = kGrad0 + kSlots, kNumEv = kJoin + 3 };
     cudaEvent_t ev[kNumEv] = {};
-    cudaError_t open(cudaStream_t u) {
+    std::vector<cudaEvent_t> prep_done;  // one per segment
+    cudaError_t open(cudaStream_t u, int nseg) {
         user = u;
         int least = 0, greatest = 0;
         cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+        const int middle = (least + greatest) / 2;
         if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&chain, cudaStreamNonBlocking, greatest);
+        if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&pre, cudaStreamNonBlocking, middle);
         if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&side, cudaStreamNonBlocking, least);
         for (int i = 0; i < kNumEv && e == cudaSuccess; ++i)
             e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+        prep_done.assign(nseg, nullptr);
+        for (int i = 0; i < nseg && e == cudaSuccess; ++i)
+            e = cudaEventCreateWithFlags(&prep_done[i], cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventRecord(ev[kFork], user);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(chain, ev[kFork], 0);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev[kFork], 0);
+        for (cudaStream_t x : {chain, pre, side})
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(x, ev[kFork], 0);
         return e;
     }
-    // Stream dst waits for all work enqueued so far on src (through event i).
-    cudaError_t after(cudaStream_t dst, cudaStream_t src, int i) {
-        cudaError_t e = cudaEventRecord(ev[i], src);
-        return e == cudaSuccess ? cudaStreamWaitEvent(dst, ev[i], 0) : e;
-    }
     cudaError_t join() {
-        cudaError_t e = after(user, chain, kJoinChain);
-        cudaError_t e2 = after(user, side, kJoinSide);
-        return e != cudaSuccess ? e : e2;
+        cudaError_t first = cudaSuccess;
+        int i = kJoin;
+        for (cudaStream_t x : {chain, pre, side}) {
+            cudaError_t e = cudaEventRecord(ev[i], x);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(user, ev[i], 0);
+            if (first == cudaSuccess) first = e;
+            ++i;
+        }
+        return first;
     }
     ~Pipe() {
         for (cudaEvent_t x : ev)
             if (x) cudaEventDestroy(x);
-        if (chain) cudaStreamDestroy(chain);
-        if (side) cudaStreamDestroy(side);
+        for (cudaEvent_t x : prep_done)
+            if (x) cudaEventDestroy(x);
+        for (cudaStream_t x : {chain, pre, side})
+            if (x) cudaStreamDestroy(x);
     }
 };
 
-// The segment chain of the tensor-core path, pipelined.  Forward: while the
-// forward scan of segment i runs on the chain stream, Pre of segment i+1 and
-// Out of segment i-1 (with the intra-chunk output gradient OG of that segment
-// when the backward follows) run on the side stream.  Backward: the parallel gradients (PG) of segment i+1 run beside the
+// The segment chain of the tensor-core path, pipelined.  Forward: Pre of every
+// segment runs ahead on its own stream; while the forward scan of segment i
+// runs on the chain stream, Out of segment i-1 (with the intra-chunk output
+// gradient OG of that segment when the backward follows) runs on the side
+// stream.  Backward: the parallel gradients (PG) of segment i+1 run beside the
 // reverse scan of segment i.  Each segment keeps its forward intermediates, so
 // the backward repeats neither Pre nor the forward state recompute.  Every
 // kernel computes exactly what it computes in sf_gdn_fwd / sf_gdn_bwd, so the
@@ -315,7 +327,7 @@ sf_status segment_run_pipelined(const sf_gdn_shape& s, const std::vector<int>& l
     }
 
     Pipe p;
-    cudaError_t e = p.open(user);
+    cudaError_t e = p.open(user, N);
     const bool opened = e == cudaSuccess;
     auto chk = [&](cudaError_t x) {
         if (e == cudaSuccess) e = x;
@@ -332,24 +344,23 @@ sf_status segment_run_pipelined(const sf_gdn_shape& s, const std::vector<int>& l
         if (e == cudaSuccess) e = cudaEventRecord(p.ev[i], src);
     };
 
-    // Forward.  Side stream order: Pre 0, Pre 1, Out 0, Pre 2, Out 1, ...
+    // Forward.  Pre of every segment first (pre stream), then the chain with
+    // Out of each segment behind its scan (side stream).
     bool any_out = false;
-    auto issue_prep = [&](int i) {
-        if (lens[i] == 0) return;
-        run(sf::TcStage::Prep, i, p.side);
-        record(p.side, Pipe::kPrep);
-        wait(p.chain, Pipe::kPrep);
-    };
+    for (int i = 0; i < N; ++i) {
+        if (lens[i] == 0) continue;
+        run(sf::TcStage::Prep, i, p.pre);
+        if (e == cudaSuccess) e = cudaEventRecord(p.prep_done[i], p.pre);
+    }
     chk(copy_state(state(0), F.S_in, nstate, p.chain));
-    issue_prep(0);
     for (int i = 0; i < N && e == cudaSuccess; ++i) {
         if (lens[i] > 0) {
+            chk(cudaStreamWaitEvent(p.chain, p.prep_done[i], 0));
             run(sf::TcStage::Scan, i, p.chain);
             record(p.chain, Pipe::kScan);
         } else {
             chk(copy_state(state(i + 1), state(i), nstate, p.chain));
         }
-        if (i + 1 < N) issue_prep(i + 1);
         if (lens[i] > 0) {
             wait(p.side, Pipe::kScan);
             run(B ? sf::TcStage::OutOg : sf::TcStage::Out, i, p.side);
@@ -376,9 +387,10 @@ sf_status segment_run_pipelined(const sf_gdn_shape& s, const std::vector<int>& l
                 if (slot_read[i % kSlots]) wait(p.chain, Pipe::kGrad0 + i % kSlots);
                 run(sf::TcStage::ScanBwd, i, p.chain);
                 record(p.chain, Pipe::kBwdScan);
-                wait(p.side, Pipe::kBwdScan);
-                run(sf::TcStage::Grad, i, p.side);
-                record(p.side, Pipe::kGrad0 + i % kSlots);
+                cudaStream_t gs = (i & 1) ? p.pre : p.side;
+                wait(gs, Pipe::kBwdScan);
+                run(sf::TcStage::Grad, i, gs);
+                record(gs, Pipe::kGrad0 + i % kSlots);
                 slot_read[i % kSlots] = true;
             } else {
                 chk(copy_state(nxt, cur, nstate, p.chain));

@@ -1190,16 +1190,17 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     const int nval = min(C, s.T - t0);
     const size_t Tp = (size_t)s.NC * C;
     const size_t ci = (size_t)bh * s.NC + c;
-    // Two copy groups: what the state products of phase S read, then Q, K, V.
+    // Two copy groups: what phase C1 reads (Q, K, dO, V_new), then the state
+    // tiles of phase S and V, which land while C1 runs.
+    load_tile<C, DK, GTH>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+    load_tile<C, DK, GTH>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
     load_tile<C, DV, GTH>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
     load_tile_swz<DV, C, GTH>(Vns, LDC, Vnt + ci * DV * C, tid);
+    if (tid < 16) cp_async16(Gs + tid * 4, Gc + bh * Tp + t0 + tid * 4, true);
+    cp_async_commit();
     load_tile_swz<DV, C, GTH>(dVns, LDC, dVnt + ci * DV * C, tid);
     load_tile_swz<DV, DK, GTH>(S0s, LDK, S0t + ci * DV * DK, tid);
     load_tile_swz<DV, DK, GTH>(dSs, LDK, dSCt + ci * DV * DK, tid);
-    if (tid < 16) cp_async16(Gs + tid * 4, Gc + bh * Tp + t0 + tid * 4, true);
-    cp_async_commit();
-    load_tile<C, DK, GTH>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
-    load_tile<C, DK, GTH>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
     load_tile<C, DV, GTH>(Vs, LDV, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
     cp_async_commit();
     for (int i = tid; i < C; i += GTH) Bs[i] = (BETA && i < nval) ? beta[bh * s.hs_g + t0 + i] : 0.f;
@@ -1212,97 +1213,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     const float gC = Gs[C - 1];
     const float dec0 = __expf(gC - Gs[r0]), dec1 = __expf(gC - Gs[r1]);
 
-    // ---- phase S: products with the chunk-entry state and the state gradient
-    float accQ[DKW / 8][4] = {}, accK[DKW / 8][4] = {};
-    {
-        float accW[DKW / 8][4] = {};
-#pragma unroll
-        for (int kv = 0; kv < DV / 16; ++kv) {
-            uint32_t aO[4], aN[4], aV[4];
-            ldA(aO, dOs, LDV, 16 * mw, 16 * kv, lane);
-            ldAt(aN, dVns, LDC, 16 * mw, 16 * kv, lane);
-            ldAt(aV, Vns, LDC, 16 * mw, 16 * kv, lane);
-#pragma unroll
-            for (int nn = 0; nn < DKW / 8; nn += 2) {
-                uint32_t b[4];
-                ldBkn(b, S0s, LDK, DKW * nw + 8 * nn, 16 * kv, lane);
-                mma(accQ[nn], aO, b[0], b[1]);
-                mma(accQ[nn + 1], aO, b[2], b[3]);
-                mma(accW[nn], aN, b[0], b[1]);
-                mma(accW[nn + 1], aN, b[2], b[3]);
-                ldBkn(b, dSs, LDK, DKW * nw + 8 * nn, 16 * kv, lane);
-                mma(accK[nn], aV, b[0], b[1]);
-                mma(accK[nn + 1], aV, b[2], b[3]);
-            }
-        }
-        cp_async_wait<0>();
-        __syncthreads();  // Q, K, V have landed
-        float pd = 0.f;  // <S0, dS_C>
-        for (int e = tid; e < DV * DK; e += GTH) {
-            const int r = e / DK, cc = e % DK;
-            pd += __bfloat162float(S0s[r * LDK + cc]) * __bfloat162float(dSs[r * LDK + cc]);
-        }
-        red[tid] = pd;
-        // dq_inter = scale gamma (dO S0^T); dK_state = dec (V_new dS_C^T)
-        const float sq0 = s.scale * gam0, sq1 = s.scale * gam1;
-        float pi0 = 0.f, pi1 = 0.f, pz0 = 0.f, pz1 = 0.f;
-#pragma unroll
-        for (int nn = 0; nn < DKW / 8; ++nn) {
-            const int col = DKW * nw + 8 * nn + 2 * tq;
-            const float2 q0 = unpack(*reinterpret_cast<const uint32_t*>(Qs + r0 * LDK + col));
-            const float2 q1 = unpack(*reinterpret_cast<const uint32_t*>(Qs + r1 * LDK + col));
-            const float2 k0 = unpack(*reinterpret_cast<const uint32_t*>(Ks + r0 * LDK + col));
-            const float2 k1 = unpack(*reinterpret_cast<const uint32_t*>(Ks + r1 * LDK + col));
-            accQ[nn][0] *= sq0;
-            accQ[nn][1] *= sq0;
-            accQ[nn][2] *= sq1;
-            accQ[nn][3] *= sq1;
-            accK[nn][0] *= dec0;
-            accK[nn][1] *= dec0;
-            accK[nn][2] *= dec1;
-            accK[nn][3] *= dec1;
-            pi0 += q0.x * accQ[nn][0] + q0.y * accQ[nn][1];
-            pi1 += q1.x * accQ[nn][2] + q1.y * accQ[nn][3];
-            pz0 += k0.x * accK[nn][0] + k0.y * accK[nn][1];
-            pz1 += k1.x * accK[nn][2] + k1.y * accK[nn][3];
-        }
-#pragma unroll
-        for (int o = 1; o < 4; o <<= 1) {
-            pi0 += __shfl_xor_sync(0xffffffffu, pi0, o);
-            pi1 += __shfl_xor_sync(0xffffffffu, pi1, o);
-            pz0 += __shfl_xor_sync(0xffffffffu, pz0, o);
-            pz1 += __shfl_xor_sync(0xffffffffu, pz1, o);
-        }
-        if (tq == 0) {
-            part[(P_INTER + nw) * C + r0] = pi0;
-            part[(P_INTER + nw) * C + r1] = pi1;
-            part[(P_Z + nw) * C + r0] = pz0;
-            part[(P_Z + nw) * C + r1] = pz1;
-        }
-        __syncthreads();  // everyone is done with S0^T and dS_C^T
-        if (BETA) {  // L of this chunk (from the prep kernel) into Lf; waited for before phase C2
-            const float* Lg = Lm + ci * C * C;
-            for (int e = tid; e < C * C / 4; e += GTH) {
-                const int i = e >> 4, j = (e & 15) * 4;
-                cp_async16(Lf + i * LDF + j, Lg + i * C + j, true);
-            }
-            cp_async_commit();
-        }
-        // dW = -dV_new S0^T into the freed region
-#pragma unroll
-        for (int nn = 0; nn < DKW / 8; ++nn) {
-            const int col = DKW * nw + 8 * nn + 2 * tq;
-            *reinterpret_cast<uint32_t*>(dWs + r0 * LDK + col) = pack(-accW[nn][0], -accW[nn][1]);
-            *reinterpret_cast<uint32_t*>(dWs + r1 * LDK + col) = pack(-accW[nn][2], -accW[nn][3]);
-        }
-    }
-    for (int o = GTH / 2; o > 0; o >>= 1) {
-        if (tid < o) red[tid] += red[tid + o];
-        __syncthreads();
-    }
-    const float sdot = red[0];
-
-    // ---- phase C1: C x C products (rows 16mw.., columns 32nw..)
+    // ---- phase C1: C x C products (rows 16mw.., columns CW nw..); reads only the first copy group
     float kkr[CW / 8][4] = {};
     {
         float qk[CW / 8][4] = {}, dp[CW / 8][4] = {};
@@ -1368,6 +1279,97 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
             part[(P_ROWP + nw) * C + r1] = row1;
         }
     }
+    cp_async_wait<0>();
+    __syncthreads();  // the state tiles and V have landed
+
+    // ---- phase S: products with the chunk-entry state and the state gradient
+    float accQ[DKW / 8][4] = {}, accK[DKW / 8][4] = {};
+    {
+        float accW[DKW / 8][4] = {};
+#pragma unroll
+        for (int kv = 0; kv < DV / 16; ++kv) {
+            uint32_t aO[4], aN[4], aV[4];
+            ldA(aO, dOs, LDV, 16 * mw, 16 * kv, lane);
+            ldAt(aN, dVns, LDC, 16 * mw, 16 * kv, lane);
+            ldAt(aV, Vns, LDC, 16 * mw, 16 * kv, lane);
+#pragma unroll
+            for (int nn = 0; nn < DKW / 8; nn += 2) {
+                uint32_t b[4];
+                ldBkn(b, S0s, LDK, DKW * nw + 8 * nn, 16 * kv, lane);
+                mma(accQ[nn], aO, b[0], b[1]);
+                mma(accQ[nn + 1], aO, b[2], b[3]);
+                mma(accW[nn], aN, b[0], b[1]);
+                mma(accW[nn + 1], aN, b[2], b[3]);
+                ldBkn(b, dSs, LDK, DKW * nw + 8 * nn, 16 * kv, lane);
+                mma(accK[nn], aV, b[0], b[1]);
+                mma(accK[nn + 1], aV, b[2], b[3]);
+            }
+        }
+        float pd = 0.f;  // <S0, dS_C>
+        for (int e = tid; e < DV * DK; e += GTH) {
+            const int r = e / DK, cc = e % DK;
+            pd += __bfloat162float(S0s[r * LDK + cc]) * __bfloat162float(dSs[r * LDK + cc]);
+        }
+        red[tid] = pd;
+        // dq_inter = scale gamma (dO S0^T); dK_state = dec (V_new dS_C^T)
+        const float sq0 = s.scale * gam0, sq1 = s.scale * gam1;
+        float pi0 = 0.f, pi1 = 0.f, pz0 = 0.f, pz1 = 0.f;
+#pragma unroll
+        for (int nn = 0; nn < DKW / 8; ++nn) {
+            const int col = DKW * nw + 8 * nn + 2 * tq;
+            const float2 q0 = unpack(*reinterpret_cast<const uint32_t*>(Qs + r0 * LDK + col));
+            const float2 q1 = unpack(*reinterpret_cast<const uint32_t*>(Qs + r1 * LDK + col));
+            const float2 k0 = unpack(*reinterpret_cast<const uint32_t*>(Ks + r0 * LDK + col));
+            const float2 k1 = unpack(*reinterpret_cast<const uint32_t*>(Ks + r1 * LDK + col));
+            accQ[nn][0] *= sq0;
+            accQ[nn][1] *= sq0;
+            accQ[nn][2] *= sq1;
+            accQ[nn][3] *= sq1;
+            accK[nn][0] *= dec0;
+            accK[nn][1] *= dec0;
+            accK[nn][2] *= dec1;
+            accK[nn][3] *= dec1;
+            pi0 += q0.x * accQ[nn][0] + q0.y * accQ[nn][1];
+            pi1 += q1.x * accQ[nn][2] + q1.y * accQ[nn][3];
+            pz0 += k0.x * accK[nn][0] + k0.y * accK[nn][1];
+            pz1 += k1.x * accK[nn][2] + k1.y * accK[nn][3];
+        }
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+            pi0 += __shfl_xor_sync(0xffffffffu, pi0, o);
+            pi1 += __shfl_xor_sync(0xffffffffu, pi1, o);
+            pz0 += __shfl_xor_sync(0xffffffffu, pz0, o);
+            pz1 += __shfl_xor_sync(0xffffffffu, pz1, o);
+        }
+        if (tq == 0) {
+            part[(P_INTER + nw) * C + r0] = pi0;
+            part[(P_INTER + nw) * C + r1] = pi1;
+            part[(P_Z + nw) * C + r0] = pz0;
+            part[(P_Z + nw) * C + r1] = pz1;
+        }
+        __syncthreads();  // everyone is done with S0^T and dS_C^T
+        if (BETA) {  // L of this chunk (from the prep kernel) into Lf; waited for before phase C2
+            const float* Lg = Lm + ci * C * C;
+            for (int e = tid; e < C * C / 4; e += GTH) {
+                const int i = e >> 4, j = (e & 15) * 4;
+                cp_async16(Lf + i * LDF + j, Lg + i * C + j, true);
+            }
+            cp_async_commit();
+        }
+        // dW = -dV_new S0^T into the freed region
+#pragma unroll
+        for (int nn = 0; nn < DKW / 8; ++nn) {
+            const int col = DKW * nw + 8 * nn + 2 * tq;
+            *reinterpret_cast<uint32_t*>(dWs + r0 * LDK + col) = pack(-accW[nn][0], -accW[nn][1]);
+            *reinterpret_cast<uint32_t*>(dWs + r1 * LDK + col) = pack(-accW[nn][2], -accW[nn][3]);
+        }
+    }
+    for (int o = GTH / 2; o > 0; o >>= 1) {
+        if (tid < o) red[tid] += red[tid + o];
+        __syncthreads();
+    }
+    const float sdot = red[0];
+
     if (BETA) cp_async_wait<0>();
     __syncthreads();
 
