@@ -59,44 +59,64 @@ def algo_bytes_per_token_head(dk, dv, esize=2, use_beta=True):
 
 def kernel_work(name, w, T_seg):
     """(bound, algorithmic flops, algorithmic bytes) of ONE launch of `name`
-    on a segment of T_seg tokens (all B*H heads)."""
+    on a segment of T_seg tokens (all B*H heads).  Flops count the products the
+    kernel contributes to the method (no recompute); bytes count what the
+    kernel must read and write: its share of the ABI tensors plus the
+    per-chunk intermediates of the chunked decomposition (bf16 tiles, fp32 G and
+    L), each once."""
     C, dk, dv = w.C, w.dk, w.dv
     es = 2 if w.io == "bf16" else 4
     n = w.B * w.H * T_seg                      # token-heads in the launch
     nch = w.B * w.H * ((T_seg + C - 1) // C)   # chunk-heads in the launch
-    wu = 4 if name.startswith("simt") else 2   # W/U/V_new storage bytes per element
-    if name.endswith("prep"):
-        flops = nch * (2 * C * C * dk + 2 * C * C * dk + 2 * C * C * dv)
-        byts = n * (es * (dk + dv) + 8 + wu * (dk + dv))
+    wu = 4 if name.startswith("simt") else 2   # intermediate storage bytes per element
+    gb = 8 if w.use_beta else 4                # g (and beta) per token
+    lb = C * C * 4 if w.use_beta else 0        # L per chunk
+    state = dk * dv * wu                       # one chunk state tile
+    if name.endswith("prep"):                  # k, v, g, beta -> G, exp G, -W, Khat, U^T, L
+        flops = nch * (2 * C * C * dk * (2 if w.use_beta else 0) + 2 * C * C * dv * (1 if w.use_beta else 0))
+        byts = n * (es * (dk + dv) + gb + 8 + wu * (2 * dk + dv)) + nch * lb
         return "hbm", flops, byts
-    if name.endswith("scan_fwd"):
+    if name.endswith("scan_fwd"):              # -W, Khat, U^T, exp G -> V_new^T, chunk states
         flops = nch * 2 * (2 * C * dk * dv)
-        byts = n * (wu * (dk + dv) + es * dk + wu * dv)
+        byts = n * (wu * (2 * dk + dv) + 4 + wu * dv) + nch * state
         return "tensor", flops, byts
-    if name.endswith("scan_bwd"):
-        flops = nch * 2 * (2 * C * dk * dv) + nch * 2 * C * dk * dv
-        byts = n * (es * (2 * dk + dv) + wu * dv * 2)
+    if name.endswith("scan_bwd"):              # -W, Khat, dVi^T, exp G, D^T -> dV_new^T, dS_C^T
+        flops = nch * 2 * (2 * C * dk * dv)
+        byts = n * (wu * (2 * dk + dv) + 4 + wu * dv) + nch * 2 * state
         return "tensor", flops, byts
-    if name.endswith("out_og"):
-        # Out plus the intra-chunk backward products: O, dVi = P^T dO, D = (gamma dO)^T Q
+    if name.endswith("out_og"):                # q, k, dO, G, V_new^T, S0^T -> o, dVi^T, D^T
         flops = nch * (2 * C * dk * dv + 2 * C * C * dk + 2 * C * C * dv) + nch * (2 * C * C * dv + 2 * C * dk * dv)
-        byts = (n * (es * (2 * dk + dv) + wu * dv + es * dv + es * dv + wu * dv)
-                + nch * dk * dv * wu * 2)
+        byts = n * (es * (2 * dk + dv) + 4 + wu * dv + es * dv + wu * dv) + nch * 2 * state
         return "hbm", flops, byts
-    if name.endswith("out"):
+    if name.endswith("out"):                   # q, k, G, V_new^T, S0^T -> o
         flops = nch * (2 * C * dk * dv + 2 * C * C * dk + 2 * C * C * dv)
-        byts = n * (es * (2 * dk + dv)) + nch * dk * dv * 4
+        byts = n * (es * 2 * dk + 4 + wu * dv + es * dv) + nch * state
         return "hbm", flops, byts
-    if name.endswith("intra"):
-        flops = nch * (2 * C * C * dk + 2 * C * C * dv)
-        byts = n * (es * (2 * dk + dv) + wu * dv)
+    if name.endswith("intra"):                 # q, k, dO, G -> dVi^T, D^T
+        flops = nch * (2 * C * C * dk + 2 * C * C * dv + 2 * C * dk * dv)
+        byts = n * (es * (2 * dk + dv) + 4 + wu * dv) + nch * state
         return "hbm", flops, byts
-    # parallel gradient kernel: dP K, dP^T Q, dW (gamma K)^T, T^T dW, dA K (C^2 dk each),
-    # dO V_new^T, dU V^T, T^T dU (C^2 dv each), dO S0^T, V_new dS^T, dV_new S0^T (C dk dv each)
+    # parallel gradients: dP K, dP^T Q, dW (gamma K)^T, T^T dW, dA K (C^2 dk each),
+    # dO V_new^T, dU V^T, T^T dU (C^2 dv each), dO S0^T, V_new dS^T, dV_new S0^T (C dk dv each);
+    # q, k, v, dO, g, beta, V_new, dV_new, S0, dS_C, L -> dq, dk, dv, dg, dbeta
     flops = nch * (2 * C * C * 5 * dk + 2 * C * C * 3 * dv + 3 * 2 * C * dk * dv)
-    byts = (n * (es * (2 * dk + 2 * dv) + 8 + 2 * wu * dv + es * (2 * dk + dv) + 8)
-            + nch * 2 * dk * dv * 4)
+    byts = (n * (es * (2 * dk + 2 * dv) + gb + 2 * wu * dv + es * (2 * dk + dv) + gb)
+            + nch * (2 * state + lb))
     return "hbm", flops, byts
+
+
+# DRAM bytes (read + write) per chunk-head measured by ncu for each kernel of the
+# tensor-core path (B=1, H=16, T=8192, d=128, one segment: 2048 chunk-heads per
+# launch; summary and command in profiles/ncu_full_h16_t8k.md).  A launch's
+# traffic is this figure times its chunk-heads.  Valid for the kernels as they
+# were when captured; an entry is removed when its kernel changes.
+MEASURED_TRAFFIC = {
+    "tc_prep": 150.90e6 / 2048,
+    "tc_scan_fwd": 161.25e6 / 2048,
+    "tc_out_og": 293.45e6 / 2048,
+    "tc_scan_bwd": 238.72e6 / 2048,
+    "tc_grad": 452.10e6 / 2048,
+}
 
 
 # ---------------------------------------------------------------- helpers ---
@@ -385,9 +405,16 @@ def run_ours(args):
     dom = max(tot, key=tot.get) if tot else None
     roof = None
     if dom:
+        # the library cuts segments into pipeline pieces, so a launch covers a
+        # share of the step: per-launch work = the step's work / launches per step
+        per_step = len(per[dom]) / args.steps
         T_seg = -(-w.T // seg)
         bound, flops, byts = kernel_work(dom, w, T_seg)
+        flops, byts = flops * seg / per_step, byts * seg / per_step
         avg_ms = tot[dom] / len(per[dom])
+        nch_launch = w.B * w.H * (-(-T_seg // w.C)) * seg / per_step
+        traffic = (MEASURED_TRAFFIC[dom] * nch_launch if dom in MEASURED_TRAFFIC and w.io == "bf16"
+                   and w.dk == 128 and w.dv == 128 and w.C == 64 else None)
         if bound == "hbm":
             ach = byts / (avg_ms * 1e-3) / 1e9
             peak = pk["hbm_gbs"]
@@ -397,7 +424,7 @@ def run_ours(args):
             peak = pk["bf16_tflops_sustained"]
             unit = "TFLOP/s"
         roof = {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
-                "traffic": None, "kernel": dom, "avg_launch_ms": avg_ms,
+                "traffic": traffic, "kernel": dom, "avg_launch_ms": avg_ms,
                 "share": tot[dom] / sum(tot.values()), "peak_source": pk["source"]}
 
     # whole-step roofline (the metric's "% of bf16 roofline")

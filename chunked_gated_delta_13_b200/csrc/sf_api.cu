@@ -201,6 +201,23 @@ bool segment_lengths(const sf_gdn_shape& s, int N, const int* seg_len, std::vect
 // segments in turn).  Offsets from a 256-byte aligned base.
 constexpr int kSlots = 3;
 
+// Pipeline pieces: every segment longer than kPiece tokens is cut into pieces
+// of kPiece tokens (a multiple of the chunk length, counted from the segment
+// start) and a shorter last piece.  A cut at a multiple of C from the segment
+// start falls on a chunk boundary, where the state handed on is exactly the
+// state the chain carries, so the pieces change no result; they give a long
+// segment the same overlap as many short ones.
+constexpr int kPiece = 4096;
+
+std::vector<int> pipe_pieces(const std::vector<int>& lens) {
+    std::vector<int> out;
+    for (int L : lens) {
+        if (L == 0) out.push_back(0);
+        for (int t = 0; t < L; t += kPiece) out.push_back(L - t < kPiece ? L - t : kPiece);
+    }
+    return out;
+}
+
 struct PipeLayout {
     size_t sstride, keep0, kstride, slot0, slstride, total;
 };
@@ -481,7 +498,7 @@ size_t sf_segment_workspace_bytes(const sf_gdn_shape* s, int N, const int* seg_l
     std::vector<int> lens;
     if (!segment_lengths(*s, N, seg_len, lens)) return 0;
     if (pick_path(*s) == Path::Tc) {
-        const PipeLayout L = pipe_layout(*s, lens);
+        const PipeLayout L = pipe_layout(*s, pipe_pieces(lens));
         return L.total + 256;
     }
     size_t per = 0;
@@ -520,7 +537,7 @@ sf_status sf_segment_run(const sf_gdn_shape* s, int N, const int* seg_len, const
         char* b = reinterpret_cast<char*>(sf::align_up(reinterpret_cast<uintptr_t>(ws), 256));
         const sf::FwdArgs F{q, k, v, g, beta, S_in, o, S_out};
         const sf::BwdArgs B{q, k, v, g, beta, S_in, dO, dS_out, dq, dk, dv, dg, dbeta, dS_in};
-        return segment_run_pipelined(*s, lens, F, dO ? &B : nullptr, b, cs);
+        return segment_run_pipelined(*s, pipe_pieces(lens), F, dO ? &B : nullptr, b, cs);
     }
 
     const size_t nstate = (size_t)s->B * s->H * s->dk * s->dv;

@@ -3,13 +3,17 @@
 //
 // Decomposition (StateFlow, arXiv 2608.06838, section 2.2: Pre / ST / Out per
 // chunk; section 3.4.2: the backward stages SR, OG, STB, PG):
-//   forward  : prep (Pre: UT/WY transform)  -> scan (ST, sequential over chunks)
-//              -> out (Out)
-//   backward : prep (Pre again, plus the intra-chunk output gradient OG)
+//   forward  : prep (Pre: UT/WY transform, also L for the gradients)
+//              -> scan (ST, sequential over chunks) -> out (Out)
+//   backward : prep (Pre again) -> intra (OG: dVi = P^T dO, and the
+//              chain-independent term D = (gamma dO)^T Q of the reverse scan)
 //              -> one launch running the forward state recompute (SR) and the
 //                 reverse state-gradient scan (STB) side by side: the two
 //                 chains do not depend on each other
 //              -> grad (PG: every input gradient of every chunk)
+//   segment chain (sf_segment_run): per segment prep, scan, out with OG fused
+//              into the same launch; then per segment, in reverse, STB and PG
+//              on the kept forward intermediates (no second Pre, no SR).
 // With G_i = sum_{s<=i} g_s inside a chunk, gamma_i = exp(G_i),
 // Gamma_ij = exp(G_i - G_j) (j <= i), Khat = K * exp(G_C - G):
 //   A = strictly-lower(diag(beta)(K K^T * Gamma)), L = (I + A)^{-1}, T = L diag(beta)
@@ -186,30 +190,26 @@ __device__ void block_inverse(const float* A, int la, float* L, int ll, float* Y
 }
 
 // ------------------------------------------------------------------ prep ---
-template <int DV, bool BWD>
+template <int DV>
 constexpr size_t prep_smem() {
-    return (size_t)C * LDK * 2 + (size_t)C * (DV + 8) * 2 + (BWD ? (size_t)C * LDK * 2 + (size_t)C * (DV + 8) * 2 : 0) +
-           (size_t)C * LDF * 4 * 2 + (size_t)C * LDC * 2 * 2 + 768 * 4 + 2 * C * 4;
+    return (size_t)C * LDK * 2 + (size_t)C * (DV + 8) * 2 + (size_t)C * LDF * 4 * 2 + (size_t)C * LDC * 2 * 2 +
+           768 * 4 + 2 * C * 4;
 }
 
-// One CTA (8 warps: rows 16*(w%4), column half w/4) per (chunk, head).  Writes G, Khat, W, U^T; in backward
-// mode also dVi^T = (P^T dO)^T with P = scale (Q K^T) * Gamma.
-template <int DV, bool BETA, bool BWD>
+// One CTA (8 warps: rows 16*(w%4), column half w/4) per (chunk, head).  Writes
+// G, exp(G), Khat, -W, L and U^T.
+template <int DV, bool BETA>
 __global__ void __launch_bounds__(256)
-tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
-               const bf16* __restrict__ v, const float* __restrict__ g,
-               const float* __restrict__ beta, const bf16* __restrict__ dO, float* __restrict__ Gc,
-               float* __restrict__ Gmo, bf16* __restrict__ Wo, float* __restrict__ Lmo, bf16* __restrict__ Kho,
-               bf16* __restrict__ Uto, bf16* __restrict__ dVito) {
+tc_prep_kernel(SeqView s, const bf16* __restrict__ k, const bf16* __restrict__ v, const float* __restrict__ g,
+               const float* __restrict__ beta, float* __restrict__ Gc, float* __restrict__ Gmo,
+               bf16* __restrict__ Wo, float* __restrict__ Lmo, bf16* __restrict__ Kho, bf16* __restrict__ Uto) {
     constexpr int LDV = DV + 8;
     extern __shared__ __align__(16) unsigned char smem[];
     bf16* Ks = reinterpret_cast<bf16*>(smem);
     bf16* Vs = Ks + C * LDK;
-    bf16* Qs = Vs + C * LDV;
-    bf16* dOs = Qs + (BWD ? C * LDK : 0);
-    float* Af = reinterpret_cast<float*>(dOs + (BWD ? C * LDV : 0));  // later: W staging
+    float* Af = reinterpret_cast<float*>(Vs + C * LDV);                // later: W staging
     float* Lf = Af + C * LDF;                                          // later: U^T staging
-    bf16* Tw = reinterpret_cast<bf16*>(Lf + C * LDF);                  // later: P
+    bf16* Tw = reinterpret_cast<bf16*>(Lf + C * LDF);
     bf16* Tu = Tw + C * LDC;
     float* Yb = reinterpret_cast<float*>(Tu + C * LDC);
     float* Gs = Yb + 768;
@@ -223,10 +223,6 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     const size_t Tp = (size_t)s.NC * C;
     load_tile<C, DK, 256>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
     load_tile<C, DV, 256>(Vs, LDV, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
-    if (BWD) {
-        load_tile<C, DK, 256>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
-        load_tile<C, DV, 256>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
-    }
     cp_async_commit();
     if (w == 0) chunk_cumsum(g + bh * s.hs_g + t0, nval, Gs, lane);
     for (int i = tid; i < C; i += 256) Bs[i] = (BETA && i < nval) ? beta[bh * s.hs_g + t0 + i] : 0.f;
@@ -1692,10 +1688,10 @@ cudaError_t smem_attr(K* kern, size_t bytes) {
 template <int DV, bool BETA>
 cudaError_t launch_prep(const char* name, const SeqView& s, const bf16* k, const bf16* v, const float* g,
                         const float* beta, const TcWs& w, cudaStream_t st) {
-    constexpr size_t sm = prep_smem<DV, false>();
-    TC_TRY(smem_attr(tc_prep_kernel<DV, BETA, false>, sm));
-    SF_LAUNCH(name, st, tc_prep_kernel<DV, BETA, false><<<dim3(s.NC, s.BH), 256, sm, st>>>(
-                            s, nullptr, k, v, g, beta, nullptr, w.Gc, w.Gm, w.W, w.Lm, w.Kh, w.Ut, nullptr));
+    constexpr size_t sm = prep_smem<DV>();
+    TC_TRY(smem_attr(tc_prep_kernel<DV, BETA>, sm));
+    SF_LAUNCH(name, st, tc_prep_kernel<DV, BETA><<<dim3(s.NC, s.BH), 256, sm, st>>>(
+                            s, k, v, g, beta, w.Gc, w.Gm, w.W, w.Lm, w.Kh, w.Ut));
     return cudaGetLastError();
 }
 

@@ -110,20 +110,39 @@ sf_status sf_gdn_bwd(const sf_gdn_shape* shape, const void* q, const void* k, co
                      const float* dS_out, void* dq, void* dk, void* dv, float* dg,
                      float* dbeta, float* dS_in, void* ws, size_t ws_bytes, void* stream);
 
-/* Workspace for sf_segment_run: the per-segment workspace of the longest
- * segment plus N+1 fp32 boundary states and N+1 boundary state gradients.
- * seg_len: host array of N lengths summing to shape->T, or NULL for the equal
- * split (the first T % N segments one token longer). */
+/* Workspace for sf_segment_run.  seg_len: host array of N lengths summing to
+ * shape->T, or NULL for the equal split (the first T % N segments one token
+ * longer).  Two cases:
+ *  - tensor-core path (bf16 I/O, dk = 128, dv in {64, 128}, C = 64): the
+ *    pipelined chain keeps every segment's forward intermediates for its
+ *    backward, so the workspace grows with T: 8 + 4 dk + 4 C + 6 dv +
+ *    4 dk dv / C bytes per token per head (2568 B at dk = dv = 128, C = 64:
+ *    2.7 GB for B = 1, H = 16, T = 65536), plus the backward tiles of three
+ *    pieces of 4096 tokens and the fp32 boundary states;
+ *  - otherwise: the per-segment workspace of the longest segment plus N+1
+ *    fp32 boundary states and two boundary state gradients. */
 size_t sf_segment_workspace_bytes(const sf_gdn_shape* full, int N, const int* seg_len);
 
 /* The segment chain on one GPU (StateFlow section 3.1): split the sequence of
- * `full` into N segments, run sf_gdn_fwd on segments 0..N-1 with each S_out
- * handed on as the next S_in, then (when dO != NULL) sf_gdn_bwd on segments
+ * `full` into N segments, run the forward on segments 0..N-1 with each S_out
+ * handed on as the next S_in, then (when dO != NULL) the backward on segments
  * N-1..0 with each dS_in handed back as the previous dS_out.  Arguments are the
  * full-sequence tensors of sf_gdn_fwd and sf_gdn_bwd; with dO == NULL the
  * backward is skipped and dq, dk, dv, dg, dbeta, dS_in are ignored.  The
  * boundary states stay fp32 on the device, so when every segment length is a
- * multiple of C the results are bit-identical to N = 1. */
+ * multiple of C the results are bit-identical to N = 1.
+ *
+ * On the tensor-core path the chain is pipelined (StateFlow section 3.4, the
+ * split-and-overlap of the state scan with the chunk-parallel kernels):
+ * segments are further cut into pieces of 4096 tokens at chunk boundaries
+ * (this changes no result); the state scans of consecutive pieces run in
+ * order on an internal high-priority stream while the chunk-parallel kernels
+ * of neighbouring pieces run on two lower-priority streams.  The streams and
+ * their events are created for the call, forked from `stream` and joined back
+ * to it before the call returns, so for the caller all work is ordered on
+ * `stream` as usual; they are released asynchronously.  The backward reuses
+ * the forward's intermediates instead of recomputing them; its results are
+ * bit-identical to sf_gdn_fwd followed by sf_gdn_bwd on the same segment. */
 sf_status sf_segment_run(const sf_gdn_shape* full, int N, const int* seg_len, const void* q,
                          const void* k, const void* v, const float* g, const float* beta,
                          const float* S_in, const void* dO, const float* dS_out, void* o,

@@ -1,0 +1,76 @@
+"""The pipelined segment chain of the tensor-core path (sf_segment_run with bf16
+I/O, dk = 128): it must compute exactly what the standalone calls compute,
+run the benchmarked configuration correctly, and handle a forward-only call.
+"""
+import pytest
+import torch
+
+import chunked_gated_delta_13_b200 as sf
+from chunked_gated_delta_13_b200.inputs import CONFIGS, Workload, make_inputs
+from gpu_util import compare, gpu_fwd_bwd, oracle_fwd_bwd, to_device
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16 = 2e-2
+
+
+def _run_segments(d, C, N):
+    o, S_out, gr = sf.segment_run(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S_in"], d["dO"],
+                                  d["dS_out"], N=N, C=C)
+    torch.cuda.synchronize()
+    sf.device_check()
+    out = {"o": o, "S_out": S_out}
+    out.update(gr)
+    return out
+
+
+def _run_calls(d, C):
+    o, S_out = sf.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S_in"], C=C)
+    gr = sf.bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S_in"], d["dO"], d["dS_out"], C=C)
+    torch.cuda.synchronize()
+    sf.device_check()
+    out = {"o": o, "S_out": S_out}
+    out.update(gr)
+    return out
+
+
+@pytest.mark.parametrize("dv,beta,T", [(128, True, 6 * 64), (128, True, 5 * 64 + 40),
+                                       (64, True, 4 * 64), (64, False, 3 * 64 + 7),
+                                       (128, False, 4 * 64)])
+def test_pipeline_bit_identical_to_standalone_calls(dv, beta, T):
+    """One-segment chain (fused Out + OG, kept intermediates, no second Pre or
+    forward recompute) against sf_gdn_fwd + sf_gdn_bwd: every output bit-equal."""
+    w = Workload(name="pipe", B=2, H=3, T=T, dk=128, dv=dv, C=64, io="bf16", use_beta=beta,
+                 S_in_std=0.05, dS_out_std=0.1, g_shift=-4.0)
+    d = to_device(make_inputs(w))
+    a = _run_segments(d, w.C, 1)
+    b = _run_calls(d, w.C)
+    for name, x in b.items():
+        if x is None:
+            assert a.get(name) is None, name
+            continue
+        assert torch.equal(a[name], x), name
+
+
+def test_headline_segment_chain_sampled_heads():
+    """The benchmarked configuration: B=1, H=16, T=65536, d=128 as 16 segments,
+    two heads checked against the oracle."""
+    w = CONFIGS["headline_h16_t64k"]
+    heads = [(0, 3), (0, 14)]
+    inp = make_inputs(w)
+    out = _run_segments(to_device(inp), w.C, 16)
+    gpu = {k: None if v is None else v.double().cpu().numpy() for k, v in out.items()}
+    compare(gpu, oracle_fwd_bwd(inp, heads=heads), TOL_BF16, heads=heads)
+
+
+def test_segment_chain_forward_only():
+    """dO = NULL runs the forward chain alone; its outputs equal those of a full run."""
+    w = Workload(name="fwd_only", B=1, H=4, T=8 * 64, dk=128, dv=128, C=64, io="bf16",
+                 S_in_std=0.05, g_shift=-4.0)
+    d = to_device(make_inputs(w))
+    o, S_out, gr = sf.segment_run(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S_in"], None, N=4, C=w.C)
+    torch.cuda.synchronize()
+    sf.device_check()
+    assert gr is None
+    full = _run_segments(d, w.C, 4)
+    assert torch.equal(o, full["o"]) and torch.equal(S_out, full["S_out"])
