@@ -111,7 +111,6 @@ def kernel_work(name, w, T_seg):
 # traffic is this figure times its chunk-heads.  Valid for the kernels as they
 # were when captured; an entry is removed when its kernel changes.
 MEASURED_TRAFFIC = {
-    "tc_prep": 150.90e6 / 2048,
     "tc_scan_fwd": 161.25e6 / 2048,
     "tc_out_og": 293.45e6 / 2048,
     "tc_scan_bwd": 238.72e6 / 2048,

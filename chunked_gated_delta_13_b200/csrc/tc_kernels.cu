@@ -191,9 +191,8 @@ __device__ void block_inverse(const float* A, int la, float* L, int ll, float* Y
 
 // ------------------------------------------------------------------ prep ---
 template <int DV>
-constexpr size_t prep_smem() {
-    return (size_t)C * LDK * 2 + (size_t)C * (DV + 8) * 2 + (size_t)C * LDF * 4 * 2 + (size_t)C * LDC * 2 * 2 +
-           768 * 4 + 2 * C * 4;
+constexpr size_t prep_smem() {  // 75.5 KB: three CTAs per SM
+    return (size_t)C * LDK * 2 * 2 + (size_t)C * LDF * 4 * 2 + 768 * 4 + 3 * C * 4;
 }
 
 // One CTA (8 warps: rows 16*(w%4), column half w/4) per (chunk, head).  Writes
@@ -205,15 +204,19 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ k, const bf16* __restrict__ v
                bf16* __restrict__ Wo, float* __restrict__ Lmo, bf16* __restrict__ Kho, bf16* __restrict__ Uto) {
     constexpr int LDV = DV + 8;
     extern __shared__ __align__(16) unsigned char smem[];
+    // Regions are reused as the chunk advances: V's region (sized for a
+    // [C][LDK] tile) holds the W staging once U is done, A's region holds the
+    // bf16 T tiles once L is known, L's region the U^T staging.
     bf16* Ks = reinterpret_cast<bf16*>(smem);
-    bf16* Vs = Ks + C * LDK;
-    float* Af = reinterpret_cast<float*>(Vs + C * LDV);                // later: W staging
-    float* Lf = Af + C * LDF;                                          // later: U^T staging
-    bf16* Tw = reinterpret_cast<bf16*>(Lf + C * LDF);
+    bf16* Vs = Ks + C * LDK;                                  // later: W staging [C][LDK]
+    float* Af = reinterpret_cast<float*>(Vs + C * LDK);      // later: T tiles
+    float* Lf = Af + C * LDF;                                 // later: U^T staging
+    bf16* Tw = reinterpret_cast<bf16*>(Af);
     bf16* Tu = Tw + C * LDC;
-    float* Yb = reinterpret_cast<float*>(Tu + C * LDC);
+    float* Yb = Lf + C * LDF;
     float* Gs = Yb + 768;
     float* Bs = Gs + C;
+    float* BGs = Bs + C;  // beta_j exp(G_j)
 
     const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int gq = lane >> 2, tq = lane & 3;
@@ -232,8 +235,10 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ k, const bf16* __restrict__ v
     __syncthreads();
 
     for (int i = tid; i < C; i += 256) {
+        const float e = __expf(Gs[i]);
         Gc[bh * Tp + t0 + i] = Gs[i];
-        Gmo[bh * Tp + t0 + i] = __expf(Gs[i]);
+        Gmo[bh * Tp + t0 + i] = e;
+        BGs[i] = Bs[i] * e;
     }
     const float gC = Gs[C - 1];
     for (int e = tid; e < C * (DK / 8); e += 256) {
@@ -278,36 +283,14 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ k, const bf16* __restrict__ v
             const int i = e >> 4, j = (e & 15) * 4;
             *reinterpret_cast<float4*>(Lg + i * C + j) = *reinterpret_cast<const float4*>(Lf + i * LDF + j);
         }
-        for (int e = tid; e < C * C; e += 256) {
+        for (int e = tid; e < C * C; e += 256) {  // A is dead: its region takes the T tiles
             const int i = e >> 6, j = e & 63;
             const float l = Lf[i * LDF + j];
-            Tw[i * LDC + j] = __float2bfloat16_rn(l * Bs[j] * __expf(Gs[j]));
+            Tw[i * LDC + j] = __float2bfloat16_rn(l * BGs[j]);
             Tu[i * LDC + j] = __float2bfloat16_rn(l * Bs[j]);
         }
         __syncthreads();
-        bf16* Wst = reinterpret_cast<bf16*>(Af);  // [C][LDK]
-        {  // W = T (gamma * K), staged negated
-            float acc[8][4] = {};
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                uint32_t a[4];
-                ldA(a, Tw, LDC, 16 * mw, 16 * kk, lane);
-#pragma unroll
-                for (int nn = 0; nn < 8; nn += 2) {
-                    uint32_t b[4];
-                    ldBkn(b, Ks, LDK, 64 * nw + 8 * nn, 16 * kk, lane);
-                    mma(acc[nn], a, b[0], b[1]);
-                    mma(acc[nn + 1], a, b[2], b[3]);
-                }
-            }
-#pragma unroll
-            for (int nn = 0; nn < 8; ++nn) {
-                const int i = 16 * mw + gq, col = 64 * nw + 8 * nn + 2 * tq;
-                *reinterpret_cast<uint32_t*>(Wst + i * LDK + col) = pack(-acc[nn][0], -acc[nn][1]);
-                *reinterpret_cast<uint32_t*>(Wst + (i + 8) * LDK + col) = pack(-acc[nn][2], -acc[nn][3]);
-            }
-        }
-        {  // U = T V, staged transposed
+        {  // U = T V, staged transposed into L's region
             float acc[DV / 16][4] = {};
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -328,6 +311,29 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ k, const bf16* __restrict__ v
                     const int i = 16 * mw + gq + 8 * (e >> 1), col = (DV / 2) * nw + 8 * nn + 2 * tq + (e & 1);
                     Ust[col * LDC + i] = __float2bfloat16_rn(acc[nn][e]);
                 }
+        }
+        __syncthreads();  // V is dead: its region takes the W staging
+        bf16* Wst = Vs;  // [C][LDK]
+        {  // W = T (gamma * K), staged negated
+            float acc[8][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                uint32_t a[4];
+                ldA(a, Tw, LDC, 16 * mw, 16 * kk, lane);
+#pragma unroll
+                for (int nn = 0; nn < 8; nn += 2) {
+                    uint32_t b[4];
+                    ldBkn(b, Ks, LDK, 64 * nw + 8 * nn, 16 * kk, lane);
+                    mma(acc[nn], a, b[0], b[1]);
+                    mma(acc[nn + 1], a, b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int nn = 0; nn < 8; ++nn) {
+                const int i = 16 * mw + gq, col = 64 * nw + 8 * nn + 2 * tq;
+                *reinterpret_cast<uint32_t*>(Wst + i * LDK + col) = pack(-acc[nn][0], -acc[nn][1]);
+                *reinterpret_cast<uint32_t*>(Wst + (i + 8) * LDK + col) = pack(-acc[nn][2], -acc[nn][3]);
+            }
         }
         __syncthreads();
         for (int e = tid; e < C * (DK / 8); e += 256) {
