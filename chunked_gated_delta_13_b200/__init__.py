@@ -23,7 +23,8 @@ import threading
 from ._build import LIB, build, needs_build
 
 __all__ = ["Shape", "SFError", "lib", "fwd", "bwd", "segment_run", "make_shape", "path", "device_check",
-           "launches", "set_launch_hook", "fwd_workspace_bytes", "bwd_workspace_bytes", "segment_workspace_bytes",
+           "launches", "set_launch_hook", "timer_enable", "timer_disable", "timer_count", "timer_results", "timer_free",
+           "fwd_workspace_bytes", "bwd_workspace_bytes", "segment_workspace_bytes",
            "EXPORTED_SYMBOLS"]
 
 SF_F32, SF_BF16 = 0, 1
@@ -35,7 +36,8 @@ EXPORTED_SYMBOLS = [
     "sf_status_str", "sf_last_cuda_error", "sf_gdn_fwd_workspace_bytes",
     "sf_gdn_bwd_workspace_bytes", "sf_gdn_fwd", "sf_gdn_bwd", "sf_segment_workspace_bytes",
     "sf_segment_run", "sf_gdn_path", "sf_gdn_launches", "sf_set_launch_hook", "sf_gdn_fwd_noalloc",
-    "sf_device_check",
+    "sf_device_check", "sf_timer_enable", "sf_timer_disable", "sf_timer_count", "sf_timer_read",
+    "sf_timer_free",
 ]
 
 HOOK_T = ctypes.CFUNCTYPE(None, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p)
@@ -102,6 +104,16 @@ def lib():
         L.sf_gdn_fwd_noalloc.restype = ctypes.c_int
         L.sf_set_launch_hook.argtypes = [HOOK_T, ctypes.c_void_p]
         L.sf_set_launch_hook.restype = None
+        L.sf_timer_enable.argtypes = [ctypes.c_int]
+        L.sf_timer_enable.restype = ctypes.c_int
+        L.sf_timer_disable.argtypes = []
+        L.sf_timer_disable.restype = None
+        L.sf_timer_count.argtypes = []
+        L.sf_timer_count.restype = ctypes.c_int
+        L.sf_timer_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float)]
+        L.sf_timer_read.restype = ctypes.c_int
+        L.sf_timer_free.argtypes = []
+        L.sf_timer_free.restype = None
         _lib = L
         return _lib
 
@@ -169,6 +181,35 @@ def set_launch_hook(fn):
 
     _hook_ref = HOOK_T(_cb)
     lib().sf_set_launch_hook(_hook_ref, None)
+
+
+def timer_enable(capacity: int):
+    """Time the next `capacity` kernel launches with CUDA events recorded by the
+    library itself on each launch's stream (see sf_timer_enable)."""
+    _check(lib().sf_timer_enable(int(capacity)))
+
+
+def timer_disable():
+    lib().sf_timer_disable()
+
+
+def timer_count() -> int:
+    return int(lib().sf_timer_count())
+
+
+def timer_results():
+    """[(kernel_name, ms)] of the recorded launches, in launch order (waits for them)."""
+    out = []
+    name = ctypes.c_char_p()
+    ms = ctypes.c_float()
+    for i in range(lib().sf_timer_count()):
+        _check(lib().sf_timer_read(i, ctypes.byref(name), ctypes.byref(ms)))
+        out.append((name.value.decode(), float(ms.value)))
+    return out
+
+
+def timer_free():
+    lib().sf_timer_free()
 
 
 # ------------------------------------------------------------ torch glue ----

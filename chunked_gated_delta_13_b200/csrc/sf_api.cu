@@ -18,6 +18,27 @@ thread_local char g_last_cuda_error[256] = "";
 sf_launch_hook g_hook = nullptr;
 void* g_hook_user = nullptr;
 
+// Native launch timer (sf_timer_*): event pairs and kernel names of the
+// recorded launches.
+struct LaunchTimer {
+    bool on = false;
+    int used = 0;
+    std::vector<cudaEvent_t> begin, end;
+    std::vector<const char*> name;
+    void destroy() {
+        for (cudaEvent_t e : begin)
+            if (e) cudaEventDestroy(e);
+        for (cudaEvent_t e : end)
+            if (e) cudaEventDestroy(e);
+        begin.clear();
+        end.clear();
+        name.clear();
+        used = 0;
+        on = false;
+    }
+};
+LaunchTimer g_timer;
+
 sf_status cuda_fail(cudaError_t e) {
     std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
                   cudaGetErrorString(e));
@@ -431,10 +452,53 @@ namespace sf {
 void launch_hook(const char* kernel, int after, cudaStream_t st) {
     sf_launch_hook h = g_hook;
     if (h) h(kernel, after, static_cast<void*>(st), g_hook_user);
+    if (g_timer.on && g_timer.used < (int)g_timer.begin.size()) {
+        const int i = g_timer.used;
+        if (!after) {
+            cudaEventRecord(g_timer.begin[i], st);
+        } else {
+            cudaEventRecord(g_timer.end[i], st);
+            g_timer.name[i] = kernel;
+            g_timer.used = i + 1;
+        }
+    }
 }
 }  // namespace sf
 
 extern "C" {
+
+sf_status sf_timer_enable(int capacity) {
+    g_timer.destroy();
+    if (capacity < 0) return SF_ERR_INVALID_ARG;
+    g_timer.begin.assign(capacity, nullptr);
+    g_timer.end.assign(capacity, nullptr);
+    g_timer.name.assign(capacity, nullptr);
+    for (int i = 0; i < capacity; ++i) {
+        cudaError_t e = cudaEventCreate(&g_timer.begin[i]);
+        if (e == cudaSuccess) e = cudaEventCreate(&g_timer.end[i]);
+        if (e != cudaSuccess) {
+            g_timer.destroy();
+            return cuda_fail(e);
+        }
+    }
+    g_timer.on = true;
+    return SF_OK;
+}
+
+void sf_timer_disable(void) { g_timer.on = false; }
+
+int sf_timer_count(void) { return g_timer.used; }
+
+sf_status sf_timer_read(int i, const char** kernel, float* ms) {
+    if (i < 0 || i >= g_timer.used || !kernel || !ms) return SF_ERR_INVALID_ARG;
+    cudaError_t e = cudaEventSynchronize(g_timer.end[i]);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(ms, g_timer.begin[i], g_timer.end[i]);
+    if (e != cudaSuccess) return cuda_fail(e);
+    *kernel = g_timer.name[i];
+    return SF_OK;
+}
+
+void sf_timer_free(void) { g_timer.destroy(); }
 
 void sf_set_launch_hook(sf_launch_hook hook, void* user) {
     g_hook_user = user;

@@ -1628,21 +1628,27 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
             }
         }
     }
-    {
-        bf16* dqb = dq + bh * s.hs_k + (size_t)t0 * DK;
-        bf16* dkb = dk + bh * s.hs_k + (size_t)t0 * DK;
+    // dq, dk: staged in the free R region, then one bulk store per row
+    __syncthreads();  // the operand reads of C7 are done
+    bf16* dqs = reinterpret_cast<bf16*>(R);  // [C][LDK]
+    bf16* dks = dqs + C * LDK;               // [C][LDK]
 #pragma unroll
-        for (int nn = 0; nn < DKW / 8; ++nn) {
-            const int col = DKW * nw + 8 * nn + 2 * tq;
-            if (r0 < nval) {
-                *reinterpret_cast<uint32_t*>(dqb + (size_t)r0 * DK + col) = pack(accQ[nn][0], accQ[nn][1]);
-                *reinterpret_cast<uint32_t*>(dkb + (size_t)r0 * DK + col) = pack(accK[nn][0], accK[nn][1]);
-            }
-            if (r1 < nval) {
-                *reinterpret_cast<uint32_t*>(dqb + (size_t)r1 * DK + col) = pack(accQ[nn][2], accQ[nn][3]);
-                *reinterpret_cast<uint32_t*>(dkb + (size_t)r1 * DK + col) = pack(accK[nn][2], accK[nn][3]);
-            }
-        }
+    for (int nn = 0; nn < DKW / 8; ++nn) {
+        const int col = DKW * nw + 8 * nn + 2 * tq;
+        *reinterpret_cast<uint32_t*>(dqs + r0 * LDK + col) = pack(accQ[nn][0], accQ[nn][1]);
+        *reinterpret_cast<uint32_t*>(dks + r0 * LDK + col) = pack(accK[nn][0], accK[nn][1]);
+        *reinterpret_cast<uint32_t*>(dqs + r1 * LDK + col) = pack(accQ[nn][2], accQ[nn][3]);
+        *reinterpret_cast<uint32_t*>(dks + r1 * LDK + col) = pack(accK[nn][2], accK[nn][3]);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    const bool storer = tid < 2 * C && (tid & (C - 1)) < nval;
+    if (storer) {
+        const int r = tid & (C - 1);
+        const bool isq = tid < C;
+        bf16* dst = (isq ? dq : dk) + bh * s.hs_k + (size_t)(t0 + r) * DK;
+        bulk_store(dst, (isq ? dqs : dks) + r * LDK, DK * 2);
+        bulk_commit();
     }
 
     // ---- phase C8: dG, dg (reverse cumsum), dbeta; warp 0, two tokens per lane
@@ -1677,6 +1683,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         if (2 * lane < nval) dgb[2 * lane] = suf;
         if (2 * lane + 1 < nval) dgb[2 * lane + 1] = suf - x[0];
     }
+    if (storer) bulk_wait_read<0>();  // the staged rows must outlive their reads
 }
 
 template <typename K>

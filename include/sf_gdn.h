@@ -183,6 +183,22 @@ sf_status sf_gdn_fwd_noalloc(const sf_gdn_shape* shape, const void* q, const voi
 typedef void (*sf_launch_hook)(const char* kernel, int after, void* stream, void* user);
 void sf_set_launch_hook(sf_launch_hook hook, void* user);
 
+/* Native launch timer, for measurement with little host overhead.  While
+ * enabled, each of the next `capacity` kernel launches of this library is
+ * bracketed by two CUDA events (timing enabled) recorded on the launch's own
+ * stream; later launches are not timed.  sf_timer_enable creates the events
+ * (and discards earlier records); sf_timer_disable stops recording and keeps
+ * the records; sf_timer_count gives how many launches were recorded;
+ * sf_timer_read(i, ...) waits for launch i to finish and returns its kernel
+ * name (a static string) and its duration in milliseconds; sf_timer_free
+ * destroys the events.  Process-wide, for one host thread at a time; the only
+ * state this library keeps between calls, and only while a caller uses it. */
+sf_status sf_timer_enable(int capacity);
+void sf_timer_disable(void);
+int sf_timer_count(void);
+sf_status sf_timer_read(int i, const char** kernel, float* ms);
+void sf_timer_free(void);
+
 /* Introspection for tests and benchmarks: the kernel family a shape runs on
  * ("tc" = tensor-core kernels, "simt" = fp32 CUDA-core kernels; NULL if the
  * shape is unsupported) and how many kernels one call launches. */

@@ -74,3 +74,17 @@ def test_segment_chain_forward_only():
     assert gr is None
     full = _run_segments(d, w.C, 4)
     assert torch.equal(o, full["o"]) and torch.equal(S_out, full["S_out"])
+
+
+def test_native_launch_timer():
+    """sf_timer_*: one record per launch, named after the kernel, with a positive duration."""
+    w = Workload(name="timer", B=1, H=2, T=3 * 64, dk=128, dv=128, C=64, io="bf16")
+    d = to_device(make_inputs(w))
+    sf.timer_enable(64)
+    _run_segments(d, w.C, 1)
+    sf.timer_disable()
+    rec = sf.timer_results()
+    sf.timer_free()
+    names = [n for n, _ in rec]
+    assert names == ["tc_prep", "tc_scan_fwd", "tc_out_og", "tc_scan_bwd", "tc_grad"], names
+    assert all(ms > 0 for _, ms in rec)
