@@ -106,15 +106,17 @@ def kernel_work(name, w, T_seg):
 
 
 # DRAM bytes (read + write) per chunk-head measured by ncu for each kernel of the
-# tensor-core path (B=1, H=16, T=8192, d=128, one segment: 2048 chunk-heads per
-# launch; summary and command in profiles/ncu_full_h16_t8k.md).  A launch's
-# traffic is this figure times its chunk-heads.  Valid for the kernels as they
-# were when captured; an entry is removed when its kernel changes.
+# tensor-core path (B=1, H=16, T=8192, d=128, one segment cut into two
+# 4096-token pieces: 1024 chunk-heads per launch, mean of the two launches;
+# summary and command in profiles/ncu_full_h16_t8k.md).  A launch's traffic is
+# this figure times its chunk-heads.  Valid for the kernels as they were when
+# captured; an entry is removed when its kernel changes.
 MEASURED_TRAFFIC = {
-    "tc_scan_fwd": 161.25e6 / 2048,
-    "tc_out_og": 293.45e6 / 2048,
-    "tc_scan_bwd": 238.72e6 / 2048,
-    "tc_grad": 452.10e6 / 2048,
+    "tc_prep": 44149.0,
+    "tc_scan_fwd": 61061.0,
+    "tc_out_og": 124965.0,
+    "tc_scan_bwd": 102704.0,
+    "tc_grad": 211599.0,
 }
 
 
