@@ -23,6 +23,8 @@
 // warp-level m16n8k16 products: each warp owns 16 state columns, so the
 // recurrence never leaves the register file; only the operands W, Khat, U
 // stream in through double-buffered asynchronous copies.
+#include <algorithm>
+
 #include "tc_kernels.cuh"
 #include "tc_mma.cuh"
 
@@ -55,6 +57,7 @@ struct TcWs {
     bf16* dVnt;  // [BH][NC][DV][C]    dV_new transposed (permuted)
     bf16* dSCt;  // [BH][NC][DV][DK]   gradient of the state leaving each chunk, transposed (permuted)
     bf16* Dt;    // [BH][NC][DV][DK]   scale (gamma * dO)^T Q per chunk, transposed (permuted)
+    int* ticket;  // chunk counter of the persistent gradient kernel
     size_t total;
 };
 
@@ -92,6 +95,7 @@ TcWs tc_parts(const SeqView& s, char* keep, char* og, char* slot, size_t* keep_b
     off = 0;
     w.dVnt = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
     w.dSCt = reinterpret_cast<bf16*>(take(BH * NC * DV * DK * 2));
+    w.ticket = reinterpret_cast<int*>(take(sizeof(int)));
     if (slot_bytes) *slot_bytes = off;
     return w;
 }
@@ -102,7 +106,10 @@ TcWs tc_layout(const SeqView& s, bool backward, char* base) {
     tc_parts(s, nullptr, nullptr, nullptr, &kb, &ob, &sb);
     TcWs w = tc_parts(s, base, base ? base + kb : nullptr, base ? base + kb + ob : nullptr, nullptr, nullptr,
                       nullptr);
-    if (!backward) w.dVit = w.dVnt = w.dSCt = w.Dt = nullptr;
+    if (!backward) {
+        w.dVit = w.dVnt = w.dSCt = w.Dt = nullptr;
+        w.ticket = nullptr;
+    }
     w.total = kb + (backward ? ob + sb : 0) + 256;
     return w;
 }
@@ -1147,7 +1154,7 @@ constexpr size_t grad_region_bytes() {
 template <int DV>
 constexpr size_t grad_smem() {
     return (size_t)C * LDK * 2 * 2 + (size_t)C * (DV + 8) * 2 * 2 + (size_t)DV * LDC * 2 * 2 +
-           grad_region_bytes<DV>() + (size_t)P_ROWS * C * 4 + GTH * 4 + 2 * C * 4;
+           grad_region_bytes<DV>() + (size_t)P_ROWS * C * 4 + GTH * 4 + 4 * C * 4 + 16;
 }
 
 // Every input gradient of one chunk (4 x GW warps: rows 16*(w%4), column group w/4).
@@ -1159,7 +1166,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
                const bf16* __restrict__ Vnt, const bf16* __restrict__ dVnt,
                const bf16* __restrict__ S0t, const bf16* __restrict__ dSCt, bf16* __restrict__ dq,
                bf16* __restrict__ dk, bf16* __restrict__ dv, float* __restrict__ dg,
-               float* __restrict__ dbeta) {
+               float* __restrict__ dbeta, int* __restrict__ ticket) {
     constexpr int LDV = DV + 8;
     extern __shared__ __align__(16) unsigned char smem[];
     bf16* Qs = reinterpret_cast<bf16*>(smem);
@@ -1182,35 +1189,91 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     bf16* Zs = Xs + C * LDC;
     float* part = reinterpret_cast<float*>(R + grad_region_bytes<DV>());  // [P_ROWS][C]
     float* red = part + P_ROWS * C;                                        // [GTH]
-    float* Gs = red + GTH;
-    float* Bs = Gs + C;
+    float* Gsb = red + GTH;  // [2][C] G of this chunk / the next
+    float* Bsb = Gsb + 2 * C;  // [2][C] beta of this chunk / the next
+    int* tk = reinterpret_cast<int*>(Bsb + 2 * C);
 
-    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    // Persistent: each CTA takes chunk tickets from `ticket` until none is
+    // left.  The next chunk's tiles are copied into regions as they die: dO and
+    // V_new after phase S, V and dV_new after C6, Q, K, G, S0 and dS_C after
+    // C7; so only the part of the first copy group that C8 cannot cover is
+    // waited for at the top of the next iteration.
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int gq = lane >> 2, tq = lane & 3;
     const int mw = w & 3, nw = w >> 2;
+    const size_t Tp = (size_t)s.NC * C;
+    const int total = s.NC * s.BH;
+    const int r0 = 16 * mw + gq, r1 = r0 + 8;  // the two rows this thread holds
+    auto where = [&](int j, int& c, int& bh) {
+        bh = j / s.NC;
+        c = j - bh * s.NC;
+    };
+    auto copy_a1 = [&](int j, int gbuf) {  // Q, K, G
+        int c, bh;
+        where(j, c, bh);
+        const int t0 = c * C, nval = min(C, s.T - t0);
+        load_tile<C, DK, GTH>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+        load_tile<C, DK, GTH>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+        if (tid < 16) cp_async16(Gsb + gbuf * C + tid * 4, Gc + bh * Tp + t0 + tid * 4, true);
+    };
+    auto copy_a2 = [&](int j) {  // dO, V_new
+        int c, bh;
+        where(j, c, bh);
+        const int t0 = c * C, nval = min(C, s.T - t0);
+        const size_t ci = (size_t)bh * s.NC + c;
+        load_tile<C, DV, GTH>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+        load_tile_swz<DV, C, GTH>(Vns, LDC, Vnt + ci * DV * C, tid);
+    };
+    auto copy_b1 = [&](int j) {  // V, dV_new
+        int c, bh;
+        where(j, c, bh);
+        const int t0 = c * C, nval = min(C, s.T - t0);
+        const size_t ci = (size_t)bh * s.NC + c;
+        load_tile_swz<DV, C, GTH>(dVns, LDC, dVnt + ci * DV * C, tid);
+        load_tile<C, DV, GTH>(Vs, LDV, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+    };
+    auto copy_b2 = [&](int j) {  // S0, dS_C
+        int c, bh;
+        where(j, c, bh);
+        const size_t ci = (size_t)bh * s.NC + c;
+        load_tile_swz<DV, DK, GTH>(S0s, LDK, S0t + ci * DV * DK, tid);
+        load_tile_swz<DV, DK, GTH>(dSs, LDK, dSCt + ci * DV * DK, tid);
+    };
+    auto beta_of = [&](int j) {
+        int c, bh;
+        where(j, c, bh);
+        const int t0 = c * C, nval = min(C, s.T - t0);
+        return (BETA && tid < nval) ? beta[bh * s.hs_g + t0 + tid] : 0.f;
+    };
+
+    if (tid == 0) tk[0] = atomicAdd(ticket, 1);
+    __syncthreads();
+    int j = tk[0];
+    if (j >= total) return;
+    // Copy groups of the first chunk: A (C1's operands), then B (the rest).
+    copy_a1(j, 0);
+    copy_a2(j);
+    cp_async_commit();
+    copy_b1(j);
+    copy_b2(j);
+    cp_async_commit();
+    if (tid < C) Bsb[tid] = beta_of(j);
+    for (int e = tid; e < P_ROWS * C; e += GTH) part[e] = 0.f;
+    int buf = 0;
+  for (;;) {
+    int c, bh;
+    where(j, c, bh);
     const int t0 = c * C;
     const int nval = min(C, s.T - t0);
-    const size_t Tp = (size_t)s.NC * C;
     const size_t ci = (size_t)bh * s.NC + c;
-    // Two copy groups: what phase C1 reads (Q, K, dO, V_new), then the state
-    // tiles of phase S and V, which land while C1 runs.
-    load_tile<C, DK, GTH>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
-    load_tile<C, DK, GTH>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
-    load_tile<C, DV, GTH>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
-    load_tile_swz<DV, C, GTH>(Vns, LDC, Vnt + ci * DV * C, tid);
-    if (tid < 16) cp_async16(Gs + tid * 4, Gc + bh * Tp + t0 + tid * 4, true);
-    cp_async_commit();
-    load_tile_swz<DV, C, GTH>(dVns, LDC, dVnt + ci * DV * C, tid);
-    load_tile_swz<DV, DK, GTH>(S0s, LDK, S0t + ci * DV * DK, tid);
-    load_tile_swz<DV, DK, GTH>(dSs, LDK, dSCt + ci * DV * DK, tid);
-    load_tile<C, DV, GTH>(Vs, LDV, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
-    cp_async_commit();
-    for (int i = tid; i < C; i += GTH) Bs[i] = (BETA && i < nval) ? beta[bh * s.hs_g + t0 + i] : 0.f;
-    for (int e = tid; e < P_ROWS * C; e += GTH) part[e] = 0.f;
-    cp_async_wait<1>();
+    float* Gs = Gsb + buf * C;
+    float* Bs = Bsb + buf * C;
+    cp_async_wait<1>();  // group A of this chunk (the state tiles may still be landing)
+    if (tid == 0) tk[1] = atomicAdd(ticket, 1);
     __syncthreads();
+    const int jn = tk[1];
+    const bool has_next = jn < total;
 
-    const int r0 = 16 * mw + gq, r1 = r0 + 8;  // the two rows this thread holds
     const float gam0 = __expf(Gs[r0]), gam1 = __expf(Gs[r1]);
     const float gC = Gs[C - 1];
     const float dec0 = __expf(gC - Gs[r0]), dec1 = __expf(gC - Gs[r1]);
@@ -1358,6 +1421,8 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
             }
             cp_async_commit();
         }
+        if (has_next) copy_a2(jn);  // dO and V_new are dead
+        cp_async_commit();
         // dW = -dV_new S0^T into the freed region
 #pragma unroll
         for (int nn = 0; nn < DKW / 8; ++nn) {
@@ -1372,7 +1437,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     }
     const float sdot = red[0];
 
-    if (BETA) cp_async_wait<0>();
+    if (BETA) cp_async_wait<1>();  // L (the next chunk's dO, V_new may still be landing)
     __syncthreads();
 
     // ---- phase C2: T = L diag(beta), L = (I + A)^{-1} as computed by the prep kernel
@@ -1599,6 +1664,8 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         }
     }
     __syncthreads();
+    if (has_next) copy_b1(jn);  // V and dV_new are dead
+    cp_async_commit();
 
     // ---- phase C7: dK += (Z + Z^T) K + Ms^T Q ; dq += Ms K
 #pragma unroll
@@ -1628,27 +1695,27 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
             }
         }
     }
-    // dq, dk: staged in the free R region, then one bulk store per row
-    __syncthreads();  // the operand reads of C7 are done
-    bf16* dqs = reinterpret_cast<bf16*>(R);  // [C][LDK]
-    bf16* dks = dqs + C * LDK;               // [C][LDK]
+    __syncthreads();  // the operand reads of C7 are done: Q, K and R are dead
+    if (has_next) copy_a1(jn, buf ^ 1);
+    cp_async_commit();
+    if (has_next) copy_b2(jn);
+    cp_async_commit();
+    const float beta_next = has_next ? beta_of(jn) : 0.f;
+    {
+        bf16* dqb = dq + bh * s.hs_k + (size_t)t0 * DK;
+        bf16* dkb = dk + bh * s.hs_k + (size_t)t0 * DK;
 #pragma unroll
-    for (int nn = 0; nn < DKW / 8; ++nn) {
-        const int col = DKW * nw + 8 * nn + 2 * tq;
-        *reinterpret_cast<uint32_t*>(dqs + r0 * LDK + col) = pack(accQ[nn][0], accQ[nn][1]);
-        *reinterpret_cast<uint32_t*>(dks + r0 * LDK + col) = pack(accK[nn][0], accK[nn][1]);
-        *reinterpret_cast<uint32_t*>(dqs + r1 * LDK + col) = pack(accQ[nn][2], accQ[nn][3]);
-        *reinterpret_cast<uint32_t*>(dks + r1 * LDK + col) = pack(accK[nn][2], accK[nn][3]);
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    const bool storer = tid < 2 * C && (tid & (C - 1)) < nval;
-    if (storer) {
-        const int r = tid & (C - 1);
-        const bool isq = tid < C;
-        bf16* dst = (isq ? dq : dk) + bh * s.hs_k + (size_t)(t0 + r) * DK;
-        bulk_store(dst, (isq ? dqs : dks) + r * LDK, DK * 2);
-        bulk_commit();
+        for (int nn = 0; nn < DKW / 8; ++nn) {
+            const int col = DKW * nw + 8 * nn + 2 * tq;
+            if (r0 < nval) {
+                *reinterpret_cast<uint32_t*>(dqb + (size_t)r0 * DK + col) = pack(accQ[nn][0], accQ[nn][1]);
+                *reinterpret_cast<uint32_t*>(dkb + (size_t)r0 * DK + col) = pack(accK[nn][0], accK[nn][1]);
+            }
+            if (r1 < nval) {
+                *reinterpret_cast<uint32_t*>(dqb + (size_t)r1 * DK + col) = pack(accQ[nn][2], accQ[nn][3]);
+                *reinterpret_cast<uint32_t*>(dkb + (size_t)r1 * DK + col) = pack(accK[nn][2], accK[nn][3]);
+            }
+        }
     }
 
     // ---- phase C8: dG, dg (reverse cumsum), dbeta; warp 0, two tokens per lane
@@ -1683,7 +1750,13 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         if (2 * lane < nval) dgb[2 * lane] = suf;
         if (2 * lane + 1 < nval) dgb[2 * lane + 1] = suf - x[0];
     }
-    if (storer) bulk_wait_read<0>();  // the staged rows must outlive their reads
+    __syncthreads();  // C8 is done with the partial sums
+    if (!has_next) break;
+    for (int e = tid; e < P_ROWS * C; e += GTH) part[e] = 0.f;
+    if (tid < C) Bsb[(buf ^ 1) * C + tid] = beta_next;
+    j = jn;
+    buf ^= 1;
+  }
 }
 
 template <typename K>
@@ -1757,15 +1830,32 @@ cudaError_t launch_scan_bwd(const SeqView& s, const BwdArgs& a, bool with_sr, co
     return cudaGetLastError();
 }
 
+int num_sms() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+            n = v;
+        else
+            n = 148;
+    }
+    return n;
+}
+
+// Persistent: one CTA per SM at most; the CTAs take chunks from w.ticket, so
+// they stay balanced when other kernels hold some of the SMs.
 template <int DV, bool BETA>
 cudaError_t launch_grad(const SeqView& s, const BwdArgs& a, const TcWs& w, cudaStream_t st) {
     constexpr size_t sm = grad_smem<DV>();
     TC_TRY(smem_attr(tc_grad_kernel<DV, BETA>, sm));
-    SF_LAUNCH("tc_grad", st, tc_grad_kernel<DV, BETA><<<dim3(s.NC, s.BH), GTH, sm, st>>>(
+    TC_TRY(cudaMemsetAsync(w.ticket, 0, sizeof(int), st));
+    const int grid = std::min(s.NC * s.BH, num_sms());
+    SF_LAUNCH("tc_grad", st, tc_grad_kernel<DV, BETA><<<grid, GTH, sm, st>>>(
                                  s, static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k),
                                  static_cast<const bf16*>(a.v), a.beta, static_cast<const bf16*>(a.dO), w.Gc,
                                  w.Lm, w.Vnt, w.dVnt, w.S0t, w.dSCt, static_cast<bf16*>(a.dq), static_cast<bf16*>(a.dk),
-                                 static_cast<bf16*>(a.dv), a.dg, a.dbeta));
+                                 static_cast<bf16*>(a.dv), a.dg, a.dbeta, w.ticket));
     return cudaGetLastError();
 }
 
