@@ -116,7 +116,6 @@ MEASURED_TRAFFIC = {
     "tc_scan_fwd": 61061.0,
     "tc_out_og": 124965.0,
     "tc_scan_bwd": 102704.0,
-    "tc_grad": 211599.0,
 }
 
 
