@@ -679,31 +679,45 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
             vn[nn][2] = u1.x;
             vn[nn][3] = u1.y;
         }
+        // own state rows first (no wait for the partner), the partner's rows into
+        // separate accumulators once its fragments are in
+        if (BETA) {
+            uint32_t bw[4][2][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int n2 = 0; n2 < 2; ++n2)
+                    ldsm_x4(bw[j][n2], Ws + sw_off(Lnk, 8 * (4 * half + 2 * n2), 2 * (4 * half + j), DK));
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int n2 = 0; n2 < 2; ++n2) {
+                    mma(vn[2 * n2], sa[j], bw[j][n2][0], bw[j][n2][1]);
+                    mma(vn[2 * n2 + 1], sa[j], bw[j][n2][2], bw[j][n2][3]);
+                }
+        }
         pair_sync(cg);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) get_frag(xslot(xch, cg, oth, kk, lane), sp[kk]);
         if (BETA) {
-            uint32_t bw[8][2][4];  // all B fragments of this phase, loaded before the first MMA
+            uint32_t bw[4][2][4];
+            float vq[4][4] = {};
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int kt = (j < 4) ? 4 * half + j : 4 * oth + (j - 4);
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
-                for (int n2 = 0; n2 < 2; ++n2) ldsm_x4(bw[j][n2], Ws + sw_off(Lnk, 8 * (4 * half + 2 * n2), 2 * kt, DK));
-            }
+                for (int n2 = 0; n2 < 2; ++n2)
+                    ldsm_x4(bw[j][n2], Ws + sw_off(Lnk, 8 * (4 * half + 2 * n2), 2 * (4 * oth + j), DK));
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {  // own state rows first, then the partner's
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int n2 = 0; n2 < 2; ++n2) {
-                    const uint32_t(&b)[4] = bw[j][n2];
-                    if (j < 4) {
-                        mma(vn[2 * n2], sa[j], b[0], b[1]);
-                        mma(vn[2 * n2 + 1], sa[j], b[2], b[3]);
-                    } else {
-                        mma(vn[2 * n2], sp[j - 4], b[0], b[1]);
-                        mma(vn[2 * n2 + 1], sp[j - 4], b[2], b[3]);
-                    }
+                    mma(vq[2 * n2], sp[j], bw[j][n2][0], bw[j][n2][1]);
+                    mma(vq[2 * n2 + 1], sp[j], bw[j][n2][2], bw[j][n2][3]);
                 }
-            }
+#pragma unroll
+            for (int nn = 0; nn < 4; ++nn)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) vn[nn][e] += vq[nn][e];
         }
         uint32_t va[2][4], vp[2][4];
 #pragma unroll
@@ -711,35 +725,42 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
             c2a(va[kk], vn[2 * kk], vn[2 * kk + 1]);
             put_frag(xslot(xch, cg, half, 4 + kk, lane), va[kk]);
         }
-        pair_sync(cg);
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) get_frag(xslot(xch, cg, oth, 4 + kk, lane), vp[kk]);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) st[j][e] *= gamC;
-        {
-            uint32_t bk[4][4][4];  // all B fragments of Khat for this phase
+        {  // own token tiles first (no wait for the partner)
+            uint32_t bk[2][4][4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int kt = (j < 2) ? 2 * half + j : 2 * oth + (j - 2);
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
-                for (int n2 = 0; n2 < 4; ++n2) ldsm_x4_t(bk[j][n2], Khs + sw_off(Lkn, 16 * kt, 8 * half + 2 * n2, DK));
-            }
+                for (int n2 = 0; n2 < 4; ++n2)
+                    ldsm_x4_t(bk[j][n2], Khs + sw_off(Lkn, 16 * (2 * half + j), 8 * half + 2 * n2, DK));
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {  // token tiles: own first, then the partner's
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
                 for (int n2 = 0; n2 < 4; ++n2) {
-                    const uint32_t(&b)[4] = bk[j][n2];
-                    if (j < 2) {
-                        mma(st[2 * n2], va[j], b[0], b[1]);
-                        mma(st[2 * n2 + 1], va[j], b[2], b[3]);
-                    } else {
-                        mma(st[2 * n2], vp[j - 2], b[0], b[1]);
-                        mma(st[2 * n2 + 1], vp[j - 2], b[2], b[3]);
-                    }
+                    mma(st[2 * n2], va[j], bk[j][n2][0], bk[j][n2][1]);
+                    mma(st[2 * n2 + 1], va[j], bk[j][n2][2], bk[j][n2][3]);
                 }
-            }
+        }
+        pair_sync(cg);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) get_frag(xslot(xch, cg, oth, 4 + kk, lane), vp[kk]);
+        {  // then the partner's
+            uint32_t bk[2][4][4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int n2 = 0; n2 < 4; ++n2)
+                    ldsm_x4_t(bk[j][n2], Khs + sw_off(Lkn, 16 * (2 * oth + j), 8 * half + 2 * n2, DK));
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int n2 = 0; n2 < 4; ++n2) {
+                    mma(st[2 * n2], vp[j], bk[j][n2][0], bk[j][n2][1]);
+                    mma(st[2 * n2 + 1], vp[j], bk[j][n2][2], bk[j][n2][3]);
+                }
         }
         // stage this chunk's outputs (own halves) while the state update is in flight
         if (S0t) {
@@ -771,7 +792,8 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
 
 // Reverse chain of the state gradient for one (head, 64 state columns):
 // per chunk, from the last, dV_new^T = dVi^T + dS^T Khat^T and
-// dS^T <- gamma_C dS^T + dO^T (scale gamma * Q) + dV_new^T (-W).
+// dS^T <- gamma_C dS^T + D^T + dV_new^T (-W), D^T = (scale (gamma * dO)^T Q)^T
+// precomputed by the intra-chunk products.
 // Outputs dV_new^T and dS_C^T per chunk (bf16, staged and bulk-stored), dS_in (fp32).
 template <int DV, bool BETA>
 __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, const bf16* __restrict__ Dt,
@@ -861,11 +883,8 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
             c2a(da[kk], ds[2 * kk], ds[2 * kk + 1]);
             put_frag(xslot(xch, cg, half, kk, lane), da[kk]);
         }
-        __syncthreads();  // the exchanged fragments are visible
         mbar_wait(&bars[cc & 1], (use >> 1) & 1, &g_tc_status, failed);
         const float gamC = Gs[C - 1];
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) get_frag(xslot(xch, cg, oth, kk, lane), dp[kk]);
         float dvn[4][4];  // dV_new^T, tokens 32*half + 8nn..
 #pragma unroll
         for (int nn = 0; nn < 4; ++nn) {
@@ -877,28 +896,43 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
             dvn[nn][2] = u1.x;
             dvn[nn][3] = u1.y;
         }
-        {
-            uint32_t bk[8][2][4];
+        {  // own state rows first (no wait for the partner)
+            uint32_t bk[4][2][4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int kt = (j < 4) ? 4 * half + j : 4 * oth + (j - 4);
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
-                for (int n2 = 0; n2 < 2; ++n2) ldsm_x4(bk[j][n2], Khs + sw_off(Lnk, 8 * (4 * half + 2 * n2), 2 * kt, DK));
-            }
+                for (int n2 = 0; n2 < 2; ++n2)
+                    ldsm_x4(bk[j][n2], Khs + sw_off(Lnk, 8 * (4 * half + 2 * n2), 2 * (4 * half + j), DK));
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int n2 = 0; n2 < 2; ++n2) {
-                    const uint32_t(&b)[4] = bk[j][n2];
-                    if (j < 4) {
-                        mma(dvn[2 * n2], da[j], b[0], b[1]);
-                        mma(dvn[2 * n2 + 1], da[j], b[2], b[3]);
-                    } else {
-                        mma(dvn[2 * n2], dp[j - 4], b[0], b[1]);
-                        mma(dvn[2 * n2 + 1], dp[j - 4], b[2], b[3]);
-                    }
+                    mma(dvn[2 * n2], da[j], bk[j][n2][0], bk[j][n2][1]);
+                    mma(dvn[2 * n2 + 1], da[j], bk[j][n2][2], bk[j][n2][3]);
                 }
-            }
+        }
+        pair_sync(cg);  // the partner's fragments are visible
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) get_frag(xslot(xch, cg, oth, kk, lane), dp[kk]);
+        {  // the partner's rows into separate accumulators
+            uint32_t bk[4][2][4];
+            float dq[4][4] = {};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int n2 = 0; n2 < 2; ++n2)
+                    ldsm_x4(bk[j][n2], Khs + sw_off(Lnk, 8 * (4 * half + 2 * n2), 2 * (4 * oth + j), DK));
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int n2 = 0; n2 < 2; ++n2) {
+                    mma(dq[2 * n2], dp[j], bk[j][n2][0], bk[j][n2][1]);
+                    mma(dq[2 * n2 + 1], dp[j], bk[j][n2][2], bk[j][n2][3]);
+                }
+#pragma unroll
+            for (int nn = 0; nn < 4; ++nn)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dvn[nn][e] += dq[nn][e];
         }
         uint32_t va[2][4], vp[2][4];
 #pragma unroll
@@ -917,31 +951,38 @@ __device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, c
             ds[j][2] = fmaf(ds[j][2], gamC, d1.x);
             ds[j][3] = fmaf(ds[j][3], gamC, d1.y);
         }
+        if (BETA) {  // own token tiles first (no wait for the partner)
+            uint32_t bw[2][4][4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int n2 = 0; n2 < 4; ++n2)
+                    ldsm_x4_t(bw[j][n2], Ws + sw_off(Lkn, 16 * (2 * half + j), 8 * half + 2 * n2, DK));
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int n2 = 0; n2 < 4; ++n2) {
+                    mma(ds[2 * n2], va[j], bw[j][n2][0], bw[j][n2][1]);
+                    mma(ds[2 * n2 + 1], va[j], bw[j][n2][2], bw[j][n2][3]);
+                }
+        }
         pair_sync(cg);
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) get_frag(xslot(xch, cg, oth, 4 + kk, lane), vp[kk]);
-        if (BETA) {
-            uint32_t bw[4][4][4];
+        if (BETA) {  // then the partner's
+            uint32_t bw[2][4][4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int kt = (j < 2) ? 2 * half + j : 2 * oth + (j - 2);
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
-                for (int n2 = 0; n2 < 4; ++n2) ldsm_x4_t(bw[j][n2], Ws + sw_off(Lkn, 16 * kt, 8 * half + 2 * n2, DK));
-            }
+                for (int n2 = 0; n2 < 4; ++n2)
+                    ldsm_x4_t(bw[j][n2], Ws + sw_off(Lkn, 16 * (2 * oth + j), 8 * half + 2 * n2, DK));
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
                 for (int n2 = 0; n2 < 4; ++n2) {
-                    const uint32_t(&b)[4] = bw[j][n2];
-                    if (j < 2) {
-                        mma(ds[2 * n2], va[j], b[0], b[1]);
-                        mma(ds[2 * n2 + 1], va[j], b[2], b[3]);
-                    } else {
-                        mma(ds[2 * n2], vp[j - 2], b[0], b[1]);
-                        mma(ds[2 * n2 + 1], vp[j - 2], b[2], b[3]);
-                    }
+                    mma(ds[2 * n2], vp[j], bw[j][n2][0], bw[j][n2][1]);
+                    mma(ds[2 * n2 + 1], vp[j], bw[j][n2][2], bw[j][n2][3]);
                 }
-            }
         }
         if (dSCt) {
 #pragma unroll
