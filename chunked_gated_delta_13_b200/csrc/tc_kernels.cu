@@ -511,9 +511,12 @@ constexpr size_t bwd_stage_bytes() {  // + the 64 rows of D^T of this block
 // (64 x DK) and the value tile (64 x C), in the permuted layout of swz().
 constexpr size_t out_stage_bytes() { return (size_t)64 * DK * 2 + (size_t)64 * C * 2; }
 constexpr int kOutBufs = 3;  // staged outputs of chunk c are flushed during step c+1 and must be read by step c+3
+constexpr int kFwdStages = 3;  // operand stages of the forward chain: chunk c+2 is in flight during step c
 constexpr size_t xch_bytes();
 template <bool BETA>
-constexpr size_t fwd_scan_smem() { return 2 * fwd_stage_bytes<BETA>() + kOutBufs * out_stage_bytes() + xch_bytes() + 16; }
+constexpr size_t fwd_scan_smem() {
+    return kFwdStages * fwd_stage_bytes<BETA>() + kOutBufs * out_stage_bytes() + xch_bytes() + 8 * kFwdStages;
+}
 template <bool BETA>
 constexpr size_t bwd_scan_smem() { return 2 * bwd_stage_bytes<BETA>() + kOutBufs * out_stage_bytes() + xch_bytes() + 16; }
 
@@ -596,7 +599,7 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
     const int vl = 16 * cg;           // first state column of this warp pair inside the block
     const int v0 = vb * 64 + vl;      // ... and inside the head
     const size_t Tp = (size_t)s.NC * C;
-    unsigned char* outs = smem + 2 * STAGE;
+    unsigned char* outs = smem + kFwdStages * STAGE;
     unsigned char* xch = outs + kOutBufs * out_stage_bytes();
     uint64_t* bars = reinterpret_cast<uint64_t*>(xch + xch_bytes());
     bool failed = false;
@@ -614,7 +617,7 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
     auto load = [&](int cc) {  // thread 0 only
         bf16 *Khs, *Ws, *Uts;
         float* Gs;
-        const int buf = cc & 1;
+        const int buf = cc % kFwdStages;
         stage(buf, Khs, Ws, Uts, Gs);
         const size_t row0 = (size_t)bh * Tp + (size_t)cc * C;
         mbar_expect_tx(&bars[buf], TX);
@@ -643,20 +646,20 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
     const bool outputs = S0t || Vnt;
 
     if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
+        for (int i = 0; i < kFwdStages; ++i) mbar_init(&bars[i], 1);
         mbar_init_fence();
     }
     __syncthreads();
-    if (tid == 0) load(0);
+    if (tid == 0)
+        for (int i = 0; i < kFwdStages - 1 && i < s.NC; ++i) load(i);
     for (int cc = 0; cc < s.NC; ++cc) {
         if (tid == 0) {
-            if (cc + 1 < s.NC) load(cc + 1);  // its buffer was released by the barrier ending step cc-1
+            if (cc + kFwdStages - 1 < s.NC) load(cc + kFwdStages - 1);  // buffer released by the barrier ending step cc-1
             if (outputs && cc > 0) flush(cc - 1);
         }
         bf16 *Khs, *Ws, *Uts;
         float* Gs;
-        stage(cc & 1, Khs, Ws, Uts, Gs);
+        stage(cc % kFwdStages, Khs, Ws, Uts, Gs);
         bf16* S0s = reinterpret_cast<bf16*>(outs + (cc % kOutBufs) * out_stage_bytes());
         bf16* Vns = S0s + 64 * DK;
         // own half of S^T as bf16 fragments, swapped with the partner
@@ -666,7 +669,7 @@ __device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, c
             c2a(sa[kk], st[2 * kk], st[2 * kk + 1]);
             put_frag(xslot(xch, cg, half, kk, lane), sa[kk]);
         }
-        mbar_wait(&bars[cc & 1], (cc >> 1) & 1, &g_tc_status, failed);
+        mbar_wait(&bars[cc % kFwdStages], (cc / kFwdStages) & 1, &g_tc_status, failed);
         const float gamC = Gs[C - 1];
         float vn[4][4];  // V_new^T, tokens 32*half + 8nn..
 #pragma unroll
