@@ -575,12 +575,6 @@ __device__ __forceinline__ void get_frag(const uint4* p, uint32_t (&a)[4]) {
     a[3] = v.w;
 }
 
-// A^T fragment (ldmatrix.trans) from a permuted tile of row length `rowlen`
-// stored [k][m] (see swz): rows k0.., columns m0.. (m0, k0 multiples of 16).
-__device__ __forceinline__ int swz_at_off(int k0, int m0, int lane, int rowlen) {
-    const int lr = (lane & 7) + ((lane >> 4) << 3), pb = (lane >> 3) & 1;
-    return (k0 + lr) * rowlen + ((((m0 >> 3) + pb) ^ (lr & 7)) << 3);
-}
 
 // Forward chain for one (head, 64 state columns): per chunk
 // V_new^T = U^T + S^T (-W)^T, S^T <- gamma_C S^T + V_new^T Khat.

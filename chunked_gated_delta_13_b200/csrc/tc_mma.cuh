@@ -64,7 +64,6 @@ __device__ __forceinline__ uint32_t scale2(uint32_t u, float s0, float s1) {
     const float2 f = unpack(u);
     return pack(f.x * s0, f.y * s1);
 }
-__device__ __forceinline__ uint32_t neg2(uint32_t u) { return u ^ 0x80008000u; }
 
 // A (16 x 16 at [m0, k0]) from a tile stored [m][k] (row-major A).
 __device__ __forceinline__ void ldA(uint32_t (&a)[4], const __nv_bfloat16* s, int ld, int m0, int k0,

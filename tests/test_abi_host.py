@@ -143,3 +143,41 @@ def test_cpu_tensors_rejected():
     q = torch.zeros(1, 1, 8, 16)
     with pytest.raises(RuntimeError):
         sf.fwd(q, q, q, torch.zeros(1, 1, 8), torch.zeros(1, 1, 8))
+
+
+def test_pipelined_segment_workspace_matches_the_documented_size():
+    """Tensor-core segment chain: every piece keeps its forward and intra-chunk
+    intermediates, 8 + 4 dk + 4 C + 6 dv + 4 dk dv / C bytes per token per head
+    (2568 at dk = dv = 128, C = 64), plus three pieces' backward tiles and the
+    fp32 boundary states; the pieces do not depend on how the caller splits T."""
+    B, H, T, d, C = 1, 16, 65536, 128, 64
+    s = sf.make_shape(B, H, T, d, d, C, "bf16")
+    assert sf.path(s) == "tc"
+    per_token = 8 + 4 * d + 4 * C + 6 * d + 4 * d * d // C
+    assert per_token == 2568
+    pieces = T // 4096
+    keep = B * H * T * per_token
+    slots = 3 * B * H * (4096 // C) * (2 * d * C + 2 * d * d)
+    states = (pieces + 3) * B * H * d * d * 4
+    expect = keep + slots + states
+    for N in (1, 4, 16):
+        got = sf.segment_workspace_bytes(s, N)
+        assert expect <= got <= expect * 1.001, (N, got, expect)
+    # a ragged split adds pieces, each with its own boundary state
+    got = sf.segment_workspace_bytes(s, 3, [100, 65336, 100])
+    assert got > expect
+
+
+def test_timer_api_without_launches():
+    """The native launch timer needs no GPU until a kernel runs: enabling with
+    zero capacity, reading nothing and freeing are host-only."""
+    L = sf.lib()
+    L.sf_timer_free()
+    assert L.sf_timer_count() == 0
+    assert L.sf_timer_enable(-1) == 1          # SF_ERR_INVALID_ARG
+    assert L.sf_timer_enable(0) == 0
+    assert L.sf_timer_count() == 0
+    name, ms = ctypes.c_char_p(), ctypes.c_float()
+    assert L.sf_timer_read(0, ctypes.byref(name), ctypes.byref(ms)) == 1
+    L.sf_timer_disable()
+    L.sf_timer_free()
