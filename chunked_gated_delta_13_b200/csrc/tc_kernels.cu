@@ -20,9 +20,10 @@
 //   W = T (gamma * K), U = T V;  V_new = U - W S0;  S_C = gamma_C S0 + Khat^T V_new
 //   O = scale (gamma * Q) S0 + scale ((Q K^T) * Gamma) V_new
 // The state chains keep S (or dS) in fp32 registers as the accumulator of
-// warp-level m16n8k16 products: each warp owns 16 state columns, so the
-// recurrence never leaves the register file; only the operands W, Khat, U
-// stream in through double-buffered asynchronous copies.
+// warp-level m16n8k16 products: each 16-column slice of the state is held by a
+// warp pair, so the recurrence never leaves the register file; only the
+// operands (W, Khat, U or dVi and D) stream in, through bulk copies three
+// (forward) or two (backward) chunks deep.
 #include <algorithm>
 
 #include "tc_kernels.cuh"

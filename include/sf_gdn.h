@@ -201,7 +201,8 @@ void sf_timer_free(void);
 
 /* Introspection for tests and benchmarks: the kernel family a shape runs on
  * ("tc" = tensor-core kernels, "simt" = fp32 CUDA-core kernels; NULL if the
- * shape is unsupported) and how many kernels one call launches. */
+ * shape is unsupported) and how many kernels one sf_gdn_fwd (backward = 0) or
+ * sf_gdn_bwd (backward = 1) call launches. */
 const char* sf_gdn_path(const sf_gdn_shape* shape);
 int sf_gdn_launches(const sf_gdn_shape* shape, int backward);
 
