@@ -129,6 +129,31 @@ def dist_env():
     return ws, rank, local
 
 
+def rank_workload(name, rank):
+    """Replicas: every rank runs its own independent batch, the named workload
+    with the seed offset by the rank (no data crosses ranks)."""
+    from chunked_gated_delta_13_b200.inputs import CONFIGS
+    w = CONFIGS[name]
+    return w.with_(seed=w.seed + rank)
+
+
+def max_over_ranks(x, ws, device):
+    """The slowest rank's value of x (all ranks take part; a no-op on one rank)."""
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_mtokens_per_s(tokens_per_rank, ws, ms):
+    """Whole-job throughput: the tokens all ranks processed over the step time
+    (already the maximum over ranks)."""
+    return tokens_per_rank * ws / (ms * 1e-3) / 1e6
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -291,7 +316,7 @@ def run_ours(args):
         dist.init_process_group("nccl", rank=rank, world_size=ws,
                                 timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    w = CONFIGS[args.workload].with_(seed=CONFIGS[args.workload].seed + rank)
+    w = rank_workload(args.workload, rank)
     seg = args.segments if args.segments else w.N
     inp_cpu = make_inputs(w)
     d = {k: None if v is None else v.to(dev).contiguous() for k, v in inp_cpu.items()}
@@ -316,12 +341,8 @@ def run_ours(args):
         if ws > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if ws == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def max_ranks(x):
+        return max_over_ranks(x, ws, dev)
 
     clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                           else local)
@@ -351,7 +372,7 @@ def run_ours(args):
     barrier()
     sf.timer_disable()
     ms = t0.elapsed_time(t1) / args.steps
-    ms = max_over_ranks(ms)
+    ms = max_ranks(ms)
     clk = clocks.stop()
 
     # per-kernel durations inside the timed region
@@ -390,10 +411,9 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e)
+    e2e_ms = max_ranks(e0.elapsed_time(e1) / n_e2e)
 
-    tokens = w.B * w.T * ws
-    value = tokens / (ms * 1e-3) / 1e6
+    value = job_mtokens_per_s(w.B * w.T, ws, ms)
     pk = peaks()
 
     # roofline of the dominant kernel
@@ -451,7 +471,7 @@ def run_ours(args):
             "kernels_ms": {k: {"launches": len(v), "total_ms": sum(v), "share": sum(v) / sum(tot.values())}
                            for k, v in per.items()},
             "cpu_baseline": cpu,
-            "e2e": {"value": tokens / (e2e_ms * 1e-3) / 1e6, "unit": UNIT,
+            "e2e": {"value": job_mtokens_per_s(w.B * w.T, ws, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches * args.steps,
             "clocks": clk,
