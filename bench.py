@@ -176,29 +176,54 @@ class ClockSampler:
     def __init__(self, device_index):
         self.proc = None
         self.idx = device_index
-        self.out = None
+        self.lines = []
+        self.mark_at = None
+        self.thread = None
 
     def start(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(self.idx)],
+                 "-lms", "50", "-i", str(self.idx)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return
+
+        def reader():
+            for line in self.proc.stdout:
+                self.lines.append(line)
+
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+
+    def mark(self, wait_s=5.0):
+        """Call just before the timed region: waits for the sampler's first line,
+        then remembers where the timed region's samples begin."""
+        t = time.time()
+        while self.proc is not None and not self.lines and time.time() - t < wait_s:
+            time.sleep(0.01)
+        self.mark_at = len(self.lines)
 
     def stop(self):
         if self.proc is None:
             return None
+        timed = len(self.lines) - (self.mark_at or 0)
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-            out, _ = self.proc.communicate()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        # the samples taken during the timed region, else (region shorter than
+        # the sampling interval) all samples of the run
+        lines = self.lines[self.mark_at:self.mark_at + timed] if self.mark_at is not None and timed > 0 \
+            else self.lines
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -213,7 +238,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "in_timed_region": bool(self.mark_at is not None and timed > 0)}
 
 
 # --------------------------------------------------------- reference arm ---
@@ -362,6 +387,7 @@ def run_ours(args):
     sf.timer_enable(per_step_launches * args.steps)
     barrier()
     torch.cuda.synchronize(dev)
+    clocks.mark()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
@@ -486,7 +512,7 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--segments", type=int, default=DEFAULT_SEGMENTS)
