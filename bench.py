@@ -4,8 +4,10 @@
 One step = one pass of the whole path on one batch of synthetic input:
 sf_segment_run over the sequence split into N segments (forward over the
 segments with the state handed on, then backward in reverse with the state
-gradient handed back), i.e. UT transform, chunk scan, output, recompute,
-reverse state-gradient scan and the parallel gradient kernel for every segment.
+gradient handed back), i.e. UT transform, chunk scan, output with the
+intra-chunk backward products, reverse state-gradient scan and the parallel
+gradient kernel for every segment.  Defaults: the B=1, H=16, T=65536, d=128
+workload as 16 segments, 3 warm-up and 50 timed steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--segments N] [--impl ours|reference]
