@@ -107,6 +107,25 @@ def kernel_work(name, w, T_seg):
     return "hbm", flops, byts
 
 
+def step_roofline(w, ms, pk):
+    """The whole step against the binding roofline (the metric's "% of bf16
+    roofline"): algorithmic flops and ABI bytes of forward + backward over every
+    token-head, at the measured peaks.  `frac` is t_roof / t_step for the binding
+    bound; `frac_tensor_sustained` is the step's algorithmic rate against the
+    sustained bf16 peak."""
+    ff, fb = algo_flops_per_token_head(w.C, w.dk, w.dv, w.use_beta)
+    bf_, bb = algo_bytes_per_token_head(w.dk, w.dv, 2 if w.io == "bf16" else 4, w.use_beta)
+    th = w.B * w.H * w.T
+    t_flop = th * (ff + fb) / (pk["bf16_tflops"] * 1e12)
+    t_hbm = th * (bf_ + bb) / (pk["hbm_gbs"] * 1e9)
+    t_roof = max(t_flop, t_hbm)
+    tflops = th * (ff + fb) / (ms * 1e-3) / 1e12
+    return {"bound": "hbm" if t_hbm >= t_flop else "tensor", "t_roof_ms": t_roof * 1e3,
+            "frac": t_roof / (ms * 1e-3), "algo_tflops": tflops,
+            "algo_gbs": th * (bf_ + bb) / (ms * 1e-3) / 1e9,
+            "frac_tensor_sustained": tflops / pk["bf16_tflops_sustained"]}
+
+
 # DRAM bytes (read + write) per chunk-head measured by ncu for each kernel of the
 # tensor-core path (B=1, H=16, T=8192, d=128, one segment cut into two
 # 4096-token pieces: 1024 chunk-heads per launch, mean of the two launches;
@@ -471,16 +490,7 @@ def run_ours(args):
                 "traffic": traffic, "kernel": dom, "avg_launch_ms": avg_ms,
                 "share": tot[dom] / sum(tot.values()), "peak_source": pk["source"]}
 
-    # whole-step roofline (the metric's "% of bf16 roofline")
-    ff, fb = algo_flops_per_token_head(w.C, w.dk, w.dv, w.use_beta)
-    bf_, bb = algo_bytes_per_token_head(w.dk, w.dv, 2 if w.io == "bf16" else 4, w.use_beta)
-    th = w.B * w.H * w.T
-    t_flop = th * (ff + fb) / (pk["bf16_tflops"] * 1e12)
-    t_hbm = th * (bf_ + bb) / (pk["hbm_gbs"] * 1e9)
-    t_roof = max(t_flop, t_hbm)
-    step_roof = {"bound": "hbm" if t_hbm >= t_flop else "tensor", "t_roof_ms": t_roof * 1e3,
-                 "frac": t_roof / (ms * 1e-3), "algo_tflops": th * (ff + fb) / (ms * 1e-3) / 1e12,
-                 "algo_gbs": th * (bf_ + bb) / (ms * 1e-3) / 1e9}
+    step_roof = step_roofline(w, ms, pk)
 
     if rank == 0:
         cpu = None

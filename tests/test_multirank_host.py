@@ -87,3 +87,21 @@ def test_reference_arm_runs_on_rank_zero_only():
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
     assert rec["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_step_roofline_headline_figures():
+    """The headline step's bound (SURVEY's figures: 8.39 MFLOP and 45.4 KB per
+    token, HBM binding at 0.46 ms per step on the measured peaks)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from chunked_gated_delta_13_b200.inputs import CONFIGS
+    w = CONFIGS["headline_h16_t64k"]
+    pk = {"hbm_gbs": 6452.5, "bf16_tflops": 1667.9, "bf16_tflops_sustained": 1378.8}
+    r = bench.step_roofline(w, 4.0, pk)
+    ff, fb = bench.algo_flops_per_token_head(w.C, w.dk, w.dv)
+    bf_, bb = bench.algo_bytes_per_token_head(w.dk, w.dv)
+    assert abs((ff + fb) * w.H / 1e6 - 8.389) < 0.01
+    assert abs((bf_ + bb) * w.H / 1e3 - 45.44) < 0.01
+    assert r["bound"] == "hbm" and abs(r["t_roof_ms"] - 0.4615) < 0.001
+    assert abs(r["frac"] - r["t_roof_ms"] / 4.0) < 1e-12
+    assert abs(r["frac_tensor_sustained"] - r["algo_tflops"] / 1378.8) < 1e-12
