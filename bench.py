@@ -60,12 +60,17 @@ def algo_bytes_per_token_head(dk, dv, esize=2, use_beta=True):
 
 
 def kernel_work(name, w, T_seg):
-    """(bound, algorithmic flops, algorithmic bytes) of ONE launch of `name`
-    on a segment of T_seg tokens (all B*H heads).  Flops count the products the
-    kernel contributes to the method (no recompute); bytes count what the
-    kernel must read and write: its share of the ABI tensors plus the
-    per-chunk intermediates of the chunked decomposition (bf16 tiles, fp32 G and
-    L), each once."""
+    """Work of ONE launch of kernel `name` on a segment of T_seg tokens (all
+    B*H heads): (bound, algorithmic flops, algorithmic bytes, intermediate bytes).
+
+    Algorithmic flops are the method's products the kernel contributes (no
+    recompute).  Algorithmic bytes are the boundary tensors the kernel reads or
+    writes (bf16 or fp32 I/O, fp32 g and beta): the state scans touch none
+    per token, the gradient kernel all of the backward's (q, k, v, dO, g, beta
+    in; dq, dk, dv, dg, dbeta out).  Intermediate bytes are the per-chunk
+    tensors of the chunked decomposition the kernel reads or writes once (bf16
+    tiles, fp32 G and L): a cost of the decomposition, reported apart and not
+    credited to the roofline."""
     C, dk, dv = w.C, w.dk, w.dv
     es = 2 if w.io == "bf16" else 4
     n = w.B * w.H * T_seg                      # token-heads in the launch
@@ -76,35 +81,28 @@ def kernel_work(name, w, T_seg):
     state = dk * dv * wu                       # one chunk state tile
     if name.endswith("prep"):                  # k, v, g, beta -> G, exp G, -W, Khat, U^T, L
         flops = nch * (2 * C * C * dk * (2 if w.use_beta else 0) + 2 * C * C * dv * (1 if w.use_beta else 0))
-        byts = n * (es * (dk + dv) + gb + 8 + wu * (2 * dk + dv)) + nch * lb
-        return "hbm", flops, byts
+        return "hbm", flops, n * (es * (dk + dv) + gb), n * (8 + wu * (2 * dk + dv)) + nch * lb
     if name.endswith("scan_fwd"):              # -W, Khat, U^T, exp G -> V_new^T, chunk states
         flops = nch * 2 * (2 * C * dk * dv)
-        byts = n * (wu * (2 * dk + dv) + 4 + wu * dv) + nch * state
-        return "tensor", flops, byts
+        return "tensor", flops, 0, n * (wu * (2 * dk + dv) + 4 + wu * dv) + nch * state
     if name.endswith("scan_bwd"):              # -W, Khat, dVi^T, exp G, D^T -> dV_new^T, dS_C^T
         flops = nch * 2 * (2 * C * dk * dv)
-        byts = n * (wu * (2 * dk + dv) + 4 + wu * dv) + nch * 2 * state
-        return "tensor", flops, byts
+        return "tensor", flops, 0, n * (wu * (2 * dk + dv) + 4 + wu * dv) + nch * 2 * state
     if name.endswith("out_og"):                # q, k, dO, G, V_new^T, S0^T -> o, dVi^T, D^T
         flops = nch * (2 * C * dk * dv + 2 * C * C * dk + 2 * C * C * dv) + nch * (2 * C * C * dv + 2 * C * dk * dv)
-        byts = n * (es * (2 * dk + dv) + 4 + wu * dv + es * dv + wu * dv) + nch * 2 * state
-        return "hbm", flops, byts
+        return "hbm", flops, n * es * (2 * dk + 2 * dv), n * (4 + 2 * wu * dv) + nch * 2 * state
     if name.endswith("out"):                   # q, k, G, V_new^T, S0^T -> o
         flops = nch * (2 * C * dk * dv + 2 * C * C * dk + 2 * C * C * dv)
-        byts = n * (es * 2 * dk + 4 + wu * dv + es * dv) + nch * state
-        return "hbm", flops, byts
+        return "hbm", flops, n * es * (2 * dk + dv), n * (4 + wu * dv) + nch * state
     if name.endswith("intra"):                 # q, k, dO, G -> dVi^T, D^T
         flops = nch * (2 * C * C * dk + 2 * C * C * dv + 2 * C * dk * dv)
-        byts = n * (es * (2 * dk + dv) + 4 + wu * dv) + nch * state
-        return "hbm", flops, byts
+        return "hbm", flops, n * es * (2 * dk + dv), n * (4 + wu * dv) + nch * state
     # parallel gradients: dP K, dP^T Q, dW (gamma K)^T, T^T dW, dA K (C^2 dk each),
     # dO V_new^T, dU V^T, T^T dU (C^2 dv each), dO S0^T, V_new dS^T, dV_new S0^T (C dk dv each);
-    # q, k, v, dO, g, beta, V_new, dV_new, S0, dS_C, L -> dq, dk, dv, dg, dbeta
+    # q, k, v, dO, g, beta -> dq, dk, dv, dg, dbeta; reads V_new, dV_new, S0, dS_C, L
     flops = nch * (2 * C * C * 5 * dk + 2 * C * C * 3 * dv + 3 * 2 * C * dk * dv)
-    byts = (n * (es * (2 * dk + 2 * dv) + gb + 2 * wu * dv + es * (2 * dk + dv) + gb)
-            + nch * (2 * state + lb))
-    return "hbm", flops, byts
+    _, abi = algo_bytes_per_token_head(dk, dv, es, w.use_beta)
+    return "hbm", flops, n * abi, n * 2 * wu * dv + nch * (2 * state + lb)
 
 
 def step_roofline(w, ms, pk):
@@ -126,11 +124,12 @@ def step_roofline(w, ms, pk):
             "frac_tensor_sustained": tflops / pk["bf16_tflops_sustained"]}
 
 
-# DRAM bytes (read + write) per chunk-head measured by ncu for each kernel of the
-# tensor-core path (B=1, H=16, T=8192, d=128, one segment cut into two
-# 4096-token pieces: 1024 chunk-heads per launch, mean of the two launches;
-# summary and command in profiles/ncu_full_h16_t8k.md).  A launch's traffic is
-# this figure times its chunk-heads.  Valid for the kernels as they were when
+# DRAM bytes (read + write) per chunk-head measured by ncu
+# (dram__bytes_read.sum + dram__bytes_write.sum) for each kernel of the
+# tensor-core path on the small case of the headline shape (B=1, H=16, T=8192,
+# d=128, one segment cut into two 4096-token pipeline pieces: 1024 chunk-heads
+# per launch, mean of the two launches).  A launch's traffic is this figure
+# times its chunk-heads.  Valid for the kernels as they were when
 # captured; an entry is removed when its kernel changes.
 MEASURED_TRAFFIC = {
     "tc_prep": 45850.0,
@@ -472,8 +471,8 @@ def run_ours(args):
         # share of the step: per-launch work = the step's work / launches per step
         per_step = len(per[dom]) / args.steps
         T_seg = -(-w.T // seg)
-        bound, flops, byts = kernel_work(dom, w, T_seg)
-        flops, byts = flops * seg / per_step, byts * seg / per_step
+        bound, flops, byts, inter = kernel_work(dom, w, T_seg)
+        flops, byts, inter = (x * seg / per_step for x in (flops, byts, inter))
         avg_ms = tot[dom] / len(per[dom])
         nch_launch = w.B * w.H * (-(-T_seg // w.C)) * seg / per_step
         traffic = (MEASURED_TRAFFIC[dom] * nch_launch if dom in MEASURED_TRAFFIC and w.io == "bf16"
@@ -488,6 +487,9 @@ def run_ours(args):
             unit = "TFLOP/s"
         roof = {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
                 "traffic": traffic, "kernel": dom, "avg_launch_ms": avg_ms,
+                "algorithmic_bytes": byts, "algorithmic_flops": flops,
+                "intermediate_bytes": inter,
+                "waste": (traffic / byts) if (traffic is not None and byts > 0) else None,
                 "share": tot[dom] / sum(tot.values()), "peak_source": pk["source"]}
 
     step_roof = step_roofline(w, ms, pk)

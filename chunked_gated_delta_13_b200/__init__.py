@@ -64,18 +64,29 @@ _lib = None
 
 
 def lib():
-    """Load libsf_gdn.so (building it in-tree first if it is missing or stale)."""
+    """Load libsf_gdn.so, building it in-tree first if it is missing or older than
+    any of its sources (a failed build raises).  The environment variable
+    SF_GDN_LIB may name a prebuilt library to load as it is instead."""
     global _lib
     with _lock:
         if _lib is not None:
             return _lib
-        if needs_build():
-            try:
-                build()
-            except Exception as exc:  # no nvcc here, or a compile error
-                if not os.path.exists(LIB):
-                    raise RuntimeError(f"libsf_gdn.so is missing and could not be built: {exc}")
-        L = ctypes.CDLL(LIB)
+        path = os.environ.get("SF_GDN_LIB")
+        if path:
+            # explicit opt-in to a prebuilt library (no rebuild, no staleness check)
+            if not os.path.exists(path):
+                raise RuntimeError(f"SF_GDN_LIB names a missing file: {path}")
+        else:
+            path = LIB
+            if needs_build():
+                # a library older than its sources is never loaded: a failed
+                # rebuild (no nvcc, a compile error) raises instead
+                try:
+                    build()
+                except Exception as exc:
+                    raise RuntimeError(f"libsf_gdn.so is missing or older than its sources and could "
+                                       f"not be rebuilt: {exc}") from exc
+        L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         SP = ctypes.POINTER(Shape)
         L.sf_status_str.argtypes = [ctypes.c_int]

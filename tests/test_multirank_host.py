@@ -90,8 +90,9 @@ def test_reference_arm_runs_on_rank_zero_only():
 
 
 def test_step_roofline_headline_figures():
-    """The headline step's bound (SURVEY's figures: 8.39 MFLOP and 45.4 KB per
-    token, HBM binding at 0.46 ms per step on the measured peaks)."""
+    """The headline step's bound: 8.39 MFLOP and 45.4 KB per token (all 16
+    heads) of algorithmic work, HBM binding at 0.46 ms per step on the measured
+    peaks."""
     sys.path.insert(0, ROOT)
     import bench
     from chunked_gated_delta_13_b200.inputs import CONFIGS
@@ -105,3 +106,22 @@ def test_step_roofline_headline_figures():
     assert r["bound"] == "hbm" and abs(r["t_roof_ms"] - 0.4615) < 0.001
     assert abs(r["frac"] - r["t_roof_ms"] / 4.0) < 1e-12
     assert abs(r["frac_tensor_sustained"] - r["algo_tflops"] / 1378.8) < 1e-12
+
+
+def test_dominant_kernel_credits_boundary_bytes_only():
+    """The per-kernel roofline credits a kernel with the boundary tensors it
+    moves: the gradient kernel with all of the backward's (1808 B per token-head
+    at d = 128, bf16), the state scans with none; the decomposition's
+    intermediates are reported apart."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from chunked_gated_delta_13_b200.inputs import CONFIGS
+    w = CONFIGS["headline_h16_t64k"]
+    th = w.B * w.H * 4096
+    bound, flops, abi, inter = bench.kernel_work("tc_grad", w, 4096)
+    assert bound == "hbm" and abi == th * 1808 and inter > 0
+    _, bwd = bench.algo_bytes_per_token_head(w.dk, w.dv, 2, True)
+    assert bwd == 1808
+    for name in ("tc_scan_fwd", "tc_scan_bwd"):
+        bound, flops, abi, inter = bench.kernel_work(name, w, 4096)
+        assert bound == "tensor" and abi == 0 and flops == w.B * w.H * 64 * 2 * (2 * 64 * 128 * 128)

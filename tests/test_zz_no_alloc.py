@@ -13,7 +13,7 @@ import torch
 
 import chunked_gated_delta_13_b200 as sf
 from chunked_gated_delta_13_b200.inputs import Workload, make_inputs
-from gpu_util import relerr, to_device
+from gpu_util import to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -37,21 +37,29 @@ def _noalloc_fwd(d, C, scale=1.0):
     return rc, o, S_out
 
 
-@pytest.mark.parametrize("w,tol", [
-    (Workload("na_bf16", B=1, H=4, T=3 * 64 + 29, dk=128, dv=128, C=64, io="bf16", S_in_std=0.05,
-              g_shift=-3.0), 2e-2),
-    (Workload("na_f32", B=2, H=2, T=150, dk=64, dv=32, C=32, io="f32", S_in_std=0.05), 1e-4),
+@pytest.mark.parametrize("w", [
+    Workload("na_bf16", B=1, H=4, T=3 * 64 + 29, dk=128, dv=128, C=64, io="bf16", S_in_std=0.05,
+             g_shift=-3.0),
+    Workload("na_f32", B=2, H=2, T=150, dk=64, dv=32, C=32, io="f32", S_in_std=0.05),
 ])
-def test_noalloc_forward_matches_workspace_forward(w, tol):
+def test_noalloc_forward_matches_workspace_forward(w):
+    """The scratch-backed forward runs the same kernels as sf_gdn_fwd, so its
+    outputs must be bit-equal.  Before each compared call the scratch is filled
+    by a call on other inputs (another seed, a longer sequence that still fits),
+    so reading anything stale would show."""
     d = to_device(make_inputs(w))
     o_ref, S_ref = sf.fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S_in"], C=w.C)
     torch.cuda.synchronize()
+    T_dirty = 4000 if w.io == "bf16" else 2000
+    dirty = to_device(make_inputs(w.with_(T=T_dirty, seed=w.seed + 1, g_shift=-4.0)))
     for _ in range(2):  # two calls in a row: the shared scratch keeps the previous call's contents
+        rc, _, _ = _noalloc_fwd(dirty, w.C)
+        assert rc == 0, sf.STATUS_NAMES[rc]
         rc, o, S_out = _noalloc_fwd(d, w.C)
         torch.cuda.synchronize()
         assert rc == 0, sf.STATUS_NAMES[rc]
-        assert relerr(o.double().cpu().numpy(), o_ref.double().cpu().numpy()) <= tol
-        assert relerr(S_out.cpu().numpy(), S_ref.cpu().numpy()) <= tol
+        assert torch.equal(o, o_ref)
+        assert torch.equal(S_out, S_ref)
 
 
 def test_noalloc_rejects_shapes_beyond_the_scratch():
