@@ -25,6 +25,7 @@
 // operands (W, Khat, U or dVi and D) stream in, through bulk copies three
 // (forward) or two (backward) chunks deep.
 #include <algorithm>
+#include <cstdlib>
 
 #include "tc_kernels.cuh"
 #include "tc_mma.cuh"
@@ -495,31 +496,48 @@ tc_intra_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
 }
 
 // ------------------------------------------------------------ state scans ---
-// Operand stages of the chains are filled by one thread with bulk copies that
-// complete on an mbarrier per stage; tiles produced by the prep kernel are
-// stored permuted (swz), so the linear copies land bank-conflict-free.
+// The forward state scan (ST) and the reverse state-gradient scan (STB) run
+// the same step on different operands.  With X, Y the two [C][DK] operand
+// tiles of a chunk and R the running state (S^T or dS^T: d_v rows, d_k
+// columns, fp32), one step is
+//     Z^T = I^T + R X^T                 product 1: d_v x C, contraction over d_k
+//     R  <- gamma_C R (+ E) + Z^T Y     product 2: d_v x d_k, contraction over C
+// forward  (chunks in order):   X = -W, Y = Khat, I = U^T, Z = V_new;
+//          per chunk the entering R (S0^T) and Z^T are written, R at the end is S_out^T;
+// backward (chunks in reverse): X = Khat, Y = -W, I = dVi^T, E = D^T, Z = dV_new;
+//          per chunk the entering R (dS_C^T) and Z^T, R at the end is dS_in^T.
+// Without the beta path W is absent: the forward has no product 1 (V_new = V),
+// the backward no product 2 (dS <- gamma_C dS + D).
+//
+// Work split (the pages' tiling of the state transition over d_v): a CTA owns
+// NCG slices of 16 state columns, each carried by four warps.  In product 1
+// warp q of a slice computes tokens 16q..16q+15 over all of d_k, in product 2
+// state rows 32q..32q+31 of d_k over all C tokens; the bf16 left-operand
+// fragments each warp needs from the other three (R for product 1, Z^T for
+// product 2) pass through shared memory, with one 128-thread barrier per
+// product.  The state never leaves the register file.  Operand tiles arrive by
+// bulk copies (the TMA engine) into kStages buffers completing on mbarriers;
+// the outputs are staged by stmatrix and written back by bulk stores.
 constexpr uint32_t kTileK = C * DK * 2;   // a [C][DK] bf16 tile
-constexpr uint32_t kTileV = 64 * C * 2;   // 64 rows of a [DV][C] bf16 tile
-template <bool BETA>
-constexpr size_t fwd_stage_bytes() {
-    return (size_t)kTileK * (BETA ? 2 : 1) + kTileV + C * 4;
-}
-template <bool BETA>
-constexpr size_t bwd_stage_bytes() {  // + the 64 rows of D^T of this block
-    return (size_t)kTileK * (BETA ? 2 : 1) + kTileV + C * 4 + kTileK;
-}
-// Output staging of one chunk step of a 64-column block: the state tile
-// (64 x DK) and the value tile (64 x C), in the permuted layout of swz().
-constexpr size_t out_stage_bytes() { return (size_t)64 * DK * 2 + (size_t)64 * C * 2; }
-constexpr int kOutBufs = 3;  // staged outputs of chunk c are flushed during step c+1 and must be read by step c+3
-constexpr int kFwdStages = 3;  // operand stages of the forward chain: chunk c+2 is in flight during step c
-constexpr size_t xch_bytes();
-template <bool BETA>
-constexpr size_t fwd_scan_smem() {
-    return kFwdStages * fwd_stage_bytes<BETA>() + kOutBufs * out_stage_bytes() + xch_bytes() + 8 * kFwdStages;
-}
-template <bool BETA>
-constexpr size_t bwd_scan_smem() { return 2 * bwd_stage_bytes<BETA>() + kOutBufs * out_stage_bytes() + xch_bytes() + 16; }
+constexpr int kOutBufs = 3;  // staged outputs of step i are flushed during step i+1 and must be read by step i+3
+
+template <int DV, bool BETA, bool BWD, int NCG>
+struct Chain {
+    static constexpr bool HAS_X = BWD || BETA;  // product 1 runs
+    static constexpr bool HAS_Y = !BWD || BETA;  // product 2 runs
+    static constexpr uint32_t kI = NCG * 16 * C * 2;                // I^T rows of this CTA
+    static constexpr uint32_t kE = BWD ? NCG * 16 * DK * 2 : 0;     // E rows of this CTA
+    static constexpr uint32_t kX = HAS_X ? kTileK : 0, kY = HAS_Y ? kTileK : 0;
+    static constexpr uint32_t TX = kX + kY + kI + C * 4 + kE;       // bytes of one stage (all copied)
+    static constexpr size_t OUT = (size_t)NCG * 16 * (DK + C) * 2;  // staged R and Z^T rows of one step
+    static constexpr size_t XCH = (size_t)NCG * 12 * 32 * 16;       // 8 R + 4 Z^T fragments per slice
+    static constexpr size_t smem(int stages) { return stages * (size_t)TX + kOutBufs * OUT + XCH + 8 * stages; }
+    // as many operand stages as fit (up to 6): a step's operands are requested
+    // kStages - 1 steps ahead, which must cover the latency of the copies
+    static constexpr int kStages = smem(6) <= 227 * 1024 ? 6 : smem(5) <= 227 * 1024 ? 5
+                                 : smem(4) <= 227 * 1024 ? 4 : smem(3) <= 227 * 1024 ? 3 : 2;
+    static constexpr size_t SMEM = smem(kStages);
+};
 
 // Per-lane parts of the addresses into permuted [rows][128] tiles.
 //   B fragments (stored [n][k], k = 16kk..): row = n0 + lr, piece 2kk + pb
@@ -551,22 +569,6 @@ __device__ __forceinline__ void stage_afrag(bf16* t, int cols, int r0, int c0, c
     stsm_x4(t + (r0 + lr) * cols + piece * 8, a);
 }
 
-// The chains use 8 warps per 64-column block: warps w and w+4 (which share an
-// SM sub-partition) own the same 16 state columns and split every chunk step,
-// the first warp taking tokens 0-31 of V_new and state rows 0-63 (of d_k),
-// the second tokens 32-63 and rows 64-127.  Each product needs the partner's
-// half of its left operand, which the pair swaps as bf16 fragments through
-// shared memory.  One warp alone can issue a warp-level MMA only every ~18
-// cycles, so two warps per sub-partition halve the step's issue time.
-constexpr size_t xch_bytes() { return (size_t)4 * 2 * (4 + 2) * 32 * 16; }  // per pair: 4 state + 2 value fragments
-
-// Pair barrier of the two warps that share a column group.
-__device__ __forceinline__ void pair_sync(int cg) { asm volatile("bar.sync %0, 64;\n" ::"r"(cg + 1) : "memory"); }
-
-// Fragment exchange slots (16 bytes per lane): [cg][half][slot 0-5][lane].
-__device__ __forceinline__ uint4* xslot(unsigned char* xch, int cg, int half, int slot, int lane) {
-    return reinterpret_cast<uint4*>(xch) + (((cg * 2 + half) * 6 + slot) * 32 + lane);
-}
 __device__ __forceinline__ void put_frag(uint4* p, const uint32_t (&a)[4]) { *p = make_uint4(a[0], a[1], a[2], a[3]); }
 __device__ __forceinline__ void get_frag(const uint4* p, uint32_t (&a)[4]) {
     const uint4 v = *p;
@@ -575,473 +577,241 @@ __device__ __forceinline__ void get_frag(const uint4* p, uint32_t (&a)[4]) {
     a[2] = v.z;
     a[3] = v.w;
 }
+// Barrier of the four warps of slice g (named barriers 1..NCG).
+__device__ __forceinline__ void slice_sync(int g) { asm volatile("bar.sync %0, 128;\n" ::"r"(g + 1) : "memory"); }
 
+// Operands of one chain launch, for one direction.
+struct ChainOps {
+    const bf16* X;      // [BH][Tp][DK] permuted: -W (forward) or Khat (backward)
+    const bf16* Y;      // [BH][Tp][DK] permuted: Khat (forward) or -W (backward)
+    const bf16* I;      // [BH][NC][DV][C] permuted: U^T or dVi^T
+    const bf16* E;      // [BH][NC][DV][DK] permuted: D^T (backward only)
+    const float* Gm;    // [BH][Tp] exp(G)
+    const float* R_in;  // [BH][DK][DV] S_in or dS_out (NULL = zeros)
+    bf16* Rt;           // [BH][NC][DV][DK] permuted: S0^T or dS_C^T per chunk (NULL = skip)
+    bf16* Zt;           // [BH][NC][DV][C] permuted: V_new^T or dV_new^T per chunk (NULL = skip)
+    float* R_out;       // [BH][DK][DV] S_out or dS_in (NULL = skip)
+};
 
-// Forward chain for one (head, 64 state columns): per chunk
-// V_new^T = U^T + S^T (-W)^T, S^T <- gamma_C S^T + V_new^T Khat.
-// Optional outputs: V_new^T and S0^T per chunk (bf16, bulk-stored from a
-// staging area by one thread), S_out (fp32).
-template <int DV, bool BETA>
-__device__ __forceinline__ void scan_fwd_cta(const SeqView& s, int bh, int vb, const float* __restrict__ Gm,
-                                             const bf16* __restrict__ Wn, const bf16* __restrict__ Kh,
-                                             const bf16* __restrict__ Ut, const float* __restrict__ S_in,
-                                             bf16* __restrict__ Vnt, bf16* __restrict__ S0t,
-                                             float* __restrict__ S_out, unsigned char* smem) {
-    constexpr size_t STAGE = fwd_stage_bytes<BETA>();
-    constexpr uint32_t TX = (BETA ? 2 : 1) * kTileK + kTileV + C * 4;
+template <int DV, bool BETA, bool BWD, int NCG>
+__device__ __forceinline__ void chain_cta(const SeqView& s, int bh, int vb, const ChainOps& op, unsigned char* smem) {
+    using CH = Chain<DV, BETA, BWD, NCG>;
+    constexpr int NS = CH::kStages;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, gq = lane >> 2, tq = lane & 3;
-    const int cg = w & 3, half = w >> 2, oth = half ^ 1;
-    const int vl = 16 * cg;           // first state column of this warp pair inside the block
-    const int v0 = vb * 64 + vl;      // ... and inside the head
+    const int g = w >> 2, q = w & 3;        // slice of this warp, warp index inside the slice
+    const int v0 = vb * 16 * NCG;           // first state column of the CTA
+    const int vr = 16 * g;                  // first row of this slice in the CTA's tiles
     const size_t Tp = (size_t)s.NC * C;
-    unsigned char* outs = smem + kFwdStages * STAGE;
-    unsigned char* xch = outs + kOutBufs * out_stage_bytes();
-    uint64_t* bars = reinterpret_cast<uint64_t*>(xch + xch_bytes());
+    unsigned char* outs = smem + NS * (size_t)CH::TX;
+    uint4* xch = reinterpret_cast<uint4*>(outs + kOutBufs * CH::OUT) + g * 12 * 32 + lane;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(outs + kOutBufs * CH::OUT + CH::XCH);
     bool failed = false;
 
-    auto stage = [&](int buf, bf16*& Khs, bf16*& Ws, bf16*& Uts, float*& Gs) {
-        unsigned char* p = smem + buf * STAGE;
-        Khs = reinterpret_cast<bf16*>(p);
-        p += kTileK;
-        Ws = reinterpret_cast<bf16*>(p);
-        if (BETA) p += kTileK;
-        Uts = reinterpret_cast<bf16*>(p);
-        p += kTileV;
-        Gs = reinterpret_cast<float*>(p);
+    auto chunk_of = [&](int i) { return BWD ? s.NC - 1 - i : i; };
+    struct Stage {
+        bf16 *X, *Y, *I, *E;
+        float* G;
     };
-    auto load = [&](int cc) {  // thread 0 only
-        bf16 *Khs, *Ws, *Uts;
-        float* Gs;
-        const int buf = cc % kFwdStages;
-        stage(buf, Khs, Ws, Uts, Gs);
+    auto stage = [&](int buf) {
+        unsigned char* p = smem + buf * (size_t)CH::TX;
+        Stage st;
+        st.X = reinterpret_cast<bf16*>(p);
+        st.Y = reinterpret_cast<bf16*>(p + CH::kX);
+        st.I = reinterpret_cast<bf16*>(p + CH::kX + CH::kY);
+        st.G = reinterpret_cast<float*>(p + CH::kX + CH::kY + CH::kI);
+        st.E = reinterpret_cast<bf16*>(p + CH::kX + CH::kY + CH::kI + C * 4);
+        return st;
+    };
+    auto load = [&](int i) {  // thread 0: bulk copies of step i's operands
+        const int cc = chunk_of(i), buf = i % NS;
+        const Stage st = stage(buf);
         const size_t row0 = (size_t)bh * Tp + (size_t)cc * C;
-        mbar_expect_tx(&bars[buf], TX);
-        bulk_load(Khs, Kh + row0 * DK, kTileK, &bars[buf]);
-        if (BETA) bulk_load(Ws, Wn + row0 * DK, kTileK, &bars[buf]);
-        bulk_load(Uts, Ut + (((size_t)bh * s.NC + cc) * DV + vb * 64) * C, kTileV, &bars[buf]);
-        bulk_load(Gs, Gm + row0, C * 4, &bars[buf]);
+        const size_t blk = ((size_t)bh * s.NC + cc) * DV + v0;
+        mbar_expect_tx(&bars[buf], CH::TX);
+        if (CH::HAS_X) bulk_load(st.X, op.X + row0 * DK, kTileK, &bars[buf]);
+        if (CH::HAS_Y) bulk_load(st.Y, op.Y + row0 * DK, kTileK, &bars[buf]);
+        bulk_load(st.I, op.I + blk * C, CH::kI, &bars[buf]);
+        bulk_load(st.G, op.Gm + row0, C * 4, &bars[buf]);
+        if (BWD) bulk_load(st.E, op.E + blk * DK, CH::kE, &bars[buf]);
     };
-    auto flush = [&](int cc) {  // thread 0 only: bulk-store the staged outputs of chunk cc
-        unsigned char* o = outs + (cc % kOutBufs) * out_stage_bytes();
-        const size_t blk = ((size_t)bh * s.NC + cc) * DV + vb * 64;
-        if (S0t) bulk_store(S0t + blk * DK, o, 64 * DK * 2);
-        if (Vnt) bulk_store(Vnt + blk * C, o + 64 * DK * 2, 64 * C * 2);
+    const bool outputs = op.Rt || op.Zt;
+    auto flush = [&](int i) {  // thread 0: bulk-store the staged outputs of step i
+        unsigned char* o = outs + (i % kOutBufs) * CH::OUT;
+        const size_t blk = ((size_t)bh * s.NC + chunk_of(i)) * DV + v0;
+        if (op.Rt) bulk_store(op.Rt + blk * DK, o, NCG * 16 * DK * 2);
+        if (op.Zt) bulk_store(op.Zt + blk * C, o + NCG * 16 * DK * 2, NCG * 16 * C * 2);
         bulk_commit();
     };
 
-    float st[8][4];  // S^T rows vl.., state rows 64*half + 8j..
+    // R: rows vr + gq (+8) of the slice, d_k columns 32q + 8j + 2tq (+1)
+    float r[4][4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const int vv = v0 + gq + 8 * (e >> 1), d = 64 * half + 8 * j + 2 * tq + (e & 1);
-            st[j][e] = S_in ? S_in[((size_t)bh * DK + d) * DV + vv] : 0.f;
+            const int vv = v0 + vr + gq + 8 * (e >> 1), d = 32 * q + 8 * j + 2 * tq + (e & 1);
+            r[j][e] = op.R_in ? op.R_in[((size_t)bh * DK + d) * DV + vv] : 0.f;
         }
     const SwLane Lnk = sw_lane_nk(lane), Lkn = sw_lane_kn(lane);
-    const bool outputs = S0t || Vnt;
 
     if (tid == 0) {
-        for (int i = 0; i < kFwdStages; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
         mbar_init_fence();
     }
     __syncthreads();
     if (tid == 0)
-        for (int i = 0; i < kFwdStages - 1 && i < s.NC; ++i) load(i);
-    for (int cc = 0; cc < s.NC; ++cc) {
+        for (int i = 0; i < NS - 1 && i < s.NC; ++i) load(i);
+    for (int i = 0; i < s.NC; ++i) {
         if (tid == 0) {
-            if (cc + kFwdStages - 1 < s.NC) load(cc + kFwdStages - 1);  // buffer released by the barrier ending step cc-1
-            if (outputs && cc > 0) flush(cc - 1);
+            if (i + NS - 1 < s.NC) load(i + NS - 1);  // its buffer was released by the barrier ending step i-1
+            if (outputs && i > 0) flush(i - 1);
         }
-        bf16 *Khs, *Ws, *Uts;
-        float* Gs;
-        stage(cc % kFwdStages, Khs, Ws, Uts, Gs);
-        bf16* S0s = reinterpret_cast<bf16*>(outs + (cc % kOutBufs) * out_stage_bytes());
-        bf16* Vns = S0s + 64 * DK;
-        // own half of S^T as bf16 fragments, swapped with the partner
-        uint32_t sa[4][4], sp[4][4];
+        const Stage st = stage(i % NS);
+        bf16* Rs = reinterpret_cast<bf16*>(outs + (i % kOutBufs) * CH::OUT);  // [16 NCG][DK]
+        bf16* Zs = Rs + NCG * 16 * DK;                                        // [16 NCG][C]
+        // the entering R as bf16 fragments of this warp's k-tiles 2q, 2q+1
+        uint32_t sa[2][4];
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            c2a(sa[kk], st[2 * kk], st[2 * kk + 1]);
-            put_frag(xslot(xch, cg, half, kk, lane), sa[kk]);
+        for (int jj = 0; jj < 2; ++jj) {
+            c2a(sa[jj], r[2 * jj], r[2 * jj + 1]);
+            if (CH::HAS_X) put_frag(xch + (2 * q + jj) * 32, sa[jj]);
+            if (op.Rt) stage_afrag(Rs, DK, vr, 16 * (2 * q + jj), sa[jj], lane);
         }
-        mbar_wait(&bars[cc % kFwdStages], (cc / kFwdStages) & 1, &g_tc_status, failed);
-        const float gamC = Gs[C - 1];
-        float vn[4][4];  // V_new^T, tokens 32*half + 8nn..
+        if (CH::HAS_X) slice_sync(g);
+        mbar_wait(&bars[i % NS], (i / NS) & 1, &g_tc_status, failed);
+        const float gamC = st.G[C - 1];
+
+        // product 1: Z^T (rows vr.., tokens 16q + 8n + 2tq ..) = I^T + R X^T
+        float z[2][4];
 #pragma unroll
-        for (int nn = 0; nn < 4; ++nn) {
-            const int po = (((4 * half + nn) ^ gq) << 3) + 2 * tq;
-            const float2 u0 = unpack(*reinterpret_cast<const uint32_t*>(Uts + (vl + gq) * C + po));
-            const float2 u1 = unpack(*reinterpret_cast<const uint32_t*>(Uts + (vl + gq + 8) * C + po));
-            vn[nn][0] = u0.x;
-            vn[nn][1] = u0.y;
-            vn[nn][2] = u1.x;
-            vn[nn][3] = u1.y;
+        for (int n = 0; n < 2; ++n) {
+            const int po = (((2 * q + n) ^ gq) << 3) + 2 * tq;
+            const float2 u0 = unpack(*reinterpret_cast<const uint32_t*>(st.I + (vr + gq) * C + po));
+            const float2 u1 = unpack(*reinterpret_cast<const uint32_t*>(st.I + (vr + gq + 8) * C + po));
+            z[n][0] = u0.x;
+            z[n][1] = u0.y;
+            z[n][2] = u1.x;
+            z[n][3] = u1.y;
         }
-        // own state rows first (no wait for the partner), the partner's rows into
-        // separate accumulators once its fragments are in
-        if (BETA) {
-            uint32_t bw[4][2][4];
+        if (CH::HAS_X) {
+            uint32_t ra[8][4];  // all eight k-tiles of R (own ones from registers)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                if ((kk >> 1) == q) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) ra[kk][e] = sa[kk & 1][e];
+                } else {
+                    get_frag(xch + kk * 32, ra[kk]);
+                }
+            }
+            float zq[2][4] = {};  // odd k-tiles: two shorter dependent chains
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                uint32_t b[4];
+                ldsm_x4(b, st.X + sw_off(Lnk, 16 * q, 2 * kk, DK));
+                if (kk & 1) {
+                    mma(zq[0], ra[kk], b[0], b[1]);
+                    mma(zq[1], ra[kk], b[2], b[3]);
+                } else {
+                    mma(z[0], ra[kk], b[0], b[1]);
+                    mma(z[1], ra[kk], b[2], b[3]);
+                }
+            }
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) z[n][e] += zq[n][e];
+        }
+        uint32_t za[4];
+        c2a(za, z[0], z[1]);
+        if (CH::HAS_Y) put_frag(xch + (8 + q) * 32, za);
+        if (op.Zt) stage_afrag(Zs, C, vr, 16 * q, za, lane);
+
+        // product 2: R <- gamma_C R (+ E) + Z^T Y
+        if (BWD) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int col = 32 * q + 8 * j + 2 * tq;
+                const float2 d0 = unpack(*reinterpret_cast<const uint32_t*>(st.E + swz(vr + gq, col, DK)));
+                const float2 d1 = unpack(*reinterpret_cast<const uint32_t*>(st.E + swz(vr + gq + 8, col, DK)));
+                r[j][0] = fmaf(r[j][0], gamC, d0.x);
+                r[j][1] = fmaf(r[j][1], gamC, d0.y);
+                r[j][2] = fmaf(r[j][2], gamC, d1.x);
+                r[j][3] = fmaf(r[j][3], gamC, d1.y);
+            }
+        } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
-                for (int n2 = 0; n2 < 2; ++n2)
-                    ldsm_x4(bw[j][n2], Ws + sw_off(Lnk, 8 * (4 * half + 2 * n2), 2 * (4 * half + j), DK));
+                for (int e = 0; e < 4; ++e) r[j][e] *= gamC;
+        }
+        if (CH::HAS_Y) {
+            slice_sync(g);
+            uint32_t zf[4][4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int kt = 0; kt < 4; ++kt) {
+                if (kt == q) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) zf[kt][e] = za[e];
+                } else {
+                    get_frag(xch + (8 + kt) * 32, zf[kt]);
+                }
+            }
+#pragma unroll
+            for (int kt = 0; kt < 4; ++kt)
 #pragma unroll
                 for (int n2 = 0; n2 < 2; ++n2) {
-                    mma(vn[2 * n2], sa[j], bw[j][n2][0], bw[j][n2][1]);
-                    mma(vn[2 * n2 + 1], sa[j], bw[j][n2][2], bw[j][n2][3]);
+                    uint32_t b[4];
+                    ldsm_x4_t(b, st.Y + sw_off(Lkn, 16 * kt, 4 * q + 2 * n2, DK));
+                    mma(r[2 * n2], zf[kt], b[0], b[1]);
+                    mma(r[2 * n2 + 1], zf[kt], b[2], b[3]);
                 }
-        }
-        pair_sync(cg);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) get_frag(xslot(xch, cg, oth, kk, lane), sp[kk]);
-        if (BETA) {
-            uint32_t bw[4][2][4];
-            float vq[4][4] = {};
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 2; ++n2)
-                    ldsm_x4(bw[j][n2], Ws + sw_off(Lnk, 8 * (4 * half + 2 * n2), 2 * (4 * oth + j), DK));
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 2; ++n2) {
-                    mma(vq[2 * n2], sp[j], bw[j][n2][0], bw[j][n2][1]);
-                    mma(vq[2 * n2 + 1], sp[j], bw[j][n2][2], bw[j][n2][3]);
-                }
-#pragma unroll
-            for (int nn = 0; nn < 4; ++nn)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) vn[nn][e] += vq[nn][e];
-        }
-        uint32_t va[2][4], vp[2][4];
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-            c2a(va[kk], vn[2 * kk], vn[2 * kk + 1]);
-            put_frag(xslot(xch, cg, half, 4 + kk, lane), va[kk]);
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) st[j][e] *= gamC;
-        {  // own token tiles first (no wait for the partner)
-            uint32_t bk[2][4][4];
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 4; ++n2)
-                    ldsm_x4_t(bk[j][n2], Khs + sw_off(Lkn, 16 * (2 * half + j), 8 * half + 2 * n2, DK));
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 4; ++n2) {
-                    mma(st[2 * n2], va[j], bk[j][n2][0], bk[j][n2][1]);
-                    mma(st[2 * n2 + 1], va[j], bk[j][n2][2], bk[j][n2][3]);
-                }
-        }
-        pair_sync(cg);
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) get_frag(xslot(xch, cg, oth, 4 + kk, lane), vp[kk]);
-        {  // then the partner's
-            uint32_t bk[2][4][4];
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 4; ++n2)
-                    ldsm_x4_t(bk[j][n2], Khs + sw_off(Lkn, 16 * (2 * oth + j), 8 * half + 2 * n2, DK));
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 4; ++n2) {
-                    mma(st[2 * n2], vp[j], bk[j][n2][0], bk[j][n2][1]);
-                    mma(st[2 * n2 + 1], vp[j], bk[j][n2][2], bk[j][n2][3]);
-                }
-        }
-        // stage this chunk's outputs (own halves) while the state update is in flight
-        if (S0t) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) stage_afrag(S0s, DK, vl, 64 * half + 16 * kk, sa[kk], lane);
-        }
-        if (Vnt) {
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk) stage_afrag(Vns, C, vl, 32 * half + 16 * kk, va[kk], lane);
         }
         if (outputs) fence_proxy_async_smem();
-        if (tid == 0 && outputs) bulk_wait_read<1>();  // chunk cc-2's outputs left their buffer
+        if (tid == 0 && outputs) bulk_wait_read<1>();  // step i-2's outputs left their buffer
         __syncthreads();
     }
     if (tid == 0) {
         if (outputs && s.NC > 0) flush(s.NC - 1);
         bulk_wait<0>();
     }
-    if (S_out) {
+    if (op.R_out) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int vv = v0 + gq + 8 * (e >> 1), d = 64 * half + 8 * j + 2 * tq + (e & 1);
-                S_out[((size_t)bh * DK + d) * DV + vv] = st[j][e];
+                const int vv = v0 + vr + gq + 8 * (e >> 1), d = 32 * q + 8 * j + 2 * tq + (e & 1);
+                op.R_out[((size_t)bh * DK + d) * DV + vv] = r[j][e];
             }
     }
 }
 
-// Reverse chain of the state gradient for one (head, 64 state columns):
-// per chunk, from the last, dV_new^T = dVi^T + dS^T Khat^T and
-// dS^T <- gamma_C dS^T + D^T + dV_new^T (-W), D^T = (scale (gamma * dO)^T Q)^T
-// precomputed by the intra-chunk products.
-// Outputs dV_new^T and dS_C^T per chunk (bf16, staged and bulk-stored), dS_in (fp32).
-template <int DV, bool BETA>
-__device__ __forceinline__ void scan_bwd_cta(const SeqView& s, int bh, int vb, const bf16* __restrict__ Dt,
-                                             const float* __restrict__ Gm,
-                                             const bf16* __restrict__ Wn, const bf16* __restrict__ Kh,
-                                             const bf16* __restrict__ dVit, const float* __restrict__ dS_out,
-                                             bf16* __restrict__ dVnt, bf16* __restrict__ dSCt,
-                                             float* __restrict__ dS_in, unsigned char* smem) {
-    constexpr size_t STAGE = bwd_stage_bytes<BETA>();
-    constexpr uint32_t TX = (BETA ? 2 : 1) * kTileK + kTileV + C * 4 + kTileK;
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, gq = lane >> 2, tq = lane & 3;
-    const int cg = w & 3, half = w >> 2, oth = half ^ 1;
-    const int vl = 16 * cg;
-    const int v0 = vb * 64 + vl;
-    const size_t Tp = (size_t)s.NC * C;
-    unsigned char* outs = smem + 2 * STAGE;
-    unsigned char* xch = outs + kOutBufs * out_stage_bytes();
-    uint64_t* bars = reinterpret_cast<uint64_t*>(xch + xch_bytes());
-    bool failed = false;
+// Chain CTAs per head for NCG slices per CTA.
+template <int DV, int NCG>
+constexpr int chain_ctas_per_head() { return DV / (16 * NCG); }
 
-    auto stage = [&](int buf, bf16*& Khs, bf16*& Ws, bf16*& dVis, float*& Gs, bf16*& Dts) {
-        unsigned char* p = smem + buf * STAGE;
-        Khs = reinterpret_cast<bf16*>(p);
-        p += kTileK;
-        Ws = reinterpret_cast<bf16*>(p);
-        if (BETA) p += kTileK;
-        dVis = reinterpret_cast<bf16*>(p);
-        p += kTileV;
-        Gs = reinterpret_cast<float*>(p);
-        p += C * 4;
-        Dts = reinterpret_cast<bf16*>(p);
-    };
-    auto load = [&](int cc) {  // thread 0: bulk copies of one chunk's operands
-        bf16 *Khs, *Ws, *dVis, *Dts;
-        float* Gs;
-        const int buf = cc & 1;
-        stage(buf, Khs, Ws, dVis, Gs, Dts);
-        const size_t row0 = (size_t)bh * Tp + (size_t)cc * C;
-        const size_t blk = ((size_t)bh * s.NC + cc) * DV + vb * 64;
-        if (tid == 0) {
-            mbar_expect_tx(&bars[buf], TX);
-            bulk_load(Khs, Kh + row0 * DK, kTileK, &bars[buf]);
-            if (BETA) bulk_load(Ws, Wn + row0 * DK, kTileK, &bars[buf]);
-            bulk_load(dVis, dVit + blk * C, kTileV, &bars[buf]);
-            bulk_load(Gs, Gm + row0, C * 4, &bars[buf]);
-            bulk_load(Dts, Dt + blk * DK, kTileK, &bars[buf]);
-        }
-    };
-    auto flush = [&](int cc) {
-        unsigned char* o = outs + (cc % kOutBufs) * out_stage_bytes();
-        const size_t blk = ((size_t)bh * s.NC + cc) * DV + vb * 64;
-        if (dSCt) bulk_store(dSCt + blk * DK, o, 64 * DK * 2);
-        if (dVnt) bulk_store(dVnt + blk * C, o + 64 * DK * 2, 64 * C * 2);
-        bulk_commit();
-    };
-
-    float ds[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int vv = v0 + gq + 8 * (e >> 1), d = 64 * half + 8 * j + 2 * tq + (e & 1);
-            ds[j][e] = dS_out ? dS_out[((size_t)bh * DK + d) * DV + vv] : 0.f;
-        }
-    const SwLane Lnk = sw_lane_nk(lane), Lkn = sw_lane_kn(lane);
-    const bool outputs = dSCt || dVnt;
-
-    if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        mbar_init_fence();
-    }
-    __syncthreads();
-    load(s.NC - 1);
-    for (int cc = s.NC - 1; cc >= 0; --cc) {
-        const int use = s.NC - 1 - cc;  // how many chunks were processed before this one
-        if (cc > 0) load(cc - 1);
-        if (tid == 0 && outputs && cc < s.NC - 1) flush(cc + 1);
-        bf16 *Khs, *Ws, *dVis, *Dts;
-        float* Gs;
-        stage(cc & 1, Khs, Ws, dVis, Gs, Dts);
-        bf16* dSs = reinterpret_cast<bf16*>(outs + (cc % kOutBufs) * out_stage_bytes());
-        bf16* dVns = dSs + 64 * DK;
-        uint32_t da[4][4], dp[4][4];
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            c2a(da[kk], ds[2 * kk], ds[2 * kk + 1]);
-            put_frag(xslot(xch, cg, half, kk, lane), da[kk]);
-        }
-        mbar_wait(&bars[cc & 1], (use >> 1) & 1, &g_tc_status, failed);
-        const float gamC = Gs[C - 1];
-        float dvn[4][4];  // dV_new^T, tokens 32*half + 8nn..
-#pragma unroll
-        for (int nn = 0; nn < 4; ++nn) {
-            const int po = (((4 * half + nn) ^ gq) << 3) + 2 * tq;
-            const float2 u0 = unpack(*reinterpret_cast<const uint32_t*>(dVis + (vl + gq) * C + po));
-            const float2 u1 = unpack(*reinterpret_cast<const uint32_t*>(dVis + (vl + gq + 8) * C + po));
-            dvn[nn][0] = u0.x;
-            dvn[nn][1] = u0.y;
-            dvn[nn][2] = u1.x;
-            dvn[nn][3] = u1.y;
-        }
-        {  // own state rows first (no wait for the partner)
-            uint32_t bk[4][2][4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 2; ++n2)
-                    ldsm_x4(bk[j][n2], Khs + sw_off(Lnk, 8 * (4 * half + 2 * n2), 2 * (4 * half + j), DK));
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 2; ++n2) {
-                    mma(dvn[2 * n2], da[j], bk[j][n2][0], bk[j][n2][1]);
-                    mma(dvn[2 * n2 + 1], da[j], bk[j][n2][2], bk[j][n2][3]);
-                }
-        }
-        pair_sync(cg);  // the partner's fragments are visible
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) get_frag(xslot(xch, cg, oth, kk, lane), dp[kk]);
-        {  // the partner's rows into separate accumulators
-            uint32_t bk[4][2][4];
-            float dq[4][4] = {};
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 2; ++n2)
-                    ldsm_x4(bk[j][n2], Khs + sw_off(Lnk, 8 * (4 * half + 2 * n2), 2 * (4 * oth + j), DK));
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 2; ++n2) {
-                    mma(dq[2 * n2], dp[j], bk[j][n2][0], bk[j][n2][1]);
-                    mma(dq[2 * n2 + 1], dp[j], bk[j][n2][2], bk[j][n2][3]);
-                }
-#pragma unroll
-            for (int nn = 0; nn < 4; ++nn)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) dvn[nn][e] += dq[nn][e];
-        }
-        uint32_t va[2][4], vp[2][4];
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-            c2a(va[kk], dvn[2 * kk], dvn[2 * kk + 1]);
-            put_frag(xslot(xch, cg, half, 4 + kk, lane), va[kk]);
-        }
-        // dS <- gamma_C dS + D (D from the intra kernel, independent of the chain)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int col = 64 * half + 8 * j + 2 * tq;
-            const float2 d0 = unpack(*reinterpret_cast<const uint32_t*>(Dts + swz(vl + gq, col, DK)));
-            const float2 d1 = unpack(*reinterpret_cast<const uint32_t*>(Dts + swz(vl + gq + 8, col, DK)));
-            ds[j][0] = fmaf(ds[j][0], gamC, d0.x);
-            ds[j][1] = fmaf(ds[j][1], gamC, d0.y);
-            ds[j][2] = fmaf(ds[j][2], gamC, d1.x);
-            ds[j][3] = fmaf(ds[j][3], gamC, d1.y);
-        }
-        if (BETA) {  // own token tiles first (no wait for the partner)
-            uint32_t bw[2][4][4];
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 4; ++n2)
-                    ldsm_x4_t(bw[j][n2], Ws + sw_off(Lkn, 16 * (2 * half + j), 8 * half + 2 * n2, DK));
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 4; ++n2) {
-                    mma(ds[2 * n2], va[j], bw[j][n2][0], bw[j][n2][1]);
-                    mma(ds[2 * n2 + 1], va[j], bw[j][n2][2], bw[j][n2][3]);
-                }
-        }
-        pair_sync(cg);
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) get_frag(xslot(xch, cg, oth, 4 + kk, lane), vp[kk]);
-        if (BETA) {  // then the partner's
-            uint32_t bw[2][4][4];
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 4; ++n2)
-                    ldsm_x4_t(bw[j][n2], Ws + sw_off(Lkn, 16 * (2 * oth + j), 8 * half + 2 * n2, DK));
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int n2 = 0; n2 < 4; ++n2) {
-                    mma(ds[2 * n2], vp[j], bw[j][n2][0], bw[j][n2][1]);
-                    mma(ds[2 * n2 + 1], vp[j], bw[j][n2][2], bw[j][n2][3]);
-                }
-        }
-        if (dSCt) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) stage_afrag(dSs, DK, vl, 64 * half + 16 * kk, da[kk], lane);
-        }
-        if (dVnt) {
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk) stage_afrag(dVns, C, vl, 32 * half + 16 * kk, va[kk], lane);
-        }
-        if (outputs) fence_proxy_async_smem();
-        if (tid == 0 && outputs) bulk_wait_read<1>();
-        __syncthreads();
-    }
-    if (tid == 0) {
-        if (outputs && s.NC > 0) flush(0);
-        bulk_wait<0>();
-    }
-    if (dS_in) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int vv = v0 + gq + 8 * (e >> 1), d = 64 * half + 8 * j + 2 * tq + (e & 1);
-                dS_in[((size_t)bh * DK + d) * DV + vv] = ds[j][e];
-            }
-    }
+template <int DV, bool BETA, int NCG>
+__global__ void __launch_bounds__(128 * NCG, 1)
+tc_scan_fwd_kernel(SeqView s, ChainOps op) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    constexpr int NB = chain_ctas_per_head<DV, NCG>();
+    chain_cta<DV, BETA, false, NCG>(s, blockIdx.x / NB, blockIdx.x % NB, op, smem);
 }
 
-template <int DV, bool BETA>
-__global__ void __launch_bounds__(256, 1)
-tc_scan_fwd_kernel(SeqView s, const float* __restrict__ Gm, const bf16* __restrict__ Wn,
-                   const bf16* __restrict__ Kh, const bf16* __restrict__ Ut,
-                   const float* __restrict__ S_in, bf16* __restrict__ Vnt, bf16* __restrict__ S0t,
-                   float* __restrict__ S_out) {
+// Backward chains in one launch: with nsr > 0, blocks [0, nsr) recompute the
+// forward states (V_new^T and the chunk-entry states, op_f) and the rest run
+// the reverse state-gradient scan (op_b); the two groups share no data.
+template <int DV, bool BETA, int NCG>
+__global__ void __launch_bounds__(128 * NCG, 1)
+tc_scan_bwd_dual_kernel(SeqView s, ChainOps op_f, ChainOps op_b, int nsr) {
     extern __shared__ __align__(16) unsigned char smem[];
-    constexpr int NVB = DV / 64;
-    scan_fwd_cta<DV, BETA>(s, blockIdx.x / NVB, blockIdx.x % NVB, Gm, Wn, Kh, Ut, S_in, Vnt, S0t, S_out, smem);
-}
-
-// Backward chains in one launch: with with_sr, blocks [0, BH*DV/64) recompute
-// the forward states (V_new and the chunk-entry states) and the rest run the
-// reverse state-gradient scan; the two groups share no data.  Without it (the
-// forward's states are kept), every block runs the reverse scan.
-template <int DV, bool BETA>
-__global__ void __launch_bounds__(256, 1)
-tc_scan_bwd_dual_kernel(SeqView s, const bf16* __restrict__ Dt,
-                        const float* __restrict__ Gm, const bf16* __restrict__ Wn,
-                        const bf16* __restrict__ Kh, const bf16* __restrict__ Ut,
-                        const bf16* __restrict__ dVit, const float* __restrict__ S_in,
-                        const float* __restrict__ dS_out, bf16* __restrict__ Vnt, bf16* __restrict__ S0t,
-                        bf16* __restrict__ dVnt, bf16* __restrict__ dSCt, float* __restrict__ dS_in,
-                        int with_sr) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    constexpr int NVB = DV / 64;
-    const int nsr = with_sr ? s.BH * NVB : 0;
+    constexpr int NB = chain_ctas_per_head<DV, NCG>();
     int id = blockIdx.x;
     if (id < nsr) {
-        scan_fwd_cta<DV, BETA>(s, id / NVB, id % NVB, Gm, Wn, Kh, Ut, S_in, Vnt, S0t, nullptr, smem);
+        chain_cta<DV, BETA, false, NCG>(s, id / NB, id % NB, op_f, smem);
     } else {
         id -= nsr;
-        scan_bwd_cta<DV, BETA>(s, id / NVB, id % NVB, Dt, Gm, Wn, Kh, dVit, dS_out, dVnt, dSCt, dS_in, smem);
+        chain_cta<DV, BETA, true, NCG>(s, id / NB, id % NB, op_b, smem);
     }
 }
 
@@ -1820,13 +1590,45 @@ cudaError_t launch_prep(const char* name, const SeqView& s, const bf16* k, const
     return cudaGetLastError();
 }
 
+// Slices of 16 state columns per chain CTA: 1 (B*H*d_v/16 CTAs of 4 warps),
+// 2 (half as many CTAs of 8 warps, the default) or 4.  Measured at B=1, H=16,
+// T=65536, d=128 on B200, each launch alone: the forward chain takes 0.80,
+// 0.96 and 1.60 ms for 1, 2 and 4 slices; the backward launch (forward
+// recompute beside the reverse chain, twice the CTAs) 1.67, 1.02 and 1.68 ms.
+// SF_GDN_CHAIN_SLICES overrides the default (read once).
+int chain_slices() {
+    static int n = 0;
+    if (n == 0) {
+        const char* e = std::getenv("SF_GDN_CHAIN_SLICES");
+        n = e ? std::atoi(e) : 2;
+        if (n != 1 && n != 4) n = 2;
+    }
+    return n;
+}
+
+ChainOps fwd_ops(const TcWs& w, const float* S_in, float* S_out) {
+    return ChainOps{w.W, w.Kh, w.Ut, nullptr, w.Gm, S_in, w.S0t, w.Vnt, S_out};
+}
+ChainOps bwd_ops(const TcWs& w, const float* dS_out, float* dS_in) {
+    return ChainOps{w.Kh, w.W, w.dVit, w.Dt, w.Gm, dS_out, w.dSCt, w.dVnt, dS_in};
+}
+
+template <int DV, bool BETA, int NCG>
+cudaError_t launch_scan_fwd_n(const SeqView& s, const float* S_in, float* S_out, const TcWs& w, cudaStream_t st) {
+    constexpr size_t sm = Chain<DV, BETA, false, NCG>::SMEM;
+    TC_TRY(smem_attr(tc_scan_fwd_kernel<DV, BETA, NCG>, sm));
+    SF_LAUNCH("tc_scan_fwd", st,
+              tc_scan_fwd_kernel<DV, BETA, NCG><<<s.BH * chain_ctas_per_head<DV, NCG>(), 128 * NCG, sm, st>>>(
+                  s, fwd_ops(w, S_in, S_out)));
+    return cudaGetLastError();
+}
 template <int DV, bool BETA>
 cudaError_t launch_scan_fwd(const SeqView& s, const float* S_in, float* S_out, const TcWs& w, cudaStream_t st) {
-    constexpr size_t sm = fwd_scan_smem<BETA>();
-    TC_TRY(smem_attr(tc_scan_fwd_kernel<DV, BETA>, sm));
-    SF_LAUNCH("tc_scan_fwd", st, tc_scan_fwd_kernel<DV, BETA><<<s.BH * (DV / 64), 256, sm, st>>>(
-                                     s, w.Gm, w.W, w.Kh, w.Ut, S_in, w.Vnt, w.S0t, S_out));
-    return cudaGetLastError();
+    switch (chain_slices()) {
+        case 4: return DV % 64 == 0 ? launch_scan_fwd_n<DV, BETA, 4>(s, S_in, S_out, w, st) : cudaErrorInvalidValue;
+        case 2: return launch_scan_fwd_n<DV, BETA, 2>(s, S_in, S_out, w, st);
+        default: return launch_scan_fwd_n<DV, BETA, 1>(s, S_in, S_out, w, st);
+    }
 }
 
 template <int DV>
@@ -1857,16 +1659,25 @@ cudaError_t launch_intra(const SeqView& s, const bf16* q, const bf16* k, const b
     return cudaGetLastError();
 }
 
+template <int DV, bool BETA, int NCG>
+cudaError_t launch_scan_bwd_n(const SeqView& s, const BwdArgs& a, bool with_sr, const TcWs& w, cudaStream_t st) {
+    constexpr size_t sm_f = Chain<DV, BETA, false, NCG>::SMEM, sm_b = Chain<DV, BETA, true, NCG>::SMEM;
+    constexpr size_t sm = sm_f > sm_b ? sm_f : sm_b;
+    TC_TRY(smem_attr(tc_scan_bwd_dual_kernel<DV, BETA, NCG>, sm));
+    const int per = s.BH * chain_ctas_per_head<DV, NCG>();
+    const int nsr = with_sr ? per : 0;
+    SF_LAUNCH("tc_scan_bwd", st,
+              tc_scan_bwd_dual_kernel<DV, BETA, NCG><<<nsr + per, 128 * NCG, sm, st>>>(
+                  s, fwd_ops(w, a.S_in, nullptr), bwd_ops(w, a.dS_out, a.dS_in), nsr));
+    return cudaGetLastError();
+}
 template <int DV, bool BETA>
 cudaError_t launch_scan_bwd(const SeqView& s, const BwdArgs& a, bool with_sr, const TcWs& w, cudaStream_t st) {
-    constexpr size_t sm_f = fwd_scan_smem<BETA>(), sm_b = bwd_scan_smem<BETA>();
-    constexpr size_t sm = sm_f > sm_b ? sm_f : sm_b;
-    TC_TRY(smem_attr(tc_scan_bwd_dual_kernel<DV, BETA>, sm));
-    const int nb = (with_sr ? 2 : 1) * s.BH * (DV / 64);
-    SF_LAUNCH("tc_scan_bwd", st, tc_scan_bwd_dual_kernel<DV, BETA><<<nb, 256, sm, st>>>(
-                                     s, w.Dt, w.Gm, w.W, w.Kh, w.Ut, w.dVit, a.S_in, a.dS_out, w.Vnt, w.S0t, w.dVnt, w.dSCt,
-                                     a.dS_in, with_sr ? 1 : 0));
-    return cudaGetLastError();
+    switch (chain_slices()) {
+        case 4: return launch_scan_bwd_n<DV, BETA, 4>(s, a, with_sr, w, st);
+        case 2: return launch_scan_bwd_n<DV, BETA, 2>(s, a, with_sr, w, st);
+        default: return launch_scan_bwd_n<DV, BETA, 1>(s, a, with_sr, w, st);
+    }
 }
 
 int num_sms() {
