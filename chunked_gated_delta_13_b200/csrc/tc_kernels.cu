@@ -26,9 +26,11 @@
 // (forward) or two (backward) chunks deep.
 #include <algorithm>
 #include <cstdlib>
+#include <string>
 
 #include "tc_kernels.cuh"
 #include "tc_mma.cuh"
+#include "tc_umma.cuh"
 
 namespace sf {
 namespace {
@@ -53,11 +55,11 @@ struct TcWs {
     float* Lm;   // [BH][NC][C][C]     L = (I + A)^{-1} per chunk (delta path), for the gradient kernel
     bf16* Kh;    // [BH][Tp][DK]       K * exp(G_C - G) (permuted)
     bf16* Ut;    // [BH][NC][DV][C]    U transposed per chunk, V^T without the beta path (permuted)
-    bf16* Vnt;   // [BH][NC][DV][C]    V_new transposed per chunk (pieces permuted, see swz)
-    bf16* S0t;   // [BH][NC][DV][DK]   state entering each chunk, transposed (permuted)
+    bf16* Vnt;   // [BH][NC][DV][C]    V_new transposed per chunk (canon, see tc_umma.cuh)
+    bf16* S0t;   // [BH][NC][DV][DK]   state entering each chunk, transposed (canon)
     bf16* dVit;  // [BH][NC][DV][C]    intra-chunk part of dV_new, transposed (permuted)
-    bf16* dVnt;  // [BH][NC][DV][C]    dV_new transposed (permuted)
-    bf16* dSCt;  // [BH][NC][DV][DK]   gradient of the state leaving each chunk, transposed (permuted)
+    bf16* dVnt;  // [BH][NC][DV][C]    dV_new transposed (canon)
+    bf16* dSCt;  // [BH][NC][DV][DK]   gradient of the state leaving each chunk, transposed (canon)
     bf16* Dt;    // [BH][NC][DV][DK]   scale (gamma * dO)^T Q per chunk, transposed (permuted)
     int* ticket;  // chunk counter of the persistent gradient kernel
     size_t total;
@@ -495,6 +497,13 @@ tc_intra_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     og_products<DV>(s, Qs, dOs, Ps, Gs, dVito + ci * DV * C, Dto + ci * DV * DK, w, lane);
 }
 
+// Copy BYTES contiguous bytes global -> shared, 16 bytes per cp.async request.
+template <int BYTES, int NT>
+__device__ __forceinline__ void copy_linear(void* s, const void* g, int tid) {
+    for (int e = tid; e < BYTES / 16; e += NT)
+        cp_async16(static_cast<char*>(s) + 16 * e, static_cast<const char*>(g) + 16 * e, true);
+}
+
 // ------------------------------------------------------------ state scans ---
 // The forward state scan (ST) and the reverse state-gradient scan (STB) run
 // the same step on different operands.  With X, Y the two [C][DK] operand
@@ -561,14 +570,6 @@ __device__ __forceinline__ int sw_off(const SwLane& L, int rowbase, int pe, int 
     return (rowbase + L.row) * rowlen + ((pe * 8) ^ L.hi8) + L.lo;
 }
 
-// Write a bf16 A-fragment block (16 rows x 16 cols at [r0, c0]) into a permuted
-// staging tile of row length `cols` with one stmatrix.
-__device__ __forceinline__ void stage_afrag(bf16* t, int cols, int r0, int c0, const uint32_t (&a)[4], int lane) {
-    const int lr = (lane & 7) + (((lane >> 3) & 1) << 3), pb = lane >> 4;
-    const int piece = ((c0 >> 3) + pb) ^ (lr & 7);
-    stsm_x4(t + (r0 + lr) * cols + piece * 8, a);
-}
-
 __device__ __forceinline__ void put_frag(uint4* p, const uint32_t (&a)[4]) { *p = make_uint4(a[0], a[1], a[2], a[3]); }
 __device__ __forceinline__ void get_frag(const uint4* p, uint32_t (&a)[4]) {
     const uint4 v = *p;
@@ -588,8 +589,8 @@ struct ChainOps {
     const bf16* E;      // [BH][NC][DV][DK] permuted: D^T (backward only)
     const float* Gm;    // [BH][Tp] exp(G)
     const float* R_in;  // [BH][DK][DV] S_in or dS_out (NULL = zeros)
-    bf16* Rt;           // [BH][NC][DV][DK] permuted: S0^T or dS_C^T per chunk (NULL = skip)
-    bf16* Zt;           // [BH][NC][DV][C] permuted: V_new^T or dV_new^T per chunk (NULL = skip)
+    bf16* Rt;           // [BH][NC][DV][DK] canon: S0^T or dS_C^T per chunk (NULL = skip)
+    bf16* Zt;           // [BH][NC][DV][C] canon: V_new^T or dV_new^T per chunk (NULL = skip)
     float* R_out;       // [BH][DK][DV] S_out or dS_in (NULL = skip)
 };
 
@@ -675,7 +676,7 @@ __device__ __forceinline__ void chain_cta(const SeqView& s, int bh, int vb, cons
         for (int jj = 0; jj < 2; ++jj) {
             c2a(sa[jj], r[2 * jj], r[2 * jj + 1]);
             if (CH::HAS_X) put_frag(xch + (2 * q + jj) * 32, sa[jj]);
-            if (op.Rt) stage_afrag(Rs, DK, vr, 16 * (2 * q + jj), sa[jj], lane);
+            if (op.Rt) umma::st_afrag_c(Rs, DK, vr, 16 * (2 * q + jj), sa[jj], lane);
         }
         if (CH::HAS_X) slice_sync(g);
         mbar_wait(&bars[i % NS], (i / NS) & 1, &g_tc_status, failed);
@@ -725,7 +726,7 @@ __device__ __forceinline__ void chain_cta(const SeqView& s, int bh, int vb, cons
         uint32_t za[4];
         c2a(za, z[0], z[1]);
         if (CH::HAS_Y) put_frag(xch + (8 + q) * 32, za);
-        if (op.Zt) stage_afrag(Zs, C, vr, 16 * q, za, lane);
+        if (op.Zt) umma::st_afrag_c(Zs, C, vr, 16 * q, za, lane);
 
         // product 2: R <- gamma_C R (+ E) + Z^T Y
         if (BWD) {
@@ -835,8 +836,8 @@ tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
     extern __shared__ __align__(16) unsigned char smem[];
     bf16* Qs = reinterpret_cast<bf16*>(smem);
     bf16* Ks = Qs + C * LDK;     // later (OG): P [C][LDC]
-    bf16* S0s = Ks + C * LDK;   // [DV][LDK]
-    bf16* Vns = S0s + DV * LDK;  // [DV][LDC]
+    bf16* S0s = Ks + C * LDK;   // [DV][DK] canon (sized [DV][LDK])
+    bf16* Vns = S0s + DV * LDK;  // [DV][C] canon (sized [DV][LDC])
     float* Gs = reinterpret_cast<float*>(Vns + DV * LDC);
     bf16* dOs = reinterpret_cast<bf16*>(Gs + C);  // [C][LDV] (OG)
     const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -846,8 +847,8 @@ tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
     const size_t Tp = (size_t)s.NC * C;
     load_tile<C, DK, 128>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
     load_tile<C, DK, 128>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
-    load_tile_swz<DV, DK, 128>(S0s, LDK, S0t + ((size_t)bh * s.NC + c) * DV * DK, tid);
-    load_tile_swz<DV, C, 128>(Vns, LDC, Vnt + ((size_t)bh * s.NC + c) * DV * C, tid);
+    copy_linear<DV * DK * 2, 128>(S0s, S0t + ((size_t)bh * s.NC + c) * DV * DK, tid);  // canon tiles
+    copy_linear<DV * C * 2, 128>(Vns, Vnt + ((size_t)bh * s.NC + c) * DV * C, tid);
     if (tid < 16) cp_async16(Gs + tid * 4, Gc + bh * Tp + t0 + tid * 4, true);
     cp_async_commit();
     if (OG) {
@@ -875,7 +876,7 @@ tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
         for (int nn = 0; nn < DV / 8; nn += 2) {
             uint32_t b[4];
-            ldBnk(b, S0s, LDK, 8 * nn, 16 * kk, lane);
+            umma::ldBnk_c(b, S0s, DK, 8 * nn, 16 * kk, lane);
             mma(acc[nn], a, b[0], b[1]);
             mma(acc[nn + 1], a, b[2], b[3]);
         }
@@ -914,7 +915,7 @@ tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
         for (int nn = 0; nn < DV / 8; nn += 2) {
             uint32_t b[4];
-            ldBnk(b, Vns, LDC, 8 * nn, 16 * kk, lane);
+            umma::ldBnk_c(b, Vns, C, 8 * nn, 16 * kk, lane);
             mma(acc[nn], a, b[0], b[1]);
             mma(acc[nn + 1], a, b[2], b[3]);
         }
@@ -982,11 +983,11 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     bf16* Ks = Qs + C * LDK;
     bf16* Vs = Ks + C * LDK;     // [C][LDV]
     bf16* dOs = Vs + C * LDV;    // [C][LDV]
-    bf16* Vns = dOs + C * LDV;   // [DV][LDC]  V_new^T
-    bf16* dVns = Vns + DV * LDC;  // [DV][LDC] dV_new^T
+    bf16* Vns = dOs + C * LDV;   // [DV][C] canon V_new^T (sized [DV][LDC])
+    bf16* dVns = Vns + DV * LDC;  // [DV][C] canon dV_new^T
     unsigned char* R = reinterpret_cast<unsigned char*>(dVns + DV * LDC);
-    bf16* S0s = reinterpret_cast<bf16*>(R);       // [DV][LDK]  (phase S)
-    bf16* dSs = S0s + DV * LDK;                   // [DV][LDK]  (phase S)
+    bf16* S0s = reinterpret_cast<bf16*>(R);       // [DV][DK] canon (phase S)
+    bf16* dSs = S0s + DV * LDK;                   // [DV][DK] canon (phase S)
     bf16* dWs = reinterpret_cast<bf16*>(R);       // [C][LDK]   (after phase S)
     float* XZ = reinterpret_cast<float*>(R + C * LDK * 2);  // X, Z (bf16 [C][LDC] each)
     float* Lf = XZ + C * LDF;                     // [C][LDF] L (fp32)
@@ -1031,22 +1032,22 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         const int t0 = c * C, nval = min(C, s.T - t0);
         const size_t ci = (size_t)bh * s.NC + c;
         load_tile<C, DV, GTH>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
-        load_tile_swz<DV, C, GTH>(Vns, LDC, Vnt + ci * DV * C, tid);
+        copy_linear<DV * C * 2, GTH>(Vns, Vnt + ci * DV * C, tid);
     };
     auto copy_b1 = [&](int j) {  // V, dV_new
         int c, bh;
         where(j, c, bh);
         const int t0 = c * C, nval = min(C, s.T - t0);
         const size_t ci = (size_t)bh * s.NC + c;
-        load_tile_swz<DV, C, GTH>(dVns, LDC, dVnt + ci * DV * C, tid);
+        copy_linear<DV * C * 2, GTH>(dVns, dVnt + ci * DV * C, tid);
         load_tile<C, DV, GTH>(Vs, LDV, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
     };
     auto copy_b2 = [&](int j) {  // S0, dS_C
         int c, bh;
         where(j, c, bh);
         const size_t ci = (size_t)bh * s.NC + c;
-        load_tile_swz<DV, DK, GTH>(S0s, LDK, S0t + ci * DV * DK, tid);
-        load_tile_swz<DV, DK, GTH>(dSs, LDK, dSCt + ci * DV * DK, tid);
+        copy_linear<DV * DK * 2, GTH>(S0s, S0t + ci * DV * DK, tid);
+        copy_linear<DV * DK * 2, GTH>(dSs, dSCt + ci * DV * DK, tid);
     };
     auto beta_of = [&](int j) {
         int c, bh;
@@ -1113,7 +1114,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 #pragma unroll
             for (int nn = 0; nn < CW / 8; nn += 2) {
                 uint32_t b[4];
-                ldBkn(b, Vns, LDC, CW * nw + 8 * nn, 16 * kv, lane);
+                umma::ldBkn_c(b, Vns, C, CW * nw + 8 * nn, 16 * kv, lane);
                 mma(dp[nn], aO, b[0], b[1]);
                 mma(dp[nn + 1], aO, b[2], b[3]);
             }
@@ -1164,26 +1165,24 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         for (int kv = 0; kv < DV / 16; ++kv) {
             uint32_t aO[4], aN[4], aV[4];
             ldA(aO, dOs, LDV, 16 * mw, 16 * kv, lane);
-            ldAt(aN, dVns, LDC, 16 * mw, 16 * kv, lane);
-            ldAt(aV, Vns, LDC, 16 * mw, 16 * kv, lane);
+            umma::ldAt_c(aN, dVns, C, 16 * mw, 16 * kv, lane);
+            umma::ldAt_c(aV, Vns, C, 16 * mw, 16 * kv, lane);
 #pragma unroll
             for (int nn = 0; nn < DKW / 8; nn += 2) {
                 uint32_t b[4];
-                ldBkn(b, S0s, LDK, DKW * nw + 8 * nn, 16 * kv, lane);
+                umma::ldBkn_c(b, S0s, DK, DKW * nw + 8 * nn, 16 * kv, lane);
                 mma(accQ[nn], aO, b[0], b[1]);
                 mma(accQ[nn + 1], aO, b[2], b[3]);
                 mma(accW[nn], aN, b[0], b[1]);
                 mma(accW[nn + 1], aN, b[2], b[3]);
-                ldBkn(b, dSs, LDK, DKW * nw + 8 * nn, 16 * kv, lane);
+                umma::ldBkn_c(b, dSs, DK, DKW * nw + 8 * nn, 16 * kv, lane);
                 mma(accK[nn], aV, b[0], b[1]);
                 mma(accK[nn + 1], aV, b[2], b[3]);
             }
         }
         float pd = 0.f;  // <S0, dS_C>
-        for (int e = tid; e < DV * DK; e += GTH) {
-            const int r = e / DK, cc = e % DK;
-            pd += __bfloat162float(S0s[r * LDK + cc]) * __bfloat162float(dSs[r * LDK + cc]);
-        }
+        for (int e = tid; e < DV * DK; e += GTH)  // both canon tiles: same element at the same offset
+            pd += __bfloat162float(S0s[e]) * __bfloat162float(dSs[e]);
         red[tid] = pd;
         // dq_inter = scale gamma (dO S0^T); dK_state = dec (V_new dS_C^T)
         const float sq0 = s.scale * gam0, sq1 = s.scale * gam1;
@@ -1312,7 +1311,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 #pragma unroll
                 for (int nn = 0; nn < NT; nn += 2) {
                     uint32_t b[4];
-                    ldBnk(b, dVns, LDC, (DV / GW) * nw + 8 * nn, 16 * kr, lane);
+                    umma::ldBnk_c(b, dVns, C, (DV / GW) * nw + 8 * nn, 16 * kr, lane);
                     mma(acc[nn], a, b[0], b[1]);
                     mma(acc[nn + 1], a, b[2], b[3]);
                 }
@@ -1326,7 +1325,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         } else {
             for (int e = tid; e < nval * DV; e += GTH) {
                 const int j = e / DV, col = e % DV;
-                dvb[(size_t)j * DV + col] = dVns[col * LDC + j];
+                dvb[(size_t)j * DV + col] = *umma::canon_at<bf16>(dVns, col, j, C);
             }
         }
     }
@@ -1353,7 +1352,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 #pragma unroll
         for (int kv = 0; kv < DV / 16; ++kv) {
             uint32_t a[4];
-            ldAt(a, dVns, LDC, 16 * mw, 16 * kv, lane);
+            umma::ldAt_c(a, dVns, C, 16 * mw, 16 * kv, lane);
 #pragma unroll
             for (int nn = 0; nn < CW / 8; nn += 2) {
                 uint32_t b[4];
@@ -1568,6 +1567,715 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
   }
 }
 
+// ------------------------------------------------- grad on tcgen05 (PG) ---
+// Every input gradient of a chunk with the products on the fifth-generation
+// tensor cores: one thread issues each product as a chain of K = 16
+// tcgen05.mma (M = 64 token rows, fp32 accumulators in TMEM, operands read
+// from canon tiles in shared memory), and the 16 warps run the elementwise
+// epilogues between them on the accumulators they load from TMEM (warp w
+// owns rows 16 (w % 4).. and the column group w / 4).  With
+//   P = scale (Q K^T) * Gamma,  M = scale (dO V_new^T) * Gamma,  T = L diag(beta),
+//   dW = -dV_new S0^T,  dT = dW (gamma K)^T + dV_new V^T,  dL = dT diag(beta),
+//   dA = -strictly-lower(L^T dL L^T),  Z = diag(beta) (dA * Gamma):
+//   dq = scale gamma (dO S0^T) + M K
+//   dk = dec (V_new dS_C^T) + gamma (T^T dW) + M^T Q + Z K + Z^T K
+//   dv = T^T dV_new   (dv = dV_new without the beta path)
+// and dG (hence dg, dbeta) from the row and column sums of the elementwise
+// terms, reduced in a fixed order (bit-reproducible).
+//
+// Persistent: a CTA takes chunk tickets from a per-launch counter and copies
+// the next chunk's tiles in while it works on the current one: Q, K, G into
+// the second of two buffers at once; dO and V_new^T once the products reading
+// them are done, then dV_new^T and V, then L; the state tiles last, into the
+// region the epilogue tiles of the current chunk leave.
+//
+// TMEM columns (512 allocated; M = 64 uses lanes 0-15 of each quarter):
+//   [0,64) Q K^T -> [0,128) dk       [64,128) K K^T        [128,192) dP -> dT_b -> dA
+//   [192,320) dq                     [320,448) dV_new S0^T -> gamma T^T dW -> dv
+//   [448,512) dW K^T -> X
+template <int DV>
+struct G5 {
+    // TMEM columns of the accumulators
+    static constexpr uint32_t QK = 0, KK = 64, DP = 128, DQ = 192, DW = 320, DTA = 448;
+    static constexpr uint32_t DKC = 0, T3 = 320, DTB = 128, DVC = 320, XC = 448, DA = 128;
+    static constexpr int SLD = 128 + 8;  // row stride of the dq / dk staging tiles (elements)
+    static constexpr size_t kQK = (size_t)2 * C * 128 * 2;  // one buffer: Q then K
+    static constexpr size_t kV = (size_t)C * DV * 2;        // V, dO, V_new^T, dV_new^T each
+    static constexpr size_t kStateB = (size_t)DV * 128 * 2 * 2;
+    static constexpr size_t kEpiB = (size_t)C * 128 * 2 + 6 * (size_t)C * C * 2;
+    static constexpr size_t kOutB = (size_t)2 * C * SLD * 2;
+    static constexpr size_t kB0 = kStateB > kEpiB ? kStateB : kEpiB;
+    static constexpr size_t kB = kB0 > kOutB ? kB0 : kOutB;
+    static constexpr size_t SMEM = 2 * kQK + 4 * kV + kB + (size_t)C * C * 4 + (size_t)C * C * 2 +
+                                   (size_t)P_ROWS * C * 4 + 16 * 4 + 4 * C * 4 + 16 * 8 + 16;
+};
+
+template <int DV, bool BETA>
+__global__ void __launch_bounds__(512, 1)
+tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
+                const float* __restrict__ beta, const bf16* __restrict__ dO, const float* __restrict__ Gc,
+                const float* __restrict__ Lm, const bf16* __restrict__ Vnt, const bf16* __restrict__ dVnt,
+                const bf16* __restrict__ S0t, const bf16* __restrict__ dSCt, bf16* __restrict__ dq,
+                bf16* __restrict__ dk, bf16* __restrict__ dv, float* __restrict__ dg, float* __restrict__ dbeta,
+                int* __restrict__ ticket) {
+    using L5 = G5<DV>;
+    extern __shared__ __align__(16) unsigned char smem[];
+    unsigned char* p = smem;
+    unsigned char* QKb = p;                   p += 2 * L5::kQK;  // [2] x (Q [C][DK], K [C][DK])
+    bf16* Vc = reinterpret_cast<bf16*>(p);   p += L5::kV;        // [C][DV]
+    bf16* dOc = reinterpret_cast<bf16*>(p);  p += L5::kV;        // [C][DV]
+    bf16* Vnc = reinterpret_cast<bf16*>(p);  p += L5::kV;        // [DV][C]  V_new^T
+    bf16* dVnc = reinterpret_cast<bf16*>(p); p += L5::kV;        // [DV][C]  dV_new^T
+    unsigned char* RB = p;                   p += L5::kB;
+    bf16* S0c = reinterpret_cast<bf16*>(RB);           // [DV][DK]
+    bf16* dSc = S0c + DV * 128;                        // [DV][DK]
+    bf16* dWs = reinterpret_cast<bf16*>(RB);           // [C][DK]   (after the state products)
+    bf16* Tpp = dWs + C * 128;                         // [C][C]    L diag(beta gamma)
+    bf16* Ts = Tpp + C * C;                            // [C][C]    L diag(beta)
+    bf16* Ls = Ts + C * C;                             // [C][C]    L
+    bf16* dLs = Ls + C * C;                            // [C][C]
+    bf16* Xs = dLs + C * C;                            // [C][C]
+    bf16* Zs = Xs + C * C;                             // [C][C]
+    bf16* Sq = reinterpret_cast<bf16*>(RB);            // [C][SLD] dq staging (row-major, at the end)
+    bf16* Sk = Sq + C * L5::SLD;                       // [C][SLD] dk staging
+    float* Lf = reinterpret_cast<float*>(p);  p += C * C * 4;   // [C][C] fp32, row-major
+    bf16* Ms = reinterpret_cast<bf16*>(p);    p += C * C * 2;   // [C][C]
+    float* part = reinterpret_cast<float*>(p); p += P_ROWS * C * 4;
+    float* red = reinterpret_cast<float*>(p);  p += 16 * 4;
+    float* Gsb = reinterpret_cast<float*>(p);  p += 2 * C * 4;  // [2][C]
+    float* Bsb = reinterpret_cast<float*>(p);  p += 2 * C * 4;  // [2][C]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(p);  p += 16 * 8;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(p);
+    int* tk = reinterpret_cast<int*>(p + 4);  // [2] chunk tickets
+    // mbarriers: copies (one phase per chunk) and product completions (one per chunk)
+    uint64_t* bVn = &bars[0];
+    uint64_t* bS = &bars[1];
+    uint64_t* bdVn = &bars[2];
+    uint64_t* bL = &bars[3];
+    uint64_t* bm = &bars[4];  // [7]
+
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int gq = lane >> 2, tq = lane & 3;
+    const int mw = w & 3, nw = w >> 2;
+    const size_t Tp = (size_t)s.NC * C;
+    const int total = s.NC * s.BH;
+    const int r0 = 16 * mw + gq, r1 = r0 + 8;  // the two rows this thread holds
+    bool failed = false;
+
+    auto where = [&](int j, int& c, int& bh) {
+        bh = j / s.NC;
+        c = j - bh * s.NC;
+    };
+    auto Qc_of = [&](int b) { return reinterpret_cast<bf16*>(QKb + b * L5::kQK); };
+    auto Kc_of = [&](int b) { return reinterpret_cast<bf16*>(QKb + b * L5::kQK) + C * 128; };
+    // copy groups (cp.async: per-thread FIFO groups; bulk: mbarriers, thread 0)
+    auto copy_qkg = [&](int j, int b) {  // Q, K, G of chunk j into buffer b
+        int c, bh;
+        where(j, c, bh);
+        const int t0 = c * C, nval = min(C, s.T - t0);
+        umma::load_canon<C, 128, 512>(Qc_of(b), q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+        umma::load_canon<C, 128, 512>(Kc_of(b), k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+        if (tid < C / 4) cp_async16(Gsb + b * C + 4 * tid, Gc + bh * Tp + t0 + 4 * tid, true);
+    };
+    auto copy_do = [&](int j) {
+        int c, bh;
+        where(j, c, bh);
+        const int t0 = c * C, nval = min(C, s.T - t0);
+        umma::load_canon<C, DV, 512>(dOc, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+    };
+    auto copy_v = [&](int j) {
+        int c, bh;
+        where(j, c, bh);
+        const int t0 = c * C, nval = min(C, s.T - t0);
+        umma::load_canon<C, DV, 512>(Vc, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+    };
+    auto bulk_vn = [&](int j) {  // thread 0
+        int c, bh;
+        where(j, c, bh);
+        mbar_expect_tx(bVn, DV * C * 2);
+        bulk_load(Vnc, Vnt + ((size_t)bh * s.NC + c) * DV * C, DV * C * 2, bVn);
+    };
+    auto bulk_state = [&](int j) {  // thread 0
+        int c, bh;
+        where(j, c, bh);
+        const size_t ci = (size_t)bh * s.NC + c;
+        mbar_expect_tx(bS, 2 * DV * 128 * 2);
+        bulk_load(S0c, S0t + ci * DV * DK, DV * 128 * 2, bS);
+        bulk_load(dSc, dSCt + ci * DV * DK, DV * 128 * 2, bS);
+    };
+    auto bulk_dvn = [&](int j) {  // thread 0
+        int c, bh;
+        where(j, c, bh);
+        mbar_expect_tx(bdVn, DV * C * 2);
+        bulk_load(dVnc, dVnt + ((size_t)bh * s.NC + c) * DV * C, DV * C * 2, bdVn);
+    };
+    auto bulk_l = [&](int j) {  // thread 0
+        int c, bh;
+        where(j, c, bh);
+        mbar_expect_tx(bL, C * C * 4);
+        bulk_load(Lf, Lm + ((size_t)bh * s.NC + c) * C * C, C * C * 4, bL);
+    };
+    auto beta_of = [&](int j) {
+        int c, bh;
+        where(j, c, bh);
+        const int t0 = c * C, nval = min(C, s.T - t0);
+        return (BETA && tid < nval) ? beta[bh * s.hs_g + t0 + tid] : 0.f;
+    };
+
+    if (tid == 0) {
+        for (int i = 0; i < 11; ++i) mbar_init(&bars[i], 1);
+        mbar_init_fence();
+        tk[0] = atomicAdd(ticket, 1);
+    }
+    __syncthreads();
+    int j = tk[0];
+    if (j >= total) return;
+    if (w == 0) umma::alloc(tslot, 512);
+    // first chunk: groups [Q K G dO] and [V]; bulk copies of its other tiles
+    copy_qkg(j, 0);
+    copy_do(j);
+    cp_async_commit();
+    copy_v(j);
+    cp_async_commit();
+    if (tid == 0) {
+        bulk_vn(j);
+        bulk_state(j);
+        bulk_dvn(j);
+        if (BETA) bulk_l(j);
+    }
+    if (tid < C) Bsb[tid] = beta_of(j);
+    for (int e = tid; e < P_ROWS * C; e += 512) part[e] = 0.f;
+    __syncthreads();  // TMEM allocated
+    umma::fence_after();
+    const uint32_t tm = *tslot;
+    const uint32_t trow = umma::taddr(tm, 32 * mw, 0);  // this warp's lane quarter
+    auto chain = [&](uint32_t col, uint32_t idesc, int nks, bool acc, auto da, auto db) {
+#pragma unroll 1
+        for (int ks = 0; ks < nks; ++ks) umma::mma(tm + col, da(ks), db(ks), idesc, acc || ks > 0);
+    };
+    constexpr uint32_t I64kk = umma::idesc_bf16(64, 64, false, false);
+    constexpr uint32_t I64km = umma::idesc_bf16(64, 64, false, true);
+    constexpr uint32_t I64mk = umma::idesc_bf16(64, 64, true, false);
+    constexpr uint32_t I64mm = umma::idesc_bf16(64, 64, true, true);
+    constexpr uint32_t I128km = umma::idesc_bf16(64, 128, false, true);
+    constexpr uint32_t I128mm = umma::idesc_bf16(64, 128, true, true);
+    constexpr uint32_t IDVmk = umma::idesc_bf16(64, DV, true, false);
+    auto sync_for_mma = [&]() {  // generic shared writes and TMEM accesses -> the next products
+        fence_proxy_async_smem();
+        umma::fence_before();
+        __syncthreads();
+    };
+
+  for (int it = 0;; ++it) {
+    const int buf = it & 1;
+    const uint32_t par = (uint32_t)(it & 1);
+    auto wait_bar = [&](uint64_t* b) {
+        mbar_wait(b, par, &g_tc_status, failed);
+        umma::fence_after();
+    };
+    int c, bh;
+    where(j, c, bh);
+    const int t0 = c * C;
+    const int nval = min(C, s.T - t0);
+    bf16* Qc = Qc_of(buf);
+    bf16* Kc = Kc_of(buf);
+    float* Gs = Gsb + buf * C;
+    float* Bs = Bsb + buf * C;
+    if (tid == 0) tk[(it + 1) & 1] = atomicAdd(ticket, 1);
+    cp_async_wait<1>();  // Q, K, G, dO of this chunk (its V may still be landing)
+    mbar_wait(bVn, par, &g_tc_status, failed);
+    sync_for_mma();
+    const int jn = tk[(it + 1) & 1];
+    const bool has_next = jn < total;
+    if (tid == 0) {  // Q K^T, K K^T, dP = dO V_new^T
+        umma::fence_after();
+        chain(L5::QK, I64kk, 8, false, [&](int ks) { return umma::desc_k(Qc, ks, 128); },
+              [&](int ks) { return umma::desc_k(Kc, ks, 128); });
+        if (BETA)
+            chain(L5::KK, I64kk, 8, false, [&](int ks) { return umma::desc_k(Kc, ks, 128); },
+                  [&](int ks) { return umma::desc_k(Kc, ks, 128); });
+        chain(L5::DP, I64km, DV / 16, false, [&](int ks) { return umma::desc_k(dOc, ks, DV); },
+              [&](int ks) { return umma::desc_mn(Vnc, ks, C); });
+        umma::commit(&bm[0]);
+    }
+    if (has_next) copy_qkg(jn, buf ^ 1);  // the other buffer's chunk is done
+    cp_async_commit();
+    const float beta_next = has_next ? beta_of(jn) : 0.f;
+    mbar_wait(bS, par, &g_tc_status, failed);
+    mbar_wait(bdVn, par, &g_tc_status, failed);
+    if (tid == 0) {  // dO S0^T, dV_new S0^T
+        umma::fence_after();
+        chain(L5::DQ, I128km, DV / 16, false, [&](int ks) { return umma::desc_k(dOc, ks, DV); },
+              [&](int ks) { return umma::desc_mn(S0c, ks, 128); });
+        if (BETA)
+            chain(L5::DW, I128mm, DV / 16, false, [&](int ks) { return umma::desc_mn(dVnc, ks, C); },
+                  [&](int ks) { return umma::desc_mn(S0c, ks, 128); });
+        umma::commit(&bm[1]);
+    }
+
+    const float gam0 = __expf(Gs[r0]), gam1 = __expf(Gs[r1]);
+    const float gC = Gs[C - 1];
+    const float dec0 = __expf(gC - Gs[r0]), dec1 = __expf(gC - Gs[r1]);
+
+    // ---- E1: M = scale dP * Gamma (bf16 tile), row/column sums of M * QK; keep K K^T
+    float kkr[2][4];
+    {
+        wait_bar(&bm[0]);
+        float qk[2][4], dp[2][4];
+        umma::ld16(trow + L5::QK + 16 * nw, qk);
+        if (BETA) umma::ld16(trow + L5::KK + 16 * nw, kkr);
+        umma::ld16(trow + L5::DP + 16 * nw, dp);
+        umma::wait_ld();
+        float row0 = 0.f, row1 = 0.f;
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+            float col[2] = {0.f, 0.f};
+            float m[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = (e >> 1) ? r1 : r0, jj = 16 * nw + 8 * n + 2 * tq + (e & 1);
+                const float gm = (jj <= i) ? __expf(Gs[i] - Gs[jj]) : 0.f;
+                m[e] = s.scale * dp[n][e] * gm;
+                const float zp = m[e] * qk[n][e];
+                if (e >> 1) row1 += zp; else row0 += zp;
+                col[e & 1] += zp;
+            }
+            const int jj = 16 * nw + 8 * n + 2 * tq;
+            *umma::canon_at<uint32_t>(Ms, r0, jj, C) = pack(m[0], m[1]);
+            *umma::canon_at<uint32_t>(Ms, r1, jj, C) = pack(m[2], m[3]);
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                col[0] += __shfl_xor_sync(0xffffffffu, col[0], o);
+                col[1] += __shfl_xor_sync(0xffffffffu, col[1], o);
+            }
+            if (gq == 0) {
+                part[(P_COLP + mw) * C + jj] = col[0];
+                part[(P_COLP + mw) * C + jj + 1] = col[1];
+            }
+        }
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+            row0 += __shfl_xor_sync(0xffffffffu, row0, o);
+            row1 += __shfl_xor_sync(0xffffffffu, row1, o);
+        }
+        if (tq == 0) {
+            part[(P_ROWP + nw) * C + r0] = row0;
+            part[(P_ROWP + nw) * C + r1] = row1;
+        }
+    }
+    sync_for_mma();
+    if (tid == 0) {  // V_new dS_C^T
+        umma::fence_after();
+        chain(L5::DKC, I128mm, DV / 16, false, [&](int ks) { return umma::desc_mn(Vnc, ks, C); },
+              [&](int ks) { return umma::desc_mn(dSc, ks, 128); });
+        umma::commit(&bm[2]);
+    }
+
+    // ---- E2a: dq <- scale gamma (dO S0^T) in place; sum_k Q dq; <S0, dS_C>
+    {
+        wait_bar(&bm[1]);
+        float a[4][4];
+        umma::ld32(trow + L5::DQ + 32 * nw, a);
+        umma::wait_ld();
+        const float sq0 = s.scale * gam0, sq1 = s.scale * gam1;
+        float pi0 = 0.f, pi1 = 0.f;
+#pragma unroll
+        for (int jq = 0; jq < 4; ++jq) {
+            const int col = 32 * nw + 8 * jq + 2 * tq;
+            const float2 q0 = unpack(*umma::canon_at<uint32_t>(Qc, r0, col, 128));
+            const float2 q1 = unpack(*umma::canon_at<uint32_t>(Qc, r1, col, 128));
+            a[jq][0] *= sq0;
+            a[jq][1] *= sq0;
+            a[jq][2] *= sq1;
+            a[jq][3] *= sq1;
+            pi0 += q0.x * a[jq][0] + q0.y * a[jq][1];
+            pi1 += q1.x * a[jq][2] + q1.y * a[jq][3];
+        }
+        umma::st32(trow + L5::DQ + 32 * nw, a);
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+            pi0 += __shfl_xor_sync(0xffffffffu, pi0, o);
+            pi1 += __shfl_xor_sync(0xffffffffu, pi1, o);
+        }
+        if (tq == 0) {
+            part[(P_INTER + nw) * C + r0] = pi0;
+            part[(P_INTER + nw) * C + r1] = pi1;
+        }
+        float pd = 0.f;  // both canon tiles: the same element at the same offset
+        for (int e = tid; e < DV * 128 / 2; e += 512) {
+            const float2 x = unpack(reinterpret_cast<const uint32_t*>(S0c)[e]);
+            const float2 y = unpack(reinterpret_cast<const uint32_t*>(dSc)[e]);
+            pd = fmaf(x.x, y.x, pd);
+            pd = fmaf(x.y, y.y, pd);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pd += __shfl_xor_sync(0xffffffffu, pd, o);
+        if (lane == 0) red[w] = pd;
+        umma::wait_st();
+    }
+    sync_for_mma();
+    if (tid == 0) {  // dq += M K
+        umma::fence_after();
+        chain(L5::DQ, I128km, C / 16, true, [&](int ks) { return umma::desc_k(Ms, ks, C); },
+              [&](int ks) { return umma::desc_mn(Kc, ks, 128); });
+    }
+
+    // ---- E2b: dk <- dec (V_new dS_C^T) in place, sum_k K dk; dW; T'', T, L tiles
+    {
+        wait_bar(&bm[2]);  // every earlier product too: dO, V_new^T and the state tiles are free
+        if (has_next) copy_do(jn);
+        cp_async_commit();
+        if (tid == 0 && has_next) bulk_vn(jn);
+        float a[4][4];
+        umma::ld32(trow + L5::DKC + 32 * nw, a);
+        umma::wait_ld();
+        float pz0 = 0.f, pz1 = 0.f;
+#pragma unroll
+        for (int jq = 0; jq < 4; ++jq) {
+            const int col = 32 * nw + 8 * jq + 2 * tq;
+            const float2 k0 = unpack(*umma::canon_at<uint32_t>(Kc, r0, col, 128));
+            const float2 k1 = unpack(*umma::canon_at<uint32_t>(Kc, r1, col, 128));
+            a[jq][0] *= dec0;
+            a[jq][1] *= dec0;
+            a[jq][2] *= dec1;
+            a[jq][3] *= dec1;
+            pz0 += k0.x * a[jq][0] + k0.y * a[jq][1];
+            pz1 += k1.x * a[jq][2] + k1.y * a[jq][3];
+        }
+        umma::st32(trow + L5::DKC + 32 * nw, a);
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+            pz0 += __shfl_xor_sync(0xffffffffu, pz0, o);
+            pz1 += __shfl_xor_sync(0xffffffffu, pz1, o);
+        }
+        if (tq == 0) {
+            part[(P_Z + nw) * C + r0] = pz0;
+            part[(P_Z + nw) * C + r1] = pz1;
+        }
+        if (BETA) {
+            umma::ld32(trow + L5::DW + 32 * nw, a);
+            umma::wait_ld();
+#pragma unroll
+            for (int jq = 0; jq < 4; ++jq) {
+                const int col = 32 * nw + 8 * jq + 2 * tq;
+                *umma::canon_at<uint32_t>(dWs, r0, col, 128) = pack(-a[jq][0], -a[jq][1]);
+                *umma::canon_at<uint32_t>(dWs, r1, col, 128) = pack(-a[jq][2], -a[jq][3]);
+            }
+            mbar_wait(bL, par, &g_tc_status, failed);
+            {  // T'' = L diag(beta gamma), T = L diag(beta), L: one 8-element row piece per thread
+                const int i = tid >> 3, j0 = (tid & 7) * 8;
+                uint32_t tpp[4], tt[4], ll[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int jj = j0 + 2 * h;
+                    const float2 l = *reinterpret_cast<const float2*>(Lf + i * C + jj);
+                    const float b0 = Bs[jj], b1 = Bs[jj + 1];
+                    tpp[h] = pack(l.x * b0 * __expf(Gs[jj]), l.y * b1 * __expf(Gs[jj + 1]));
+                    tt[h] = pack(l.x * b0, l.y * b1);
+                    ll[h] = pack(l.x, l.y);
+                }
+                *umma::canon_at<uint4>(Tpp, i, j0, C) = make_uint4(tpp[0], tpp[1], tpp[2], tpp[3]);
+                *umma::canon_at<uint4>(Ts, i, j0, C) = make_uint4(tt[0], tt[1], tt[2], tt[3]);
+                *umma::canon_at<uint4>(Ls, i, j0, C) = make_uint4(ll[0], ll[1], ll[2], ll[3]);
+            }
+        }
+        umma::wait_st();
+    }
+    if (BETA) cp_async_wait<2>();  // this chunk's V (the next chunk's Q, K, dO may still be landing)
+    sync_for_mma();
+    if (tid == 0) {
+        umma::fence_after();
+        if (BETA) {  // gamma T^T dW, dW K^T, dV_new V^T
+            chain(L5::T3, I128mm, C / 16, false, [&](int ks) { return umma::desc_mn(Tpp, ks, C); },
+                  [&](int ks) { return umma::desc_mn(dWs, ks, 128); });
+            chain(L5::DTA, I64kk, 8, false, [&](int ks) { return umma::desc_k(dWs, ks, 128); },
+                  [&](int ks) { return umma::desc_k(Kc, ks, 128); });
+            chain(L5::DTB, I64mk, DV / 16, false, [&](int ks) { return umma::desc_mn(dVnc, ks, C); },
+                  [&](int ks) { return umma::desc_k(Vc, ks, DV); });
+        } else {  // dk += M^T Q
+            chain(L5::DKC, I128mm, C / 16, true, [&](int ks) { return umma::desc_mn(Ms, ks, C); },
+                  [&](int ks) { return umma::desc_mn(Qc, ks, 128); });
+        }
+        umma::commit(&bm[3]);
+    }
+
+    if (BETA) {
+        // ---- E3: dk += gamma T^T dW, sum_k K (gamma T^T dW); E4: dT, dL, dbeta (column part)
+        wait_bar(&bm[3]);
+        {
+            float t3[4][4], a[4][4];
+            umma::ld32(trow + L5::T3 + 32 * nw, t3);
+            umma::ld32(trow + L5::DKC + 32 * nw, a);
+            umma::wait_ld();
+            float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+            for (int jq = 0; jq < 4; ++jq) {
+                const int col = 32 * nw + 8 * jq + 2 * tq;
+                const float2 k0 = unpack(*umma::canon_at<uint32_t>(Kc, r0, col, 128));
+                const float2 k1 = unpack(*umma::canon_at<uint32_t>(Kc, r1, col, 128));
+                p0 += k0.x * t3[jq][0] + k0.y * t3[jq][1];
+                p1 += k1.x * t3[jq][2] + k1.y * t3[jq][3];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) a[jq][e] += t3[jq][e];
+            }
+            umma::st32(trow + L5::DKC + 32 * nw, a);
+#pragma unroll
+            for (int o = 1; o < 4; o <<= 1) {
+                p0 += __shfl_xor_sync(0xffffffffu, p0, o);
+                p1 += __shfl_xor_sync(0xffffffffu, p1, o);
+            }
+            if (tq == 0) {
+                part[(P_KT + nw) * C + r0] = p0;
+                part[(P_KT + nw) * C + r1] = p1;
+            }
+        }
+        {
+            float ta[2][4], tb[2][4];
+            umma::ld16(trow + L5::DTA + 16 * nw, ta);
+            umma::ld16(trow + L5::DTB + 16 * nw, tb);
+            umma::wait_ld();
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+                float col[2] = {0.f, 0.f};
+                float dl[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = (e >> 1) ? r1 : r0, jj = 16 * nw + 8 * n + 2 * tq + (e & 1);
+                    const float dt = fmaf(ta[n][e], __expf(Gs[jj]), tb[n][e]);
+                    col[e & 1] += dt * Lf[r * C + jj];
+                    dl[e] = dt * Bs[jj];
+                }
+                const int jj = 16 * nw + 8 * n + 2 * tq;
+                *umma::canon_at<uint32_t>(dLs, r0, jj, C) = pack(dl[0], dl[1]);
+                *umma::canon_at<uint32_t>(dLs, r1, jj, C) = pack(dl[2], dl[3]);
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) {
+                    col[0] += __shfl_xor_sync(0xffffffffu, col[0], o);
+                    col[1] += __shfl_xor_sync(0xffffffffu, col[1], o);
+                }
+                if (gq == 0) {
+                    part[(P_DBC + mw) * C + jj] = col[0];
+                    part[(P_DBC + mw) * C + jj + 1] = col[1];
+                }
+            }
+        }
+        umma::wait_st();
+        sync_for_mma();  // L (fp32) is read for the last time above
+        if (tid == 0) {  // dv = T^T dV_new, X = L^T dL, dk += M^T Q
+            umma::fence_after();
+            chain(L5::DVC, IDVmk, C / 16, false, [&](int ks) { return umma::desc_mn(Ts, ks, C); },
+                  [&](int ks) { return umma::desc_k(dVnc, ks, C); });
+            chain(L5::XC, I64mm, C / 16, false, [&](int ks) { return umma::desc_mn(Ls, ks, C); },
+                  [&](int ks) { return umma::desc_mn(dLs, ks, C); });
+            chain(L5::DKC, I128mm, C / 16, true, [&](int ks) { return umma::desc_mn(Ms, ks, C); },
+                  [&](int ks) { return umma::desc_mn(Qc, ks, 128); });
+            umma::commit(&bm[4]);
+            if (has_next) bulk_l(jn);
+        }
+        // ---- E5: X (bf16 tile); dv out
+        wait_bar(&bm[4]);  // V, dV_new^T are free
+        if (has_next) copy_v(jn);
+        cp_async_commit();
+        if (tid == 0 && has_next) bulk_dvn(jn);
+        {
+            float x[2][4];
+            umma::ld16(trow + L5::XC + 16 * nw, x);
+            umma::wait_ld();
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+                const int jj = 16 * nw + 8 * n + 2 * tq;
+                *umma::canon_at<uint32_t>(Xs, r0, jj, C) = pack(x[n][0], x[n][1]);
+                *umma::canon_at<uint32_t>(Xs, r1, jj, C) = pack(x[n][2], x[n][3]);
+            }
+            bf16* dvb = dv + bh * s.hs_v + (size_t)t0 * DV;
+            if (DV == 128) {
+                float a[4][4];
+                umma::ld32(trow + L5::DVC + 32 * nw, a);
+                umma::wait_ld();
+#pragma unroll
+                for (int jq = 0; jq < 4; ++jq) {
+                    const int col = 32 * nw + 8 * jq + 2 * tq;
+                    if (r0 < nval) *reinterpret_cast<uint32_t*>(dvb + (size_t)r0 * DV + col) = pack(a[jq][0], a[jq][1]);
+                    if (r1 < nval) *reinterpret_cast<uint32_t*>(dvb + (size_t)r1 * DV + col) = pack(a[jq][2], a[jq][3]);
+                }
+            } else {
+                float a[2][4];
+                umma::ld16(trow + L5::DVC + 16 * nw, a);
+                umma::wait_ld();
+#pragma unroll
+                for (int jq = 0; jq < 2; ++jq) {
+                    const int col = 16 * nw + 8 * jq + 2 * tq;
+                    if (r0 < nval) *reinterpret_cast<uint32_t*>(dvb + (size_t)r0 * DV + col) = pack(a[jq][0], a[jq][1]);
+                    if (r1 < nval) *reinterpret_cast<uint32_t*>(dvb + (size_t)r1 * DV + col) = pack(a[jq][2], a[jq][3]);
+                }
+            }
+        }
+        sync_for_mma();
+        if (tid == 0) {  // dA' = X L^T
+            umma::fence_after();
+            chain(L5::DA, I64kk, C / 16, false, [&](int ks) { return umma::desc_k(Xs, ks, C); },
+                  [&](int ks) { return umma::desc_k(Ls, ks, C); });
+            umma::commit(&bm[5]);
+        }
+        // ---- E6: dA = strictly-lower(-X L^T); Z = dA beta_i Gamma; dbeta (row part); Z sums
+        wait_bar(&bm[5]);
+        {
+            float da[2][4];
+            umma::ld16(trow + L5::DA + 16 * nw, da);
+            umma::wait_ld();
+            float rz0 = 0.f, rz1 = 0.f, rb0 = 0.f, rb1 = 0.f;
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+                float col[2] = {0.f, 0.f};
+                float zz[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = (e >> 1) ? r1 : r0, jj = 16 * nw + 8 * n + 2 * tq + (e & 1);
+                    float z = 0.f, bterm = 0.f;
+                    if (jj < i) {
+                        const float gm = __expf(Gs[i] - Gs[jj]);
+                        const float dav = -da[n][e];
+                        bterm = dav * gm * kkr[n][e];
+                        z = dav * Bs[i] * gm;
+                    }
+                    zz[e] = z;
+                    const float za = z * kkr[n][e];
+                    if (e >> 1) {
+                        rz1 += za;
+                        rb1 += bterm;
+                    } else {
+                        rz0 += za;
+                        rb0 += bterm;
+                    }
+                    col[e & 1] += za;
+                }
+                const int jj = 16 * nw + 8 * n + 2 * tq;
+                *umma::canon_at<uint32_t>(Zs, r0, jj, C) = pack(zz[0], zz[1]);
+                *umma::canon_at<uint32_t>(Zs, r1, jj, C) = pack(zz[2], zz[3]);
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) {
+                    col[0] += __shfl_xor_sync(0xffffffffu, col[0], o);
+                    col[1] += __shfl_xor_sync(0xffffffffu, col[1], o);
+                }
+                if (gq == 0) {
+                    part[(P_COLA + mw) * C + jj] = col[0];
+                    part[(P_COLA + mw) * C + jj + 1] = col[1];
+                }
+            }
+#pragma unroll
+            for (int o = 1; o < 4; o <<= 1) {
+                rz0 += __shfl_xor_sync(0xffffffffu, rz0, o);
+                rz1 += __shfl_xor_sync(0xffffffffu, rz1, o);
+                rb0 += __shfl_xor_sync(0xffffffffu, rb0, o);
+                rb1 += __shfl_xor_sync(0xffffffffu, rb1, o);
+            }
+            if (tq == 0) {
+                part[(P_ROWA + nw) * C + r0] = rz0;
+                part[(P_ROWA + nw) * C + r1] = rz1;
+                part[(P_DBR + nw) * C + r0] = rb0;
+                part[(P_DBR + nw) * C + r1] = rb1;
+            }
+        }
+        sync_for_mma();
+        if (tid == 0) {  // dk += Z K + Z^T K
+            umma::fence_after();
+            chain(L5::DKC, I128km, C / 16, true, [&](int ks) { return umma::desc_k(Zs, ks, C); },
+                  [&](int ks) { return umma::desc_mn(Kc, ks, 128); });
+            chain(L5::DKC, I128mm, C / 16, true, [&](int ks) { return umma::desc_mn(Zs, ks, C); },
+                  [&](int ks) { return umma::desc_mn(Kc, ks, 128); });
+            umma::commit(&bm[6]);
+        }
+        wait_bar(&bm[6]);
+    } else {
+        wait_bar(&bm[3]);
+        bf16* dvb = dv + bh * s.hs_v + (size_t)t0 * DV;
+        for (int e = tid; e < nval * DV; e += 512) {
+            const int jj = e / DV, col = e % DV;
+            dvb[(size_t)jj * DV + col] = *umma::canon_at<bf16>(dVnc, col, jj, C);
+        }
+        __syncthreads();  // V (unused here) and dV_new^T are free
+        if (has_next) copy_v(jn);
+        cp_async_commit();
+        if (tid == 0 && has_next) bulk_dvn(jn);
+    }
+
+    // ---- E7: dq, dk staged row-major in the free state region, then bulk-stored by rows
+    {
+        float a[4][4], b[4][4];
+        umma::ld32(trow + L5::DQ + 32 * nw, a);
+        umma::ld32(trow + L5::DKC + 32 * nw, b);
+        umma::wait_ld();
+#pragma unroll
+        for (int jq = 0; jq < 4; ++jq) {
+            const int col = 32 * nw + 8 * jq + 2 * tq;
+            *reinterpret_cast<uint32_t*>(Sq + r0 * L5::SLD + col) = pack(a[jq][0], a[jq][1]);
+            *reinterpret_cast<uint32_t*>(Sq + r1 * L5::SLD + col) = pack(a[jq][2], a[jq][3]);
+            *reinterpret_cast<uint32_t*>(Sk + r0 * L5::SLD + col) = pack(b[jq][0], b[jq][1]);
+            *reinterpret_cast<uint32_t*>(Sk + r1 * L5::SLD + col) = pack(b[jq][2], b[jq][3]);
+        }
+    }
+    fence_proxy_async_smem();
+    umma::fence_before();
+    __syncthreads();  // staging written, partial sums written, TMEM reads done
+    if (tid < 2 * C) {  // one row of dq or dk per thread
+        const int r = tid & (C - 1);
+        if (r < nval) {
+            const bool isk = tid >= C;
+            bf16* dst = (isk ? dk : dq) + bh * s.hs_k + (size_t)(t0 + r) * DK;
+            bulk_store(dst, (isk ? Sk : Sq) + r * L5::SLD, DK * 2);
+        }
+        bulk_commit();
+    }
+    if (w == 15) {
+        // ---- dG, dg (chunk-local reverse cumsum), dbeta; two tokens per lane
+        auto P = [&](int row, int n, int i) {
+            float x = 0.f;
+            for (int u = 0; u < n; ++u) x += part[(row + u) * C + i];
+            return x;
+        };
+        float x[2], zs = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int i = 2 * lane + h;
+            x[h] = P(P_INTER, GW, i) + P(P_ROWP, GW, i) - P(P_COLP, 4, i) - P(P_Z, GW, i);
+            zs += P(P_Z, GW, i);
+            if (BETA) {
+                x[h] += P(P_ROWA, GW, i) - P(P_COLA, 4, i) + P(P_KT, GW, i);
+                if (i < nval) dbeta[bh * s.hs_g + t0 + i] = P(P_DBC, 4, i) + P(P_DBR, GW, i);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
+        float sdot = 0.f;
+        for (int u = 0; u < 16; ++u) sdot += red[u];
+        if (lane == 31) x[1] += __expf(gC) * sdot + zs;
+        float suf = x[0] + x[1];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_down_sync(0xffffffffu, suf, o);
+            if (lane + o < 32) suf += y;
+        }
+        float* dgb = dg + bh * s.hs_g + t0;
+        if (2 * lane < nval) dgb[2 * lane] = suf;
+        if (2 * lane + 1 < nval) dgb[2 * lane + 1] = suf - x[0];
+    }
+    if (tid < 2 * C) bulk_wait_read<0>();  // the staging region is read out
+    __syncthreads();  // partial sums consumed; the state region is free
+    if (tid == 0 && has_next) bulk_state(jn);
+    if (!has_next) break;
+    for (int e = tid; e < P_ROWS * C; e += 512) part[e] = 0.f;
+    if (tid < C) Bsb[(buf ^ 1) * C + tid] = beta_next;
+    j = jn;
+  }
+    if (tid < 2 * C) bulk_wait<0>();
+    umma::fence_before();
+    __syncthreads();
+    if (w == 0) {
+        umma::fence_after();
+        umma::dealloc(tm, 512);
+    }
+}
+
 template <typename K>
 cudaError_t smem_attr(K* kern, size_t bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -1710,6 +2418,36 @@ cudaError_t launch_grad(const SeqView& s, const BwdArgs& a, const TcWs& w, cudaS
 }
 
 template <int DV, bool BETA>
+cudaError_t launch_grad5(const SeqView& s, const BwdArgs& a, const TcWs& w, cudaStream_t st) {
+    constexpr size_t sm = G5<DV>::SMEM;
+    TC_TRY(smem_attr(tc_grad5_kernel<DV, BETA>, sm));
+    TC_TRY(cudaMemsetAsync(w.ticket, 0, sizeof(int), st));
+    const int grid = std::min(s.NC * s.BH, num_sms());
+    SF_LAUNCH("tc_grad", st, tc_grad5_kernel<DV, BETA><<<grid, 512, sm, st>>>(
+                                 s, static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k),
+                                 static_cast<const bf16*>(a.v), a.beta, static_cast<const bf16*>(a.dO), w.Gc,
+                                 w.Lm, w.Vnt, w.dVnt, w.S0t, w.dSCt, static_cast<bf16*>(a.dq), static_cast<bf16*>(a.dk),
+                                 static_cast<bf16*>(a.dv), a.dg, a.dbeta, w.ticket));
+    return cudaGetLastError();
+}
+
+// Gradient kernel: the tcgen05 one (default) or the warp-level persistent one
+// (SF_GDN_GRAD=warp), read once.
+bool grad_tcgen05() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = std::getenv("SF_GDN_GRAD");
+        v = (e && std::string(e) == "warp") ? 0 : 1;
+    }
+    return v == 1;
+}
+
+template <int DV, bool BETA>
+cudaError_t launch_grad_any(const SeqView& s, const BwdArgs& a, const TcWs& w, cudaStream_t st) {
+    return grad_tcgen05() ? launch_grad5<DV, BETA>(s, a, w, st) : launch_grad<DV, BETA>(s, a, w, st);
+}
+
+template <int DV, bool BETA>
 cudaError_t fwd_impl(const SeqView& s, const FwdArgs& a, void* ws, cudaStream_t st) {
     char* base = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), 256));
     const TcWs w = tc_layout(s, false, base);
@@ -1729,7 +2467,7 @@ cudaError_t bwd_impl(const SeqView& s, const BwdArgs& a, void* ws, cudaStream_t 
     TC_TRY((launch_prep<DV, BETA>("tc_prep_bwd", s, k, static_cast<const bf16*>(a.v), a.g, a.beta, w, st)));
     TC_TRY((launch_intra<DV>(s, q, k, static_cast<const bf16*>(a.dO), w, st)));
     TC_TRY((launch_scan_bwd<DV, BETA>(s, a, true, w, st)));
-    return launch_grad<DV, BETA>(s, a, w, st);
+    return launch_grad_any<DV, BETA>(s, a, w, st);
 }
 
 template <int DV, bool BETA>
@@ -1754,7 +2492,7 @@ cudaError_t stage_impl(TcStage stage, const SeqView& s, const FwdArgs* f, const 
             return launch_intra<DV>(s, static_cast<const bf16*>(b->q), static_cast<const bf16*>(b->k),
                                     static_cast<const bf16*>(b->dO), w, st);
         case TcStage::ScanBwd: return launch_scan_bwd<DV, BETA>(s, *b, false, w, st);
-        case TcStage::Grad: return launch_grad<DV, BETA>(s, *b, w, st);
+        case TcStage::Grad: return launch_grad_any<DV, BETA>(s, *b, w, st);
     }
     return cudaErrorInvalidValue;
 }
