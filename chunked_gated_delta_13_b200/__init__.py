@@ -10,6 +10,8 @@ Entry points mirror the C ABI in ``include/sf_gdn.h``:
   fwd(q, k, v, g, beta, S_in)                       -> (o, S_out)
   bwd(q, k, v, g, beta, S_in, dO, dS_out)           -> dict of gradients
   segment_run(..., N or seg_len)                    -> (o, S_out, gradients)
+  conv_fwd / conv_bwd / conv_segment_run            the short causal convolution
+                                                    with its boundary state
 The operations are StateFlow's chunk Fwd/Bwd and its sequence split with the
 state handed forward and the state gradient handed backward (arXiv 2608.06838,
 sections 2.1 and 3.1).
@@ -22,7 +24,7 @@ import threading
 
 from ._build import LIB, build, needs_build
 
-__all__ = ["Shape", "SFError", "lib", "fwd", "bwd", "segment_run", "make_shape", "path", "device_check",
+__all__ = ["Shape", "ConvShape", "make_conv_shape", "conv_fwd", "conv_bwd", "conv_segment_run", "SFError", "lib", "fwd", "bwd", "segment_run", "make_shape", "path", "device_check",
            "launches", "set_launch_hook", "timer_enable", "timer_disable", "timer_count", "timer_results", "timer_free",
            "fwd_workspace_bytes", "bwd_workspace_bytes", "segment_workspace_bytes",
            "EXPORTED_SYMBOLS"]
@@ -37,7 +39,8 @@ EXPORTED_SYMBOLS = [
     "sf_gdn_bwd_workspace_bytes", "sf_gdn_fwd", "sf_gdn_bwd", "sf_segment_workspace_bytes",
     "sf_segment_run", "sf_gdn_path", "sf_gdn_launches", "sf_set_launch_hook", "sf_gdn_fwd_noalloc",
     "sf_device_check", "sf_timer_enable", "sf_timer_disable", "sf_timer_count", "sf_timer_read",
-    "sf_timer_free",
+    "sf_timer_free", "sf_conv_workspace_bytes", "sf_conv_fwd", "sf_conv_bwd",
+    "sf_conv_segment_workspace_bytes", "sf_conv_segment_run",
 ]
 
 HOOK_T = ctypes.CFUNCTYPE(None, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p)
@@ -48,6 +51,12 @@ class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int),
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("C", ctypes.c_int),
                 ("io", ctypes.c_int), ("use_beta", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+class ConvShape(ctypes.Structure):
+    """Mirror of ``sf_conv_shape``."""
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("d", ctypes.c_int),
+                ("K", ctypes.c_int), ("io", ctypes.c_int), ("act", ctypes.c_int)]
 
 
 class SFError(RuntimeError):
@@ -125,6 +134,18 @@ def lib():
         L.sf_timer_read.restype = ctypes.c_int
         L.sf_timer_free.argtypes = []
         L.sf_timer_free.restype = None
+        CP = ctypes.POINTER(ConvShape)
+        L.sf_conv_workspace_bytes.argtypes = [CP]
+        L.sf_conv_workspace_bytes.restype = ctypes.c_size_t
+        L.sf_conv_fwd.argtypes = [CP] + [P] * 5 + [P]
+        L.sf_conv_fwd.restype = ctypes.c_int
+        L.sf_conv_bwd.argtypes = [CP] + [P] * 9 + [P, ctypes.c_size_t, P]
+        L.sf_conv_bwd.restype = ctypes.c_int
+        L.sf_conv_segment_workspace_bytes.argtypes = [CP, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+        L.sf_conv_segment_workspace_bytes.restype = ctypes.c_size_t
+        L.sf_conv_segment_run.argtypes = ([CP, ctypes.c_int, ctypes.POINTER(ctypes.c_int)] + [P] * 10
+                                          + [P, ctypes.c_size_t, P])
+        L.sf_conv_segment_run.restype = ctypes.c_int
         _lib = L
         return _lib
 
@@ -354,3 +375,82 @@ def segment_run(q, k, v, g, beta, S_in, dO, dS_out=None, *, N=1, seg_len=None, C
     if dO is not None:
         grads = {n: out[n] for n in ("dq", "dk", "dv", "dg", "dbeta", "dS_in")}
     return out["o"], out["S_out"], grads
+
+
+# ------------------------------------------------- short convolution glue ---
+
+def make_conv_shape(B, H, T, d, K, io="bf16", act="silu") -> ConvShape:
+    io_code = {"bf16": SF_BF16, "f32": SF_F32}[io]
+    return ConvShape(int(B), int(H), int(T), int(d), int(K), io_code, {"none": 0, "silu": 1}[act])
+
+
+def _conv_shape_of(x, w, act):
+    B, H, T, d = x.shape
+    return make_conv_shape(B, H, T, d, w.shape[-1], _io_of(x), act)
+
+
+def conv_fwd(x, w, conv_in=None, *, act="silu", y=None, conv_out=None, stream=None):
+    """Short causal convolution of one segment with its boundary state.
+    x: [B,H,T,d] (bf16 or fp32); w: [H,d,K] fp32; conv_in: [B,H,K-1,d] (x's dtype)
+    or None.  Returns (y, conv_out)."""
+    torch = _torch()
+    _need_cuda(x, w, conv_in)
+    shape = _conv_shape_of(x, w, act)
+    B, H, T, d = x.shape
+    K = w.shape[-1]
+    if y is None:
+        y = torch.empty_like(x)
+    if conv_out is None:
+        conv_out = torch.empty(B, H, K - 1, d, dtype=x.dtype, device=x.device)
+    _check(lib().sf_conv_fwd(ctypes.byref(shape), _ptr(x), _ptr(w), _ptr(conv_in), _ptr(y),
+                             _ptr(conv_out), _stream(stream)))
+    return y, conv_out
+
+
+def conv_bwd(x, w, conv_in, dy, dconv_out=None, *, act="silu", dw_in=None, out=None, workspace=None,
+             stream=None):
+    """Backward of one segment.  Returns a dict: dx, dw (= dw_in + this segment's
+    weight gradient) and dconv_in."""
+    torch = _torch()
+    _need_cuda(x, w, conv_in, dy, dconv_out, dw_in)
+    shape = _conv_shape_of(x, w, act)
+    B, H, T, d = x.shape
+    K = w.shape[-1]
+    if out is None:
+        out = {"dx": torch.empty_like(x), "dw": torch.empty_like(w),
+               "dconv_in": torch.empty(B, H, K - 1, d, dtype=torch.float32, device=x.device)}
+    ws = _workspace(int(lib().sf_conv_workspace_bytes(ctypes.byref(shape))), x.device, workspace)
+    nbytes = 0 if ws is None else ws.numel()
+    _check(lib().sf_conv_bwd(ctypes.byref(shape), _ptr(x), _ptr(w), _ptr(conv_in), _ptr(dy),
+                             _ptr(dconv_out), _ptr(out["dx"]), _ptr(dw_in), _ptr(out["dw"]),
+                             _ptr(out["dconv_in"]), _ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+def conv_segment_run(x, w, conv_in, dy, dconv_out=None, *, N=1, seg_len=None, act="silu",
+                     workspace=None, stream=None):
+    """The convolution's segment chain: N segments forward with the state handed
+    on, then (dy given) backward in reverse with its gradient handed back.
+    Returns (y, conv_out, grads) with grads None when dy is None."""
+    torch = _torch()
+    _need_cuda(x, w, conv_in, dy, dconv_out)
+    shape = _conv_shape_of(x, w, act)
+    B, H, T, d = x.shape
+    K = w.shape[-1]
+    segs = _seg_array(N, seg_len)
+    y = torch.empty_like(x)
+    conv_out = torch.empty(B, H, K - 1, d, dtype=x.dtype, device=x.device)
+    grads = None
+    if dy is not None:
+        grads = {"dx": torch.empty_like(x), "dw": torch.empty_like(w),
+                 "dconv_in": torch.empty(B, H, K - 1, d, dtype=torch.float32, device=x.device)}
+    need = int(lib().sf_conv_segment_workspace_bytes(ctypes.byref(shape), int(N), segs))
+    if need == 0:
+        raise SFError(1, "invalid convolution shape or segment lengths")
+    ws = _workspace(need, x.device, workspace)
+    g_ = (lambda n: _ptr(grads[n])) if grads is not None else (lambda n: None)
+    _check(lib().sf_conv_segment_run(ctypes.byref(shape), int(N), segs, _ptr(x), _ptr(w),
+                                     _ptr(conv_in), _ptr(dy), _ptr(dconv_out), _ptr(y),
+                                     _ptr(conv_out), g_("dx"), g_("dw"), g_("dconv_in"), _ptr(ws),
+                                     ws.numel(), _stream(stream)))
+    return y, conv_out, grads

@@ -1589,15 +1589,19 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 // them are done, then dV_new^T and V, then L; the state tiles last, into the
 // region the epilogue tiles of the current chunk leave.
 //
+// The term gamma (T^T dW) of dk accumulates in place; its share of dG,
+// sum_k K_ik gamma_i (T^T dW)_ik = gamma_i beta_i sum_j L_ji (dW K^T)_ji, is a
+// column sum of L * (dW K^T), taken where dT is formed.
+//
 // TMEM columns (512 allocated; M = 64 uses lanes 0-15 of each quarter):
 //   [0,64) Q K^T -> [0,128) dk       [64,128) K K^T        [128,192) dP -> dT_b -> dA
-//   [192,320) dq                     [320,448) dV_new S0^T -> gamma T^T dW -> dv
+//   [192,320) dq                     [320,448) dV_new S0^T -> dv
 //   [448,512) dW K^T -> X
 template <int DV>
 struct G5 {
     // TMEM columns of the accumulators
     static constexpr uint32_t QK = 0, KK = 64, DP = 128, DQ = 192, DW = 320, DTA = 448;
-    static constexpr uint32_t DKC = 0, T3 = 320, DTB = 128, DVC = 320, XC = 448, DA = 128;
+    static constexpr uint32_t DKC = 0, DTB = 128, DVC = 320, XC = 448, DA = 128;
     static constexpr int SLD = 128 + 8;  // row stride of the dq / dk staging tiles (elements)
     static constexpr size_t kQK = (size_t)2 * C * 128 * 2;  // one buffer: Q then K
     static constexpr size_t kV = (size_t)C * DV * 2;        // V, dO, V_new^T, dV_new^T each
@@ -1985,13 +1989,17 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     sync_for_mma();
     if (tid == 0) {
         umma::fence_after();
-        if (BETA) {  // gamma T^T dW, dW K^T, dV_new V^T
-            chain(L5::T3, I128mm, C / 16, false, [&](int ks) { return umma::desc_mn(Tpp, ks, C); },
+        if (BETA) {  // dk += gamma T^T dW, dk += M^T Q, dW K^T, dV_new V^T, dv = T^T dV_new
+            chain(L5::DKC, I128mm, C / 16, true, [&](int ks) { return umma::desc_mn(Tpp, ks, C); },
                   [&](int ks) { return umma::desc_mn(dWs, ks, 128); });
+            chain(L5::DKC, I128mm, C / 16, true, [&](int ks) { return umma::desc_mn(Ms, ks, C); },
+                  [&](int ks) { return umma::desc_mn(Qc, ks, 128); });
             chain(L5::DTA, I64kk, 8, false, [&](int ks) { return umma::desc_k(dWs, ks, 128); },
                   [&](int ks) { return umma::desc_k(Kc, ks, 128); });
             chain(L5::DTB, I64mk, DV / 16, false, [&](int ks) { return umma::desc_mn(dVnc, ks, C); },
                   [&](int ks) { return umma::desc_k(Vc, ks, DV); });
+            chain(L5::DVC, IDVmk, C / 16, false, [&](int ks) { return umma::desc_mn(Ts, ks, C); },
+                  [&](int ks) { return umma::desc_k(dVnc, ks, C); });
         } else {  // dk += M^T Q
             chain(L5::DKC, I128mm, C / 16, true, [&](int ks) { return umma::desc_mn(Ms, ks, C); },
                   [&](int ks) { return umma::desc_mn(Qc, ks, 128); });
@@ -2000,35 +2008,11 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     }
 
     if (BETA) {
-        // ---- E3: dk += gamma T^T dW, sum_k K (gamma T^T dW); E4: dT, dL, dbeta (column part)
-        wait_bar(&bm[3]);
-        {
-            float t3[4][4], a[4][4];
-            umma::ld32(trow + L5::T3 + 32 * nw, t3);
-            umma::ld32(trow + L5::DKC + 32 * nw, a);
-            umma::wait_ld();
-            float p0 = 0.f, p1 = 0.f;
-#pragma unroll
-            for (int jq = 0; jq < 4; ++jq) {
-                const int col = 32 * nw + 8 * jq + 2 * tq;
-                const float2 k0 = unpack(*umma::canon_at<uint32_t>(Kc, r0, col, 128));
-                const float2 k1 = unpack(*umma::canon_at<uint32_t>(Kc, r1, col, 128));
-                p0 += k0.x * t3[jq][0] + k0.y * t3[jq][1];
-                p1 += k1.x * t3[jq][2] + k1.y * t3[jq][3];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) a[jq][e] += t3[jq][e];
-            }
-            umma::st32(trow + L5::DKC + 32 * nw, a);
-#pragma unroll
-            for (int o = 1; o < 4; o <<= 1) {
-                p0 += __shfl_xor_sync(0xffffffffu, p0, o);
-                p1 += __shfl_xor_sync(0xffffffffu, p1, o);
-            }
-            if (tq == 0) {
-                part[(P_KT + nw) * C + r0] = p0;
-                part[(P_KT + nw) * C + r1] = p1;
-            }
-        }
+        // ---- E4: dT = dW (gamma K)^T + dV_new V^T, dL, dbeta (column part), the gamma T^T dW share of dG
+        wait_bar(&bm[3]);  // V, dV_new^T are free
+        if (has_next) copy_v(jn);
+        cp_async_commit();
+        if (tid == 0 && has_next) bulk_dvn(jn);
         {
             float ta[2][4], tb[2][4];
             umma::ld16(trow + L5::DTA + 16 * nw, ta);
@@ -2036,13 +2020,15 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
             umma::wait_ld();
 #pragma unroll
             for (int n = 0; n < 2; ++n) {
-                float col[2] = {0.f, 0.f};
+                float col[2] = {0.f, 0.f}, ckt[2] = {0.f, 0.f};
                 float dl[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int r = (e >> 1) ? r1 : r0, jj = 16 * nw + 8 * n + 2 * tq + (e & 1);
+                    const float l = Lf[r * C + jj];
                     const float dt = fmaf(ta[n][e], __expf(Gs[jj]), tb[n][e]);
-                    col[e & 1] += dt * Lf[r * C + jj];
+                    col[e & 1] += dt * l;
+                    ckt[e & 1] += ta[n][e] * l;
                     dl[e] = dt * Bs[jj];
                 }
                 const int jj = 16 * nw + 8 * n + 2 * tq;
@@ -2052,41 +2038,18 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
                 for (int o = 4; o < 32; o <<= 1) {
                     col[0] += __shfl_xor_sync(0xffffffffu, col[0], o);
                     col[1] += __shfl_xor_sync(0xffffffffu, col[1], o);
+                    ckt[0] += __shfl_xor_sync(0xffffffffu, ckt[0], o);
+                    ckt[1] += __shfl_xor_sync(0xffffffffu, ckt[1], o);
                 }
                 if (gq == 0) {
                     part[(P_DBC + mw) * C + jj] = col[0];
                     part[(P_DBC + mw) * C + jj + 1] = col[1];
+                    part[(P_KT + mw) * C + jj] = ckt[0];
+                    part[(P_KT + mw) * C + jj + 1] = ckt[1];
                 }
             }
         }
-        umma::wait_st();
-        sync_for_mma();  // L (fp32) is read for the last time above
-        if (tid == 0) {  // dv = T^T dV_new, X = L^T dL, dk += M^T Q
-            umma::fence_after();
-            chain(L5::DVC, IDVmk, C / 16, false, [&](int ks) { return umma::desc_mn(Ts, ks, C); },
-                  [&](int ks) { return umma::desc_k(dVnc, ks, C); });
-            chain(L5::XC, I64mm, C / 16, false, [&](int ks) { return umma::desc_mn(Ls, ks, C); },
-                  [&](int ks) { return umma::desc_mn(dLs, ks, C); });
-            chain(L5::DKC, I128mm, C / 16, true, [&](int ks) { return umma::desc_mn(Ms, ks, C); },
-                  [&](int ks) { return umma::desc_mn(Qc, ks, 128); });
-            umma::commit(&bm[4]);
-            if (has_next) bulk_l(jn);
-        }
-        // ---- E5: X (bf16 tile); dv out
-        wait_bar(&bm[4]);  // V, dV_new^T are free
-        if (has_next) copy_v(jn);
-        cp_async_commit();
-        if (tid == 0 && has_next) bulk_dvn(jn);
-        {
-            float x[2][4];
-            umma::ld16(trow + L5::XC + 16 * nw, x);
-            umma::wait_ld();
-#pragma unroll
-            for (int n = 0; n < 2; ++n) {
-                const int jj = 16 * nw + 8 * n + 2 * tq;
-                *umma::canon_at<uint32_t>(Xs, r0, jj, C) = pack(x[n][0], x[n][1]);
-                *umma::canon_at<uint32_t>(Xs, r1, jj, C) = pack(x[n][2], x[n][3]);
-            }
+        {  // dv out
             bf16* dvb = dv + bh * s.hs_v + (size_t)t0 * DV;
             if (DV == 128) {
                 float a[4][4];
@@ -2108,6 +2071,27 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
                     if (r0 < nval) *reinterpret_cast<uint32_t*>(dvb + (size_t)r0 * DV + col) = pack(a[jq][0], a[jq][1]);
                     if (r1 < nval) *reinterpret_cast<uint32_t*>(dvb + (size_t)r1 * DV + col) = pack(a[jq][2], a[jq][3]);
                 }
+            }
+        }
+        sync_for_mma();  // L (fp32) is read for the last time above
+        if (tid == 0) {  // X = L^T dL
+            umma::fence_after();
+            chain(L5::XC, I64mm, C / 16, false, [&](int ks) { return umma::desc_mn(Ls, ks, C); },
+                  [&](int ks) { return umma::desc_mn(dLs, ks, C); });
+            umma::commit(&bm[4]);
+            if (has_next) bulk_l(jn);
+        }
+        // ---- E5: X (bf16 tile)
+        wait_bar(&bm[4]);
+        {
+            float x[2][4];
+            umma::ld16(trow + L5::XC + 16 * nw, x);
+            umma::wait_ld();
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+                const int jj = 16 * nw + 8 * n + 2 * tq;
+                *umma::canon_at<uint32_t>(Xs, r0, jj, C) = pack(x[n][0], x[n][1]);
+                *umma::canon_at<uint32_t>(Xs, r1, jj, C) = pack(x[n][2], x[n][3]);
             }
         }
         sync_for_mma();
@@ -2240,7 +2224,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
             x[h] = P(P_INTER, GW, i) + P(P_ROWP, GW, i) - P(P_COLP, 4, i) - P(P_Z, GW, i);
             zs += P(P_Z, GW, i);
             if (BETA) {
-                x[h] += P(P_ROWA, GW, i) - P(P_COLA, 4, i) + P(P_KT, GW, i);
+                x[h] += P(P_ROWA, GW, i) - P(P_COLA, 4, i) + __expf(Gs[i]) * Bs[i] * P(P_KT, 4, i);
                 if (i < nval) dbeta[bh * s.hs_g + t0 + i] = P(P_DBC, 4, i) + P(P_DBR, GW, i);
             }
         }

@@ -127,3 +127,41 @@ def as_f64(inputs: dict) -> dict:
     for name, t in inputs.items():
         out[name] = None if t is None else t.to(torch.float64).numpy()
     return out
+
+
+@dataclass(frozen=True)
+class ConvWorkload:
+    """Synthetic inputs of the short causal convolution: x ~ N(0,1), taps
+    w ~ N(0, 1/K), boundary state ~ N(0,1) (or none), dy ~ N(0,1), boundary-state
+    gradient ~ N(0, 0.1) (or none)."""
+    name: str
+    B: int
+    H: int
+    T: int
+    d: int
+    K: int = 4
+    io: str = "bf16"
+    act: str = "silu"
+    with_state: bool = True
+    seed: int = 0
+
+    def with_(self, **kw) -> "ConvWorkload":
+        return replace(self, **kw)
+
+
+def make_conv_inputs(w: ConvWorkload) -> dict:
+    """Draw order: x, taps, conv_in, dy, dconv_out (CPU generator, fp32 draws)."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(w.seed)
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=gen, dtype=torch.float32)
+
+    x = randn(w.B, w.H, w.T, w.d)
+    taps = randn(w.H, w.d, w.K) / w.K ** 0.5
+    ci = randn(w.B, w.H, w.K - 1, w.d)
+    dy = randn(w.B, w.H, w.T, w.d)
+    dco = randn(w.B, w.H, w.K - 1, w.d) * 0.1
+    return {"x": _round_io(x, w.io), "w": taps.contiguous(),
+            "conv_in": _round_io(ci, w.io) if w.with_state else None,
+            "dy": _round_io(dy, w.io), "dconv_out": dco if w.with_state else None}

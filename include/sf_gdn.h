@@ -174,6 +174,62 @@ sf_status sf_gdn_fwd_noalloc(const sf_gdn_shape* shape, const void* q, const voi
                              const float* g, const float* beta, const float* S_in, void* o,
                              float* S_out, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Short causal convolution with a boundary state: the local-convolution state
+ * a sequence chunk hands to the next beside the recurrent state (StateFlow
+ * section 1: chunks must keep the boundary states of local convolution
+ * modules; section 3.3: the boundary tensor B_r holds recurrent and
+ * local-convolution boundary states).  The pages do not define the
+ * convolution; it is the causal depthwise short convolution that Gated
+ * DeltaNet-style layers apply per channel of q, k and v before the recurrence.
+ * Per (batch b, head h, channel c), with taps w[h][c][j] (tap j multiplies the
+ * input j steps back) and the extended input xe_p = conv_in[K-1+p] for p < 0,
+ * x_p otherwise:
+ *     pre_t = sum_j w_j xe_{t-j},  y_t = act(pre_t)  (act: identity or SiLU)
+ *     conv_out = xe_{T-K+1} .. xe_{T-1}   (the state handed to the next segment)
+ * The backward gives the gradients of sum_t <y_t, dy_t> + <conv_out, dconv_out>.
+ *
+ * Layouts: x, y, dy, dx [B,H,T,d] (I/O dtype); w, dw [H,d,K] fp32; conv_in,
+ * conv_out [B,H,K-1,d] (I/O dtype, oldest input first); dconv_out, dconv_in
+ * [B,H,K-1,d] fp32.  Pointers 8-byte aligned, the workspace 16-byte aligned;
+ * conv_out must not overlap x or conv_in.  Summation orders are fixed, so a
+ * sequence split into segments gives bit-identical y, conv_out, dx and
+ * dconv_in for any segment lengths, and a bit-identical dw when every segment
+ * length is a multiple of 64 (the weight gradient is folded per 64 tokens,
+ * from the last block to the first, continuing from dw_in). */
+typedef struct {
+    int B, H, T;   /* batch, heads, tokens (>= 0) */
+    int d;         /* channels per head: even, 2..1024 */
+    int K;         /* taps: 2..8 */
+    sf_dtype io;   /* dtype of x, y, dy, dx, conv_in, conv_out */
+    int act;       /* 0: identity, 1: SiLU */
+} sf_conv_shape;
+
+/* Workspace of sf_conv_bwd (0 when the shape is invalid). */
+size_t sf_conv_workspace_bytes(const sf_conv_shape* shape);
+
+/* Forward of one segment.  conv_in NULL = zeros (the start of a sequence);
+ * conv_out NULL = not written. */
+sf_status sf_conv_fwd(const sf_conv_shape* shape, const void* x, const float* w, const void* conv_in,
+                      void* y, void* conv_out, void* stream);
+
+/* Backward of one segment: dx (I/O dtype), dconv_in (fp32; NULL = not
+ * written) and dw_out = dw_in + this segment's weight gradient (dw_in NULL =
+ * zeros; dw_in == dw_out is allowed).  dconv_out NULL = zeros. */
+sf_status sf_conv_bwd(const sf_conv_shape* shape, const void* x, const float* w, const void* conv_in,
+                      const void* dy, const float* dconv_out, void* dx, const float* dw_in, float* dw_out,
+                      float* dconv_in, void* ws, size_t ws_bytes, void* stream);
+
+/* The segment chain of the convolution (as sf_segment_run for the recurrent
+ * state): forward over N segments with conv_out handed on as the next conv_in,
+ * then (dy != NULL) backward in reverse with dconv_in handed back as the
+ * previous dconv_out and the weight gradient accumulated into dw. */
+size_t sf_conv_segment_workspace_bytes(const sf_conv_shape* full, int N, const int* seg_len);
+sf_status sf_conv_segment_run(const sf_conv_shape* full, int N, const int* seg_len, const void* x,
+                              const float* w, const void* conv_in, const void* dy, const float* dconv_out,
+                              void* y, void* conv_out, void* dx, float* dw, float* dconv_in, void* ws,
+                              size_t ws_bytes, void* stream);
+
 /* Optional launch observer, for profiling.  When set, every kernel this
  * library launches is bracketed by hook(name, 0, stream, user) just before the
  * launch and hook(name, 1, stream, user) just after it, on the calling thread,
