@@ -37,7 +37,7 @@ STATUS_NAMES = ["SF_OK", "SF_ERR_INVALID_ARG", "SF_ERR_UNSUPPORTED", "SF_ERR_ALI
 EXPORTED_SYMBOLS = [
     "sf_status_str", "sf_last_cuda_error", "sf_gdn_fwd_workspace_bytes",
     "sf_gdn_bwd_workspace_bytes", "sf_gdn_fwd", "sf_gdn_bwd", "sf_segment_workspace_bytes",
-    "sf_segment_run", "sf_gdn_path", "sf_gdn_launches", "sf_set_launch_hook", "sf_gdn_fwd_noalloc",
+    "sf_segment_run", "sf_segment_min_workspace_bytes", "sf_gdn_path", "sf_gdn_launches", "sf_set_launch_hook", "sf_gdn_fwd_noalloc",
     "sf_device_check", "sf_timer_enable", "sf_timer_disable", "sf_timer_count", "sf_timer_read",
     "sf_timer_free", "sf_conv_workspace_bytes", "sf_conv_fwd", "sf_conv_bwd",
     "sf_conv_segment_workspace_bytes", "sf_conv_segment_run",
@@ -105,8 +105,9 @@ def lib():
         for name in ("sf_gdn_fwd_workspace_bytes", "sf_gdn_bwd_workspace_bytes"):
             getattr(L, name).argtypes = [SP]
             getattr(L, name).restype = ctypes.c_size_t
-        L.sf_segment_workspace_bytes.argtypes = [SP, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
-        L.sf_segment_workspace_bytes.restype = ctypes.c_size_t
+        for name in ("sf_segment_workspace_bytes", "sf_segment_min_workspace_bytes"):
+            getattr(L, name).argtypes = [SP, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+            getattr(L, name).restype = ctypes.c_size_t
         L.sf_gdn_fwd.argtypes = [SP] + [P] * 8 + [P, ctypes.c_size_t, P]
         L.sf_gdn_fwd.restype = ctypes.c_int
         L.sf_gdn_bwd.argtypes = [SP] + [P] * 14 + [P, ctypes.c_size_t, P]
@@ -183,8 +184,11 @@ def _seg_array(N, seg_len):
     return (ctypes.c_int * N)(*[int(x) for x in seg_len])
 
 
-def segment_workspace_bytes(shape: Shape, N: int, seg_len=None) -> int:
-    return int(lib().sf_segment_workspace_bytes(ctypes.byref(shape), int(N), _seg_array(N, seg_len)))
+def segment_workspace_bytes(shape: Shape, N: int, seg_len=None, bounded_memory=False) -> int:
+    """Workspace of segment_run: the fastest mode, or with bounded_memory the
+    mode that keeps only the boundary states and recomputes each segment."""
+    f = lib().sf_segment_min_workspace_bytes if bounded_memory else lib().sf_segment_workspace_bytes
+    return int(f(ctypes.byref(shape), int(N), _seg_array(N, seg_len)))
 
 
 def path(shape: Shape):
@@ -342,9 +346,11 @@ def bwd(q, k, v, g, beta, S_in, dO, dS_out=None, *, C=64, scale=1.0, out=None, w
 
 
 def segment_run(q, k, v, g, beta, S_in, dO, dS_out=None, *, N=1, seg_len=None, C=64, scale=1.0,
-                out=None, workspace=None, stream=None):
+                out=None, workspace=None, stream=None, bounded_memory=False):
     """Run the sequence as N segments in order with state handoff (forward), then
     in reverse with state-gradient handoff (backward, skipped when dO is None).
+    bounded_memory=True allocates only the bounded-memory workspace (boundary
+    states plus one segment); a caller workspace picks the mode by its size.
 
     Returns (o, S_out, grads) where grads is None when dO is None."""
     torch = _torch()
@@ -363,7 +369,7 @@ def segment_run(q, k, v, g, beta, S_in, dO, dS_out=None, *, N=1, seg_len=None, C
                                                                device=q.device),
                 "dS_in": torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)})
     segs = _seg_array(N, seg_len)
-    ws = _workspace(segment_workspace_bytes(shape, N, seg_len), q.device, workspace)
+    ws = _workspace(segment_workspace_bytes(shape, N, seg_len, bounded_memory), q.device, workspace)
     nbytes = 0 if ws is None else ws.numel()
     g_ = lambda name: _ptr(out.get(name)) if dO is not None else None
     _check(lib().sf_segment_run(ctypes.byref(shape), int(N), segs, _ptr(q), _ptr(k), _ptr(v),

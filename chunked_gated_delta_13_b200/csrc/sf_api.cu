@@ -557,14 +557,10 @@ sf_status sf_gdn_bwd(const sf_gdn_shape* s, const void* q, const void* k, const 
     return bwd_segment(*s, s->T, 0, s->T, a, ws, static_cast<cudaStream_t>(stream));
 }
 
-size_t sf_segment_workspace_bytes(const sf_gdn_shape* s, int N, const int* seg_len) {
-    if (check_shape(s) != SF_OK) return 0;
-    std::vector<int> lens;
-    if (!segment_lengths(*s, N, seg_len, lens)) return 0;
-    if (pick_path(*s) == Path::Tc) {
-        const PipeLayout L = pipe_layout(*s, pipe_pieces(lens));
-        return L.total + 256;
-    }
+// Workspace of the sequential chain: N+1 boundary states, two boundary state
+// gradients (ping-pong) and the per-call workspace of the longest segment.
+static size_t sequential_workspace_bytes(const sf_gdn_shape* s, const std::vector<int>& lens) {
+    const int N = (int)lens.size();
     size_t per = 0;
     for (int L : lens) {
         const size_t f = call_ws(*s, L, false), b = call_ws(*s, L, true);
@@ -575,6 +571,24 @@ size_t sf_segment_workspace_bytes(const sf_gdn_shape* s, int N, const int* seg_l
     // N+1 boundary states, two boundary state gradients (ping-pong), then the
     // per-segment workspace; every piece 256-byte aligned.
     return sf::align_up(nstate * sizeof(float), 256) * (size_t)(N + 3) + per + 256;
+}
+
+size_t sf_segment_workspace_bytes(const sf_gdn_shape* s, int N, const int* seg_len) {
+    if (check_shape(s) != SF_OK) return 0;
+    std::vector<int> lens;
+    if (!segment_lengths(*s, N, seg_len, lens)) return 0;
+    if (pick_path(*s) == Path::Tc) {
+        const PipeLayout L = pipe_layout(*s, pipe_pieces(lens));
+        return L.total + 256;
+    }
+    return sequential_workspace_bytes(s, lens);
+}
+
+size_t sf_segment_min_workspace_bytes(const sf_gdn_shape* s, int N, const int* seg_len) {
+    if (check_shape(s) != SF_OK) return 0;
+    std::vector<int> lens;
+    if (!segment_lengths(*s, N, seg_len, lens)) return 0;
+    return sequential_workspace_bytes(s, lens);
 }
 
 sf_status sf_segment_run(const sf_gdn_shape* s, int N, const int* seg_len, const void* q,
@@ -592,12 +606,16 @@ sf_status sf_segment_run(const sf_gdn_shape* s, int N, const int* seg_len, const
         st = check_bwd_ptrs(*s, q, k, v, g, beta, S_in, dO, dS_out, dq, dk, dv, dg, dbeta, dS_in);
         if (st != SF_OK) return st;
     }
-    const size_t need = sf_segment_workspace_bytes(s, N, seg_len);
-    st = check_ws(need, ws, ws_bytes);
+    // the pipelined chain when the workspace holds every segment's forward
+    // intermediates, else the sequential chain (boundary states only, each
+    // segment's backward recomputing its forward)
+    const size_t need_min = sf_segment_min_workspace_bytes(s, N, seg_len);
+    const bool pipelined = pick_path(*s) == Path::Tc && ws_bytes >= sf_segment_workspace_bytes(s, N, seg_len);
+    st = check_ws(need_min, ws, ws_bytes);
     if (st != SF_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (s->B * s->H == 0) return SF_OK;
-    if (pick_path(*s) == Path::Tc) {
+    if (pipelined) {
         char* b = reinterpret_cast<char*>(sf::align_up(reinterpret_cast<uintptr_t>(ws), 256));
         const sf::FwdArgs F{q, k, v, g, beta, S_in, o, S_out};
         const sf::BwdArgs B{q, k, v, g, beta, S_in, dO, dS_out, dq, dk, dv, dg, dbeta, dS_in};

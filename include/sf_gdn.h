@@ -112,7 +112,10 @@ sf_status sf_gdn_bwd(const sf_gdn_shape* shape, const void* q, const void* k, co
 
 /* Workspace for sf_segment_run.  seg_len: host array of N lengths summing to
  * shape->T, or NULL for the equal split (the first T % N segments one token
- * longer).  Two cases:
+ * longer).  sf_segment_workspace_bytes gives the size of the fastest mode,
+ * sf_segment_min_workspace_bytes the size of the bounded-memory mode;
+ * sf_segment_run picks the fastest mode the workspace it is given allows.
+ * Two cases for the fastest mode:
  *  - tensor-core path (bf16 I/O, dk = 128, dv in {64, 128}, C = 64): the
  *    pipelined chain keeps every segment's forward intermediates for its
  *    backward, so the workspace grows with T: 8 + 4 dk + 4 C + 6 dv +
@@ -123,6 +126,18 @@ sf_status sf_gdn_bwd(const sf_gdn_shape* shape, const void* q, const void* k, co
  *    fp32 boundary states and two boundary state gradients. */
 size_t sf_segment_workspace_bytes(const sf_gdn_shape* full, int N, const int* seg_len);
 
+/* Bounded-memory mode of sf_segment_run (StateFlow section 3.1: each chunk's
+ * activations are released after its backward; section 3.3: the retained
+ * activation is bounded by the boundary states plus one chunk): the N+1 fp32
+ * boundary states, two boundary state gradients and the workspace of one
+ * sf_gdn_bwd call on the longest segment.  With a workspace of at least this
+ * size but less than sf_segment_workspace_bytes, sf_segment_run runs the
+ * segments one after another, each backward recomputing its forward from the
+ * saved boundary state; the results are bit-identical to the pipelined mode.
+ * At B=1, H=16, d=128 in 16 segments: 0.24 GB instead of 2.9 GB at T = 65536,
+ * 0.89 GB instead of 11.0 GB at T = 262144. */
+size_t sf_segment_min_workspace_bytes(const sf_gdn_shape* full, int N, const int* seg_len);
+
 /* The segment chain on one GPU (StateFlow section 3.1): split the sequence of
  * `full` into N segments, run the forward on segments 0..N-1 with each S_out
  * handed on as the next S_in, then (when dO != NULL) the backward on segments
@@ -132,7 +147,8 @@ size_t sf_segment_workspace_bytes(const sf_gdn_shape* full, int N, const int* se
  * boundary states stay fp32 on the device, so when every segment length is a
  * multiple of C the results are bit-identical to N = 1.
  *
- * On the tensor-core path the chain is pipelined (StateFlow section 3.4, the
+ * On the tensor-core path, given the workspace of sf_segment_workspace_bytes,
+ * the chain is pipelined (StateFlow section 3.4, the
  * split-and-overlap of the state scan with the chunk-parallel kernels):
  * segments are further cut into pieces of 4096 tokens at chunk boundaries
  * (this changes no result); the state scans of consecutive pieces run in

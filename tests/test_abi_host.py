@@ -181,3 +181,19 @@ def test_timer_api_without_launches():
     assert L.sf_timer_read(0, ctypes.byref(name), ctypes.byref(ms)) == 1
     L.sf_timer_disable()
     L.sf_timer_free()
+
+
+def test_bounded_memory_workspace():
+    """The bounded-memory chain needs the boundary states plus one segment's
+    backward workspace: far less than the pipelined chain on the tensor-core
+    path, the same on the CUDA-core path (which always runs sequentially)."""
+    tc = sf.make_shape(1, 16, 65536, 128, 128, 64, "bf16")
+    full = sf.segment_workspace_bytes(tc, 16)
+    small = sf.segment_workspace_bytes(tc, 16, bounded_memory=True)
+    one = sf.bwd_workspace_bytes(sf.make_shape(1, 16, 4096, 128, 128, 64, "bf16"))
+    state = 16 * 128 * 128 * 4
+    assert small == 19 * state + one + 256
+    assert small * 10 < full
+    simt = sf.make_shape(1, 2, 256, 64, 64, 64, "f32")
+    assert sf.segment_workspace_bytes(simt, 2) == sf.segment_workspace_bytes(simt, 2, bounded_memory=True)
+    assert sf.lib().sf_segment_min_workspace_bytes(ctypes.byref(tc), 0, None) == 0

@@ -14,9 +14,9 @@ pytestmark = pytest.mark.gpu
 TOL_BF16 = 2e-2
 
 
-def _run_segments(d, C, N):
+def _run_segments(d, C, N, seg_len=None):
     o, S_out, gr = sf.segment_run(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S_in"], d["dO"],
-                                  d["dS_out"], N=N, C=C)
+                                  d["dS_out"], N=N, seg_len=seg_len, C=C)
     torch.cuda.synchronize()
     sf.device_check()
     out = {"o": o, "S_out": S_out}
@@ -88,3 +88,43 @@ def test_native_launch_timer():
     names = [n for n, _ in rec]
     assert names == ["tc_prep", "tc_scan_fwd", "tc_out_og", "tc_scan_bwd", "tc_grad"], names
     assert all(ms > 0 for _, ms in rec)
+
+
+@pytest.mark.parametrize("dv,beta,T,N", [(128, True, 6 * 64, 2), (64, False, 5 * 64 + 40, 3),
+                                         (128, True, 9000, 3)])
+def test_bounded_memory_chain_bit_identical(dv, beta, T, N):
+    """The bounded-memory mode (boundary states only, each segment's backward
+    recomputing its forward) gives the same bits as the pipelined mode."""
+    w = Workload(name="bounded", B=1, H=3, T=T, dk=128, dv=dv, C=64, io="bf16", use_beta=beta,
+                 S_in_std=0.05, dS_out_std=0.1, g_shift=-4.0)
+    d = to_device(make_inputs(w))
+    seg = [T // N // 64 * 64] * (N - 1)
+    seg.append(T - sum(seg))
+    a = _run_segments(d, w.C, N, seg_len=seg)
+    o, S_out, gr = sf.segment_run(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S_in"], d["dO"],
+                                  d["dS_out"], N=N, seg_len=seg, C=w.C, bounded_memory=True)
+    torch.cuda.synchronize()
+    sf.device_check()
+    b = {"o": o, "S_out": S_out}
+    b.update(gr)
+    for name, x in b.items():
+        if x is None:
+            assert a.get(name) is None, name
+            continue
+        assert torch.equal(a[name], x), name
+
+
+def test_bounded_memory_headline_chain():
+    """The headline chain (B=1, H=16, T=65536, d=128, 16 segments) in the
+    bounded-memory mode: bit-identical to the pipelined mode."""
+    w = CONFIGS["headline_h16_t64k"].with_(S_in_std=0.02, g_mode="softplus", g_shift=-4.0)
+    d = to_device(make_inputs(w))
+    a = _run_segments(d, w.C, 16)
+    o, S_out, gr = sf.segment_run(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S_in"], d["dO"],
+                                  d["dS_out"], N=16, C=w.C, bounded_memory=True)
+    torch.cuda.synchronize()
+    sf.device_check()
+    assert torch.equal(a["o"], o) and torch.equal(a["S_out"], S_out)
+    for name, x in gr.items():
+        if x is not None:
+            assert torch.equal(a[name], x), name
