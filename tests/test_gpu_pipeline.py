@@ -128,3 +128,38 @@ def test_bounded_memory_headline_chain():
     for name, x in gr.items():
         if x is not None:
             assert torch.equal(a[name], x), name
+
+
+def test_rank_pipeline_cuda_stage_single_rank():
+    """The multi-rank sequence pipeline with the CUDA segment arithmetic, on the
+    one GPU a run here has (world size 1, NCCL): every microbatch's outputs are
+    bit-identical to the standalone calls.  Two or more ranks are covered on the
+    CPU (gloo, oracle arithmetic) in the host tests."""
+    import datetime
+    import os
+
+    import torch.distributed as dist
+
+    from chunked_gated_delta_13_b200 import pipeline
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29517")
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        segs, refs = [], []
+        for a in range(2):
+            w = Workload(name="ranks", B=1, H=2, T=5 * 64 + 9, dk=128, dv=128, C=64, io="bf16",
+                         S_in_std=0.05, dS_out_std=0.1, g_shift=-4.0, seed=a)
+            d = to_device(make_inputs(w))
+            segs.append(pipeline.SegmentData(q=d["q"], k=d["k"], v=d["v"], g=d["g"], beta=d["beta"], dO=d["dO"],
+                                             S_in=d["S_in"], dS_out=d["dS_out"]))
+            refs.append(_run_calls(d, 64))
+        res = pipeline.run_pipeline(pipeline.CudaStage(C=64), segs)
+        torch.cuda.synchronize()
+        for r, ref in zip(res, refs):
+            assert torch.equal(r["o"], ref["o"]) and torch.equal(r["S_out"], ref["S_out"])
+            for name in ("dq", "dk", "dv", "dg", "dbeta", "dS_in"):
+                assert torch.equal(r["grads"][name], ref[name]), name
+            assert torch.equal(r["dS_in"], ref["dS_in"])
+    finally:
+        dist.destroy_process_group()
