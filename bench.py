@@ -132,11 +132,11 @@ def step_roofline(w, ms, pk):
 # times its chunk-heads.  Valid for the kernels as they were when
 # captured; an entry is removed when its kernel changes.
 MEASURED_TRAFFIC = {
-    "tc_prep": 45850.0,
-    "tc_scan_fwd": 59810.0,
-    "tc_out_og": 123471.0,
-    "tc_scan_bwd": 103061.0,
-    "tc_grad": 208855.0,
+    "tc_prep": 47729.0,
+    "tc_scan_fwd": 60554.0,
+    "tc_out_og": 123065.0,
+    "tc_scan_bwd": 103362.0,
+    "tc_grad": 209383.0,
 }
 
 
@@ -149,11 +149,14 @@ def dist_env():
     return ws, rank, local
 
 
-def rank_workload(name, rank):
+def rank_workload(name, rank, chunk=0):
     """Replicas: every rank runs its own independent batch, the named workload
-    with the seed offset by the rank (no data crosses ranks)."""
+    with the seed offset by the rank (no data crosses ranks); `chunk` > 0
+    overrides the kernel chunk length."""
     from chunked_gated_delta_13_b200.inputs import CONFIGS
     w = CONFIGS[name]
+    if chunk:
+        w = w.with_(C=chunk)
     return w.with_(seed=w.seed + rank)
 
 
@@ -273,6 +276,8 @@ def run_reference(args):
     from chunked_gated_delta_13_b200.inputs import CONFIGS, as_f64, make_inputs
 
     w = CONFIGS[args.workload]
+    if args.chunk:
+        w = w.with_(C=args.chunk)
     seg = args.segments if args.segments else w.N
     budget_s = float(os.environ.get("SF_REF_STEP_SECONDS", "1.5"))
 
@@ -361,7 +366,7 @@ def run_ours(args):
         dist.init_process_group("nccl", rank=rank, world_size=ws,
                                 timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    w = rank_workload(args.workload, rank)
+    w = rank_workload(args.workload, rank, args.chunk)
     seg = args.segments if args.segments else w.N
     inp_cpu = make_inputs(w)
     d = {k: None if v is None else v.to(dev).contiguous() for k, v in inp_cpu.items()}
@@ -497,7 +502,7 @@ def run_ours(args):
     if rank == 0:
         cpu = None
         if ws == 1 and not args.no_cpu_baseline:
-            cpu = cpu_baseline(CONFIGS[args.workload], seg)
+            cpu = cpu_baseline(w.with_(seed=CONFIGS[args.workload].seed), seg)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -530,6 +535,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--segments", type=int, default=DEFAULT_SEGMENTS)
+    ap.add_argument("--chunk", type=int, default=0, help="kernel chunk length C (0 = the workload's)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

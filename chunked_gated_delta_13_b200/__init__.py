@@ -12,6 +12,8 @@ Entry points mirror the C ABI in ``include/sf_gdn.h``:
   segment_run(..., N or seg_len)                    -> (o, S_out, gradients)
   conv_fwd / conv_bwd / conv_segment_run            the short causal convolution
                                                     with its boundary state
+  kda_fwd / kda_bwd                                 the delta rule with a per-channel
+                                                    (diagonal) decay
 The operations are StateFlow's chunk Fwd/Bwd and its sequence split with the
 state handed forward and the state gradient handed backward (arXiv 2608.06838,
 sections 2.1 and 3.1).
@@ -24,7 +26,7 @@ import threading
 
 from ._build import LIB, build, needs_build
 
-__all__ = ["Shape", "ConvShape", "make_conv_shape", "conv_fwd", "conv_bwd", "conv_segment_run", "SFError", "lib", "fwd", "bwd", "segment_run", "make_shape", "path", "device_check",
+__all__ = ["Shape", "ConvShape", "KdaShape", "kda_fwd", "kda_bwd", "make_conv_shape", "conv_fwd", "conv_bwd", "conv_segment_run", "SFError", "lib", "fwd", "bwd", "segment_run", "make_shape", "path", "device_check",
            "launches", "set_launch_hook", "timer_enable", "timer_disable", "timer_count", "timer_results", "timer_free",
            "fwd_workspace_bytes", "bwd_workspace_bytes", "segment_workspace_bytes",
            "EXPORTED_SYMBOLS"]
@@ -40,7 +42,8 @@ EXPORTED_SYMBOLS = [
     "sf_segment_run", "sf_segment_min_workspace_bytes", "sf_gdn_path", "sf_gdn_launches", "sf_set_launch_hook", "sf_gdn_fwd_noalloc",
     "sf_device_check", "sf_timer_enable", "sf_timer_disable", "sf_timer_count", "sf_timer_read",
     "sf_timer_free", "sf_conv_workspace_bytes", "sf_conv_fwd", "sf_conv_bwd",
-    "sf_conv_segment_workspace_bytes", "sf_conv_segment_run",
+    "sf_conv_segment_workspace_bytes", "sf_conv_segment_run", "sf_kda_workspace_bytes", "sf_kda_fwd",
+    "sf_kda_bwd",
 ]
 
 HOOK_T = ctypes.CFUNCTYPE(None, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p)
@@ -57,6 +60,12 @@ class ConvShape(ctypes.Structure):
     """Mirror of ``sf_conv_shape``."""
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("d", ctypes.c_int),
                 ("K", ctypes.c_int), ("io", ctypes.c_int), ("act", ctypes.c_int)]
+
+
+class KdaShape(ctypes.Structure):
+    """Mirror of ``sf_kda_shape``."""
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("dk", ctypes.c_int),
+                ("dv", ctypes.c_int), ("io", ctypes.c_int), ("use_beta", ctypes.c_int), ("scale", ctypes.c_float)]
 
 
 class SFError(RuntimeError):
@@ -147,6 +156,13 @@ def lib():
         L.sf_conv_segment_run.argtypes = ([CP, ctypes.c_int, ctypes.POINTER(ctypes.c_int)] + [P] * 10
                                           + [P, ctypes.c_size_t, P])
         L.sf_conv_segment_run.restype = ctypes.c_int
+        KP = ctypes.POINTER(KdaShape)
+        L.sf_kda_workspace_bytes.argtypes = [KP, ctypes.c_int]
+        L.sf_kda_workspace_bytes.restype = ctypes.c_size_t
+        L.sf_kda_fwd.argtypes = [KP] + [P] * 8 + [P]
+        L.sf_kda_fwd.restype = ctypes.c_int
+        L.sf_kda_bwd.argtypes = [KP] + [P] * 14 + [P, ctypes.c_size_t, P]
+        L.sf_kda_bwd.restype = ctypes.c_int
         _lib = L
         return _lib
 
@@ -460,3 +476,43 @@ def conv_segment_run(x, w, conv_in, dy, dconv_out=None, *, N=1, seg_len=None, ac
                                      _ptr(conv_out), g_("dx"), g_("dw"), g_("dconv_in"), _ptr(ws),
                                      ws.numel(), _stream(stream)))
     return y, conv_out, grads
+
+
+# ------------------------------------------------ per-channel decay glue ---
+
+def _kda_shape_of(q, v, beta, scale):
+    B, H, T, dk = q.shape
+    return KdaShape(B, H, T, dk, v.shape[-1], SF_BF16 if _io_of(q) == "bf16" else SF_F32,
+                    int(beta is not None), float(scale))
+
+
+def kda_fwd(q, k, v, g, beta=None, S_in=None, *, scale=1.0, stream=None):
+    """Forward of the delta rule with a per-channel decay; g: [B,H,T,dk] fp32.
+    Returns (o, S_out)."""
+    torch = _torch()
+    _need_cuda(q, k, v, g, beta, S_in)
+    shape = _kda_shape_of(q, v, beta, scale)
+    B, H, T, dk = q.shape
+    o = torch.empty(B, H, T, v.shape[-1], dtype=q.dtype, device=q.device)
+    S_out = torch.empty(B, H, dk, v.shape[-1], dtype=torch.float32, device=q.device)
+    _check(lib().sf_kda_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S_in),
+                            _ptr(o), _ptr(S_out), _stream(stream)))
+    return o, S_out
+
+
+def kda_bwd(q, k, v, g, beta, S_in, dO, dS_out=None, *, scale=1.0, workspace=None, stream=None):
+    """Backward: dict dq, dk, dv, dg ([B,H,T,dk] fp32), dbeta, dS_in."""
+    torch = _torch()
+    _need_cuda(q, k, v, g, beta, S_in, dO, dS_out)
+    shape = _kda_shape_of(q, v, beta, scale)
+    B, H, T, dk = q.shape
+    out = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+           "dg": torch.empty_like(g), "dbeta": None if beta is None else torch.empty_like(beta),
+           "dS_in": torch.empty(B, H, dk, v.shape[-1], dtype=torch.float32, device=q.device)}
+    ws = _workspace(int(lib().sf_kda_workspace_bytes(ctypes.byref(shape), 1)), q.device, workspace)
+    nbytes = 0 if ws is None else ws.numel()
+    _check(lib().sf_kda_bwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S_in),
+                            _ptr(dO), _ptr(dS_out), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                            _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["dS_in"]), _ptr(ws), nbytes,
+                            _stream(stream)))
+    return out

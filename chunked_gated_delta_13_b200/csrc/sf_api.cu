@@ -588,7 +588,10 @@ size_t sf_segment_min_workspace_bytes(const sf_gdn_shape* s, int N, const int* s
     if (check_shape(s) != SF_OK) return 0;
     std::vector<int> lens;
     if (!segment_lengths(*s, N, seg_len, lens)) return 0;
-    return sequential_workspace_bytes(s, lens);
+    const size_t seq = sequential_workspace_bytes(s, lens);
+    if (pick_path(*s) != Path::Tc) return seq;
+    const size_t pipe = sf_segment_workspace_bytes(s, N, seg_len);
+    return pipe < seq ? pipe : seq;
 }
 
 sf_status sf_segment_run(const sf_gdn_shape* s, int N, const int* seg_len, const void* q,
@@ -609,9 +612,9 @@ sf_status sf_segment_run(const sf_gdn_shape* s, int N, const int* seg_len, const
     // the pipelined chain when the workspace holds every segment's forward
     // intermediates, else the sequential chain (boundary states only, each
     // segment's backward recomputing its forward)
-    const size_t need_min = sf_segment_min_workspace_bytes(s, N, seg_len);
     const bool pipelined = pick_path(*s) == Path::Tc && ws_bytes >= sf_segment_workspace_bytes(s, N, seg_len);
-    st = check_ws(need_min, ws, ws_bytes);
+    st = check_ws(pipelined ? sf_segment_workspace_bytes(s, N, seg_len) : sequential_workspace_bytes(s, lens), ws,
+                  ws_bytes);
     if (st != SF_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (s->B * s->H == 0) return SF_OK;

@@ -165,3 +165,37 @@ def make_conv_inputs(w: ConvWorkload) -> dict:
     return {"x": _round_io(x, w.io), "w": taps.contiguous(),
             "conv_in": _round_io(ci, w.io) if w.with_state else None,
             "dy": _round_io(dy, w.io), "dconv_out": dco if w.with_state else None}
+
+
+def make_kda_inputs(w: Workload) -> dict:
+    """Inputs of the per-channel-decay variant: as make_inputs, with the
+    log-decay drawn per key channel, g = -softplus(N(0,1) + g_shift) of shape
+    [B,H,T,dk] (g_mode "zero": all zeros).  Draw order: q, k, v, beta-logits,
+    g-logits, S_in, dO, dS_out."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(w.seed)
+    B, H, T, dk, dv = w.B, w.H, w.T, w.dk, w.dv
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=gen, dtype=torch.float32)
+
+    q = randn(B, H, T, dk)
+    k = randn(B, H, T, dk)
+    if w.qk == "l2norm":
+        q = q / q.norm(dim=-1, keepdim=True).clamp_min(1e-12)
+        k = k / k.norm(dim=-1, keepdim=True).clamp_min(1e-12)
+    else:
+        q = q / dk ** 0.5
+        k = k / dk ** 0.5
+    v = randn(B, H, T, dv)
+    beta_logit = randn(B, H, T)
+    g_logit = randn(B, H, T, dk)
+    beta = torch.sigmoid(beta_logit) if w.use_beta else None
+    g = (-torch.nn.functional.softplus(g_logit + w.g_shift) if w.g_mode == "softplus"
+         else torch.zeros(B, H, T, dk))
+    S_in = randn(B, H, dk, dv) * w.S_in_std if w.S_in_std > 0 else None
+    dO = randn(B, H, T, dv)
+    dS_out = randn(B, H, dk, dv) * w.dS_out_std if w.dS_out_std > 0 else None
+    return {"q": _round_io(q, w.io), "k": _round_io(k, w.io), "v": _round_io(v, w.io),
+            "g": g.contiguous(), "beta": None if beta is None else beta.contiguous(),
+            "S_in": S_in, "dO": _round_io(dO, w.io), "dS_out": dS_out}

@@ -113,7 +113,7 @@ sf_status sf_gdn_bwd(const sf_gdn_shape* shape, const void* q, const void* k, co
 /* Workspace for sf_segment_run.  seg_len: host array of N lengths summing to
  * shape->T, or NULL for the equal split (the first T % N segments one token
  * longer).  sf_segment_workspace_bytes gives the size of the fastest mode,
- * sf_segment_min_workspace_bytes the size of the bounded-memory mode;
+ * sf_segment_min_workspace_bytes the smallest size the call accepts;
  * sf_segment_run picks the fastest mode the workspace it is given allows.
  * Two cases for the fastest mode:
  *  - tensor-core path (bf16 I/O, dk = 128, dv in {64, 128}, C = 64): the
@@ -130,10 +130,13 @@ size_t sf_segment_workspace_bytes(const sf_gdn_shape* full, int N, const int* se
  * activations are released after its backward; section 3.3: the retained
  * activation is bounded by the boundary states plus one chunk): the N+1 fp32
  * boundary states, two boundary state gradients and the workspace of one
- * sf_gdn_bwd call on the longest segment.  With a workspace of at least this
- * size but less than sf_segment_workspace_bytes, sf_segment_run runs the
+ * sf_gdn_bwd call on the longest segment.  Given a workspace below
+ * sf_segment_workspace_bytes but at least this size, sf_segment_run runs the
  * segments one after another, each backward recomputing its forward from the
  * saved boundary state; the results are bit-identical to the pipelined mode.
+ * sf_segment_min_workspace_bytes returns the smaller of this size and the
+ * pipelined one (a single long segment needs less in the pipelined mode, which
+ * works in pieces of 4096 tokens).
  * At B=1, H=16, d=128 in 16 segments: 0.24 GB instead of 2.9 GB at T = 65536,
  * 0.89 GB instead of 11.0 GB at T = 262144. */
 size_t sf_segment_min_workspace_bytes(const sf_gdn_shape* full, int N, const int* seg_len);
@@ -245,6 +248,42 @@ sf_status sf_conv_segment_run(const sf_conv_shape* full, int N, const int* seg_l
                               const float* w, const void* conv_in, const void* dy, const float* dconv_out,
                               void* y, void* conv_out, void* dx, float* dw, float* dconv_in, void* ws,
                               size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Delta rule with a per-channel (diagonal) decay: the diagonal-plus-low-rank
+ * transition StateFlow lists beside the scalar-plus-low-rank one (section 2.1:
+ * Kimi Delta Attention), in this library's state orientation:
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp(g_t)) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = scale * S_t^T q_t     (use_beta = 0: S_t = Diag(exp(g_t)) S_{t-1} + k_t v_t^T)
+ * with a log-decay g_t per key channel.  Same layouts as sf_gdn_* except
+ * g, dg: [B,H,T,dk] fp32.  With every channel's log-decay equal this is the
+ * sf_gdn_* layer.  The computation is fp32 token by token on the CUDA cores
+ * (see csrc/kda_kernels.cu), so splitting a sequence at any token gives
+ * bit-identical results.  dk in {32, 64, 128}; dv a multiple of 32 up to 1024;
+ * pointers 16-byte aligned. */
+typedef struct {
+    int B, H, T;
+    int dk, dv;
+    sf_dtype io;
+    int use_beta;
+    float scale;
+} sf_kda_shape;
+
+/* Workspace bytes: forward (backward = 0) needs none; the backward holds a
+ * checkpoint every 64 tokens, a window scratch per CTA and the per-column-block
+ * partial sums (at B=1, H=16, T=65536, dk=dv=128: about 6.5 GB). */
+size_t sf_kda_workspace_bytes(const sf_kda_shape* shape, int backward);
+
+/* Forward of one segment: o, and S_out (NULL = not written); S_in NULL = zeros. */
+sf_status sf_kda_fwd(const sf_kda_shape* shape, const void* q, const void* k, const void* v, const float* g,
+                     const float* beta, const float* S_in, void* o, float* S_out, void* stream);
+
+/* Backward of one segment: gradients of sum <o, dO> + <S_out, dS_out>; dS_in
+ * NULL = not written; dS_out NULL = zeros. */
+sf_status sf_kda_bwd(const sf_kda_shape* shape, const void* q, const void* k, const void* v, const float* g,
+                     const float* beta, const float* S_in, const void* dO, const float* dS_out, void* dq,
+                     void* dk, void* dv, float* dg, float* dbeta, float* dS_in, void* ws, size_t ws_bytes,
+                     void* stream);
 
 /* Optional launch observer, for profiling.  When set, every kernel this
  * library launches is bracketed by hook(name, 0, stream, user) just before the
