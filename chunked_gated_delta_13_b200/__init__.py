@@ -27,7 +27,7 @@ import threading
 from ._build import LIB, build, needs_build
 
 __all__ = ["Shape", "ConvShape", "KdaShape", "kda_fwd", "kda_bwd", "make_conv_shape", "conv_fwd", "conv_bwd", "conv_segment_run", "SFError", "lib", "fwd", "bwd", "segment_run", "make_shape", "path", "device_check",
-           "launches", "set_launch_hook", "timer_enable", "timer_disable", "timer_count", "timer_results", "timer_free",
+           "launches", "set_launch_hook", "timer_enable", "timer_disable", "timer_count", "timer_results", "timer_timeline", "timer_free",
            "fwd_workspace_bytes", "bwd_workspace_bytes", "segment_workspace_bytes",
            "EXPORTED_SYMBOLS"]
 
@@ -41,7 +41,7 @@ EXPORTED_SYMBOLS = [
     "sf_gdn_bwd_workspace_bytes", "sf_gdn_fwd", "sf_gdn_bwd", "sf_segment_workspace_bytes",
     "sf_segment_run", "sf_segment_min_workspace_bytes", "sf_gdn_path", "sf_gdn_launches", "sf_set_launch_hook", "sf_gdn_fwd_noalloc",
     "sf_device_check", "sf_timer_enable", "sf_timer_disable", "sf_timer_count", "sf_timer_read",
-    "sf_timer_free", "sf_conv_workspace_bytes", "sf_conv_fwd", "sf_conv_bwd",
+    "sf_timer_free", "sf_timer_read_at", "sf_conv_workspace_bytes", "sf_conv_fwd", "sf_conv_bwd",
     "sf_conv_segment_workspace_bytes", "sf_conv_segment_run", "sf_kda_workspace_bytes", "sf_kda_fwd",
     "sf_kda_bwd",
 ]
@@ -142,6 +142,9 @@ def lib():
         L.sf_timer_count.restype = ctypes.c_int
         L.sf_timer_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float)]
         L.sf_timer_read.restype = ctypes.c_int
+        L.sf_timer_read_at.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_char_p),
+                                       ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]
+        L.sf_timer_read_at.restype = ctypes.c_int
         L.sf_timer_free.argtypes = []
         L.sf_timer_free.restype = None
         CP = ctypes.POINTER(ConvShape)
@@ -257,6 +260,19 @@ def timer_results():
     for i in range(lib().sf_timer_count()):
         _check(lib().sf_timer_read(i, ctypes.byref(name), ctypes.byref(ms)))
         out.append((name.value.decode(), float(ms.value)))
+    return out
+
+
+def timer_timeline():
+    """[(kernel_name, start_ms, ms)] of the recorded launches, starts relative to
+    the first launch's start (waits for them)."""
+    out = []
+    name = ctypes.c_char_p()
+    t0 = ctypes.c_float()
+    ms = ctypes.c_float()
+    for i in range(lib().sf_timer_count()):
+        _check(lib().sf_timer_read_at(i, ctypes.byref(name), ctypes.byref(t0), ctypes.byref(ms)))
+        out.append((name.value.decode(), float(t0.value), float(ms.value)))
     return out
 
 

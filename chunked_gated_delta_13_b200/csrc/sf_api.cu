@@ -498,6 +498,16 @@ sf_status sf_timer_read(int i, const char** kernel, float* ms) {
     return SF_OK;
 }
 
+sf_status sf_timer_read_at(int i, const char** kernel, float* start_ms, float* ms) {
+    if (i < 0 || i >= g_timer.used || !kernel || !start_ms || !ms) return SF_ERR_INVALID_ARG;
+    cudaError_t e = cudaEventSynchronize(g_timer.end[i]);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(ms, g_timer.begin[i], g_timer.end[i]);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(start_ms, g_timer.begin[0], g_timer.begin[i]);
+    if (e != cudaSuccess) return cuda_fail(e);
+    *kernel = g_timer.name[i];
+    return SF_OK;
+}
+
 void sf_timer_free(void) { g_timer.destroy(); }
 
 void sf_set_launch_hook(sf_launch_hook hook, void* user) {

@@ -308,6 +308,9 @@ sf_status sf_timer_enable(int capacity);
 void sf_timer_disable(void);
 int sf_timer_count(void);
 sf_status sf_timer_read(int i, const char** kernel, float* ms);
+/* As sf_timer_read, plus the launch's start relative to the first recorded
+ * launch's start (a timeline of the recorded launches). */
+sf_status sf_timer_read_at(int i, const char** kernel, float* start_ms, float* ms);
 void sf_timer_free(void);
 
 /* Introspection for tests and benchmarks: the kernel family a shape runs on
