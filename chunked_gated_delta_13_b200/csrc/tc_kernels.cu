@@ -1753,10 +1753,6 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     umma::fence_after();
     const uint32_t tm = *tslot;
     const uint32_t trow = umma::taddr(tm, 32 * mw, 0);  // this warp's lane quarter
-    auto chain = [&](uint32_t col, uint32_t idesc, int nks, bool acc, auto da, auto db) {
-#pragma unroll 1
-        for (int ks = 0; ks < nks; ++ks) umma::mma(tm + col, da(ks), db(ks), idesc, acc || ks > 0);
-    };
     constexpr uint32_t I64kk = umma::idesc_bf16(64, 64, false, false);
     constexpr uint32_t I64km = umma::idesc_bf16(64, 64, false, true);
     constexpr uint32_t I64mk = umma::idesc_bf16(64, 64, true, false);
@@ -1793,13 +1789,10 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     const bool has_next = jn < total;
     if (tid == 0) {  // Q K^T, K K^T, dP = dO V_new^T
         umma::fence_after();
-        chain(L5::QK, I64kk, 8, false, [&](int ks) { return umma::desc_k(Qc, ks, 128); },
-              [&](int ks) { return umma::desc_k(Kc, ks, 128); });
+        umma::chain<8>(tm + L5::QK, I64kk, false, umma::op_k(Qc, 128), umma::op_k(Kc, 128));
         if (BETA)
-            chain(L5::KK, I64kk, 8, false, [&](int ks) { return umma::desc_k(Kc, ks, 128); },
-                  [&](int ks) { return umma::desc_k(Kc, ks, 128); });
-        chain(L5::DP, I64km, DV / 16, false, [&](int ks) { return umma::desc_k(dOc, ks, DV); },
-              [&](int ks) { return umma::desc_mn(Vnc, ks, C); });
+            umma::chain<8>(tm + L5::KK, I64kk, false, umma::op_k(Kc, 128), umma::op_k(Kc, 128));
+        umma::chain<DV / 16>(tm + L5::DP, I64km, false, umma::op_k(dOc, DV), umma::op_mn(Vnc, C));
         umma::commit(&bm[0]);
     }
     if (has_next) copy_qkg(jn, buf ^ 1);  // the other buffer's chunk is done
@@ -1809,11 +1802,9 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     mbar_wait(bdVn, par, &g_tc_status, failed);
     if (tid == 0) {  // dO S0^T, dV_new S0^T
         umma::fence_after();
-        chain(L5::DQ, I128km, DV / 16, false, [&](int ks) { return umma::desc_k(dOc, ks, DV); },
-              [&](int ks) { return umma::desc_mn(S0c, ks, 128); });
+        umma::chain<DV / 16>(tm + L5::DQ, I128km, false, umma::op_k(dOc, DV), umma::op_mn(S0c, 128));
         if (BETA)
-            chain(L5::DW, I128mm, DV / 16, false, [&](int ks) { return umma::desc_mn(dVnc, ks, C); },
-                  [&](int ks) { return umma::desc_mn(S0c, ks, 128); });
+            umma::chain<DV / 16>(tm + L5::DW, I128mm, false, umma::op_mn(dVnc, C), umma::op_mn(S0c, 128));
         umma::commit(&bm[1]);
     }
 
@@ -1870,8 +1861,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     sync_for_mma();
     if (tid == 0) {  // V_new dS_C^T
         umma::fence_after();
-        chain(L5::DKC, I128mm, DV / 16, false, [&](int ks) { return umma::desc_mn(Vnc, ks, C); },
-              [&](int ks) { return umma::desc_mn(dSc, ks, 128); });
+        umma::chain<DV / 16>(tm + L5::DKC, I128mm, false, umma::op_mn(Vnc, C), umma::op_mn(dSc, 128));
         umma::commit(&bm[2]);
     }
 
@@ -1920,8 +1910,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     sync_for_mma();
     if (tid == 0) {  // dq += M K
         umma::fence_after();
-        chain(L5::DQ, I128km, C / 16, true, [&](int ks) { return umma::desc_k(Ms, ks, C); },
-              [&](int ks) { return umma::desc_mn(Kc, ks, 128); });
+        umma::chain<C / 16>(tm + L5::DQ, I128km, true, umma::op_k(Ms, C), umma::op_mn(Kc, 128));
     }
 
     // ---- E2b: dk <- dec (V_new dS_C^T) in place, sum_k K dk; dW; T'', T, L tiles
@@ -1990,19 +1979,13 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     if (tid == 0) {
         umma::fence_after();
         if (BETA) {  // dk += gamma T^T dW, dk += M^T Q, dW K^T, dV_new V^T, dv = T^T dV_new
-            chain(L5::DKC, I128mm, C / 16, true, [&](int ks) { return umma::desc_mn(Tpp, ks, C); },
-                  [&](int ks) { return umma::desc_mn(dWs, ks, 128); });
-            chain(L5::DKC, I128mm, C / 16, true, [&](int ks) { return umma::desc_mn(Ms, ks, C); },
-                  [&](int ks) { return umma::desc_mn(Qc, ks, 128); });
-            chain(L5::DTA, I64kk, 8, false, [&](int ks) { return umma::desc_k(dWs, ks, 128); },
-                  [&](int ks) { return umma::desc_k(Kc, ks, 128); });
-            chain(L5::DTB, I64mk, DV / 16, false, [&](int ks) { return umma::desc_mn(dVnc, ks, C); },
-                  [&](int ks) { return umma::desc_k(Vc, ks, DV); });
-            chain(L5::DVC, IDVmk, C / 16, false, [&](int ks) { return umma::desc_mn(Ts, ks, C); },
-                  [&](int ks) { return umma::desc_k(dVnc, ks, C); });
+            umma::chain<C / 16>(tm + L5::DKC, I128mm, true, umma::op_mn(Tpp, C), umma::op_mn(dWs, 128));
+            umma::chain<C / 16>(tm + L5::DKC, I128mm, true, umma::op_mn(Ms, C), umma::op_mn(Qc, 128));
+            umma::chain<8>(tm + L5::DTA, I64kk, false, umma::op_k(dWs, 128), umma::op_k(Kc, 128));
+            umma::chain<DV / 16>(tm + L5::DTB, I64mk, false, umma::op_mn(dVnc, C), umma::op_k(Vc, DV));
+            umma::chain<C / 16>(tm + L5::DVC, IDVmk, false, umma::op_mn(Ts, C), umma::op_k(dVnc, C));
         } else {  // dk += M^T Q
-            chain(L5::DKC, I128mm, C / 16, true, [&](int ks) { return umma::desc_mn(Ms, ks, C); },
-                  [&](int ks) { return umma::desc_mn(Qc, ks, 128); });
+            umma::chain<C / 16>(tm + L5::DKC, I128mm, true, umma::op_mn(Ms, C), umma::op_mn(Qc, 128));
         }
         umma::commit(&bm[3]);
     }
@@ -2076,8 +2059,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
         sync_for_mma();  // L (fp32) is read for the last time above
         if (tid == 0) {  // X = L^T dL
             umma::fence_after();
-            chain(L5::XC, I64mm, C / 16, false, [&](int ks) { return umma::desc_mn(Ls, ks, C); },
-                  [&](int ks) { return umma::desc_mn(dLs, ks, C); });
+            umma::chain<C / 16>(tm + L5::XC, I64mm, false, umma::op_mn(Ls, C), umma::op_mn(dLs, C));
             umma::commit(&bm[4]);
             if (has_next) bulk_l(jn);
         }
@@ -2097,8 +2079,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
         sync_for_mma();
         if (tid == 0) {  // dA' = X L^T
             umma::fence_after();
-            chain(L5::DA, I64kk, C / 16, false, [&](int ks) { return umma::desc_k(Xs, ks, C); },
-                  [&](int ks) { return umma::desc_k(Ls, ks, C); });
+            umma::chain<C / 16>(tm + L5::DA, I64kk, false, umma::op_k(Xs, C), umma::op_k(Ls, C));
             umma::commit(&bm[5]);
         }
         // ---- E6: dA = strictly-lower(-X L^T); Z = dA beta_i Gamma; dbeta (row part); Z sums
@@ -2163,10 +2144,8 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
         sync_for_mma();
         if (tid == 0) {  // dk += Z K + Z^T K
             umma::fence_after();
-            chain(L5::DKC, I128km, C / 16, true, [&](int ks) { return umma::desc_k(Zs, ks, C); },
-                  [&](int ks) { return umma::desc_mn(Kc, ks, 128); });
-            chain(L5::DKC, I128mm, C / 16, true, [&](int ks) { return umma::desc_mn(Zs, ks, C); },
-                  [&](int ks) { return umma::desc_mn(Kc, ks, 128); });
+            umma::chain<C / 16>(tm + L5::DKC, I128km, true, umma::op_k(Zs, C), umma::op_mn(Kc, 128));
+            umma::chain<C / 16>(tm + L5::DKC, I128mm, true, umma::op_mn(Zs, C), umma::op_mn(Kc, 128));
             umma::commit(&bm[6]);
         }
         wait_bar(&bm[6]);

@@ -77,6 +77,29 @@ __device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a, uint64_t b, uin
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
         "l"(a), "l"(b), "r"(idesc), "r"((uint32_t)accumulate));
 }
+// A K-sliced operand for a chain of MMAs: the descriptor of slice 0 and the
+// step of its address field (byte address / 16) from one K = 16 slice to the
+// next: 256 bytes in a K-major canon [R][K] tile, 32 R bytes in an MN-major
+// canon [K][R] tile.  Shared addresses stay below 2^18 bytes, so adding to the
+// field never carries into the next one.
+struct Op {
+    uint64_t d;
+    uint32_t step;
+};
+__device__ __forceinline__ Op op_k(const void* base, int K) { return {desc_k(base, 0, K), 16u}; }
+__device__ __forceinline__ Op op_mn(const void* base, int R) { return {desc_mn(base, 0, R), 2u * (uint32_t)R}; }
+// D (+)= A B over NKS slices of K = 16, issued back to back by one thread:
+// the descriptors are formed once and advanced by one addition per MMA, so the
+// issue keeps ahead of the tensor core (forming each descriptor afresh costs
+// about 100 cycles of dependent integer work per MMA, more than an M = 64 MMA
+// takes to run).
+template <int NKS>
+__device__ __forceinline__ void chain(uint32_t d_tmem, uint32_t idesc, bool accumulate, Op a, Op b) {
+#pragma unroll
+    for (int ks = 0; ks < NKS; ++ks)
+        mma(d_tmem, a.d + (uint64_t)(ks * a.step), b.d + (uint64_t)(ks * b.step), idesc, accumulate || ks > 0);
+}
+
 // The mbarrier gets one arrival once every MMA this thread issued before has completed.
 __device__ __forceinline__ void commit(void* mbar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
