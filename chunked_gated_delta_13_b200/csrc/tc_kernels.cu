@@ -24,8 +24,12 @@
 // warp pair, so the recurrence never leaves the register file; only the
 // operands (W, Khat, U or dVi and D) stream in, through bulk copies three
 // (forward) or two (backward) chunks deep.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 #include <cstdlib>
+#include <cstring>
 #include <string>
 
 #include "tc_kernels.cuh"
@@ -43,6 +47,14 @@ constexpr int DK = 128;      // key head size
 constexpr int LDK = DK + 8;  // shared row stride of [*][DK] tiles
 constexpr int LDC = C + 8;   // shared row stride of [*][C] tiles
 constexpr int LDF = 72;      // shared row stride of fp32 [C][C] tiles
+
+// Offset of element (i, j) of the per-chunk fp32 L = (I + A)^{-1} as Pre
+// stores it for the gradient kernels: row i, its 16-byte piece p at position
+// p ^ (i % 8), so that the gradient kernel, which copies the tile linearly into
+// shared memory, reads a column of it for eight rows without bank conflicts.
+__host__ __device__ __forceinline__ int l_off(int i, int j) {
+    return i * C + ((((j >> 2) ^ (i & 7))) << 2) + (j & 3);
+}
 
 // Set (bit 0) by a kernel that gave up waiting for one of its own bulk copies;
 // read and cleared by sf_device_check().
@@ -292,7 +304,7 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ k, const bf16* __restrict__ v
         float* Lg = Lmo + ((size_t)bh * s.NC + c) * C * C;
         for (int e = tid; e < C * C / 4; e += 256) {
             const int i = e >> 4, j = (e & 15) * 4;
-            *reinterpret_cast<float4*>(Lg + i * C + j) = *reinterpret_cast<const float4*>(Lf + i * LDF + j);
+            *reinterpret_cast<float4*>(Lg + l_off(i, j)) = *reinterpret_cast<const float4*>(Lf + i * LDF + j);
         }
         for (int e = tid; e < C * C; e += 256) {  // A is dead: its region takes the T tiles
             const int i = e >> 6, j = e & 63;
@@ -1225,7 +1237,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
             const float* Lg = Lm + ci * C * C;
             for (int e = tid; e < C * C / 4; e += GTH) {
                 const int i = e >> 4, j = (e & 15) * 4;
-                cp_async16(Lf + i * LDF + j, Lg + i * C + j, true);
+                cp_async16(Lf + i * LDF + j, Lg + l_off(i, j), true);
             }
             cp_async_commit();
         }
@@ -1597,19 +1609,30 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 //   [0,64) Q K^T -> [0,128) dk       [64,128) K K^T        [128,192) dP -> dT_b -> dA
 //   [192,320) dq                     [320,448) dV_new S0^T -> dv
 //   [448,512) dW K^T -> X
+// Tensor maps of the gradient kernel's token-major tiles (q, k, v, dO in; dq,
+// dk out), each a five-dimensional view of a [BH][T][D] bf16 tensor ordered
+// (column within 8, row within 8, column block, row block, head), so that one
+// box of (8, 8, D/8, C/8, 1) is a whole chunk tile and lands in shared memory
+// (or is read from it) in the canonical core-matrix layout the tcgen05
+// descriptors read.  `on` is 0 when the maps could not be made; the kernel
+// then copies every tile with per-thread cp.async, as it always does for a
+// chunk shorter than C (a box cannot stop at a row that is not a multiple of
+// 8, so partial chunks never use the maps).
+struct G5Maps {
+    CUtensorMap q, k, v, dO, dq, dk;
+    int on;
+};
+
 template <int DV>
 struct G5 {
     // TMEM columns of the accumulators
     static constexpr uint32_t QK = 0, KK = 64, DP = 128, DQ = 192, DW = 320, DTA = 448;
     static constexpr uint32_t DKC = 0, DTB = 128, DVC = 320, XC = 448, DA = 128;
-    static constexpr int SLD = 128 + 8;  // row stride of the dq / dk staging tiles (elements)
     static constexpr size_t kQK = (size_t)2 * C * 128 * 2;  // one buffer: Q then K
     static constexpr size_t kV = (size_t)C * DV * 2;        // V, dO, V_new^T, dV_new^T each
     static constexpr size_t kStateB = (size_t)DV * 128 * 2 * 2;
     static constexpr size_t kEpiB = (size_t)C * 128 * 2 + 6 * (size_t)C * C * 2;
-    static constexpr size_t kOutB = (size_t)2 * C * SLD * 2;
-    static constexpr size_t kB0 = kStateB > kEpiB ? kStateB : kEpiB;
-    static constexpr size_t kB = kB0 > kOutB ? kB0 : kOutB;
+    static constexpr size_t kB = kStateB > kEpiB ? kStateB : kEpiB;
     static constexpr size_t SMEM = 2 * kQK + 4 * kV + kB + (size_t)C * C * 4 + (size_t)C * C * 2 +
                                    (size_t)P_ROWS * C * 4 + 16 * 4 + 4 * C * 4 + 16 * 8 + 16;
 };
@@ -1621,7 +1644,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
                 const float* __restrict__ Lm, const bf16* __restrict__ Vnt, const bf16* __restrict__ dVnt,
                 const bf16* __restrict__ S0t, const bf16* __restrict__ dSCt, bf16* __restrict__ dq,
                 bf16* __restrict__ dk, bf16* __restrict__ dv, float* __restrict__ dg, float* __restrict__ dbeta,
-                int* __restrict__ ticket) {
+                int* __restrict__ ticket, const __grid_constant__ G5Maps maps) {
     using L5 = G5<DV>;
     extern __shared__ __align__(16) unsigned char smem[];
     unsigned char* p = smem;
@@ -1640,8 +1663,6 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     bf16* dLs = Ls + C * C;                            // [C][C]
     bf16* Xs = dLs + C * C;                            // [C][C]
     bf16* Zs = Xs + C * C;                             // [C][C]
-    bf16* Sq = reinterpret_cast<bf16*>(RB);            // [C][SLD] dq staging (row-major, at the end)
-    bf16* Sk = Sq + C * L5::SLD;                       // [C][SLD] dk staging
     float* Lf = reinterpret_cast<float*>(p);  p += C * C * 4;   // [C][C] fp32, row-major
     bf16* Ms = reinterpret_cast<bf16*>(p);    p += C * C * 2;   // [C][C]
     float* part = reinterpret_cast<float*>(p); p += P_ROWS * C * 4;
@@ -1657,6 +1678,9 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     uint64_t* bdVn = &bars[2];
     uint64_t* bL = &bars[3];
     uint64_t* bm = &bars[4];  // [7]
+    uint64_t* bQK = &bars[11];  // [2] Q, K, G of the chunk in buffer b
+    uint64_t* bDO = &bars[13];
+    uint64_t* bV = &bars[14];
 
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int gq = lane >> 2, tq = lane & 3;
@@ -1673,25 +1697,54 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     auto Qc_of = [&](int b) { return reinterpret_cast<bf16*>(QKb + b * L5::kQK); };
     auto Kc_of = [&](int b) { return reinterpret_cast<bf16*>(QKb + b * L5::kQK) + C * 128; };
     // copy groups (cp.async: per-thread FIFO groups; bulk: mbarriers, thread 0)
+    // Q, K, G, dO and V complete on mbarriers: by tensor-map copies of thread 0
+    // for whole chunks, else by cp.async (waited for in the threads' FIFO
+    // groups) with a plain arrival of thread 0.
     auto copy_qkg = [&](int j, int b) {  // Q, K, G of chunk j into buffer b
         int c, bh;
         where(j, c, bh);
         const int t0 = c * C, nval = min(C, s.T - t0);
+        if (maps.on && nval == C) {
+            if (tid == 0) {
+                mbar_expect_tx(&bQK[b], 2 * C * DK * 2 + C * 4);
+                tma_load5(Qc_of(b), &maps.q, 0, t0 / 8, bh, &bQK[b]);
+                tma_load5(Kc_of(b), &maps.k, 0, t0 / 8, bh, &bQK[b]);
+                bulk_load(Gsb + b * C, Gc + bh * Tp + t0, C * 4, &bQK[b]);
+            }
+            return;
+        }
         umma::load_canon<C, 128, 512>(Qc_of(b), q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
         umma::load_canon<C, 128, 512>(Kc_of(b), k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
         if (tid < C / 4) cp_async16(Gsb + b * C + 4 * tid, Gc + bh * Tp + t0 + 4 * tid, true);
+        if (tid == 0) mbar_arrive(&bQK[b]);
     };
     auto copy_do = [&](int j) {
         int c, bh;
         where(j, c, bh);
         const int t0 = c * C, nval = min(C, s.T - t0);
+        if (maps.on && nval == C) {
+            if (tid == 0) {
+                mbar_expect_tx(bDO, C * DV * 2);
+                tma_load5(dOc, &maps.dO, 0, t0 / 8, bh, bDO);
+            }
+            return;
+        }
         umma::load_canon<C, DV, 512>(dOc, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+        if (tid == 0) mbar_arrive(bDO);
     };
-    auto copy_v = [&](int j) {
+    auto copy_v = [&](int j) {  // the delta path only: V is read by dV_new V^T alone
         int c, bh;
         where(j, c, bh);
         const int t0 = c * C, nval = min(C, s.T - t0);
+        if (maps.on && nval == C) {
+            if (tid == 0) {
+                mbar_expect_tx(bV, C * DV * 2);
+                tma_load5(Vc, &maps.v, 0, t0 / 8, bh, bV);
+            }
+            return;
+        }
         umma::load_canon<C, DV, 512>(Vc, v + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+        if (tid == 0) mbar_arrive(bV);
     };
     auto bulk_vn = [&](int j) {  // thread 0
         int c, bh;
@@ -1727,7 +1780,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     };
 
     if (tid == 0) {
-        for (int i = 0; i < 11; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 15; ++i) mbar_init(&bars[i], 1);
         mbar_init_fence();
         tk[0] = atomicAdd(ticket, 1);
     }
@@ -1739,7 +1792,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     copy_qkg(j, 0);
     copy_do(j);
     cp_async_commit();
-    copy_v(j);
+    if (BETA) copy_v(j);
     cp_async_commit();
     if (tid == 0) {
         bulk_vn(j);
@@ -1783,6 +1836,8 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     float* Bs = Bsb + buf * C;
     if (tid == 0) tk[(it + 1) & 1] = atomicAdd(ticket, 1);
     cp_async_wait<1>();  // Q, K, G, dO of this chunk (its V may still be landing)
+    mbar_wait(&bQK[buf], (uint32_t)((it >> 1) & 1), &g_tc_status, failed);
+    mbar_wait(bDO, par, &g_tc_status, failed);
     mbar_wait(bVn, par, &g_tc_status, failed);
     sync_for_mma();
     const int jn = tk[(it + 1) & 1];
@@ -1814,6 +1869,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
 
     // ---- E1: M = scale dP * Gamma (bf16 tile), row/column sums of M * QK; keep K K^T
     float kkr[2][4];
+    float gmr[2][4];  // Gamma_ij = exp(G_i - G_j) (j <= i) of this thread's elements, for E6
     {
         wait_bar(&bm[0]);
         float qk[2][4], dp[2][4];
@@ -1830,6 +1886,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
             for (int e = 0; e < 4; ++e) {
                 const int i = (e >> 1) ? r1 : r0, jj = 16 * nw + 8 * n + 2 * tq + (e & 1);
                 const float gm = (jj <= i) ? __expf(Gs[i] - Gs[jj]) : 0.f;
+                gmr[n][e] = gm;
                 m[e] = s.scale * dp[n][e] * gm;
                 const float zp = m[e] * qk[n][e];
                 if (e >> 1) row1 += zp; else row0 += zp;
@@ -1961,7 +2018,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     const int jj = j0 + 2 * h;
-                    const float2 l = *reinterpret_cast<const float2*>(Lf + i * C + jj);
+                    const float2 l = *reinterpret_cast<const float2*>(Lf + l_off(i, jj));
                     const float b0 = Bs[jj], b1 = Bs[jj + 1];
                     tpp[h] = pack(l.x * b0 * __expf(Gs[jj]), l.y * b1 * __expf(Gs[jj + 1]));
                     tt[h] = pack(l.x * b0, l.y * b1);
@@ -1974,7 +2031,10 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
         }
         umma::wait_st();
     }
-    if (BETA) cp_async_wait<2>();  // this chunk's V (the next chunk's Q, K, dO may still be landing)
+    if (BETA) {  // this chunk's V (the next chunk's Q, K, dO may still be landing)
+        cp_async_wait<2>();
+        mbar_wait(bV, par, &g_tc_status, failed);
+    }
     sync_for_mma();
     if (tid == 0) {
         umma::fence_after();
@@ -2008,7 +2068,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int r = (e >> 1) ? r1 : r0, jj = 16 * nw + 8 * n + 2 * tq + (e & 1);
-                    const float l = Lf[r * C + jj];
+                    const float l = Lf[l_off(r, jj)];
                     const float dt = fmaf(ta[n][e], __expf(Gs[jj]), tb[n][e]);
                     col[e & 1] += dt * l;
                     ckt[e & 1] += ta[n][e] * l;
@@ -2098,7 +2158,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
                     const int i = (e >> 1) ? r1 : r0, jj = 16 * nw + 8 * n + 2 * tq + (e & 1);
                     float z = 0.f, bterm = 0.f;
                     if (jj < i) {
-                        const float gm = __expf(Gs[i] - Gs[jj]);
+                        const float gm = gmr[n][e];
                         const float dav = -da[n][e];
                         bterm = dav * gm * kkr[n][e];
                         z = dav * Bs[i] * gm;
@@ -2148,21 +2208,26 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
             umma::chain<C / 16>(tm + L5::DKC, I128mm, true, umma::op_mn(Zs, C), umma::op_mn(Kc, 128));
             umma::commit(&bm[6]);
         }
-        wait_bar(&bm[6]);
+        wait_bar(&bm[6]);  // the last product: the state region is free
+        if (tid == 0 && has_next) bulk_state(jn);
     } else {
-        wait_bar(&bm[3]);
+        wait_bar(&bm[3]);  // the last product: the state region is free
+        if (tid == 0 && has_next) bulk_state(jn);
         bf16* dvb = dv + bh * s.hs_v + (size_t)t0 * DV;
         for (int e = tid; e < nval * DV; e += 512) {
             const int jj = e / DV, col = e % DV;
             dvb[(size_t)jj * DV + col] = *umma::canon_at<bf16>(dVnc, col, jj, C);
         }
-        __syncthreads();  // V (unused here) and dV_new^T are free
-        if (has_next) copy_v(jn);
+        __syncthreads();  // dV_new^T is free
         cp_async_commit();
         if (tid == 0 && has_next) bulk_dvn(jn);
     }
 
-    // ---- E7: dq, dk staged row-major in the free state region, then bulk-stored by rows
+    // ---- E7: dq, dk staged as canon tiles in this chunk's Q and K buffer (no
+    // product reads it any more), then written out 16 bytes per thread: piece e
+    // of a canon [C][128] tile holds row 8 (e / 128) + e % 8, columns
+    // 8 ((e / 8) % 16) + 0..7, so the shared reads are linear and a warp writes
+    // whole 32-byte sectors of eight rows.
     {
         float a[4][4], b[4][4];
         umma::ld32(trow + L5::DQ + 32 * nw, a);
@@ -2171,23 +2236,32 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
 #pragma unroll
         for (int jq = 0; jq < 4; ++jq) {
             const int col = 32 * nw + 8 * jq + 2 * tq;
-            *reinterpret_cast<uint32_t*>(Sq + r0 * L5::SLD + col) = pack(a[jq][0], a[jq][1]);
-            *reinterpret_cast<uint32_t*>(Sq + r1 * L5::SLD + col) = pack(a[jq][2], a[jq][3]);
-            *reinterpret_cast<uint32_t*>(Sk + r0 * L5::SLD + col) = pack(b[jq][0], b[jq][1]);
-            *reinterpret_cast<uint32_t*>(Sk + r1 * L5::SLD + col) = pack(b[jq][2], b[jq][3]);
+            *umma::canon_at<uint32_t>(Qc, r0, col, 128) = pack(a[jq][0], a[jq][1]);
+            *umma::canon_at<uint32_t>(Qc, r1, col, 128) = pack(a[jq][2], a[jq][3]);
+            *umma::canon_at<uint32_t>(Kc, r0, col, 128) = pack(b[jq][0], b[jq][1]);
+            *umma::canon_at<uint32_t>(Kc, r1, col, 128) = pack(b[jq][2], b[jq][3]);
         }
     }
     fence_proxy_async_smem();
     umma::fence_before();
     __syncthreads();  // staging written, partial sums written, TMEM reads done
-    if (tid < 2 * C) {  // one row of dq or dk per thread
-        const int r = tid & (C - 1);
-        if (r < nval) {
-            const bool isk = tid >= C;
-            bf16* dst = (isk ? dk : dq) + bh * s.hs_k + (size_t)(t0 + r) * DK;
-            bulk_store(dst, (isk ? Sk : Sq) + r * L5::SLD, DK * 2);
+    if (maps.on && nval == C) {
+        if (tid == 0) {
+            tma_store5(&maps.dq, 0, t0 / 8, bh, Qc);
+            tma_store5(&maps.dk, 0, t0 / 8, bh, Kc);
+            bulk_commit();
         }
-        bulk_commit();
+    } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = tid + 512 * u, pe = e & 1023;
+            const int r = ((pe >> 7) << 3) + (pe & 7), cb = (pe >> 3) & 15;
+            if (r < nval) {
+                const uint4 x = reinterpret_cast<const uint4*>(u < 2 ? Qc : Kc)[pe];
+                bf16* dst = (u < 2 ? dq : dk) + bh * s.hs_k + (size_t)(t0 + r) * DK + 8 * cb;
+                *reinterpret_cast<uint4*>(dst) = x;
+            }
+        }
     }
     if (w == 15) {
         // ---- dG, dg (chunk-local reverse cumsum), dbeta; two tokens per lane
@@ -2222,15 +2296,14 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
         if (2 * lane < nval) dgb[2 * lane] = suf;
         if (2 * lane + 1 < nval) dgb[2 * lane + 1] = suf - x[0];
     }
-    if (tid < 2 * C) bulk_wait_read<0>();  // the staging region is read out
-    __syncthreads();  // partial sums consumed; the state region is free
-    if (tid == 0 && has_next) bulk_state(jn);
+    if (tid == 0) bulk_wait_read<0>();  // the tensor-map stores have read the staging
+    __syncthreads();  // partial sums consumed, the staging read out
     if (!has_next) break;
     for (int e = tid; e < P_ROWS * C; e += 512) part[e] = 0.f;
     if (tid < C) Bsb[(buf ^ 1) * C + tid] = beta_next;
     j = jn;
   }
-    if (tid < 2 * C) bulk_wait<0>();
+    if (tid == 0) bulk_wait<0>();
     umma::fence_before();
     __syncthreads();
     if (w == 0) {
@@ -2380,17 +2453,53 @@ cudaError_t launch_grad(const SeqView& s, const BwdArgs& a, const TcWs& w, cudaS
     return cudaGetLastError();
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (the
+// library does not link the driver library); null if the driver lacks it.
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// The five-dimensional canon view of a [BH][T][D] bf16 tensor (head stride hs
+// elements) described at G5Maps; false if it cannot be made (no driver entry
+// point, a base not 16-byte aligned, fewer than C tokens).
+bool canon_map(CUtensorMap* m, const void* base, int BH, int T, int D, long long hs) {
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = encode_tiled();
+    if (!enc || T < C || BH < 1 || (reinterpret_cast<uintptr_t>(base) & 15)) return false;
+    const cuuint64_t dims[5] = {8, 8, (cuuint64_t)(D / 8), (cuuint64_t)(T / 8), (cuuint64_t)BH};
+    const cuuint64_t strides[4] = {(cuuint64_t)D * 2, 16, (cuuint64_t)D * 16, (cuuint64_t)hs * 2};
+    const cuuint32_t box[5] = {8, 8, (cuuint32_t)(D / 8), C / 8, 1};
+    const cuuint32_t unit[5] = {1, 1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, unit,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int DV, bool BETA>
 cudaError_t launch_grad5(const SeqView& s, const BwdArgs& a, const TcWs& w, cudaStream_t st) {
     constexpr size_t sm = G5<DV>::SMEM;
     TC_TRY(smem_attr(tc_grad5_kernel<DV, BETA>, sm));
     TC_TRY(cudaMemsetAsync(w.ticket, 0, sizeof(int), st));
     const int grid = std::min(s.NC * s.BH, num_sms());
+    G5Maps maps;
+    memset(&maps, 0, sizeof(maps));
+    maps.on = canon_map(&maps.q, a.q, s.BH, s.T, DK, s.hs_k) && canon_map(&maps.k, a.k, s.BH, s.T, DK, s.hs_k) &&
+              canon_map(&maps.dO, a.dO, s.BH, s.T, DV, s.hs_v) &&
+              (!BETA || canon_map(&maps.v, a.v, s.BH, s.T, DV, s.hs_v)) &&
+              canon_map(&maps.dq, a.dq, s.BH, s.T, DK, s.hs_k) && canon_map(&maps.dk, a.dk, s.BH, s.T, DK, s.hs_k);
     SF_LAUNCH("tc_grad", st, tc_grad5_kernel<DV, BETA><<<grid, 512, sm, st>>>(
                                  s, static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k),
                                  static_cast<const bf16*>(a.v), a.beta, static_cast<const bf16*>(a.dO), w.Gc,
                                  w.Lm, w.Vnt, w.dVnt, w.S0t, w.dSCt, static_cast<bf16*>(a.dq), static_cast<bf16*>(a.dk),
-                                 static_cast<bf16*>(a.dv), a.dg, a.dbeta, w.ticket));
+                                 static_cast<bf16*>(a.dv), a.dg, a.dbeta, w.ticket, maps));
     return cudaGetLastError();
 }
 

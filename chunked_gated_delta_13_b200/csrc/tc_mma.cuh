@@ -141,6 +141,27 @@ __device__ __forceinline__ void bulk_load(void* sdst, const void* gsrc, uint32_t
                  "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
 }
+// One arrival without a transaction count (a phase whose copies went another way).
+__device__ __forceinline__ void mbar_arrive(void* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+// Tensor-map (TMA) copies of one box of a five-dimensional tensor map, issued
+// by one thread: global -> shared completing on an mbarrier, shared -> global
+// in the bulk group of the issuing thread.  `map` is the generic address of a
+// __grid_constant__ CUtensorMap parameter; the innermost coordinate is 0.
+__device__ __forceinline__ void tma_load5(void* sdst, const void* map, int c2, int c3, int c4, void* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, "
+        "%6}], [%7];\n" ::"r"(smem_u32(sdst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(0), "r"(c2), "r"(c3), "r"(c4), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_store5(const void* map, int c2, int c3, int c4, const void* ssrc) {
+    asm volatile("cp.async.bulk.tensor.5d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4, %5}], [%6];\n" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(0), "r"(0), "r"(c2), "r"(c3), "r"(c4), "r"(smem_u32(ssrc))
+                 : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(void* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
