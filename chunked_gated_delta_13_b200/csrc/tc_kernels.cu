@@ -74,6 +74,7 @@ struct TcWs {
     bf16* dSCt;  // [BH][NC][DV][DK]   gradient of the state leaving each chunk, transposed (canon)
     bf16* Dt;    // [BH][NC][DV][DK]   scale (gamma * dO)^T Q per chunk, transposed (permuted)
     int* ticket;  // chunk counter of the persistent gradient kernel
+    int* oticket;  // chunk counter of the persistent Out kernel
     size_t total;
 };
 
@@ -101,6 +102,7 @@ TcWs tc_parts(const SeqView& s, char* keep, char* og, char* slot, size_t* keep_b
     w.Ut = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
     w.Vnt = reinterpret_cast<bf16*>(take(BH * NC * DV * C * 2));
     w.S0t = reinterpret_cast<bf16*>(take(BH * NC * DV * DK * 2));
+    w.oticket = reinterpret_cast<int*>(take(sizeof(int)));
     if (keep_bytes) *keep_bytes = off;
     base = og;
     off = 0;
@@ -829,121 +831,255 @@ tc_scan_bwd_dual_kernel(SeqView s, ChainOps op_f, ChainOps op_b, int nsr) {
 }
 
 // ------------------------------------------------------------------- out ---
-template <int DV, bool OG>
-constexpr size_t out_smem() {
-    return (size_t)C * LDK * 2 * 2 + (size_t)DV * LDK * 2 + (size_t)DV * LDC * 2 + C * 4 +
-           (OG ? (size_t)C * (DV + 8) * 2 : 0);
-}
+// Tensor maps of the token-major tiles a kernel copies by TMA (see canon_map):
+// q, k and dO in canon layout; `on` is 0 when they could not be made, and
+// chunks shorter than C always take per-thread cp.async.
+struct TokMaps {
+    CUtensorMap q, k, dO;
+    int on;
+};
 
-// O = scale (gamma * Q) S0 + (scale (Q K^T) * Gamma) V_new; 4 warps x 16 rows.
-// With OG (the forward of a segment whose backward follows), the same CTA also
-// writes the intra-chunk backward products of og_products, reusing Q and P.
 template <int DV, bool OG>
-__global__ void __launch_bounds__(128)
-tc_out_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k,
-              const float* __restrict__ Gc, const bf16* __restrict__ Vnt,
-              const bf16* __restrict__ S0t, bf16* __restrict__ o, const bf16* __restrict__ dO,
-              bf16* __restrict__ dVito, bf16* __restrict__ Dto) {
-    constexpr int LDV = DV + 8;
-    extern __shared__ __align__(16) unsigned char smem[];
-    bf16* Qs = reinterpret_cast<bf16*>(smem);
-    bf16* Ks = Qs + C * LDK;     // later (OG): P [C][LDC]
-    bf16* S0s = Ks + C * LDK;   // [DV][DK] canon (sized [DV][LDK])
-    bf16* Vns = S0s + DV * LDK;  // [DV][C] canon (sized [DV][LDC])
-    float* Gs = reinterpret_cast<float*>(Vns + DV * LDC);
-    bf16* dOs = reinterpret_cast<bf16*>(Gs + C);  // [C][LDV] (OG)
-    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+struct O2 {
+    static constexpr size_t kQ = (size_t)C * DK * 2;          // Q, K (canon [C][DK])
+    static constexpr size_t kS = (size_t)DV * DK * 2;         // S0^T (canon [DV][DK])
+    static constexpr size_t kVn = (size_t)DV * C * 2;         // V_new^T (canon [DV][C])
+    static constexpr size_t kdO = OG ? (size_t)C * DV * 2 : 0;  // dO (canon [C][DV])
+    static constexpr size_t kBuf = 2 * kQ + kS + kVn + kdO + C * 4;
+    static constexpr size_t SMEM = 2 * kBuf + (size_t)C * C * 2 + 2 * 8 + 2 * 4;
+};
+
+// Intra-chunk backward products of one chunk from canon tiles, 8 warps:
+// dVi^T = (P^T dO)^T and D^T = (scale (gamma * dO)^T Q)^T, each warp one
+// 16-row tile of d_v (d_v = 128) or one tile and half the columns (d_v = 64).
+template <int DV>
+__device__ __forceinline__ void og_products8(const SeqView& s, const bf16* Qs, const bf16* dOs, const bf16* Ps,
+                                             const float* Gs, bf16* dVi, bf16* Dg, int w, int lane) {
     const int gq = lane >> 2, tq = lane & 3;
-    const int t0 = c * C;
-    const int nval = min(C, s.T - t0);
-    const size_t Tp = (size_t)s.NC * C;
-    load_tile<C, DK, 128>(Qs, LDK, q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
-    load_tile<C, DK, 128>(Ks, LDK, k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
-    copy_linear<DV * DK * 2, 128>(S0s, S0t + ((size_t)bh * s.NC + c) * DV * DK, tid);  // canon tiles
-    copy_linear<DV * C * 2, 128>(Vns, Vnt + ((size_t)bh * s.NC + c) * DV * C, tid);
-    if (tid < 16) cp_async16(Gs + tid * 4, Gc + bh * Tp + t0 + tid * 4, true);
-    cp_async_commit();
-    if (OG) {
-        load_tile<C, DV, 128>(dOs, LDV, dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
-        cp_async_commit();
-        cp_async_wait<1>();
-    } else {
-        cp_async_wait<0>();
-    }
-    __syncthreads();
-
-    float p[8][4] = {};
-    float acc[DV / 8][4] = {};
+    const int m0 = DV == 128 ? 16 * w : 16 * (w & 3);
+    constexpr int NVI = DV == 128 ? 8 : 4;   // n-tiles of dVi^T per warp
+    const int n0 = DV == 128 ? 0 : 32 * (w >> 2);
+    {  // dVi^T[v][j] = sum_i dO[i][v] P[i][j]
+        float acc[NVI][4] = {};
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-        uint32_t a[4];
-        ldA(a, Qs, LDK, 16 * w, 16 * kk, lane);
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t a[4];
+            umma::ldAt_c(a, dOs, DV, m0, 16 * kk, lane);
 #pragma unroll
-        for (int nn = 0; nn < 8; nn += 2) {
-            uint32_t b[4];
-            ldBnk(b, Ks, LDK, 8 * nn, 16 * kk, lane);
-            mma(p[nn], a, b[0], b[1]);
-            mma(p[nn + 1], a, b[2], b[3]);
+            for (int nn = 0; nn < NVI; nn += 2) {
+                uint32_t b[4];
+                umma::ldBkn_c(b, Ps, C, n0 + 8 * nn, 16 * kk, lane);
+                mma(acc[nn], a, b[0], b[1]);
+                mma(acc[nn + 1], a, b[2], b[3]);
+            }
         }
 #pragma unroll
-        for (int nn = 0; nn < DV / 8; nn += 2) {
-            uint32_t b[4];
-            umma::ldBnk_c(b, S0s, DK, 8 * nn, 16 * kk, lane);
-            mma(acc[nn], a, b[0], b[1]);
-            mma(acc[nn + 1], a, b[2], b[3]);
+        for (int nn = 0; nn < NVI; ++nn) {
+            const int r = m0 + gq, j = n0 + 8 * nn + 2 * tq;
+            *reinterpret_cast<uint32_t*>(dVi + swz(r, j, C)) = pack(acc[nn][0], acc[nn][1]);
+            *reinterpret_cast<uint32_t*>(dVi + swz(r + 8, j, C)) = pack(acc[nn][2], acc[nn][3]);
         }
     }
-    const int i0 = 16 * w + gq, i1 = i0 + 8;
-    const float G0 = Gs[i0], G1 = Gs[i1];
-    const float sg0 = s.scale * __expf(G0), sg1 = s.scale * __expf(G1);
-#pragma unroll
-    for (int nn = 0; nn < DV / 8; ++nn) {
-        acc[nn][0] *= sg0;
-        acc[nn][1] *= sg0;
-        acc[nn][2] *= sg1;
-        acc[nn][3] *= sg1;
-    }
-#pragma unroll
-    for (int nn = 0; nn < 8; ++nn)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int i = (e >> 1) ? i1 : i0, j = 8 * nn + 2 * tq + (e & 1);
-            p[nn][e] = (j <= i) ? s.scale * __expf(((e >> 1) ? G1 : G0) - Gs[j]) * p[nn][e] : 0.f;
-        }
-    bf16* Ps = Ks;
-    if (OG) {
-        __syncthreads();  // every warp is done reading K
-#pragma unroll
-        for (int nn = 0; nn < 8; ++nn) {
-            const int j = 8 * nn + 2 * tq;
-            *reinterpret_cast<uint32_t*>(Ps + i0 * LDC + j) = pack(p[nn][0], p[nn][1]);
-            *reinterpret_cast<uint32_t*>(Ps + i1 * LDC + j) = pack(p[nn][2], p[nn][3]);
-        }
-    }
+    // D^T[v][d] = sum_t scale gamma_t dO[t][v] Q[t][d]
+    uint32_t a[4][4];
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
-        uint32_t a[4];
-        c2a(a, p[2 * kk], p[2 * kk + 1]);
+        umma::ldAt_c(a[kk], dOs, DV, m0, 16 * kk, lane);
+        const int tk = 16 * kk + 2 * tq;
+        const float g0 = s.scale * __expf(Gs[tk]), g1 = s.scale * __expf(Gs[tk + 1]);
+        const float g2 = s.scale * __expf(Gs[tk + 8]), g3 = s.scale * __expf(Gs[tk + 9]);
+        a[kk][0] = scale2(a[kk][0], g0, g1);
+        a[kk][1] = scale2(a[kk][1], g0, g1);
+        a[kk][2] = scale2(a[kk][2], g2, g3);
+        a[kk][3] = scale2(a[kk][3], g2, g3);
+    }
+    constexpr int NH = DV == 128 ? 2 : 1;  // 64-column halves of D^T per warp
+#pragma unroll 1
+    for (int nh = 0; nh < NH; ++nh) {
+        const int d0 = DV == 128 ? 64 * nh : 64 * (w >> 2);
+        float acc[8][4] = {};
 #pragma unroll
-        for (int nn = 0; nn < DV / 8; nn += 2) {
-            uint32_t b[4];
-            umma::ldBnk_c(b, Vns, C, 8 * nn, 16 * kk, lane);
-            mma(acc[nn], a, b[0], b[1]);
-            mma(acc[nn + 1], a, b[2], b[3]);
+        for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+            for (int nn = 0; nn < 8; nn += 2) {
+                uint32_t b[4];
+                umma::ldBkn_c(b, Qs, DK, d0 + 8 * nn, 16 * kk, lane);
+                mma(acc[nn], a[kk], b[0], b[1]);
+                mma(acc[nn + 1], a[kk], b[2], b[3]);
+            }
+        }
+#pragma unroll
+        for (int nn = 0; nn < 8; ++nn) {
+            const int r = m0 + gq, d = d0 + 8 * nn + 2 * tq;
+            *reinterpret_cast<uint32_t*>(Dg + swz(r, d, DK)) = pack(acc[nn][0], acc[nn][1]);
+            *reinterpret_cast<uint32_t*>(Dg + swz(r + 8, d, DK)) = pack(acc[nn][2], acc[nn][3]);
         }
     }
-    bf16* ob = o + bh * s.hs_v + (size_t)t0 * DV;
-#pragma unroll
-    for (int nn = 0; nn < DV / 8; ++nn) {
-        const int col = 8 * nn + 2 * tq;
-        if (i0 < nval) *reinterpret_cast<uint32_t*>(ob + (size_t)i0 * DV + col) = pack(acc[nn][0], acc[nn][1]);
-        if (i1 < nval) *reinterpret_cast<uint32_t*>(ob + (size_t)i1 * DV + col) = pack(acc[nn][2], acc[nn][3]);
-    }
-    if (OG) {
-        cp_async_wait<0>();
-        __syncthreads();  // P and dO are visible
+}
+
+// O = scale (gamma * Q) S0 + (scale (Q K^T) * Gamma) V_new.  Persistent: a CTA
+// of 8 warps takes chunk tickets and copies the next chunk's tiles (Q, K, dO
+// by tensor maps, S0^T, V_new^T, G by bulk copies) into the second of two
+// buffers while it works on the current one.  Warp w computes rows
+// 16 (w % 4).. of P = scale (Q K^T) * Gamma for columns 32 (w / 4).. and of O
+// for half of d_v; P goes to shared memory, from where every warp reads the
+// whole rows it needs for P V_new.  With OG (the forward of a segment whose
+// backward follows) the same CTA also writes the intra-chunk backward products
+// (og_products8), reusing Q and P.
+template <int DV, bool OG>
+__global__ void __launch_bounds__(256, 1)
+tc_out2_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k, const float* __restrict__ Gc,
+               const bf16* __restrict__ Vnt, const bf16* __restrict__ S0t, bf16* __restrict__ o,
+               const bf16* __restrict__ dO, bf16* __restrict__ dVito, bf16* __restrict__ Dto,
+               int* __restrict__ ticket, const __grid_constant__ TokMaps maps) {
+    using L = O2<DV, OG>;
+    extern __shared__ __align__(16) unsigned char smem[];
+    bf16* Ps = reinterpret_cast<bf16*>(smem + 2 * L::kBuf);                          // [C][C] canon
+    uint64_t* bIn = reinterpret_cast<uint64_t*>(smem + 2 * L::kBuf + (size_t)C * C * 2);  // [2]
+    int* tk = reinterpret_cast<int*>(bIn + 2);                                         // [2]
+    auto Qb = [&](int b) { return reinterpret_cast<bf16*>(smem + b * L::kBuf); };
+    auto Kb = [&](int b) { return reinterpret_cast<bf16*>(smem + b * L::kBuf + L::kQ); };
+    auto Sb = [&](int b) { return reinterpret_cast<bf16*>(smem + b * L::kBuf + 2 * L::kQ); };
+    auto Vb = [&](int b) { return reinterpret_cast<bf16*>(smem + b * L::kBuf + 2 * L::kQ + L::kS); };
+    auto dOb = [&](int b) { return reinterpret_cast<bf16*>(smem + b * L::kBuf + 2 * L::kQ + L::kS + L::kVn); };
+    auto Gb = [&](int b) {
+        return reinterpret_cast<float*>(smem + b * L::kBuf + 2 * L::kQ + L::kS + L::kVn + L::kdO);
+    };
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int gq = lane >> 2, tq = lane & 3, mw = w & 3, nh = w >> 2;
+    const int total = s.NC * s.BH;
+    const size_t Tp = (size_t)s.NC * C;
+    bool failed = false;
+    auto where = [&](int j, int& c, int& bh) {
+        bh = j / s.NC;
+        c = j - bh * s.NC;
+    };
+    // every tile of chunk j into buffer b, completing on bIn[b] (cp.async
+    // copies of a short chunk complete in the threads' FIFO groups)
+    auto issue = [&](int j, int b) {
+        int c, bh;
+        where(j, c, bh);
+        const int t0 = c * C, nval = min(C, s.T - t0);
         const size_t ci = (size_t)bh * s.NC + c;
-        og_products<DV>(s, Qs, dOs, Ps, Gs, dVito + ci * DV * C, Dto + ci * DV * DK, w, lane);
+        const bool tma = maps.on && nval == C;
+        if (!tma) {
+            umma::load_canon<C, DK, 256>(Qb(b), q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+            umma::load_canon<C, DK, 256>(Kb(b), k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+            if (OG) umma::load_canon<C, DV, 256>(dOb(b), dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+        }
+        cp_async_commit();
+        if (tid == 0) {
+            mbar_expect_tx(&bIn[b], (uint32_t)(L::kS + L::kVn + C * 4 + (tma ? 2 * L::kQ + L::kdO : 0)));
+            bulk_load(Sb(b), S0t + ci * DV * DK, (uint32_t)L::kS, &bIn[b]);
+            bulk_load(Vb(b), Vnt + ci * DV * C, (uint32_t)L::kVn, &bIn[b]);
+            bulk_load(Gb(b), Gc + bh * Tp + t0, C * 4, &bIn[b]);
+            if (tma) {
+                tma_load5(Qb(b), &maps.q, 0, t0 / 8, bh, &bIn[b]);
+                tma_load5(Kb(b), &maps.k, 0, t0 / 8, bh, &bIn[b]);
+                if (OG) tma_load5(dOb(b), &maps.dO, 0, t0 / 8, bh, &bIn[b]);
+            }
+        }
+    };
+
+    if (tid == 0) {
+        mbar_init(&bIn[0], 1);
+        mbar_init(&bIn[1], 1);
+        mbar_init_fence();
+        tk[0] = atomicAdd(ticket, 1);
+    }
+    __syncthreads();
+    int j = tk[0];
+    if (j >= total) return;
+    issue(j, 0);
+    constexpr int NO = DV / 16;  // 8-column n-tiles of O per warp (half of d_v)
+    for (int it = 0;; ++it) {
+        const int buf = it & 1;
+        if (tid == 0) tk[(it + 1) & 1] = atomicAdd(ticket, 1);
+        cp_async_wait<0>();
+        mbar_wait(&bIn[buf], (uint32_t)((it >> 1) & 1), &g_tc_status, failed);
+        __syncthreads();  // this chunk's tiles are in; the other buffer is free
+        const int jn = tk[(it + 1) & 1];
+        const bool has_next = jn < total;
+        if (has_next) issue(jn, buf ^ 1);
+
+        int c, bh;
+        where(j, c, bh);
+        const int t0 = c * C, nval = min(C, s.T - t0);
+        const bf16* Qs = Qb(buf);
+        const bf16* Ks = Kb(buf);
+        const bf16* S0s = Sb(buf);
+        const bf16* Vns = Vb(buf);
+        const float* Gs = Gb(buf);
+        const int pc0 = 32 * nh, oc0 = (DV / 2) * nh;
+        float p[4][4] = {};
+        float acc[NO][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            uint32_t a[4];
+            umma::ldA_c(a, Qs, DK, 16 * mw, 16 * kk, lane);
+#pragma unroll
+            for (int nn = 0; nn < 4; nn += 2) {
+                uint32_t b[4];
+                umma::ldBnk_c(b, Ks, DK, pc0 + 8 * nn, 16 * kk, lane);
+                mma(p[nn], a, b[0], b[1]);
+                mma(p[nn + 1], a, b[2], b[3]);
+            }
+#pragma unroll
+            for (int nn = 0; nn < NO; nn += 2) {
+                uint32_t b[4];
+                umma::ldBnk_c(b, S0s, DK, oc0 + 8 * nn, 16 * kk, lane);
+                mma(acc[nn], a, b[0], b[1]);
+                mma(acc[nn + 1], a, b[2], b[3]);
+            }
+        }
+        const int i0 = 16 * mw + gq, i1 = i0 + 8;
+        const float G0 = Gs[i0], G1 = Gs[i1];
+        const float sg0 = s.scale * __expf(G0), sg1 = s.scale * __expf(G1);
+#pragma unroll
+        for (int nn = 0; nn < NO; ++nn) {
+            acc[nn][0] *= sg0;
+            acc[nn][1] *= sg0;
+            acc[nn][2] *= sg1;
+            acc[nn][3] *= sg1;
+        }
+#pragma unroll
+        for (int nn = 0; nn < 4; ++nn) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = (e >> 1) ? i1 : i0, jj = pc0 + 8 * nn + 2 * tq + (e & 1);
+                p[nn][e] = (jj <= i) ? s.scale * __expf(((e >> 1) ? G1 : G0) - Gs[jj]) * p[nn][e] : 0.f;
+            }
+            const int jj = pc0 + 8 * nn + 2 * tq;
+            *umma::canon_at<uint32_t>(Ps, i0, jj, C) = pack(p[nn][0], p[nn][1]);
+            *umma::canon_at<uint32_t>(Ps, i1, jj, C) = pack(p[nn][2], p[nn][3]);
+        }
+        __syncthreads();  // P complete
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t a[4];
+            umma::ldA_c(a, Ps, C, 16 * mw, 16 * kk, lane);
+#pragma unroll
+            for (int nn = 0; nn < NO; nn += 2) {
+                uint32_t b[4];
+                umma::ldBnk_c(b, Vns, C, oc0 + 8 * nn, 16 * kk, lane);
+                mma(acc[nn], a, b[0], b[1]);
+                mma(acc[nn + 1], a, b[2], b[3]);
+            }
+        }
+        bf16* ob = o + bh * s.hs_v + (size_t)t0 * DV;
+#pragma unroll
+        for (int nn = 0; nn < NO; ++nn) {
+            const int col = oc0 + 8 * nn + 2 * tq;
+            if (i0 < nval) *reinterpret_cast<uint32_t*>(ob + (size_t)i0 * DV + col) = pack(acc[nn][0], acc[nn][1]);
+            if (i1 < nval) *reinterpret_cast<uint32_t*>(ob + (size_t)i1 * DV + col) = pack(acc[nn][2], acc[nn][3]);
+        }
+        if (OG) {
+            const size_t ci = (size_t)bh * s.NC + c;
+            og_products8<DV>(s, Qs, dOb(buf), Ps, Gs, dVito + ci * DV * C, Dto + ci * DV * DK, w, lane);
+        }
+        __syncthreads();  // buffer `buf` and P are free
+        if (!has_next) break;
+        j = jn;
     }
 }
 
@@ -2375,23 +2511,79 @@ cudaError_t launch_scan_fwd(const SeqView& s, const float* S_in, float* S_out, c
     }
 }
 
-template <int DV>
-cudaError_t launch_out(const SeqView& s, const bf16* q, const bf16* k, bf16* o, const TcWs& w, cudaStream_t st) {
-    constexpr size_t sm = out_smem<DV, false>();
-    TC_TRY(smem_attr(tc_out_kernel<DV, false>, sm));
-    SF_LAUNCH("tc_out", st, tc_out_kernel<DV, false><<<dim3(s.NC, s.BH), 128, sm, st>>>(
-                                s, q, k, w.Gc, w.Vnt, w.S0t, o, nullptr, nullptr, nullptr));
-    return cudaGetLastError();
+int num_sms() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+            n = v;
+        else
+            n = 148;
+    }
+    return n;
 }
 
+// CTAs of a persistent kernel that takes chunk tickets: one per SM at most.
+// (Measured at the headline segment chain: capping the chunks a CTA takes, so
+// that the chain launches get SMs sooner, made the step slower at every cap.)
+int persistent_grid(const SeqView& s) { return std::min(s.NC * s.BH, num_sms()); }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (the
+// library does not link the driver library); null if the driver lacks it.
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// The five-dimensional canon view of a [BH][T][D] bf16 tensor (head stride hs
+// elements) described at G5Maps; false if it cannot be made (no driver entry
+// point, a base not 16-byte aligned, fewer than C tokens).
+bool canon_map(CUtensorMap* m, const void* base, int BH, int T, int D, long long hs) {
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = encode_tiled();
+    if (!enc || T < C || BH < 1 || (reinterpret_cast<uintptr_t>(base) & 15)) return false;
+    const cuuint64_t dims[5] = {8, 8, (cuuint64_t)(D / 8), (cuuint64_t)(T / 8), (cuuint64_t)BH};
+    const cuuint64_t strides[4] = {(cuuint64_t)D * 2, 16, (cuuint64_t)D * 16, (cuuint64_t)hs * 2};
+    const cuuint32_t box[5] = {8, 8, (cuuint32_t)(D / 8), C / 8, 1};
+    const cuuint32_t unit[5] = {1, 1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, unit,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Persistent Out: one CTA per SM at most, chunks from w.oticket.
+template <int DV, bool OG>
+cudaError_t launch_out2(const char* name, const SeqView& s, const bf16* q, const bf16* k, bf16* o, const bf16* dO,
+                        const TcWs& w, cudaStream_t st) {
+    constexpr size_t sm = O2<DV, OG>::SMEM;
+    TC_TRY(smem_attr(tc_out2_kernel<DV, OG>, sm));
+    TC_TRY(cudaMemsetAsync(w.oticket, 0, sizeof(int), st));
+    const int grid = persistent_grid(s);
+    TokMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    maps.on = canon_map(&maps.q, q, s.BH, s.T, DK, s.hs_k) && canon_map(&maps.k, k, s.BH, s.T, DK, s.hs_k) &&
+              (!OG || canon_map(&maps.dO, dO, s.BH, s.T, DV, s.hs_v));
+    SF_LAUNCH(name, st, tc_out2_kernel<DV, OG><<<grid, 256, sm, st>>>(
+                            s, q, k, w.Gc, w.Vnt, w.S0t, o, dO, OG ? w.dVit : nullptr, OG ? w.Dt : nullptr,
+                            w.oticket, maps));
+    return cudaGetLastError();
+}
+template <int DV>
+cudaError_t launch_out(const SeqView& s, const bf16* q, const bf16* k, bf16* o, const TcWs& w, cudaStream_t st) {
+    return launch_out2<DV, false>("tc_out", s, q, k, o, nullptr, w, st);
+}
 template <int DV>
 cudaError_t launch_out_og(const SeqView& s, const bf16* q, const bf16* k, bf16* o, const bf16* dO, const TcWs& w,
                           cudaStream_t st) {
-    constexpr size_t sm = out_smem<DV, true>();
-    TC_TRY(smem_attr(tc_out_kernel<DV, true>, sm));
-    SF_LAUNCH("tc_out_og", st, tc_out_kernel<DV, true><<<dim3(s.NC, s.BH), 128, sm, st>>>(
-                                   s, q, k, w.Gc, w.Vnt, w.S0t, o, dO, w.dVit, w.Dt));
-    return cudaGetLastError();
+    return launch_out2<DV, true>("tc_out_og", s, q, k, o, dO, w, st);
 }
 
 template <int DV>
@@ -2424,18 +2616,6 @@ cudaError_t launch_scan_bwd(const SeqView& s, const BwdArgs& a, bool with_sr, co
     }
 }
 
-int num_sms() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0, v = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess &&
-            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
-            n = v;
-        else
-            n = 148;
-    }
-    return n;
-}
 
 // Persistent: one CTA per SM at most; the CTAs take chunks from w.ticket, so
 // they stay balanced when other kernels hold some of the SMs.
@@ -2453,42 +2633,12 @@ cudaError_t launch_grad(const SeqView& s, const BwdArgs& a, const TcWs& w, cudaS
     return cudaGetLastError();
 }
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (the
-// library does not link the driver library); null if the driver lacks it.
-PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
-    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q{};
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            p = nullptr;
-        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }();
-    return fn;
-}
-
-// The five-dimensional canon view of a [BH][T][D] bf16 tensor (head stride hs
-// elements) described at G5Maps; false if it cannot be made (no driver entry
-// point, a base not 16-byte aligned, fewer than C tokens).
-bool canon_map(CUtensorMap* m, const void* base, int BH, int T, int D, long long hs) {
-    const PFN_cuTensorMapEncodeTiled_v12000 enc = encode_tiled();
-    if (!enc || T < C || BH < 1 || (reinterpret_cast<uintptr_t>(base) & 15)) return false;
-    const cuuint64_t dims[5] = {8, 8, (cuuint64_t)(D / 8), (cuuint64_t)(T / 8), (cuuint64_t)BH};
-    const cuuint64_t strides[4] = {(cuuint64_t)D * 2, 16, (cuuint64_t)D * 16, (cuuint64_t)hs * 2};
-    const cuuint32_t box[5] = {8, 8, (cuuint32_t)(D / 8), C / 8, 1};
-    const cuuint32_t unit[5] = {1, 1, 1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, unit,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int DV, bool BETA>
 cudaError_t launch_grad5(const SeqView& s, const BwdArgs& a, const TcWs& w, cudaStream_t st) {
     constexpr size_t sm = G5<DV>::SMEM;
     TC_TRY(smem_attr(tc_grad5_kernel<DV, BETA>, sm));
     TC_TRY(cudaMemsetAsync(w.ticket, 0, sizeof(int), st));
-    const int grid = std::min(s.NC * s.BH, num_sms());
+    const int grid = persistent_grid(s);
     G5Maps maps;
     memset(&maps, 0, sizeof(maps));
     maps.on = canon_map(&maps.q, a.q, s.BH, s.T, DK, s.hs_k) && canon_map(&maps.k, a.k, s.BH, s.T, DK, s.hs_k) &&
