@@ -63,16 +63,16 @@ __device__ int g_tc_status = 0;
 struct TcWs {
     float* Gc;   // [BH][Tp]           chunk-local cumulative log-decay G
     float* Gm;   // [BH][Tp]           exp(G)
-    bf16* W;     // [BH][Tp][DK]       -W (negated: the scans only ever subtract W products; permuted, see swz)
+    bf16* W;     // [BH][Tp][DK]       -W (negated: the scans only ever subtract W products; canon per chunk)
     float* Lm;   // [BH][NC][C][C]     L = (I + A)^{-1} per chunk (delta path), for the gradient kernel
-    bf16* Kh;    // [BH][Tp][DK]       K * exp(G_C - G) (permuted)
-    bf16* Ut;    // [BH][NC][DV][C]    U transposed per chunk, V^T without the beta path (permuted)
+    bf16* Kh;    // [BH][Tp][DK]       K * exp(G_C - G) (canon per chunk)
+    bf16* Ut;    // [BH][NC][DV][C]    U transposed per chunk, V^T without the beta path (canon)
     bf16* Vnt;   // [BH][NC][DV][C]    V_new transposed per chunk (canon, see tc_umma.cuh)
     bf16* S0t;   // [BH][NC][DV][DK]   state entering each chunk, transposed (canon)
-    bf16* dVit;  // [BH][NC][DV][C]    intra-chunk part of dV_new, transposed (permuted)
+    bf16* dVit;  // [BH][NC][DV][C]    intra-chunk part of dV_new, transposed (canon)
     bf16* dVnt;  // [BH][NC][DV][C]    dV_new transposed (canon)
     bf16* dSCt;  // [BH][NC][DV][DK]   gradient of the state leaving each chunk, transposed (canon)
-    bf16* Dt;    // [BH][NC][DV][DK]   scale (gamma * dO)^T Q per chunk, transposed (permuted)
+    bf16* Dt;    // [BH][NC][DV][DK]   scale (gamma * dO)^T Q per chunk, transposed (canon)
     int* ticket;  // chunk counter of the persistent gradient kernel
     int* oticket;  // chunk counter of the persistent Out kernel
     size_t total;
@@ -254,8 +254,11 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ k, const bf16* __restrict__ v
     cp_async_commit();
     if (w == 0) chunk_cumsum(g + bh * s.hs_g + t0, nval, Gs, lane);
     for (int i = tid; i < C; i += 256) Bs[i] = (BETA && i < nval) ? beta[bh * s.hs_g + t0 + i] : 0.f;
-    if (BETA)
-        for (int e = tid; e < C * LDF; e += 256) Lf[e] = 0.f;
+    if (BETA)  // the blocks above the diagonal of L (block_inverse writes the others)
+        for (int e = tid; e < C * C / 4; e += 256) {
+            const int i = e >> 4, j = (e & 15) * 4;
+            if (j >= 16 * ((i >> 4) + 1)) *reinterpret_cast<float4*>(Lf + i * LDF + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     cp_async_wait<0>();
     __syncthreads();
 
@@ -266,15 +269,16 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ k, const bf16* __restrict__ v
         BGs[i] = Bs[i] * e;
     }
     const float gC = Gs[C - 1];
-    for (int e = tid; e < C * (DK / 8); e += 256) {
-        const int r = e >> 4, cc = (e & 15) * 8;
+    for (int e = tid; e < C * (DK / 8); e += 256) {  // canon tile, written in address order
+        int r, cc;
+        umma::canon_piece(e, DK, r, cc);
         const float d = __expf(gC - Gs[r]);
         uint4 x = *reinterpret_cast<const uint4*>(Ks + r * LDK + cc);
         x.x = scale2(x.x, d, d);
         x.y = scale2(x.y, d, d);
         x.z = scale2(x.z, d, d);
         x.w = scale2(x.w, d, d);
-        *reinterpret_cast<uint4*>(Kho + (bh * Tp + t0) * DK + swz(r, cc, DK)) = x;
+        reinterpret_cast<uint4*>(Kho + (bh * Tp + t0) * DK)[e] = x;
     }
 
     bf16* Ust = reinterpret_cast<bf16*>(Lf);  // [DV][LDC]
@@ -296,9 +300,12 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ k, const bf16* __restrict__ v
 #pragma unroll
             for (int nn = 0; nn < 4; ++nn)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = 16 * mw + gq + 8 * (e >> 1), j = 32 * nw + 8 * nn + 2 * tq + (e & 1);
-                    Af[i * LDF + j] = (j < i) ? Bs[i] * __expf(Gs[i] - Gs[j]) * acc[nn][e] : 0.f;
+                for (int h = 0; h < 2; ++h) {
+                    const int i = 16 * mw + gq + 8 * h, j = 32 * nw + 8 * nn + 2 * tq;
+                    float2 a2;
+                    a2.x = (j < i) ? Bs[i] * __expf(Gs[i] - Gs[j]) * acc[nn][2 * h] : 0.f;
+                    a2.y = (j + 1 < i) ? Bs[i] * __expf(Gs[i] - Gs[j + 1]) * acc[nn][2 * h + 1] : 0.f;
+                    *reinterpret_cast<float2*>(Af + i * LDF + j) = a2;
                 }
         }
         __syncthreads();
@@ -308,11 +315,23 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ k, const bf16* __restrict__ v
             const int i = e >> 4, j = (e & 15) * 4;
             *reinterpret_cast<float4*>(Lg + l_off(i, j)) = *reinterpret_cast<const float4*>(Lf + i * LDF + j);
         }
-        for (int e = tid; e < C * C; e += 256) {  // A is dead: its region takes the T tiles
-            const int i = e >> 6, j = e & 63;
-            const float l = Lf[i * LDF + j];
-            Tw[i * LDC + j] = __float2bfloat16_rn(l * BGs[j]);
-            Tu[i * LDC + j] = __float2bfloat16_rn(l * Bs[j]);
+        for (int e = tid; e < C * C / 8; e += 256) {  // A is dead: its region takes the T tiles
+            const int i = e >> 3, j = (e & 7) * 8;
+            float l[8], bg[8], b[8];
+            *reinterpret_cast<float4*>(l) = *reinterpret_cast<const float4*>(Lf + i * LDF + j);
+            *reinterpret_cast<float4*>(l + 4) = *reinterpret_cast<const float4*>(Lf + i * LDF + j + 4);
+            *reinterpret_cast<float4*>(bg) = *reinterpret_cast<const float4*>(BGs + j);
+            *reinterpret_cast<float4*>(bg + 4) = *reinterpret_cast<const float4*>(BGs + j + 4);
+            *reinterpret_cast<float4*>(b) = *reinterpret_cast<const float4*>(Bs + j);
+            *reinterpret_cast<float4*>(b + 4) = *reinterpret_cast<const float4*>(Bs + j + 4);
+            uint32_t tw[4], tu[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                tw[h] = pack(l[2 * h] * bg[2 * h], l[2 * h + 1] * bg[2 * h + 1]);
+                tu[h] = pack(l[2 * h] * b[2 * h], l[2 * h + 1] * b[2 * h + 1]);
+            }
+            *reinterpret_cast<uint4*>(Tw + i * LDC + j) = make_uint4(tw[0], tw[1], tw[2], tw[3]);
+            *reinterpret_cast<uint4*>(Tu + i * LDC + j) = make_uint4(tu[0], tu[1], tu[2], tu[3]);
         }
         __syncthreads();
         {  // U = T V, staged transposed into L's region
@@ -329,13 +348,15 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ k, const bf16* __restrict__ v
                     mma(acc[nn + 1], a, b[2], b[3]);
                 }
             }
+            // transposed by stmatrix: matrix m = (row half m % 2, n-tile nn + m / 2)
 #pragma unroll
-            for (int nn = 0; nn < DV / 16; ++nn)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = 16 * mw + gq + 8 * (e >> 1), col = (DV / 2) * nw + 8 * nn + 2 * tq + (e & 1);
-                    Ust[col * LDC + i] = __float2bfloat16_rn(acc[nn][e]);
-                }
+            for (int nn = 0; nn < DV / 16; nn += 2) {
+                const uint32_t fr[4] = {pack(acc[nn][0], acc[nn][1]), pack(acc[nn][2], acc[nn][3]),
+                                        pack(acc[nn + 1][0], acc[nn + 1][1]), pack(acc[nn + 1][2], acc[nn + 1][3])};
+                const int m = lane >> 3;
+                const int col = (DV / 2) * nw + 8 * (nn + (m >> 1)) + (lane & 7), i = 16 * mw + 8 * (m & 1);
+                stsm_x4_t(Ust + col * LDC + i, fr);
+            }
         }
         __syncthreads();  // V is dead: its region takes the W staging
         bf16* Wst = Vs;  // [C][LDK]
@@ -361,10 +382,10 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ k, const bf16* __restrict__ v
             }
         }
         __syncthreads();
-        for (int e = tid; e < C * (DK / 8); e += 256) {
-            const int r = e >> 4, cc = (e & 15) * 8;
-            *reinterpret_cast<uint4*>(Wo + (bh * Tp + t0) * DK + swz(r, cc, DK)) =
-                *reinterpret_cast<const uint4*>(Wst + r * LDK + cc);
+        for (int e = tid; e < C * (DK / 8); e += 256) {  // canon, in address order
+            int r, cc;
+            umma::canon_piece(e, DK, r, cc);
+            reinterpret_cast<uint4*>(Wo + (bh * Tp + t0) * DK)[e] = *reinterpret_cast<const uint4*>(Wst + r * LDK + cc);
         }
     } else {
         for (int e = tid; e < C * DV; e += 256) {
@@ -374,9 +395,10 @@ tc_prep_kernel(SeqView s, const bf16* __restrict__ k, const bf16* __restrict__ v
         __syncthreads();
     }
     bf16* Utg = Uto + ((size_t)bh * s.NC + c) * DV * C;
-    for (int e = tid; e < DV * (C / 8); e += 256) {
-        const int r = e >> 3, cc = (e & 7) * 8;
-        *reinterpret_cast<uint4*>(Utg + swz(r, cc, C)) = *reinterpret_cast<const uint4*>(Ust + r * LDC + cc);
+    for (int e = tid; e < DV * (C / 8); e += 256) {  // canon, in address order
+        int r, cc;
+        umma::canon_piece(e, C, r, cc);
+        reinterpret_cast<uint4*>(Utg)[e] = *reinterpret_cast<const uint4*>(Ust + r * LDC + cc);
     }
 }
 
@@ -409,8 +431,8 @@ __device__ __forceinline__ void og_products(const SeqView& s, const bf16* Qs, co
 #pragma unroll
         for (int nn = 0; nn < 8; ++nn) {
             const int r = m0 + gq, j = 8 * nn + 2 * tq;
-            *reinterpret_cast<uint32_t*>(dVi + swz(r, j, C)) = pack(acc[nn][0], acc[nn][1]);
-            *reinterpret_cast<uint32_t*>(dVi + swz(r + 8, j, C)) = pack(acc[nn][2], acc[nn][3]);
+            *reinterpret_cast<uint32_t*>(dVi + umma::canon_el(r, j, C)) = pack(acc[nn][0], acc[nn][1]);
+            *reinterpret_cast<uint32_t*>(dVi + umma::canon_el(r + 8, j, C)) = pack(acc[nn][2], acc[nn][3]);
         }
     }
     // D^T[v][d] = sum_t scale gamma_t dO[t][v] Q[t][d]
@@ -445,8 +467,8 @@ __device__ __forceinline__ void og_products(const SeqView& s, const bf16* Qs, co
 #pragma unroll
             for (int nn = 0; nn < 8; ++nn) {
                 const int r = m0 + gq, d = 64 * nh + 8 * nn + 2 * tq;
-                *reinterpret_cast<uint32_t*>(Dg + swz(r, d, DK)) = pack(acc[nn][0], acc[nn][1]);
-                *reinterpret_cast<uint32_t*>(Dg + swz(r + 8, d, DK)) = pack(acc[nn][2], acc[nn][3]);
+                *reinterpret_cast<uint32_t*>(Dg + umma::canon_el(r, d, DK)) = pack(acc[nn][0], acc[nn][1]);
+                *reinterpret_cast<uint32_t*>(Dg + umma::canon_el(r + 8, d, DK)) = pack(acc[nn][2], acc[nn][3]);
             }
         }
     }
@@ -562,28 +584,6 @@ struct Chain {
     static constexpr size_t SMEM = smem(kStages);
 };
 
-// Per-lane parts of the addresses into permuted [rows][128] tiles.
-//   B fragments (stored [n][k], k = 16kk..): row = n0 + lr, piece 2kk + pb
-//   B fragments (stored [k][n], trans):      row = k0 + lr, piece nn + pb (nn even)
-// with lr, pb the lane's row/piece offsets; the piece is XOR-ed with lr & 7.
-struct SwLane {
-    int row;   // lane row offset inside a 16-row group (times the row length is added by callers)
-    int lo;    // (pb ^ (lr & 1)) * 8   element offset of the low bit of the permuted piece
-    int hi8;   // (lr & 6) * 8          XOR mask for the even part of the piece
-};
-__device__ __forceinline__ SwLane sw_lane_nk(int lane) {  // ldmatrix non-trans, row = n, piece from k
-    const int lr = (lane & 7) + ((lane >> 4) << 3), pb = (lane >> 3) & 1;
-    return {lr, (pb ^ (lr & 1)) * 8, (lr & 6) * 8};
-}
-__device__ __forceinline__ SwLane sw_lane_kn(int lane) {  // ldmatrix trans, row = k, piece from n
-    const int lr = (lane & 7) + (((lane >> 3) & 1) << 3), pb = lane >> 4;
-    return {lr, (pb ^ (lr & 1)) * 8, (lr & 6) * 8};
-}
-// Element offset of the fragment row/piece for an even logical piece `pe`.
-__device__ __forceinline__ int sw_off(const SwLane& L, int rowbase, int pe, int rowlen) {
-    return (rowbase + L.row) * rowlen + ((pe * 8) ^ L.hi8) + L.lo;
-}
-
 __device__ __forceinline__ void put_frag(uint4* p, const uint32_t (&a)[4]) { *p = make_uint4(a[0], a[1], a[2], a[3]); }
 __device__ __forceinline__ void get_frag(const uint4* p, uint32_t (&a)[4]) {
     const uint4 v = *p;
@@ -597,10 +597,10 @@ __device__ __forceinline__ void slice_sync(int g) { asm volatile("bar.sync %0, 1
 
 // Operands of one chain launch, for one direction.
 struct ChainOps {
-    const bf16* X;      // [BH][Tp][DK] permuted: -W (forward) or Khat (backward)
-    const bf16* Y;      // [BH][Tp][DK] permuted: Khat (forward) or -W (backward)
-    const bf16* I;      // [BH][NC][DV][C] permuted: U^T or dVi^T
-    const bf16* E;      // [BH][NC][DV][DK] permuted: D^T (backward only)
+    const bf16* X;      // [BH][Tp][DK] canon per chunk: -W (forward) or Khat (backward)
+    const bf16* Y;      // [BH][Tp][DK] canon per chunk: Khat (forward) or -W (backward)
+    const bf16* I;      // [BH][NC][DV][C] canon: U^T or dVi^T
+    const bf16* E;      // [BH][NC][DV][DK] canon: D^T (backward only)
     const float* Gm;    // [BH][Tp] exp(G)
     const float* R_in;  // [BH][DK][DV] S_in or dS_out (NULL = zeros)
     bf16* Rt;           // [BH][NC][DV][DK] canon: S0^T or dS_C^T per chunk (NULL = skip)
@@ -667,7 +667,6 @@ __device__ __forceinline__ void chain_cta(const SeqView& s, int bh, int vb, cons
             const int vv = v0 + vr + gq + 8 * (e >> 1), d = 32 * q + 8 * j + 2 * tq + (e & 1);
             r[j][e] = op.R_in ? op.R_in[((size_t)bh * DK + d) * DV + vv] : 0.f;
         }
-    const SwLane Lnk = sw_lane_nk(lane), Lkn = sw_lane_kn(lane);
 
     if (tid == 0) {
         for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
@@ -700,9 +699,9 @@ __device__ __forceinline__ void chain_cta(const SeqView& s, int bh, int vb, cons
         float z[2][4];
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
-            const int po = (((2 * q + n) ^ gq) << 3) + 2 * tq;
-            const float2 u0 = unpack(*reinterpret_cast<const uint32_t*>(st.I + (vr + gq) * C + po));
-            const float2 u1 = unpack(*reinterpret_cast<const uint32_t*>(st.I + (vr + gq + 8) * C + po));
+            const int tc0 = 16 * q + 8 * n + 2 * tq;
+            const float2 u0 = unpack(*umma::canon_at<uint32_t>(st.I, vr + gq, tc0, C));
+            const float2 u1 = unpack(*umma::canon_at<uint32_t>(st.I, vr + gq + 8, tc0, C));
             z[n][0] = u0.x;
             z[n][1] = u0.y;
             z[n][2] = u1.x;
@@ -723,7 +722,7 @@ __device__ __forceinline__ void chain_cta(const SeqView& s, int bh, int vb, cons
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 uint32_t b[4];
-                ldsm_x4(b, st.X + sw_off(Lnk, 16 * q, 2 * kk, DK));
+                umma::ldBnk_c(b, st.X, DK, 16 * q, 16 * kk, lane);
                 if (kk & 1) {
                     mma(zq[0], ra[kk], b[0], b[1]);
                     mma(zq[1], ra[kk], b[2], b[3]);
@@ -747,8 +746,8 @@ __device__ __forceinline__ void chain_cta(const SeqView& s, int bh, int vb, cons
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int col = 32 * q + 8 * j + 2 * tq;
-                const float2 d0 = unpack(*reinterpret_cast<const uint32_t*>(st.E + swz(vr + gq, col, DK)));
-                const float2 d1 = unpack(*reinterpret_cast<const uint32_t*>(st.E + swz(vr + gq + 8, col, DK)));
+                const float2 d0 = unpack(*umma::canon_at<uint32_t>(st.E, vr + gq, col, DK));
+                const float2 d1 = unpack(*umma::canon_at<uint32_t>(st.E, vr + gq + 8, col, DK));
                 r[j][0] = fmaf(r[j][0], gamC, d0.x);
                 r[j][1] = fmaf(r[j][1], gamC, d0.y);
                 r[j][2] = fmaf(r[j][2], gamC, d1.x);
@@ -777,7 +776,7 @@ __device__ __forceinline__ void chain_cta(const SeqView& s, int bh, int vb, cons
 #pragma unroll
                 for (int n2 = 0; n2 < 2; ++n2) {
                     uint32_t b[4];
-                    ldsm_x4_t(b, st.Y + sw_off(Lkn, 16 * kt, 4 * q + 2 * n2, DK));
+                    umma::ldBkn_c(b, st.Y, DK, 32 * q + 16 * n2, 16 * kt, lane);
                     mma(r[2 * n2], zf[kt], b[0], b[1]);
                     mma(r[2 * n2 + 1], zf[kt], b[2], b[3]);
                 }
@@ -830,6 +829,243 @@ tc_scan_bwd_dual_kernel(SeqView s, ChainOps op_f, ChainOps op_b, int nsr) {
     }
 }
 
+// ------------------------------------------------- state scans, tcgen05 ---
+// The same step (see chain_cta) with the whole state of a head in one CTA, on
+// the fifth-generation tensor cores (d_v = 128): R (S^T or dS^T, fp32) lives
+// in TMEM, lane v = state row v, columns 0..127 = d_k; warp w's threads own
+// lanes 32 w.. (thread = state row).  Per chunk:
+//   every thread loads its row of R, writes it as bf16 into a canon [d_v][d_k]
+//   tile (the A operand of product 1 and the chunk's R output) and stores
+//   gamma_C R (+ E) back;
+//   product 1: Z^T = R X^T, M = 128, N = C, K = d_k, into TMEM columns 128..;
+//   every thread adds its row of I^T and writes Z^T as bf16 into a canon
+//   [d_v][C] tile (the A operand of product 2 and the chunk's Z output);
+//   product 2: R += Z^T Y, M = 128, N = d_k, K = C, accumulating on the
+//   scaled R.
+// One CTA per head instead of d_v / 32 CTAs of warp-level products: a quarter
+// of the SMs and of the operand reads (each head's X and Y tiles are read
+// once), the products at the full M = 128 rate.
+template <bool BETA, bool BWD>
+struct Chain5 {
+    static constexpr bool HAS_X = BWD || BETA;
+    static constexpr bool HAS_Y = !BWD || BETA;
+    static constexpr uint32_t kI = 128 * C * 2;              // I^T, canon [d_v][C]
+    static constexpr uint32_t kE = BWD ? 128 * DK * 2 : 0;   // E, canon [d_v][d_k]
+    static constexpr uint32_t kX = HAS_X ? kTileK : 0, kY = HAS_Y ? kTileK : 0;
+    static constexpr uint32_t TX = kX + kY + kI + C * 4 + kE;  // one stage, all copied
+    static constexpr size_t kR = (size_t)128 * DK * 2;         // R as bf16, canon [d_v][d_k]
+    static constexpr size_t kZ = (size_t)128 * C * 2;          // Z^T as bf16, canon [d_v][C]
+    static constexpr size_t smem(int st) { return st * (size_t)TX + kR + kZ + 8 * (st + 2) + 16; }
+    static constexpr int kStages = smem(4) <= 227 * 1024 ? 4 : smem(3) <= 227 * 1024 ? 3 : 2;
+    static constexpr size_t SMEM = smem(kStages);
+};
+
+template <bool BETA, bool BWD>
+__device__ __forceinline__ void chain5_cta(const SeqView& s, int bh, const ChainOps& op, unsigned char* smem) {
+    using CH = Chain5<BETA, BWD>;
+    constexpr int NS = CH::kStages;
+    constexpr int DV = 128;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int v = 32 * w + lane;  // this thread's state row = TMEM lane
+    const size_t Tp = (size_t)s.NC * C;
+    bf16* Rb = reinterpret_cast<bf16*>(smem + NS * (size_t)CH::TX);
+    bf16* Zb = reinterpret_cast<bf16*>(smem + NS * (size_t)CH::TX + CH::kR);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NS * (size_t)CH::TX + CH::kR + CH::kZ);  // [NS]
+    uint64_t* bM1 = bars + NS;
+    uint64_t* bM2 = bars + NS + 1;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + NS + 2);
+    bool failed = false;
+    const bool outputs = op.Rt || op.Zt;
+
+    auto chunk_of = [&](int i) { return BWD ? s.NC - 1 - i : i; };
+    struct Stage {
+        bf16 *X, *Y, *I, *E;
+        float* G;
+    };
+    auto stage = [&](int buf) {
+        unsigned char* p = smem + buf * (size_t)CH::TX;
+        Stage st;
+        st.X = reinterpret_cast<bf16*>(p);
+        st.Y = reinterpret_cast<bf16*>(p + CH::kX);
+        st.I = reinterpret_cast<bf16*>(p + CH::kX + CH::kY);
+        st.G = reinterpret_cast<float*>(p + CH::kX + CH::kY + CH::kI);
+        st.E = reinterpret_cast<bf16*>(p + CH::kX + CH::kY + CH::kI + C * 4);
+        return st;
+    };
+    auto load = [&](int i) {  // thread 0: bulk copies of step i's operands
+        const int cc = chunk_of(i), buf = i % NS;
+        const Stage st = stage(buf);
+        const size_t row0 = (size_t)bh * Tp + (size_t)cc * C;
+        const size_t blk = ((size_t)bh * s.NC + cc) * DV;
+        mbar_expect_tx(&bars[buf], CH::TX);
+        if (CH::HAS_X) bulk_load(st.X, op.X + row0 * DK, kTileK, &bars[buf]);
+        if (CH::HAS_Y) bulk_load(st.Y, op.Y + row0 * DK, kTileK, &bars[buf]);
+        bulk_load(st.I, op.I + blk * C, CH::kI, &bars[buf]);
+        bulk_load(st.G, op.Gm + row0, C * 4, &bars[buf]);
+        if (BWD) bulk_load(st.E, op.E + blk * DK, CH::kE, &bars[buf]);
+    };
+
+    if (tid == 0) {
+        for (int i = 0; i < NS + 2; ++i) mbar_init(&bars[i], 1);
+        mbar_init_fence();
+    }
+    if (w == 0) umma::alloc(tslot, 256);
+    __syncthreads();
+    umma::fence_after();
+    const uint32_t tm = *tslot;
+    const uint32_t trow = umma::taddr(tm, 32 * w, 0);
+    constexpr uint32_t ZC = 128;  // TMEM column of Z^T
+    if (tid == 0)
+        for (int i = 0; i < NS - 1 && i < s.NC; ++i) load(i);
+    // the entering state: R[v][d] = R_in[d][v]
+#pragma unroll 1
+    for (int g = 0; g < 4; ++g) {
+        float x[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = op.R_in ? op.R_in[((size_t)bh * DK + 32 * g + j) * DV + v] : 0.f;
+        umma::st_row32(trow + 32 * g, x);
+    }
+    umma::wait_st();
+
+    constexpr uint32_t I1 = umma::idesc_bf16(128, C, false, false);
+    constexpr uint32_t I2 = umma::idesc_bf16(128, DK, false, true);
+    for (int i = 0; i < s.NC; ++i) {
+        const Stage st = stage(i % NS);
+        mbar_wait(&bars[i % NS], (i / NS) & 1, &g_tc_status, failed);
+        if (CH::HAS_Y && i > 0) mbar_wait(bM2, (i - 1) & 1, &g_tc_status, failed);  // R updated
+        umma::fence_after();
+        if (tid == 0) {
+            // step i-1's buffer is free (its product 2 has completed)
+            if (i + NS - 1 < s.NC) load(i + NS - 1);
+            if (outputs && i > 0) bulk_wait_read<0>();  // step i-1's outputs have left Rb, Zb
+        }
+        __syncthreads();
+        const float gamC = st.G[C - 1];
+        // R -> bf16 canon row (product 1's A, the chunk's R output); gamma_C R (+ E) back into TMEM
+#pragma unroll 1
+        for (int g = 0; g < 4; ++g) {
+            float x[32];
+            umma::ld_row32(trow + 32 * g, x);
+            umma::wait_ld();
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                uint4 o;
+                o.x = pack(x[8 * p], x[8 * p + 1]);
+                o.y = pack(x[8 * p + 2], x[8 * p + 3]);
+                o.z = pack(x[8 * p + 4], x[8 * p + 5]);
+                o.w = pack(x[8 * p + 6], x[8 * p + 7]);
+                *umma::canon_at<uint4>(Rb, v, 32 * g + 8 * p, DK) = o;
+            }
+            if (BWD) {
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const uint4 e = *umma::canon_at<uint4>(st.E, v, 32 * g + 8 * p, DK);
+                    const uint32_t ev[4] = {e.x, e.y, e.z, e.w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const float2 f = unpack(ev[h]);
+                        x[8 * p + 2 * h] = fmaf(x[8 * p + 2 * h], gamC, f.x);
+                        x[8 * p + 2 * h + 1] = fmaf(x[8 * p + 2 * h + 1], gamC, f.y);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) x[j] *= gamC;
+            }
+            umma::st_row32(trow + 32 * g, x);
+        }
+        fence_proxy_async_smem();
+        umma::wait_st();
+        umma::fence_before();
+        __syncthreads();  // Rb complete, R scaled
+        if (tid == 0) {
+            umma::fence_after();
+            if (CH::HAS_X) {
+                umma::chain<DK / 16>(tm + ZC, I1, false, umma::op_k(Rb, DK), umma::op_k(st.X, DK));
+                umma::commit(bM1);
+            }
+            if (op.Rt) bulk_store(op.Rt + ((size_t)bh * s.NC + chunk_of(i)) * DV * DK, Rb, (uint32_t)CH::kR);
+        }
+        // Z^T = I^T (+ R X^T) -> bf16 canon row
+        {
+            if (CH::HAS_X) {
+                mbar_wait(bM1, i & 1, &g_tc_status, failed);
+                umma::fence_after();
+            }
+#pragma unroll 1
+            for (int g = 0; g < 2; ++g) {
+                float z[32];
+                if (CH::HAS_X) {
+                    umma::ld_row32(trow + ZC + 32 * g, z);
+                    umma::wait_ld();
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) z[j] = 0.f;
+                }
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const uint4 u = *umma::canon_at<uint4>(st.I, v, 32 * g + 8 * p, C);
+                    const uint32_t uv[4] = {u.x, u.y, u.z, u.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const float2 f = unpack(uv[h]);
+                        o[h] = pack(f.x + z[8 * p + 2 * h], f.y + z[8 * p + 2 * h + 1]);
+                    }
+                    *umma::canon_at<uint4>(Zb, v, 32 * g + 8 * p, C) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        umma::fence_before();
+        __syncthreads();  // Zb complete; I, E, G of this stage read
+        if (tid == 0) {
+            umma::fence_after();
+            if (CH::HAS_Y) {
+                umma::chain<C / 16>(tm, I2, true, umma::op_k(Zb, C), umma::op_mn(st.Y, DK));
+                umma::commit(bM2);
+            }
+            if (op.Zt) bulk_store(op.Zt + ((size_t)bh * s.NC + chunk_of(i)) * DV * C, Zb, (uint32_t)CH::kZ);
+            if (outputs) bulk_commit();
+        }
+    }
+    if (CH::HAS_Y && s.NC > 0) mbar_wait(bM2, (s.NC - 1) & 1, &g_tc_status, failed);
+    umma::fence_after();
+    if (op.R_out) {
+#pragma unroll 1
+        for (int g = 0; g < 4; ++g) {
+            float x[32];
+            umma::ld_row32(trow + 32 * g, x);
+            umma::wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) op.R_out[((size_t)bh * DK + 32 * g + j) * DV + v] = x[j];
+        }
+    }
+    if (tid == 0 && outputs) bulk_wait<0>();
+    umma::fence_before();
+    __syncthreads();
+    if (w == 0) {
+        umma::fence_after();
+        umma::dealloc(tm, 256);
+    }
+}
+
+template <bool BETA>
+__global__ void __launch_bounds__(128, 1) tc_chain5_fwd_kernel(SeqView s, ChainOps op) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    chain5_cta<BETA, false>(s, blockIdx.x, op, smem);
+}
+// Blocks [0, nsr) recompute the forward states (op_f), the rest run the
+// reverse state-gradient scan (op_b).
+template <bool BETA>
+__global__ void __launch_bounds__(128, 1) tc_chain5_bwd_kernel(SeqView s, ChainOps op_f, ChainOps op_b, int nsr) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    if ((int)blockIdx.x < nsr)
+        chain5_cta<BETA, false>(s, blockIdx.x, op_f, smem);
+    else
+        chain5_cta<BETA, true>(s, blockIdx.x - nsr, op_b, smem);
+}
+
 // ------------------------------------------------------------------- out ---
 // Tensor maps of the token-major tiles a kernel copies by TMA (see canon_map):
 // q, k and dO in canon layout; `on` is 0 when they could not be made, and
@@ -876,8 +1112,8 @@ __device__ __forceinline__ void og_products8(const SeqView& s, const bf16* Qs, c
 #pragma unroll
         for (int nn = 0; nn < NVI; ++nn) {
             const int r = m0 + gq, j = n0 + 8 * nn + 2 * tq;
-            *reinterpret_cast<uint32_t*>(dVi + swz(r, j, C)) = pack(acc[nn][0], acc[nn][1]);
-            *reinterpret_cast<uint32_t*>(dVi + swz(r + 8, j, C)) = pack(acc[nn][2], acc[nn][3]);
+            *reinterpret_cast<uint32_t*>(dVi + umma::canon_el(r, j, C)) = pack(acc[nn][0], acc[nn][1]);
+            *reinterpret_cast<uint32_t*>(dVi + umma::canon_el(r + 8, j, C)) = pack(acc[nn][2], acc[nn][3]);
         }
     }
     // D^T[v][d] = sum_t scale gamma_t dO[t][v] Q[t][d]
@@ -911,8 +1147,8 @@ __device__ __forceinline__ void og_products8(const SeqView& s, const bf16* Qs, c
 #pragma unroll
         for (int nn = 0; nn < 8; ++nn) {
             const int r = m0 + gq, d = d0 + 8 * nn + 2 * tq;
-            *reinterpret_cast<uint32_t*>(Dg + swz(r, d, DK)) = pack(acc[nn][0], acc[nn][1]);
-            *reinterpret_cast<uint32_t*>(Dg + swz(r + 8, d, DK)) = pack(acc[nn][2], acc[nn][3]);
+            *reinterpret_cast<uint32_t*>(Dg + umma::canon_el(r, d, DK)) = pack(acc[nn][0], acc[nn][1]);
+            *reinterpret_cast<uint32_t*>(Dg + umma::canon_el(r + 8, d, DK)) = pack(acc[nn][2], acc[nn][3]);
         }
     }
 }
@@ -2502,8 +2738,40 @@ cudaError_t launch_scan_fwd_n(const SeqView& s, const float* S_in, float* S_out,
                   s, fwd_ops(w, S_in, S_out)));
     return cudaGetLastError();
 }
+// The state chains of d_v = 128 run on tcgen05 (one CTA per head) unless
+// SF_GDN_CHAIN=warp selects the warp-level chains (read once); d_v = 64 always
+// takes the warp-level chains.
+bool chain_tcgen05() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = std::getenv("SF_GDN_CHAIN");
+        v = (e && std::string(e) == "tcgen05") ? 1 : 0;
+    }
+    return v == 1;
+}
+
+template <bool BETA>
+cudaError_t launch_chain5_fwd(const SeqView& s, const float* S_in, float* S_out, const TcWs& w, cudaStream_t st) {
+    constexpr size_t sm = Chain5<BETA, false>::SMEM;
+    TC_TRY(smem_attr(tc_chain5_fwd_kernel<BETA>, sm));
+    SF_LAUNCH("tc_scan_fwd", st, tc_chain5_fwd_kernel<BETA><<<s.BH, 128, sm, st>>>(s, fwd_ops(w, S_in, S_out)));
+    return cudaGetLastError();
+}
+template <bool BETA>
+cudaError_t launch_chain5_bwd(const SeqView& s, const BwdArgs& a, bool with_sr, const TcWs& w, cudaStream_t st) {
+    constexpr size_t sm_f = Chain5<BETA, false>::SMEM, sm_b = Chain5<BETA, true>::SMEM;
+    constexpr size_t sm = sm_f > sm_b ? sm_f : sm_b;
+    TC_TRY(smem_attr(tc_chain5_bwd_kernel<BETA>, sm));
+    const int nsr = with_sr ? s.BH : 0;
+    SF_LAUNCH("tc_scan_bwd", st,
+              tc_chain5_bwd_kernel<BETA><<<nsr + s.BH, 128, sm, st>>>(
+                  s, fwd_ops(w, a.S_in, nullptr), bwd_ops(w, a.dS_out, a.dS_in), nsr));
+    return cudaGetLastError();
+}
+
 template <int DV, bool BETA>
 cudaError_t launch_scan_fwd(const SeqView& s, const float* S_in, float* S_out, const TcWs& w, cudaStream_t st) {
+    if (DV == 128 && chain_tcgen05()) return launch_chain5_fwd<BETA>(s, S_in, S_out, w, st);
     switch (chain_slices()) {
         case 4: return DV % 64 == 0 ? launch_scan_fwd_n<DV, BETA, 4>(s, S_in, S_out, w, st) : cudaErrorInvalidValue;
         case 2: return launch_scan_fwd_n<DV, BETA, 2>(s, S_in, S_out, w, st);
@@ -2609,6 +2877,7 @@ cudaError_t launch_scan_bwd_n(const SeqView& s, const BwdArgs& a, bool with_sr, 
 }
 template <int DV, bool BETA>
 cudaError_t launch_scan_bwd(const SeqView& s, const BwdArgs& a, bool with_sr, const TcWs& w, cudaStream_t st) {
+    if (DV == 128 && chain_tcgen05()) return launch_chain5_bwd<BETA>(s, a, with_sr, w, st);
     switch (chain_slices()) {
         case 4: return launch_scan_bwd_n<DV, BETA, 4>(s, a, with_sr, w, st);
         case 2: return launch_scan_bwd_n<DV, BETA, 2>(s, a, with_sr, w, st);

@@ -124,6 +124,14 @@ __device__ __forceinline__ void stsm_x4(void* p, const uint32_t (&r)[4]) {
                  : "memory");
 }
 
+// stmatrix with transpose: matrix m's row r (address from lane 8 m + r)
+// receives column r of the fragment-layout 8x8 block held in register m.
+__device__ __forceinline__ void stsm_x4_t(void* p, const uint32_t (&r)[4]) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};\n" ::"r"(smem_u32(p)),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+                 : "memory");
+}
+
 // mbarrier-tracked bulk asynchronous global -> shared copy (issued by one thread).
 __device__ __forceinline__ void mbar_init(void* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -186,15 +194,6 @@ __device__ __forceinline__ void mbar_wait(void* bar, uint32_t parity, int* statu
     }
 }
 
-// Tiles written by the state scans are stored with the 16-byte pieces of every
-// row permuted, piece p of row r at position p ^ (r & 7), so that the scan can
-// stage them in shared memory without bank conflicts and write them out with
-// one linear bulk copy.  Element offset of (r, col) in such a tile of row
-// length `cols` (a multiple of 64):
-__device__ __forceinline__ int swz(int r, int col, int cols) {
-    return r * cols + ((((col >> 3) ^ (r & 7))) << 3) + (col & 7);
-}
-
 // Copy a [rows][cols] bf16 global tile (row stride gld elements) into shared
 // memory (row stride sld), 16 bytes per request, rows >= nrows zero-filled.
 template <int ROWS, int COLS, int NT>
@@ -205,16 +204,6 @@ __device__ __forceinline__ void load_tile(__nv_bfloat16* s, int sld, const __nv_
         const int r = e / CPR, c = (e % CPR) * 8;
         const bool ok = r < nrows;
         cp_async16(s + r * sld + c, g + (ok ? (long long)r * gld : 0) + c, ok);
-    }
-}
-
-// As load_tile, for a global tile stored with the piece permutation of swz().
-template <int ROWS, int COLS, int NT>
-__device__ __forceinline__ void load_tile_swz(__nv_bfloat16* s, int sld, const __nv_bfloat16* g, int tid) {
-    constexpr int CPR = COLS / 8;
-    for (int e = tid; e < ROWS * CPR; e += NT) {
-        const int r = e / CPR, c = e % CPR;
-        cp_async16(s + r * sld + c * 8, g + (long long)r * COLS + ((c ^ (r & 7)) << 3), true);
     }
 }
 

@@ -37,6 +37,15 @@ using tc::smem_u32;
 __host__ __device__ __forceinline__ uint32_t canon_off(int r, int c, int rowlen) {
     return (uint32_t)((r >> 3) * (16 * rowlen) + (c >> 3) * 128 + (r & 7) * 16 + (c & 7) * 2);
 }
+// Element offset of (r, c) in a canon bf16 tile.
+__host__ __device__ __forceinline__ int canon_el(int r, int c, int rowlen) { return (int)(canon_off(r, c, rowlen) >> 1); }
+// Row and column of the e-th 16-byte piece of a canon [rows][rowlen] tile
+// (pieces in address order), for copies that write the tile linearly.
+__host__ __device__ __forceinline__ void canon_piece(int e, int rowlen, int& r, int& c) {
+    const int per_rb = rowlen;  // pieces in one 8-row block: 8 rows x rowlen / 8
+    r = (e / per_rb) * 8 + (e & 7);
+    c = ((e % per_rb) >> 3) * 8;
+}
 template <typename T>
 __device__ __forceinline__ T* canon_at(void* base, int r, int c, int rowlen) {
     return reinterpret_cast<T*>(static_cast<char*>(base) + canon_off(r, c, rowlen));
@@ -161,6 +170,37 @@ __device__ __forceinline__ void st32(uint32_t ta, const float (&c)[4][4]) {
         "r"(__float_as_uint(c[2][1])), "r"(__float_as_uint(c[2][2])), "r"(__float_as_uint(c[2][3])),
         "r"(__float_as_uint(c[3][0])), "r"(__float_as_uint(c[3][1])), "r"(__float_as_uint(c[3][2])),
         "r"(__float_as_uint(c[3][3]))
+        : "memory");
+}
+// 32 TMEM columns of this thread's lane (the 32x32b shape: warp w % 4 reads
+// lanes 32 (w % 4).., thread t lane 32 (w % 4) + t; register j = column + j).
+__device__ __forceinline__ void ld_row32(uint32_t ta, float (&c)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%"
+        "19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(ta));
+#pragma unroll
+    for (int j = 0; j < 32; ++j) c[j] = __uint_as_float(r[j]);
+}
+__device__ __forceinline__ void st_row32(uint32_t ta, const float (&c)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(ta),
+        "r"(__float_as_uint(c[0])), "r"(__float_as_uint(c[1])), "r"(__float_as_uint(c[2])), "r"(__float_as_uint(c[3])),
+        "r"(__float_as_uint(c[4])), "r"(__float_as_uint(c[5])), "r"(__float_as_uint(c[6])), "r"(__float_as_uint(c[7])),
+        "r"(__float_as_uint(c[8])), "r"(__float_as_uint(c[9])), "r"(__float_as_uint(c[10])), "r"(__float_as_uint(c[11])),
+        "r"(__float_as_uint(c[12])), "r"(__float_as_uint(c[13])), "r"(__float_as_uint(c[14])),
+        "r"(__float_as_uint(c[15])), "r"(__float_as_uint(c[16])), "r"(__float_as_uint(c[17])),
+        "r"(__float_as_uint(c[18])), "r"(__float_as_uint(c[19])), "r"(__float_as_uint(c[20])),
+        "r"(__float_as_uint(c[21])), "r"(__float_as_uint(c[22])), "r"(__float_as_uint(c[23])),
+        "r"(__float_as_uint(c[24])), "r"(__float_as_uint(c[25])), "r"(__float_as_uint(c[26])),
+        "r"(__float_as_uint(c[27])), "r"(__float_as_uint(c[28])), "r"(__float_as_uint(c[29])),
+        "r"(__float_as_uint(c[30])), "r"(__float_as_uint(c[31]))
         : "memory");
 }
 __device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }

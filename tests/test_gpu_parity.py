@@ -96,7 +96,7 @@ def test_empty_inputs():
 
 # --------------------------------------------------------- bf16 I/O mode ---
 
-@pytest.mark.parametrize("dk,dv,beta", [(128, 128, True), (128, 64, False), (128, 64, True),
+@pytest.mark.parametrize("dk,dv,beta", [(128, 128, True), (128, 128, False), (128, 64, False), (128, 64, True),
                                         (64, 64, True)])
 def test_bf16_small(dk, dv, beta):
     w = small(io="bf16", dk=dk, dv=dv, use_beta=beta, qk="l2norm" if beta else "scaled",
