@@ -832,8 +832,9 @@ tc_scan_bwd_dual_kernel(SeqView s, ChainOps op_f, ChainOps op_b, int nsr) {
 // ------------------------------------------------- state scans, tcgen05 ---
 // The same step (see chain_cta) with the whole state of a head in one CTA, on
 // the fifth-generation tensor cores (d_v = 128): R (S^T or dS^T, fp32) lives
-// in TMEM, lane v = state row v, columns 0..127 = d_k; warp w's threads own
-// lanes 32 w.. (thread = state row).  Per chunk:
+// in TMEM, lane v = state row v, columns 0..127 = d_k; 8 warps, warp w's
+// threads own lanes 32 (w % 4).. (thread = state row) and half of each row's
+// columns (w / 4).  Per chunk:
 //   every thread loads its row of R, writes it as bf16 into a canon [d_v][d_k]
 //   tile (the A operand of product 1 and the chunk's R output) and stores
 //   gamma_C R (+ E) back;
@@ -866,7 +867,8 @@ __device__ __forceinline__ void chain5_cta(const SeqView& s, int bh, const Chain
     constexpr int NS = CH::kStages;
     constexpr int DV = 128;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    const int v = 32 * w + lane;  // this thread's state row = TMEM lane
+    const int v = 32 * (w & 3) + lane;  // this thread's state row = TMEM lane
+    const int hf = w >> 2;              // the half of the row's columns this thread handles
     const size_t Tp = (size_t)s.NC * C;
     bf16* Rb = reinterpret_cast<bf16*>(smem + NS * (size_t)CH::TX);
     bf16* Zb = reinterpret_cast<bf16*>(smem + NS * (size_t)CH::TX + CH::kR);
@@ -913,17 +915,18 @@ __device__ __forceinline__ void chain5_cta(const SeqView& s, int bh, const Chain
     __syncthreads();
     umma::fence_after();
     const uint32_t tm = *tslot;
-    const uint32_t trow = umma::taddr(tm, 32 * w, 0);
+    const uint32_t trow = umma::taddr(tm, 32 * (w & 3), 0);
+    const int rc0 = 64 * hf, zc0 = 32 * hf;  // first R and Z^T column of this thread
     constexpr uint32_t ZC = 128;  // TMEM column of Z^T
     if (tid == 0)
         for (int i = 0; i < NS - 1 && i < s.NC; ++i) load(i);
     // the entering state: R[v][d] = R_in[d][v]
 #pragma unroll 1
-    for (int g = 0; g < 4; ++g) {
+    for (int g = 0; g < 2; ++g) {
         float x[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = op.R_in ? op.R_in[((size_t)bh * DK + 32 * g + j) * DV + v] : 0.f;
-        umma::st_row32(trow + 32 * g, x);
+        for (int j = 0; j < 32; ++j) x[j] = op.R_in ? op.R_in[((size_t)bh * DK + rc0 + 32 * g + j) * DV + v] : 0.f;
+        umma::st_row32(trow + rc0 + 32 * g, x);
     }
     umma::wait_st();
 
@@ -934,50 +937,28 @@ __device__ __forceinline__ void chain5_cta(const SeqView& s, int bh, const Chain
         mbar_wait(&bars[i % NS], (i / NS) & 1, &g_tc_status, failed);
         if (CH::HAS_Y && i > 0) mbar_wait(bM2, (i - 1) & 1, &g_tc_status, failed);  // R updated
         umma::fence_after();
+        float x[64];  // this thread's half row of R
+#pragma unroll
+        for (int g = 0; g < 2; ++g) umma::ld_row32(trow + rc0 + 32 * g, *reinterpret_cast<float(*)[32]>(x + 32 * g));
         if (tid == 0) {
-            // step i-1's buffer is free (its product 2 has completed)
+            // step i-1's buffer is free (its products have completed)
             if (i + NS - 1 < s.NC) load(i + NS - 1);
             if (outputs && i > 0) bulk_wait_read<0>();  // step i-1's outputs have left Rb, Zb
         }
-        __syncthreads();
-        const float gamC = st.G[C - 1];
-        // R -> bf16 canon row (product 1's A, the chunk's R output); gamma_C R (+ E) back into TMEM
-#pragma unroll 1
-        for (int g = 0; g < 4; ++g) {
-            float x[32];
-            umma::ld_row32(trow + 32 * g, x);
-            umma::wait_ld();
+        umma::wait_ld();
+        __syncthreads();  // Rb and Zb may be rewritten
+        // R as bf16 into its canon row: product 1's A and the chunk's R output
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                uint4 o;
-                o.x = pack(x[8 * p], x[8 * p + 1]);
-                o.y = pack(x[8 * p + 2], x[8 * p + 3]);
-                o.z = pack(x[8 * p + 4], x[8 * p + 5]);
-                o.w = pack(x[8 * p + 6], x[8 * p + 7]);
-                *umma::canon_at<uint4>(Rb, v, 32 * g + 8 * p, DK) = o;
-            }
-            if (BWD) {
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const uint4 e = *umma::canon_at<uint4>(st.E, v, 32 * g + 8 * p, DK);
-                    const uint32_t ev[4] = {e.x, e.y, e.z, e.w};
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const float2 f = unpack(ev[h]);
-                        x[8 * p + 2 * h] = fmaf(x[8 * p + 2 * h], gamC, f.x);
-                        x[8 * p + 2 * h + 1] = fmaf(x[8 * p + 2 * h + 1], gamC, f.y);
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) x[j] *= gamC;
-            }
-            umma::st_row32(trow + 32 * g, x);
+        for (int p = 0; p < 8; ++p) {
+            uint4 o;
+            o.x = pack(x[8 * p], x[8 * p + 1]);
+            o.y = pack(x[8 * p + 2], x[8 * p + 3]);
+            o.z = pack(x[8 * p + 4], x[8 * p + 5]);
+            o.w = pack(x[8 * p + 6], x[8 * p + 7]);
+            *umma::canon_at<uint4>(Rb, v, rc0 + 8 * p, DK) = o;
         }
         fence_proxy_async_smem();
-        umma::wait_st();
-        umma::fence_before();
-        __syncthreads();  // Rb complete, R scaled
+        __syncthreads();  // Rb complete
         if (tid == 0) {
             umma::fence_after();
             if (CH::HAS_X) {
@@ -986,39 +967,56 @@ __device__ __forceinline__ void chain5_cta(const SeqView& s, int bh, const Chain
             }
             if (op.Rt) bulk_store(op.Rt + ((size_t)bh * s.NC + chunk_of(i)) * DV * DK, Rb, (uint32_t)CH::kR);
         }
-        // Z^T = I^T (+ R X^T) -> bf16 canon row
-        {
-            if (CH::HAS_X) {
-                mbar_wait(bM1, i & 1, &g_tc_status, failed);
-                umma::fence_after();
-            }
-#pragma unroll 1
-            for (int g = 0; g < 2; ++g) {
-                float z[32];
-                if (CH::HAS_X) {
-                    umma::ld_row32(trow + ZC + 32 * g, z);
-                    umma::wait_ld();
-                } else {
+        // while product 1 runs: gamma_C R (+ E) back into TMEM, this thread's row of I^T
+        const float gamC = st.G[C - 1];
+        if (BWD) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) z[j] = 0.f;
-                }
+            for (int p = 0; p < 8; ++p) {
+                const uint4 e = *umma::canon_at<uint4>(st.E, v, rc0 + 8 * p, DK);
+                const uint32_t ev[4] = {e.x, e.y, e.z, e.w};
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const uint4 u = *umma::canon_at<uint4>(st.I, v, 32 * g + 8 * p, C);
-                    const uint32_t uv[4] = {u.x, u.y, u.z, u.w};
-                    uint32_t o[4];
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const float2 f = unpack(uv[h]);
-                        o[h] = pack(f.x + z[8 * p + 2 * h], f.y + z[8 * p + 2 * h + 1]);
-                    }
-                    *umma::canon_at<uint4>(Zb, v, 32 * g + 8 * p, C) = make_uint4(o[0], o[1], o[2], o[3]);
+                for (int h = 0; h < 4; ++h) {
+                    const float2 f = unpack(ev[h]);
+                    x[8 * p + 2 * h] = fmaf(x[8 * p + 2 * h], gamC, f.x);
+                    x[8 * p + 2 * h + 1] = fmaf(x[8 * p + 2 * h + 1], gamC, f.y);
                 }
             }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) x[j] *= gamC;
+        }
+#pragma unroll
+        for (int g = 0; g < 2; ++g)
+            umma::st_row32(trow + rc0 + 32 * g, *reinterpret_cast<const float(*)[32]>(x + 32 * g));
+        uint4 irow[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) irow[p] = *umma::canon_at<uint4>(st.I, v, zc0 + 8 * p, C);
+        umma::wait_st();
+        // Z^T = I^T (+ R X^T) as bf16 into its canon row: product 2's A and the chunk's Z output
+        float z[32];
+        if (CH::HAS_X) {
+            mbar_wait(bM1, i & 1, &g_tc_status, failed);
+            umma::fence_after();
+            umma::ld_row32(trow + ZC + zc0, z);
+            umma::wait_ld();
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) z[j] = 0.f;
+        }
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const uint32_t uv[4] = {irow[p].x, irow[p].y, irow[p].z, irow[p].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float2 f = unpack(uv[h]);
+                o[h] = pack(f.x + z[8 * p + 2 * h], f.y + z[8 * p + 2 * h + 1]);
+            }
+            *umma::canon_at<uint4>(Zb, v, zc0 + 8 * p, C) = make_uint4(o[0], o[1], o[2], o[3]);
         }
         fence_proxy_async_smem();
         umma::fence_before();
-        __syncthreads();  // Zb complete; I, E, G of this stage read
+        __syncthreads();  // Zb complete, R scaled; I, E, G of this stage read
         if (tid == 0) {
             umma::fence_after();
             if (CH::HAS_Y) {
@@ -1033,12 +1031,12 @@ __device__ __forceinline__ void chain5_cta(const SeqView& s, int bh, const Chain
     umma::fence_after();
     if (op.R_out) {
 #pragma unroll 1
-        for (int g = 0; g < 4; ++g) {
+        for (int g = 0; g < 2; ++g) {
             float x[32];
-            umma::ld_row32(trow + 32 * g, x);
+            umma::ld_row32(trow + rc0 + 32 * g, x);
             umma::wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) op.R_out[((size_t)bh * DK + 32 * g + j) * DV + v] = x[j];
+            for (int j = 0; j < 32; ++j) op.R_out[((size_t)bh * DK + rc0 + 32 * g + j) * DV + v] = x[j];
         }
     }
     if (tid == 0 && outputs) bulk_wait<0>();
@@ -1051,14 +1049,14 @@ __device__ __forceinline__ void chain5_cta(const SeqView& s, int bh, const Chain
 }
 
 template <bool BETA>
-__global__ void __launch_bounds__(128, 1) tc_chain5_fwd_kernel(SeqView s, ChainOps op) {
+__global__ void __launch_bounds__(256, 1) tc_chain5_fwd_kernel(SeqView s, ChainOps op) {
     extern __shared__ __align__(16) unsigned char smem[];
     chain5_cta<BETA, false>(s, blockIdx.x, op, smem);
 }
 // Blocks [0, nsr) recompute the forward states (op_f), the rest run the
 // reverse state-gradient scan (op_b).
 template <bool BETA>
-__global__ void __launch_bounds__(128, 1) tc_chain5_bwd_kernel(SeqView s, ChainOps op_f, ChainOps op_b, int nsr) {
+__global__ void __launch_bounds__(256, 1) tc_chain5_bwd_kernel(SeqView s, ChainOps op_f, ChainOps op_b, int nsr) {
     extern __shared__ __align__(16) unsigned char smem[];
     if ((int)blockIdx.x < nsr)
         chain5_cta<BETA, false>(s, blockIdx.x, op_f, smem);
@@ -2754,7 +2752,7 @@ template <bool BETA>
 cudaError_t launch_chain5_fwd(const SeqView& s, const float* S_in, float* S_out, const TcWs& w, cudaStream_t st) {
     constexpr size_t sm = Chain5<BETA, false>::SMEM;
     TC_TRY(smem_attr(tc_chain5_fwd_kernel<BETA>, sm));
-    SF_LAUNCH("tc_scan_fwd", st, tc_chain5_fwd_kernel<BETA><<<s.BH, 128, sm, st>>>(s, fwd_ops(w, S_in, S_out)));
+    SF_LAUNCH("tc_scan_fwd", st, tc_chain5_fwd_kernel<BETA><<<s.BH, 256, sm, st>>>(s, fwd_ops(w, S_in, S_out)));
     return cudaGetLastError();
 }
 template <bool BETA>
@@ -2764,7 +2762,7 @@ cudaError_t launch_chain5_bwd(const SeqView& s, const BwdArgs& a, bool with_sr, 
     TC_TRY(smem_attr(tc_chain5_bwd_kernel<BETA>, sm));
     const int nsr = with_sr ? s.BH : 0;
     SF_LAUNCH("tc_scan_bwd", st,
-              tc_chain5_bwd_kernel<BETA><<<nsr + s.BH, 128, sm, st>>>(
+              tc_chain5_bwd_kernel<BETA><<<nsr + s.BH, 256, sm, st>>>(
                   s, fwd_ops(w, a.S_in, nullptr), bwd_ops(w, a.dS_out, a.dS_in), nsr));
     return cudaGetLastError();
 }
