@@ -128,15 +128,15 @@ def step_roofline(w, ms, pk):
 # (dram__bytes_read.sum + dram__bytes_write.sum) for each kernel of the
 # tensor-core path on the small case of the headline shape (B=1, H=16, T=8192,
 # d=128, one segment cut into two 4096-token pipeline pieces: 1024 chunk-heads
-# per launch, mean of the two launches).  A launch's traffic is this figure
+# per launch, one launch of the timed step).  A launch's traffic is this figure
 # times its chunk-heads.  Valid for the kernels as they were when
 # captured; an entry is removed when its kernel changes.
 MEASURED_TRAFFIC = {
-    "tc_prep": 47729.0,
-    "tc_scan_fwd": 60554.0,
-    "tc_out_og": 123065.0,
-    "tc_scan_bwd": 103362.0,
-    "tc_grad": 209383.0,
+    "tc_prep": 45119.0,
+    "tc_scan_fwd": 60994.0,
+    "tc_out_og": 122950.0,
+    "tc_scan_bwd": 102798.0,
+    "tc_grad": 207216.0,
 }
 
 
