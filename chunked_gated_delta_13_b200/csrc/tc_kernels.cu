@@ -564,7 +564,6 @@ __device__ __forceinline__ void copy_linear(void* s, const void* g, int tid) {
 // bulk copies (the TMA engine) into kStages buffers completing on mbarriers;
 // the outputs are staged by stmatrix and written back by bulk stores.
 constexpr uint32_t kTileK = C * DK * 2;   // a [C][DK] bf16 tile
-constexpr int kOutBufs = 3;  // staged outputs of step i are flushed during step i+1 and must be read by step i+3
 
 template <int DV, bool BETA, bool BWD, int NCG>
 struct Chain {
@@ -576,11 +575,20 @@ struct Chain {
     static constexpr uint32_t TX = kX + kY + kI + C * 4 + kE;       // bytes of one stage (all copied)
     static constexpr size_t OUT = (size_t)NCG * 16 * (DK + C) * 2;  // staged R and Z^T rows of one step
     static constexpr size_t XCH = (size_t)NCG * 12 * 32 * 16;       // 8 R + 4 Z^T fragments per slice
+    // staged outputs of step i are flushed during step i+1 and must have been
+    // read when step i + kOutBufs writes the buffer again
+    static constexpr int kOutBufs = BWD ? 3 : 2;
     static constexpr size_t smem(int stages) { return stages * (size_t)TX + kOutBufs * OUT + XCH + 8 * stages; }
     // as many operand stages as fit (up to 6): a step's operands are requested
-    // kStages - 1 steps ahead, which must cover the latency of the copies
-    static constexpr int kStages = smem(6) <= 227 * 1024 ? 6 : smem(5) <= 227 * 1024 ? 5
-                                 : smem(4) <= 227 * 1024 ? 4 : smem(3) <= 227 * 1024 ? 3 : 2;
+    // kStages - 1 steps ahead, which must cover the latency of the copies.  The
+    // forward chain keeps 3 stages and 2 output buffers (145 KB at d_v = 128,
+    // two slices) so that a Pre CTA (75.5 KB) fits beside it on its SM: the Pre
+    // of later pieces then also runs on the chain's SMs (headline forward 1.49
+    // instead of 1.54 ms, measured); the reverse chain runs beside the gradient
+    // kernel, which leaves no room on an SM, and keeps as many stages as fit.
+    static constexpr int kFit = smem(6) <= 227 * 1024 ? 6 : smem(5) <= 227 * 1024 ? 5
+                              : smem(4) <= 227 * 1024 ? 4 : smem(3) <= 227 * 1024 ? 3 : 2;
+    static constexpr int kStages = BWD ? kFit : (kFit < 3 ? kFit : 3);
     static constexpr size_t SMEM = smem(kStages);
 };
 
@@ -618,8 +626,8 @@ __device__ __forceinline__ void chain_cta(const SeqView& s, int bh, int vb, cons
     const int vr = 16 * g;                  // first row of this slice in the CTA's tiles
     const size_t Tp = (size_t)s.NC * C;
     unsigned char* outs = smem + NS * (size_t)CH::TX;
-    uint4* xch = reinterpret_cast<uint4*>(outs + kOutBufs * CH::OUT) + g * 12 * 32 + lane;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(outs + kOutBufs * CH::OUT + CH::XCH);
+    uint4* xch = reinterpret_cast<uint4*>(outs + CH::kOutBufs * CH::OUT) + g * 12 * 32 + lane;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(outs + CH::kOutBufs * CH::OUT + CH::XCH);
     bool failed = false;
 
     auto chunk_of = [&](int i) { return BWD ? s.NC - 1 - i : i; };
@@ -651,7 +659,7 @@ __device__ __forceinline__ void chain_cta(const SeqView& s, int bh, int vb, cons
     };
     const bool outputs = op.Rt || op.Zt;
     auto flush = [&](int i) {  // thread 0: bulk-store the staged outputs of step i
-        unsigned char* o = outs + (i % kOutBufs) * CH::OUT;
+        unsigned char* o = outs + (i % CH::kOutBufs) * CH::OUT;
         const size_t blk = ((size_t)bh * s.NC + chunk_of(i)) * DV + v0;
         if (op.Rt) bulk_store(op.Rt + blk * DK, o, NCG * 16 * DK * 2);
         if (op.Zt) bulk_store(op.Zt + blk * C, o + NCG * 16 * DK * 2, NCG * 16 * C * 2);
@@ -681,7 +689,7 @@ __device__ __forceinline__ void chain_cta(const SeqView& s, int bh, int vb, cons
             if (outputs && i > 0) flush(i - 1);
         }
         const Stage st = stage(i % NS);
-        bf16* Rs = reinterpret_cast<bf16*>(outs + (i % kOutBufs) * CH::OUT);  // [16 NCG][DK]
+        bf16* Rs = reinterpret_cast<bf16*>(outs + (i % CH::kOutBufs) * CH::OUT);  // [16 NCG][DK]
         bf16* Zs = Rs + NCG * 16 * DK;                                        // [16 NCG][C]
         // the entering R as bf16 fragments of this warp's k-tiles 2q, 2q+1
         uint32_t sa[2][4];
@@ -782,7 +790,7 @@ __device__ __forceinline__ void chain_cta(const SeqView& s, int bh, int vb, cons
                 }
         }
         if (outputs) fence_proxy_async_smem();
-        if (tid == 0 && outputs) bulk_wait_read<1>();  // step i-2's outputs left their buffer
+        if (tid == 0 && outputs) bulk_wait_read<CH::kOutBufs - 2>();  // the buffer step i+1 writes is read out
         __syncthreads();
     }
     if (tid == 0) {
