@@ -1228,6 +1228,11 @@ tc_out2_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
         mbar_init(&bIn[1], 1);
         mbar_init_fence();
         tk[0] = atomicAdd(ticket, 1);
+        if (maps.on) {
+            tma_prefetch_map(&maps.q);
+            tma_prefetch_map(&maps.k);
+            if (OG) tma_prefetch_map(&maps.dO);
+        }
     }
     __syncthreads();
     int j = tk[0];
@@ -2012,7 +2017,7 @@ struct G5 {
     static constexpr size_t kEpiB = (size_t)C * 128 * 2 + 6 * (size_t)C * C * 2;
     static constexpr size_t kB = kStateB > kEpiB ? kStateB : kEpiB;
     static constexpr size_t SMEM = 2 * kQK + 4 * kV + kB + (size_t)C * C * 4 + (size_t)C * C * 2 +
-                                   (size_t)P_ROWS * C * 4 + 16 * 4 + 4 * C * 4 + 16 * 8 + 16;
+                                   (size_t)P_ROWS * C * 4 + 20 * 4 + 4 * C * 4 + 16 * 8 + 16;
 };
 
 template <int DV, bool BETA>
@@ -2044,7 +2049,7 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
     float* Lf = reinterpret_cast<float*>(p);  p += C * C * 4;   // [C][C] fp32, row-major
     bf16* Ms = reinterpret_cast<bf16*>(p);    p += C * C * 2;   // [C][C]
     float* part = reinterpret_cast<float*>(p); p += P_ROWS * C * 4;
-    float* red = reinterpret_cast<float*>(p);  p += 16 * 4;
+    float* red = reinterpret_cast<float*>(p);  p += 20 * 4;  // [16] per-warp <S0, dS_C>, [3] for the dG warps
     float* Gsb = reinterpret_cast<float*>(p);  p += 2 * C * 4;  // [2][C]
     float* Bsb = reinterpret_cast<float*>(p);  p += 2 * C * 4;  // [2][C]
     uint64_t* bars = reinterpret_cast<uint64_t*>(p);  p += 16 * 8;
@@ -2161,6 +2166,14 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
         for (int i = 0; i < 15; ++i) mbar_init(&bars[i], 1);
         mbar_init_fence();
         tk[0] = atomicAdd(ticket, 1);
+        if (maps.on) {
+            tma_prefetch_map(&maps.q);
+            tma_prefetch_map(&maps.k);
+            tma_prefetch_map(&maps.dO);
+            if (BETA) tma_prefetch_map(&maps.v);
+            tma_prefetch_map(&maps.dq);
+            tma_prefetch_map(&maps.dk);
+        }
     }
     __syncthreads();
     int j = tk[0];
@@ -2641,38 +2654,39 @@ tc_grad5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ 
             }
         }
     }
-    if (w == 15) {
-        // ---- dG, dg (chunk-local reverse cumsum), dbeta; two tokens per lane
+    if (w >= 14) {
+        // ---- dG, dg (chunk-local reverse cumsum), dbeta; warps 14 and 15, one token per lane
         auto P = [&](int row, int n, int i) {
             float x = 0.f;
             for (int u = 0; u < n; ++u) x += part[(row + u) * C + i];
             return x;
         };
-        float x[2], zs = 0.f;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int i = 2 * lane + h;
-            x[h] = P(P_INTER, GW, i) + P(P_ROWP, GW, i) - P(P_COLP, 4, i) - P(P_Z, GW, i);
-            zs += P(P_Z, GW, i);
-            if (BETA) {
-                x[h] += P(P_ROWA, GW, i) - P(P_COLA, 4, i) + __expf(Gs[i]) * Bs[i] * P(P_KT, 4, i);
-                if (i < nval) dbeta[bh * s.hs_g + t0 + i] = P(P_DBC, 4, i) + P(P_DBR, GW, i);
-            }
+        const int half = w - 14, i = 32 * half + lane;
+        float x = P(P_INTER, GW, i) + P(P_ROWP, GW, i) - P(P_COLP, 4, i) - P(P_Z, GW, i);
+        float zs = P(P_Z, GW, i);
+        if (BETA) {
+            x += P(P_ROWA, GW, i) - P(P_COLA, 4, i) + __expf(Gs[i]) * Bs[i] * P(P_KT, 4, i);
+            if (i < nval) dbeta[bh * s.hs_g + t0 + i] = P(P_DBC, 4, i) + P(P_DBR, GW, i);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
-        float sdot = 0.f;
-        for (int u = 0; u < 16; ++u) sdot += red[u];
-        if (lane == 31) x[1] += __expf(gC) * sdot + zs;
-        float suf = x[0] + x[1];
+        if (lane == 0) red[16 + half] = zs;
+        asm volatile("bar.sync 1, 64;\n" ::: "memory");
+        if (half == 1 && lane == 31) {  // the last token carries the state terms
+            float sdot = 0.f;
+            for (int u = 0; u < 16; ++u) sdot += red[u];
+            x += __expf(gC) * sdot + (red[16] + red[17]);
+        }
+        float suf = x;  // sum over this warp's tokens from this one on
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float y = __shfl_down_sync(0xffffffffu, suf, o);
             if (lane + o < 32) suf += y;
         }
-        float* dgb = dg + bh * s.hs_g + t0;
-        if (2 * lane < nval) dgb[2 * lane] = suf;
-        if (2 * lane + 1 < nval) dgb[2 * lane + 1] = suf - x[0];
+        if (half == 1 && lane == 0) red[18] = suf;
+        asm volatile("bar.sync 1, 64;\n" ::: "memory");
+        if (half == 0) suf += red[18];
+        if (i < nval) dg[bh * s.hs_g + t0 + i] = suf;
     }
     if (tid == 0) bulk_wait_read<0>();  // the tensor-map stores have read the staging
     __syncthreads();  // partial sums consumed, the staging read out

@@ -164,6 +164,11 @@ __device__ __forceinline__ void tma_load5(void* sdst, const void* map, int c2, i
         "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(0), "r"(c2), "r"(c3), "r"(c4), "r"(smem_u32(bar))
         : "memory");
 }
+// Bring a tensor map (a __grid_constant__ parameter) into the TMA unit's
+// descriptor cache ahead of its first copy.
+__device__ __forceinline__ void tma_prefetch_map(const void* map) {
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
 __device__ __forceinline__ void tma_store5(const void* map, int c2, int c3, int c4, const void* ssrc) {
     asm volatile("cp.async.bulk.tensor.5d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4, %5}], [%6];\n" ::"l"(
                      reinterpret_cast<uint64_t>(map)),
