@@ -1992,6 +1992,250 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
 //   [0,64) Q K^T -> [0,128) dk       [64,128) K K^T        [128,192) dP -> dT_b -> dA
 //   [192,320) dq                     [320,448) dV_new S0^T -> dv
 //   [448,512) dW K^T -> X
+// Out (+ OG) on tcgen05 (d_v = 128): the same products as tc_out2_kernel,
+// issued by one thread into TMEM accumulators: P' = Q K^T and O1 = Q S0
+// (M = 64 token rows), with OG D^T = (scale gamma * dO)^T Q (M = 128 d_v rows);
+// then, from P (the masked, scaled bf16 tile the 8 warps build from P'),
+// O2 = P V_new (M = 64) and with OG dVi^T = dO^T P (M = 128).  O = scale gamma O1
+// + O2.  Persistent with two buffers of all input tiles (Q, K, dO by tensor
+// maps, S0^T, V_new^T, G by bulk copies), like tc_out2_kernel.
+// TMEM columns: P' [0, 64), O1 [64, 192), O2 [192, 320), dVi^T [320, 384),
+// D^T [384, 512).
+template <bool OG>
+struct O5 {
+    static constexpr int DV = 128;
+    static constexpr size_t kQ = (size_t)C * DK * 2;
+    static constexpr size_t kS = (size_t)DV * DK * 2;
+    static constexpr size_t kVn = (size_t)DV * C * 2;
+    static constexpr size_t kdO = OG ? (size_t)C * DV * 2 : 0;
+    static constexpr size_t kBuf = 2 * kQ + kS + kVn + kdO + C * 4;
+    static constexpr size_t SMEM = 2 * kBuf + (size_t)C * C * 2 + kdO + 4 * 8 + 16;
+    static constexpr uint32_t TP = 0, TO1 = 64, TO2 = 192, TDVI = 320, TDT = 384;
+};
+
+template <bool OG>
+__global__ void __launch_bounds__(256, 1)
+tc_out5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k, const float* __restrict__ Gc,
+               const bf16* __restrict__ Vnt, const bf16* __restrict__ S0t, bf16* __restrict__ o,
+               const bf16* __restrict__ dO, bf16* __restrict__ dVito, bf16* __restrict__ Dto,
+               int* __restrict__ ticket, const __grid_constant__ TokMaps maps) {
+    using L = O5<OG>;
+    constexpr int DV = L::DV;
+    extern __shared__ __align__(16) unsigned char smem[];
+    bf16* Ps = reinterpret_cast<bf16*>(smem + 2 * L::kBuf);                 // [C][C] canon
+    bf16* dOg = reinterpret_cast<bf16*>(smem + 2 * L::kBuf + C * C * 2);     // [C][DV] canon, scale gamma dO
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * L::kBuf + C * C * 2 + L::kdO);
+    uint64_t* bIn = bars;  // [2]
+    uint64_t* bm1 = bars + 2;
+    uint64_t* bm2 = bars + 3;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
+    int* tk = reinterpret_cast<int*>(bars + 4) + 1;  // [2]
+    auto Qb = [&](int b) { return reinterpret_cast<bf16*>(smem + b * L::kBuf); };
+    auto Kb = [&](int b) { return reinterpret_cast<bf16*>(smem + b * L::kBuf + L::kQ); };
+    auto Sb = [&](int b) { return reinterpret_cast<bf16*>(smem + b * L::kBuf + 2 * L::kQ); };
+    auto Vb = [&](int b) { return reinterpret_cast<bf16*>(smem + b * L::kBuf + 2 * L::kQ + L::kS); };
+    auto dOb = [&](int b) { return reinterpret_cast<bf16*>(smem + b * L::kBuf + 2 * L::kQ + L::kS + L::kVn); };
+    auto Gb = [&](int b) {
+        return reinterpret_cast<float*>(smem + b * L::kBuf + 2 * L::kQ + L::kS + L::kVn + L::kdO);
+    };
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int gq = lane >> 2, tq = lane & 3, mw = w & 3, nh = w >> 2;
+    const int total = s.NC * s.BH;
+    const size_t Tp = (size_t)s.NC * C;
+    bool failed = false;
+    auto where = [&](int j, int& c, int& bh) {
+        bh = j / s.NC;
+        c = j - bh * s.NC;
+    };
+    auto issue = [&](int j, int b) {
+        int c, bh;
+        where(j, c, bh);
+        const int t0 = c * C, nval = min(C, s.T - t0);
+        const size_t ci = (size_t)bh * s.NC + c;
+        const bool tma = maps.on && nval == C;
+        if (!tma) {
+            umma::load_canon<C, DK, 256>(Qb(b), q + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+            umma::load_canon<C, DK, 256>(Kb(b), k + bh * s.hs_k + (size_t)t0 * DK, DK, nval, tid);
+            if (OG) umma::load_canon<C, DV, 256>(dOb(b), dO + bh * s.hs_v + (size_t)t0 * DV, DV, nval, tid);
+        }
+        cp_async_commit();
+        if (tid == 0) {
+            mbar_expect_tx(&bIn[b], (uint32_t)(L::kS + L::kVn + C * 4 + (tma ? 2 * L::kQ + L::kdO : 0)));
+            bulk_load(Sb(b), S0t + ci * DV * DK, (uint32_t)L::kS, &bIn[b]);
+            bulk_load(Vb(b), Vnt + ci * DV * C, (uint32_t)L::kVn, &bIn[b]);
+            bulk_load(Gb(b), Gc + bh * Tp + t0, C * 4, &bIn[b]);
+            if (tma) {
+                tma_load5(Qb(b), &maps.q, 0, t0 / 8, bh, &bIn[b]);
+                tma_load5(Kb(b), &maps.k, 0, t0 / 8, bh, &bIn[b]);
+                if (OG) tma_load5(dOb(b), &maps.dO, 0, t0 / 8, bh, &bIn[b]);
+            }
+        }
+    };
+
+    if (tid == 0) {
+        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        mbar_init_fence();
+        tk[0] = atomicAdd(ticket, 1);
+        if (maps.on) {
+            tma_prefetch_map(&maps.q);
+            tma_prefetch_map(&maps.k);
+            if (OG) tma_prefetch_map(&maps.dO);
+        }
+    }
+    if (w == 0) umma::alloc(tslot, 512);
+    __syncthreads();
+    umma::fence_after();
+    const uint32_t tm = *tslot;
+    const uint32_t trow = umma::taddr(tm, 32 * mw, 0);  // this warp's lane quarter
+    int j = tk[0];
+    if (j < total) issue(j, 0);
+    constexpr uint32_t IP = umma::idesc_bf16(64, 64, false, false);
+    constexpr uint32_t IO = umma::idesc_bf16(64, 128, false, false);
+    constexpr uint32_t IDT = umma::idesc_bf16(128, 128, true, true);
+    constexpr uint32_t IDVI = umma::idesc_bf16(128, 64, true, true);
+    for (int it = 0; j < total; ++it) {
+        const int buf = it & 1;
+        const uint32_t par = (uint32_t)(it & 1);
+        if (tid == 0) tk[(it + 1) & 1] = atomicAdd(ticket, 1);
+        cp_async_wait<0>();
+        mbar_wait(&bIn[buf], (uint32_t)((it >> 1) & 1), &g_tc_status, failed);
+        __syncthreads();  // this chunk's tiles are in; the other buffer is free
+        const int jn = tk[(it + 1) & 1];
+        const bool has_next = jn < total;
+        if (has_next) issue(jn, buf ^ 1);
+
+        int c, bh;
+        where(j, c, bh);
+        const int t0 = c * C, nval = min(C, s.T - t0);
+        const bf16* Qs = Qb(buf);
+        const float* Gs = Gb(buf);
+        if (OG) {  // scale gamma_t dO[t][:], canon like dO (every thread 4 pieces)
+            const uint4* src = reinterpret_cast<const uint4*>(dOb(buf));
+            uint4* dst = reinterpret_cast<uint4*>(dOg);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = tid + 256 * u;
+                int r, cc;
+                umma::canon_piece(e, DV, r, cc);
+                const float gs = s.scale * __expf(Gs[r]);
+                uint4 x = src[e];
+                x.x = scale2(x.x, gs, gs);
+                x.y = scale2(x.y, gs, gs);
+                x.z = scale2(x.z, gs, gs);
+                x.w = scale2(x.w, gs, gs);
+                dst[e] = x;
+            }
+            fence_proxy_async_smem();
+            __syncthreads();
+        }
+        if (tid == 0) {  // P' = Q K^T, O1 = Q S0, D^T = (scale gamma dO)^T Q
+            umma::fence_after();
+            umma::chain<DK / 16>(tm + L::TP, IP, false, umma::op_k(Qs, DK), umma::op_k(Kb(buf), DK));
+            umma::chain<DK / 16>(tm + L::TO1, IO, false, umma::op_k(Qs, DK), umma::op_k(Sb(buf), DK));
+            if (OG) umma::chain<C / 16>(tm + L::TDT, IDT, false, umma::op_mn(dOg, DV), umma::op_mn(Qs, DK));
+            umma::commit(bm1);
+        }
+        // P = scale (Q K^T) * Gamma (masked), bf16 canon; warp w: rows of its quarter, columns 32 (w / 4)..
+        mbar_wait(bm1, par, &g_tc_status, failed);
+        umma::fence_after();
+        const int r0 = 16 * mw + gq, r1 = r0 + 8;
+        {
+            float pf[4][4];
+            umma::ld32(trow + L::TP + 32 * nh, pf);
+            umma::wait_ld();
+            const float G0 = Gs[r0], G1 = Gs[r1];
+#pragma unroll
+            for (int jq = 0; jq < 4; ++jq) {
+                const int col = 32 * nh + 8 * jq + 2 * tq;
+                float v[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = (e >> 1) ? r1 : r0, jj = col + (e & 1);
+                    v[e] = (jj <= i) ? s.scale * __expf(((e >> 1) ? G1 : G0) - Gs[jj]) * pf[jq][e] : 0.f;
+                }
+                *umma::canon_at<uint32_t>(Ps, r0, col, C) = pack(v[0], v[1]);
+                *umma::canon_at<uint32_t>(Ps, r1, col, C) = pack(v[2], v[3]);
+            }
+        }
+        fence_proxy_async_smem();
+        umma::fence_before();
+        __syncthreads();  // P complete
+        if (tid == 0) {  // O2 = P V_new, dVi^T = dO^T P
+            umma::fence_after();
+            umma::chain<C / 16>(tm + L::TO2, IO, false, umma::op_k(Ps, C), umma::op_k(Vb(buf), C));
+            if (OG) umma::chain<C / 16>(tm + L::TDVI, IDVI, false, umma::op_mn(dOb(buf), DV), umma::op_mn(Ps, C));
+            umma::commit(bm2);
+        }
+        const size_t ci = (size_t)bh * s.NC + c;
+        const int v = 32 * mw + lane;  // d_v row of the M = 128 accumulators this thread reads
+        if (OG) {  // D^T out while the second products run: row v, columns 64 (w / 4)..
+            bf16* Dg = Dto + ci * DV * DK;
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                float x[32];
+                umma::ld_row32(trow + L::TDT + 64 * nh + 32 * g, x);
+                umma::wait_ld();
+#pragma unroll
+                for (int p4 = 0; p4 < 4; ++p4) {
+                    uint4 u;
+                    u.x = pack(x[8 * p4], x[8 * p4 + 1]);
+                    u.y = pack(x[8 * p4 + 2], x[8 * p4 + 3]);
+                    u.z = pack(x[8 * p4 + 4], x[8 * p4 + 5]);
+                    u.w = pack(x[8 * p4 + 6], x[8 * p4 + 7]);
+                    *reinterpret_cast<uint4*>(Dg + umma::canon_el(v, 64 * nh + 32 * g + 8 * p4, DK)) = u;
+                }
+            }
+        }
+        mbar_wait(bm2, par, &g_tc_status, failed);
+        umma::fence_after();
+        {  // O = scale gamma O1 + O2: rows of this warp's quarter, columns 64 (w / 4)..
+            bf16* ob = o + bh * s.hs_v + (size_t)t0 * DV;
+            const float sg0 = s.scale * __expf(Gs[r0]), sg1 = s.scale * __expf(Gs[r1]);
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                float a[4][4], b[4][4];
+                umma::ld32(trow + L::TO1 + 64 * nh + 32 * g, a);
+                umma::ld32(trow + L::TO2 + 64 * nh + 32 * g, b);
+                umma::wait_ld();
+#pragma unroll
+                for (int jq = 0; jq < 4; ++jq) {
+                    const int col = 64 * nh + 32 * g + 8 * jq + 2 * tq;
+                    if (r0 < nval)
+                        *reinterpret_cast<uint32_t*>(ob + (size_t)r0 * DV + col) =
+                            pack(fmaf(a[jq][0], sg0, b[jq][0]), fmaf(a[jq][1], sg0, b[jq][1]));
+                    if (r1 < nval)
+                        *reinterpret_cast<uint32_t*>(ob + (size_t)r1 * DV + col) =
+                            pack(fmaf(a[jq][2], sg1, b[jq][2]), fmaf(a[jq][3], sg1, b[jq][3]));
+                }
+            }
+        }
+        if (OG) {  // dVi^T out: row v, columns 32 (w / 4)..
+            float x[32];
+            umma::ld_row32(trow + L::TDVI + 32 * nh, x);
+            umma::wait_ld();
+            bf16* dvi = dVito + ci * DV * C;
+#pragma unroll
+            for (int p4 = 0; p4 < 4; ++p4) {
+                uint4 u;
+                u.x = pack(x[8 * p4], x[8 * p4 + 1]);
+                u.y = pack(x[8 * p4 + 2], x[8 * p4 + 3]);
+                u.z = pack(x[8 * p4 + 4], x[8 * p4 + 5]);
+                u.w = pack(x[8 * p4 + 6], x[8 * p4 + 7]);
+                *reinterpret_cast<uint4*>(dvi + umma::canon_el(v, 32 * nh + 8 * p4, C)) = u;
+            }
+        }
+        umma::fence_before();
+        __syncthreads();  // buffer `buf`, P, dOg and TMEM are free
+        j = jn;
+    }
+    umma::fence_before();
+    __syncthreads();
+    if (w == 0) {
+        umma::fence_after();
+        umma::dealloc(tm, 512);
+    }
+}
+
 // Tensor maps of the gradient kernel's token-major tiles (q, k, v, dO in; dq,
 // dk out), each a five-dimensional view of a [BH][T][D] bf16 tensor ordered
 // (column within 8, row within 8, column block, row block, head), so that one
@@ -2864,13 +3108,41 @@ cudaError_t launch_out2(const char* name, const SeqView& s, const bf16* q, const
                             w.oticket, maps));
     return cudaGetLastError();
 }
+// Out on tcgen05 (d_v = 128) unless SF_GDN_OUT=warp selects the warp-level
+// kernel (read once); d_v = 64 always takes the warp-level kernel.
+bool out_tcgen05() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = std::getenv("SF_GDN_OUT");
+        v = (e && std::string(e) == "warp") ? 0 : 1;
+    }
+    return v == 1;
+}
+template <bool OG>
+cudaError_t launch_out5(const char* name, const SeqView& s, const bf16* q, const bf16* k, bf16* o, const bf16* dO,
+                        const TcWs& w, cudaStream_t st) {
+    constexpr size_t sm = O5<OG>::SMEM;
+    TC_TRY(smem_attr(tc_out5_kernel<OG>, sm));
+    TC_TRY(cudaMemsetAsync(w.oticket, 0, sizeof(int), st));
+    const int grid = persistent_grid(s);
+    TokMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    maps.on = canon_map(&maps.q, q, s.BH, s.T, DK, s.hs_k) && canon_map(&maps.k, k, s.BH, s.T, DK, s.hs_k) &&
+              (!OG || canon_map(&maps.dO, dO, s.BH, s.T, 128, s.hs_v));
+    SF_LAUNCH(name, st, tc_out5_kernel<OG><<<grid, 256, sm, st>>>(
+                            s, q, k, w.Gc, w.Vnt, w.S0t, o, dO, OG ? w.dVit : nullptr, OG ? w.Dt : nullptr,
+                            w.oticket, maps));
+    return cudaGetLastError();
+}
 template <int DV>
 cudaError_t launch_out(const SeqView& s, const bf16* q, const bf16* k, bf16* o, const TcWs& w, cudaStream_t st) {
+    if (DV == 128 && out_tcgen05()) return launch_out5<false>("tc_out", s, q, k, o, nullptr, w, st);
     return launch_out2<DV, false>("tc_out", s, q, k, o, nullptr, w, st);
 }
 template <int DV>
 cudaError_t launch_out_og(const SeqView& s, const bf16* q, const bf16* k, bf16* o, const bf16* dO, const TcWs& w,
                           cudaStream_t st) {
+    if (DV == 128 && out_tcgen05()) return launch_out5<true>("tc_out_og", s, q, k, o, dO, w, st);
     return launch_out2<DV, true>("tc_out_og", s, q, k, o, dO, w, st);
 }
 

@@ -1,6 +1,7 @@
 """The kernels selected by environment switches, read once per process: the
-TMEM-resident tcgen05 state chains (SF_GDN_CHAIN=tcgen05) and the warp-level
-gradient kernel (SF_GDN_GRAD=warp).  Each runs in a child process through the
+TMEM-resident tcgen05 state chains (SF_GDN_CHAIN=tcgen05), the warp-level
+gradient kernel (SF_GDN_GRAD=warp) and the warp-level Out kernel
+(SF_GDN_OUT=warp).  Each runs in a child process through the
 same parity, bit-identity and live-state tests as the default kernels."""
 import os
 import subprocess
@@ -15,8 +16,8 @@ SELECT = ("bf16_small or chunk_sizes or config2 or bit_identical_to_standalone o
           "bounded_memory_chain_bit_identical or live_state_standalone")
 
 
-@pytest.mark.parametrize("env", [{"SF_GDN_CHAIN": "tcgen05"}, {"SF_GDN_GRAD": "warp"}],
-                         ids=["tcgen05_chains", "warp_grad"])
+@pytest.mark.parametrize("env", [{"SF_GDN_CHAIN": "tcgen05"}, {"SF_GDN_GRAD": "warp"}, {"SF_GDN_OUT": "warp"}],
+                         ids=["tcgen05_chains", "warp_grad", "warp_out"])
 def test_switched_kernels(env):
     e = dict(os.environ)
     e.update(env)
