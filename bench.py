@@ -134,7 +134,7 @@ def step_roofline(w, ms, pk):
 MEASURED_TRAFFIC = {
     "tc_prep": 45119.0,
     "tc_scan_fwd": 60996.0,
-    "tc_out_og": 122989.0,
+    "tc_out_og": 123340.0,
     "tc_scan_bwd": 102798.0,
     "tc_grad": 206943.0,
 }
