@@ -1159,7 +1159,9 @@ __device__ __forceinline__ void og_products8(const SeqView& s, const bf16* Qs, c
     }
 }
 
-// O = scale (gamma * Q) S0 + (scale (Q K^T) * Gamma) V_new.  Persistent: a CTA
+// O = scale (gamma * Q) S0 + (scale (Q K^T) * Gamma) V_new on warp-level MMAs
+// (d_v = 64, and d_v = 128 when SF_GDN_OUT=warp; tc_out5_kernel below is the
+// tcgen05 version).  Persistent: a CTA
 // of 8 warps takes chunk tickets and copies the next chunk's tiles (Q, K, dO
 // by tensor maps, S0^T, V_new^T, G by bulk copies) into the second of two
 // buffers while it works on the current one.  Warp w computes rows
