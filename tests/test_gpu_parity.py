@@ -104,6 +104,16 @@ def test_bf16_small(dk, dv, beta):
     check(w, TOL_BF16)
 
 
+@pytest.mark.parametrize("T", [1, 17, 63])
+@pytest.mark.parametrize("beta", [True, False])
+def test_bf16_shorter_than_a_chunk(T, beta):
+    """A sequence shorter than one chunk: no tensor map can be made, every tile
+    takes the per-thread copies."""
+    w = small(io="bf16", dk=128, dv=128, T=T, use_beta=beta, qk="l2norm" if beta else "scaled",
+              g_shift=-4.0)
+    check(w, TOL_BF16)
+
+
 @pytest.mark.parametrize("C", [32, 64, 128])
 def test_bf16_chunk_sizes(C):
     check(small(io="bf16", dk=128, dv=128, C=C, T=3 * C + 11, g_shift=-4.0), TOL_BF16)
