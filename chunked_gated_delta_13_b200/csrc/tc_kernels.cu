@@ -1964,36 +1964,7 @@ tc_grad_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
   }
 }
 
-// ------------------------------------------------- grad on tcgen05 (PG) ---
-// Every input gradient of a chunk with the products on the fifth-generation
-// tensor cores: one thread issues each product as a chain of K = 16
-// tcgen05.mma (M = 64 token rows, fp32 accumulators in TMEM, operands read
-// from canon tiles in shared memory), and the 16 warps run the elementwise
-// epilogues between them on the accumulators they load from TMEM (warp w
-// owns rows 16 (w % 4).. and the column group w / 4).  With
-//   P = scale (Q K^T) * Gamma,  M = scale (dO V_new^T) * Gamma,  T = L diag(beta),
-//   dW = -dV_new S0^T,  dT = dW (gamma K)^T + dV_new V^T,  dL = dT diag(beta),
-//   dA = -strictly-lower(L^T dL L^T),  Z = diag(beta) (dA * Gamma):
-//   dq = scale gamma (dO S0^T) + M K
-//   dk = dec (V_new dS_C^T) + gamma (T^T dW) + M^T Q + Z K + Z^T K
-//   dv = T^T dV_new   (dv = dV_new without the beta path)
-// and dG (hence dg, dbeta) from the row and column sums of the elementwise
-// terms, reduced in a fixed order (bit-reproducible).
-//
-// Persistent: a CTA takes chunk tickets from a per-launch counter and copies
-// the next chunk's tiles in while it works on the current one: Q, K, G into
-// the second of two buffers at once; dO and V_new^T once the products reading
-// them are done, then dV_new^T and V, then L; the state tiles last, into the
-// region the epilogue tiles of the current chunk leave.
-//
-// The term gamma (T^T dW) of dk accumulates in place; its share of dG,
-// sum_k K_ik gamma_i (T^T dW)_ik = gamma_i beta_i sum_j L_ji (dW K^T)_ji, is a
-// column sum of L * (dW K^T), taken where dT is formed.
-//
-// TMEM columns (512 allocated; M = 64 uses lanes 0-15 of each quarter):
-//   [0,64) Q K^T -> [0,128) dk       [64,128) K K^T        [128,192) dP -> dT_b -> dA
-//   [192,320) dq                     [320,448) dV_new S0^T -> dv
-//   [448,512) dW K^T -> X
+// ------------------------------------------------------- out on tcgen05 ---
 // Out (+ OG) on tcgen05 (d_v = 128): the same products as tc_out2_kernel,
 // issued by one thread into TMEM accumulators: P' = Q K^T and O1 = Q S0
 // (M = 64 token rows), with OG D^T = (scale gamma * dO)^T Q (M = 128 d_v rows);
@@ -2238,6 +2209,38 @@ tc_out5_kernel(SeqView s, const bf16* __restrict__ q, const bf16* __restrict__ k
     }
 }
 
+// ------------------------------------------------- grad on tcgen05 (PG) ---
+// Every input gradient of a chunk with the products on the fifth-generation
+// tensor cores: one thread issues each product as a chain of K = 16
+// tcgen05.mma (M = 64 token rows, fp32 accumulators in TMEM, operands read
+// from canon tiles in shared memory), and the 16 warps run the elementwise
+// epilogues between them on the accumulators they load from TMEM (warp w
+// owns rows 16 (w % 4).. and the column group w / 4).  With
+//   P = scale (Q K^T) * Gamma,  M = scale (dO V_new^T) * Gamma,  T = L diag(beta),
+//   dW = -dV_new S0^T,  dT = dW (gamma K)^T + dV_new V^T,  dL = dT diag(beta),
+//   dA = -strictly-lower(L^T dL L^T),  Z = diag(beta) (dA * Gamma):
+//   dq = scale gamma (dO S0^T) + M K
+//   dk = dec (V_new dS_C^T) + gamma (T^T dW) + M^T Q + Z K + Z^T K
+//   dv = T^T dV_new   (dv = dV_new without the beta path)
+// and dG (hence dg, dbeta) from the row and column sums of the elementwise
+// terms, reduced in a fixed order (bit-reproducible).
+//
+// Persistent: a CTA takes chunk tickets from a per-launch counter and copies
+// the next chunk's tiles in while it works on the current one: Q, K, G into
+// the second of two buffers at once; dO and V_new^T once the products reading
+// them are done, then dV_new^T and V, then L; the state tiles as soon as the
+// last product completes, into the region the epilogue tiles leave.  Q, K, dO,
+// V arrive and dq, dk leave by tensor-map copies (whole chunks; a short last
+// chunk takes per-thread copies), the rest by bulk copies.
+//
+// The term gamma (T^T dW) of dk accumulates in place; its share of dG,
+// sum_k K_ik gamma_i (T^T dW)_ik = gamma_i beta_i sum_j L_ji (dW K^T)_ji, is a
+// column sum of L * (dW K^T), taken where dT is formed.
+//
+// TMEM columns (512 allocated; M = 64 uses lanes 0-15 of each quarter):
+//   [0,64) Q K^T -> [0,128) dk       [64,128) K K^T        [128,192) dP -> dT_b -> dA
+//   [192,320) dq                     [320,448) dV_new S0^T -> dv
+//   [448,512) dW K^T -> X
 // Tensor maps of the gradient kernel's token-major tiles (q, k, v, dO in; dq,
 // dk out), each a five-dimensional view of a [BH][T][D] bf16 tensor ordered
 // (column within 8, row within 8, column block, row block, head), so that one
